@@ -1,0 +1,288 @@
+"""CPU oracle for the AAAC per-layer codebook fit -- TEST INFRASTRUCTURE.
+
+Only tests/, ``__graft_entry__.smoke()`` and bench.py's cpu_baseline /
+reference legs may import this package.  The product path (the CUDA library
+``activation_aware_codebook_b200``) never imports, links or calls it, and the
+two share no code.  The arithmetic lives in ``aaac_oracle.c`` (plain C, fp64
+and exact integer arithmetic); this module only marshals numpy arrays.
+
+What each entry point follows ("Technical summary: AAAC", gist.science/ko/
+paper/2605.08692) and what pins it (tests/test_oracle_*.py):
+
+  importance        section 2 mech. 2 (I_k = sum_t X^2).  Pinned by an exact
+                    rational sum rounded to fp32 in Python (fractions), on
+                    random and hand-made boundary cases.
+  scales            section 1 / 4 (g=128 INT4, g=16 NVFP4 group scales).
+                    Pinned by torch's own bf16 / float8_e4m3fn conversions.
+  u                 section 2 mech. 4 (normalised weights).  Pinned by numpy
+                    fp32 arithmetic.
+  init_codebooks    section 2 mech. 4, initialisation (quantiles, T1 offset
+                    by half a step).  Pinned by numpy.sort at the ranks.
+  assign            section 2 mech. 4, assign (nearest entry).  Pinned by a
+                    brute-force exact (fractions) argmin, midpoint ties,
+                    duplicates, signed zeros.
+  group_error       section 2 mech. 2 (lower activation-weighted error).
+                    Pinned by exact rational errors and brute-force choice.
+  rint_mul          exact fixed-point terms of the refine sums.  Pinned by
+                    exact rational rounding (half to even).
+  fit               section 2 mech. 4 (alternating assign / refine).  Pinned
+                    by: the RTN special case (fixed uniform INT4 grid), the
+                    plain 1-D k-means special case (equal importance, one
+                    codebook, equal scales), the weighted-mean closed form of
+                    one refine, monotone objective, sorted codebooks.
+  pack / unpack     section 2 mech. 3 and section 4 (BF16 tables, sign-bit
+                    choice, S=16 at 0.0625 bpw).  Pinned by the printed
+                    storage arithmetic (tests/golden/storage_arithmetic.txt)
+                    and by a round trip that recomputes err_final.
+  Final fitted values of a whole run: parity unpinned by the pages (they print
+  no worked example); held only by the pins above.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+INT4 = 0
+NVFP4 = 1
+FREEZE_T0 = 1
+FREEZE_T1 = 2
+SINGLE_CODEBOOK = 4
+
+_lib = None
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [("near_ties", ctypes.c_int64), ("groups_t1", ctypes.c_int64),
+                ("empty_cells", ctypes.c_int64), ("dead_groups", ctypes.c_int64),
+                ("L", ctypes.c_int32), ("pad", ctypes.c_int32)]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        i32 = ctypes.c_int
+        L.orc_bf16_to_f32.restype = ctypes.c_float
+        L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.orc_f32_to_bf16_rn.restype = ctypes.c_uint16
+        L.orc_f32_to_bf16_rn.argtypes = [ctypes.c_float]
+        L.orc_e4m3_to_f32.restype = ctypes.c_float
+        L.orc_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+        L.orc_f32_to_e4m3_rn_sat.restype = ctypes.c_uint8
+        L.orc_f32_to_e4m3_rn_sat.argtypes = [ctypes.c_float]
+        L.orc_exact_sumsq_bf16.restype = ctypes.c_float
+        L.orc_exact_sumsq_bf16.argtypes = [P, i64, i64, ctypes.c_float]
+        L.orc_importance.restype = None
+        L.orc_importance.argtypes = [P, i64, i64, i64, P, P]
+        L.orc_scales.restype = None
+        L.orc_scales.argtypes = [P, i64, i64, i32, i32, P]
+        L.orc_u.restype = None
+        L.orc_u.argtypes = [P, i64, i64, i32, i32, P, P]
+        L.orc_rank_t0.restype = i64
+        L.orc_rank_t0.argtypes = [i64, i32, i32]
+        L.orc_rank_t1.restype = i64
+        L.orc_rank_t1.argtypes = [i64, i32, i32]
+        L.orc_init_codebooks.restype = i32
+        L.orc_init_codebooks.argtypes = [P, i64, i64, i32, i32, P, P]
+        L.orc_assign.restype = None
+        L.orc_assign.argtypes = [P, i32, P, i64, P]
+        L.orc_group_error.restype = ctypes.c_double
+        L.orc_group_error.argtypes = [P, P, P, P, i32]
+        L.orc_rint_mul.restype = i64
+        L.orc_rint_mul.argtypes = [ctypes.c_double, ctypes.c_float]
+        L.orc_fixed_point_L.restype = i32
+        L.orc_fixed_point_L.argtypes = [i64, ctypes.c_double, ctypes.c_double, ctypes.c_double]
+        L.orc_fit.restype = i32
+        L.orc_fit.argtypes = [P, i64, i64, P, P, i32, i32, i32, i32, ctypes.c_uint, P, P, P]
+        L.orc_pack.restype = i32
+        L.orc_pack.argtypes = [P, i64, i64, P, P, i32, i32, i32, ctypes.c_uint, P, P, P, P, P,
+                               P, P]
+        L.orc_unpack.restype = None
+        L.orc_unpack.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, P]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+def ncodes(fmt):
+    return 16 if fmt == INT4 else 15
+
+
+def scale_dtype(fmt):
+    return np.uint16 if fmt == INT4 else np.uint8
+
+
+# --- scalar formats ---------------------------------------------------------
+
+def bf16_to_f32(h):
+    h = np.asarray(h, dtype=np.uint16)
+    return (h.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16_rn(x):
+    x = np.asarray(x, dtype=np.float32).ravel()
+    return np.array([lib().orc_f32_to_bf16_rn(float(v)) for v in x], dtype=np.uint16)
+
+
+def f32_to_e4m3_rn_sat(x):
+    x = np.asarray(x, dtype=np.float32).ravel()
+    return np.array([lib().orc_f32_to_e4m3_rn_sat(float(v)) for v in x], dtype=np.uint8)
+
+
+def e4m3_to_f32(b):
+    b = np.asarray(b, dtype=np.uint8).ravel()
+    return np.array([lib().orc_e4m3_to_f32(int(v)) for v in b], dtype=np.float32)
+
+
+def decode_scales(scales, fmt):
+    """Decoded magnitudes (sign / tag bit ignored), fp32."""
+    s = np.asarray(scales)
+    if fmt == INT4:
+        return bf16_to_f32(s.astype(np.uint16) & 0x7FFF)
+    table = e4m3_to_f32(np.arange(256, dtype=np.uint8))
+    return table[s.astype(np.uint8) & 0x7F]
+
+
+# --- the path ---------------------------------------------------------------
+
+def exact_sumsq_bf16(x_u16, init=0.0):
+    x = _u16(x_u16)
+    return lib().orc_exact_sumsq_bf16(_p(x), x.size, 1, float(init))
+
+
+def importance(X_u16, I_in=None, ldx=None):
+    X = _u16(X_u16)
+    T, K = X.shape
+    out = np.empty(K, dtype=np.float32)
+    I_in = None if I_in is None else np.ascontiguousarray(I_in, dtype=np.float32)
+    lib().orc_importance(_p(X), T, K, ldx if ldx is not None else K, _p(I_in), _p(out))
+    return out
+
+
+def scales(W_u16, fmt, g):
+    W = _u16(W_u16)
+    N, K = W.shape
+    out = np.empty((N, K // g), dtype=scale_dtype(fmt))
+    lib().orc_scales(_p(W), N, K, fmt, g, _p(out))
+    return out
+
+
+def u_values(W_u16, scl, fmt, g):
+    W = _u16(W_u16)
+    N, K = W.shape
+    scl = np.ascontiguousarray(scl, dtype=scale_dtype(fmt))
+    out = np.empty((N, K), dtype=np.float32)
+    lib().orc_u(_p(W), N, K, fmt, g, _p(scl), _p(out))
+    return out
+
+
+def rank_t0(M, n, j):
+    return lib().orc_rank_t0(M, n, j)
+
+
+def rank_t1(M, n, j):
+    return lib().orc_rank_t1(M, n, j)
+
+
+def init_codebooks(W_u16, fmt, g):
+    W = _u16(W_u16)
+    N, K = W.shape
+    scl = np.empty((N, K // g), dtype=scale_dtype(fmt))
+    T = np.zeros((2, 16), dtype=np.float32)
+    rc = lib().orc_init_codebooks(_p(W), N, K, fmt, g, _p(scl), _p(T))
+    assert rc == 0
+    return scl, T
+
+
+def assign(T, n, u):
+    T = np.ascontiguousarray(T, dtype=np.float32)
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    q = np.empty(u.shape, dtype=np.uint8)
+    lib().orc_assign(_p(T), n, _p(u), u.size, _p(q))
+    return q
+
+
+def group_error(u, Ik, Tc, q):
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    Ik = np.ascontiguousarray(Ik, dtype=np.float32)
+    Tc = np.ascontiguousarray(Tc, dtype=np.float32)
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    return lib().orc_group_error(_p(u), _p(Ik), _p(Tc), _p(q), u.size)
+
+
+def rint_mul(a, u):
+    return lib().orc_rint_mul(float(a), float(u))
+
+
+def fixed_point_L(M, I_max, S2_max, U_max):
+    return lib().orc_fixed_point_L(M, I_max, S2_max, U_max)
+
+
+def fit(W_u16, I, scl, T_init, fmt, g, S, iters, flags=0):
+    W = _u16(W_u16)
+    N, K = W.shape
+    I = np.ascontiguousarray(I, dtype=np.float32)
+    scl = np.ascontiguousarray(scl, dtype=scale_dtype(fmt))
+    T = np.array(T_init, dtype=np.float32).reshape(2, 16).copy()
+    err = np.zeros(max(iters, 1), dtype=np.float64)
+    st = Stats()
+    rc = lib().orc_fit(_p(W), N, K, _p(I), _p(scl), fmt, g, S, iters, flags, _p(T), _p(err),
+                       ctypes.cast(ctypes.pointer(st), ctypes.c_void_p))
+    assert rc == 0
+    return T, err[:iters], st
+
+
+def pack(W_u16, I, scl, T, fmt, g, S, flags=0):
+    W = _u16(W_u16)
+    N, K = W.shape
+    I = np.ascontiguousarray(I, dtype=np.float32)
+    scl = np.ascontiguousarray(scl, dtype=scale_dtype(fmt))
+    T = np.ascontiguousarray(T, dtype=np.float32).reshape(2, 16)
+    T_bf16 = np.zeros((2, 16), dtype=np.uint16)
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    tagged = np.zeros_like(scl)
+    nb = (K // S + 7) // 8
+    bits = np.zeros((N, nb), dtype=np.uint8) if S != g else None
+    err = np.zeros(1, dtype=np.float64)
+    ties = np.zeros(1, dtype=np.int64)
+    rc = lib().orc_pack(_p(W), N, K, _p(I), _p(scl), fmt, g, S, flags, _p(T), _p(T_bf16),
+                        _p(codes), _p(tagged), _p(bits), _p(err), _p(ties))
+    assert rc == 0
+    return dict(T_bf16=T_bf16, codes=codes, scales_tagged=tagged, choice_bits=bits,
+                err_final=float(err[0]), near_ties=int(ties[0]))
+
+
+def unpack(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    tagged = np.ascontiguousarray(scales_tagged, dtype=scale_dtype(fmt))
+    bits = None if choice_bits is None else np.ascontiguousarray(choice_bits, dtype=np.uint8)
+    T_bf16 = np.ascontiguousarray(T_bf16, dtype=np.uint16)
+    w_hat = np.empty((N, K), dtype=np.float32)
+    ch = np.empty((N, K // S), dtype=np.uint8)
+    lib().orc_unpack(_p(codes), _p(tagged), _p(bits), _p(T_bf16), N, K, fmt, g, S, _p(w_hat),
+                     _p(ch))
+    return w_hat, ch
+
+
+def run_layer(W_u16, X_u16, fmt, g, S, iters, flags=0):
+    """importance -> init -> fit -> pack, all on the CPU."""
+    I = importance(X_u16)
+    scl, T0 = init_codebooks(W_u16, fmt, g)
+    T, err, st = fit(W_u16, I, scl, T0, fmt, g, S, iters, flags)
+    out = pack(W_u16, I, scl, T, fmt, g, S, flags)
+    out.update(I=I, scales=scl, T_init=T0, T=T, err_hist=err, stats=st)
+    return out
