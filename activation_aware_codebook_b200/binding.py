@@ -1,0 +1,254 @@
+"""Thin Python binding of libaaac.so (include/aaac.h).
+
+Argument marshalling only: torch supplies device memory and the current
+stream, every step of the fit runs in the library's CUDA kernels.  There is no
+CPU fallback: without the built library or a CUDA device every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+INT4 = 0
+NVFP4 = 1
+FREEZE_T0 = 1
+FREEZE_T1 = 2
+SINGLE_CODEBOOK = 4
+IMPORTANCE_ACCUMULATE = 1
+IMPORTANCE_EXACT = 2
+
+STATUS = {0: "AAAC_OK", 1: "AAAC_ERR_INVALID_ARG", 2: "AAAC_ERR_SHAPE", 3: "AAAC_ERR_ALIGN",
+          4: "AAAC_ERR_UNSUPPORTED", 5: "AAAC_ERR_CUDA", 6: "AAAC_ERR_WORKSPACE",
+          7: "AAAC_ERR_TIMEOUT"}
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaaac.so")
+
+EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaac_fit_layer",
+           "aaac_pack", "aaac_last_error", "aaac_version", "aaac_kernel_launches")
+
+
+class AaacError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class CConfig(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("g", ctypes.c_int32), ("S", ctypes.c_int32),
+                ("iters", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+class CStats(ctypes.Structure):
+    _fields_ = [("near_ties", ctypes.c_int64), ("groups_t1", ctypes.c_int64),
+                ("empty_cells", ctypes.c_int64), ("dead_groups", ctypes.c_int64),
+                ("exact_groups", ctypes.c_int64), ("L", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+STATS_BYTES = ctypes.sizeof(CStats)
+
+
+@dataclasses.dataclass
+class Config:
+    fmt: int = INT4
+    g: int = 128
+    S: int = 128
+    iters: int = 20
+    flags: int = 0
+
+    def c(self) -> CConfig:
+        return CConfig(self.fmt, self.g, self.S, self.iters, self.flags)
+
+    @property
+    def n(self) -> int:
+        return 16 if self.fmt == INT4 else 15
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libaaac.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libaaac.so not built ({path}); run "
+                           "python -m activation_aware_codebook_b200.csrc.build")
+    L = ctypes.CDLL(path)
+    P, i64, sz, u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint32
+    L.aaac_workspace_size.restype = sz
+    L.aaac_workspace_size.argtypes = [P, i64, i64, i64]
+    L.aaac_importance.restype = ctypes.c_int
+    L.aaac_importance.argtypes = [P, i64, i64, i64, u32, P, P, sz, P]
+    L.aaac_init_codebooks.restype = ctypes.c_int
+    L.aaac_init_codebooks.argtypes = [P, i64, i64, P, P, P, P, sz, P]
+    L.aaac_fit_layer.restype = ctypes.c_int
+    L.aaac_fit_layer.argtypes = [P, i64, i64, P, P, P, P, P, P, P, sz, P]
+    L.aaac_pack.restype = ctypes.c_int
+    L.aaac_pack.argtypes = [P, i64, i64, P, P, P, P, P, P, P, P, P, P, sz, P]
+    L.aaac_last_error.restype = ctypes.c_char_p
+    L.aaac_last_error.argtypes = []
+    L.aaac_version.restype = ctypes.c_char_p
+    L.aaac_version.argtypes = []
+    L.aaac_kernel_launches.restype = ctypes.c_uint64
+    L.aaac_kernel_launches.argtypes = []
+    _lib = L
+    return L
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(load().aaac_kernel_launches())
+
+
+def _check(status: int):
+    if status != 0:
+        raise AaacError(status, load().aaac_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libaaac takes device tensors only")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda():
+    if not torch.cuda.is_available():
+        raise RuntimeError("libaaac needs a CUDA device; there is no CPU path")
+
+
+def workspace_size(cfg: Optional[Config], N: int = 0, K: int = 0, T: int = 0) -> int:
+    c = cfg.c() if cfg is not None else None
+    return int(load().aaac_workspace_size(ctypes.byref(c) if c is not None else None, N, K, T))
+
+
+def workspace(cfg: Optional[Config], N: int = 0, K: int = 0, T: int = 0,
+              device="cuda") -> torch.Tensor:
+    return torch.empty(workspace_size(cfg, N, K, T), dtype=torch.uint8, device=device)
+
+
+def _bits16(t: torch.Tensor) -> torch.Tensor:
+    assert t.dtype in (torch.bfloat16, torch.int16, torch.uint16), t.dtype
+    return t.contiguous()
+
+
+def importance(X: torch.Tensor, I: Optional[torch.Tensor] = None, accumulate: bool = False,
+               exact: bool = False, ws: Optional[torch.Tensor] = None, stream=None,
+               ncols: Optional[int] = None) -> torch.Tensor:
+    """I_k = sum_t X[t,k]^2 (fp32, exact sum rounded once).  X: [T, ldx] bf16."""
+    _need_cuda()
+    T, ldx = X.shape
+    K = ldx if ncols is None else ncols
+    if X.stride(1) != 1:
+        raise ValueError("X must be row-major")
+    ldx = X.stride(0)
+    if I is None:
+        I = torch.zeros(K, dtype=torch.float32, device=X.device)
+    if ws is None:
+        ws = workspace(None, 0, K, T, X.device)
+    flags = (IMPORTANCE_ACCUMULATE if accumulate else 0) | (IMPORTANCE_EXACT if exact else 0)
+    _check(load().aaac_importance(_ptr(X), T, K, ldx, flags, _ptr(I), _ptr(ws), ws.numel(),
+                                  _stream(stream)))
+    return I
+
+
+def init_codebooks(W: torch.Tensor, cfg: Config, ws: Optional[torch.Tensor] = None,
+                   scales: Optional[torch.Tensor] = None, T: Optional[torch.Tensor] = None,
+                   stream=None):
+    """Absmax scales and quantile codebooks.  Returns (scales, T[2,16])."""
+    _need_cuda()
+    W = _bits16(W)
+    N, K = W.shape
+    sdt = torch.int16 if cfg.fmt == INT4 else torch.uint8
+    if scales is None:
+        scales = torch.empty(N, K // cfg.g, dtype=sdt, device=W.device)
+    if T is None:
+        T = torch.empty(2, 16, dtype=torch.float32, device=W.device)
+    if ws is None:
+        ws = workspace(cfg, N, K, 0, W.device)
+    c = cfg.c()
+    _check(load().aaac_init_codebooks(_ptr(W), N, K, ctypes.byref(c), _ptr(scales), _ptr(T),
+                                      _ptr(ws), ws.numel(), _stream(stream)))
+    return scales, T
+
+
+def fit_layer(W: torch.Tensor, I: torch.Tensor, scales: torch.Tensor, T: torch.Tensor,
+              cfg: Config, ws: Optional[torch.Tensor] = None,
+              err_hist: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
+              stream=None):
+    """cfg.iters assign/refine rounds; T [2,16] fp32 is updated in place.
+    Returns (T, err_hist[iters] fp64, stats bytes)."""
+    _need_cuda()
+    W = _bits16(W)
+    N, K = W.shape
+    if err_hist is None:
+        err_hist = torch.zeros(max(cfg.iters, 1), dtype=torch.float64, device=W.device)
+    if stats is None:
+        stats = torch.zeros(STATS_BYTES, dtype=torch.uint8, device=W.device)
+    if ws is None:
+        ws = workspace(cfg, N, K, 0, W.device)
+    c = cfg.c()
+    _check(load().aaac_fit_layer(_ptr(W), N, K, _ptr(I), _ptr(scales), ctypes.byref(c), _ptr(T),
+                                 _ptr(err_hist), _ptr(stats), _ptr(ws), ws.numel(),
+                                 _stream(stream)))
+    return T, err_hist, stats
+
+
+def decode_stats(stats: torch.Tensor) -> dict:
+    raw = bytes(stats.cpu().numpy().tobytes())
+    s = CStats.from_buffer_copy(raw)
+    return {f: getattr(s, f) for f, _ in CStats._fields_ if f != "reserved"}
+
+
+def pack(W: torch.Tensor, I: torch.Tensor, scales: torch.Tensor, T: torch.Tensor, cfg: Config,
+         ws: Optional[torch.Tensor] = None, out: Optional[dict] = None, stream=None) -> dict:
+    """bf16 tables, final assign, 4-bit codes, sign-tagged scales, choice bits."""
+    _need_cuda()
+    W = _bits16(W)
+    N, K = W.shape
+    dev = W.device
+    if out is None:
+        nb = (K // cfg.S + 7) // 8
+        out = dict(T_bf16=torch.zeros(2, 16, dtype=torch.int16, device=dev),
+                   codes=torch.empty(N, K // 2, dtype=torch.uint8, device=dev),
+                   scales_tagged=torch.empty_like(scales),
+                   choice_bits=(torch.empty(N, nb, dtype=torch.uint8, device=dev)
+                                if cfg.S != cfg.g else None),
+                   err_final=torch.zeros(1, dtype=torch.float64, device=dev))
+    if ws is None:
+        ws = workspace(cfg, N, K, 0, dev)
+    c = cfg.c()
+    _check(load().aaac_pack(_ptr(W), N, K, _ptr(I), _ptr(scales), ctypes.byref(c), _ptr(T),
+                            _ptr(out["T_bf16"]), _ptr(out["codes"]), _ptr(out["scales_tagged"]),
+                            _ptr(out["choice_bits"]), _ptr(out["err_final"]), _ptr(ws),
+                            ws.numel(), _stream(stream)))
+    return out
+
+
+def run_layer(W: torch.Tensor, X: torch.Tensor, cfg: Config, ws: Optional[torch.Tensor] = None,
+              stream=None) -> dict:
+    """importance -> init -> fit -> pack for one linear, all on the GPU."""
+    N, K = W.shape
+    if ws is None:
+        ws = workspace(cfg, N, K, X.shape[0], W.device)
+    I = importance(X, ws=ws, stream=stream)
+    scales, T = init_codebooks(W, cfg, ws=ws, stream=stream)
+    T_init = T.clone()
+    T, err_hist, stats = fit_layer(W, I, scales, T, cfg, ws=ws, stream=stream)
+    out = pack(W, I, scales, T, cfg, ws=ws, stream=stream)
+    out.update(I=I, scales=scales, T_init=T_init, T=T, err_hist=err_hist[:cfg.iters],
+               stats=stats)
+    return out

@@ -1,0 +1,193 @@
+// api.cu -- the extern "C" entry points of libaaac.so (declared in aaac.h):
+// argument validation on the host, workspace carving, and kernel launches.
+// No call allocates memory; every check runs before the first launch, so an
+// invalid call leaves all outputs untouched.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <string>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace aaac {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+}  // namespace aaac
+
+namespace {
+
+thread_local std::string g_last_error;
+
+aaac_status fail(aaac_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+aaac_status ok() {
+  g_last_error.clear();
+  return AAAC_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+aaac_status check_cfg(const aaac_config* cfg) {
+  if (!cfg) return fail(AAAC_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->fmt != AAAC_INT4 && cfg->fmt != AAAC_NVFP4)
+    return fail(AAAC_ERR_UNSUPPORTED, "fmt %d is not AAAC_INT4 or AAAC_NVFP4", cfg->fmt);
+  if (cfg->fmt == AAAC_NVFP4 && cfg->g != 16)
+    return fail(AAAC_ERR_UNSUPPORTED, "NVFP4 needs g == 16 (got %d)", cfg->g);
+  if (!pow2(cfg->g) || cfg->g < 16 || cfg->g > 256)
+    return fail(AAAC_ERR_UNSUPPORTED, "g must be a power of two in [16, 256] (got %d)", cfg->g);
+  if (!pow2(cfg->S) || cfg->S < 8 || cfg->S > cfg->g)
+    return fail(AAAC_ERR_SHAPE, "S must be a power of two with 8 <= S <= g (S=%d, g=%d)",
+                cfg->S, cfg->g);
+  if (cfg->iters < 0) return fail(AAAC_ERR_INVALID_ARG, "iters < 0 (%d)", cfg->iters);
+  if (cfg->flags & ~7u) return fail(AAAC_ERR_INVALID_ARG, "unknown flags 0x%x", cfg->flags);
+  return AAAC_OK;
+}
+
+aaac_status check_layer(int64_t N, int64_t K, const aaac_config* cfg) {
+  if (N <= 0 || K <= 0) return fail(AAAC_ERR_SHAPE, "N and K must be positive (N=%lld K=%lld)",
+                                    (long long)N, (long long)K);
+  if (K % cfg->g) return fail(AAAC_ERR_SHAPE, "K=%lld is not a multiple of g=%d", (long long)K,
+                              cfg->g);
+  if (N > INT32_MAX || K > INT32_MAX || N * K >= ((int64_t)1 << 31))
+    return fail(AAAC_ERR_SHAPE, "N*K must be < 2^31 (N=%lld K=%lld)", (long long)N,
+                (long long)K);
+  return AAAC_OK;
+}
+
+aaac_status check_ptr(const void* p, const char* name, bool required = true) {
+  if (!p) return required ? fail(AAAC_ERR_INVALID_ARG, "%s is NULL", name) : AAAC_OK;
+  if (!aligned16(p)) return fail(AAAC_ERR_ALIGN, "%s is not 16-byte aligned", name);
+  return AAAC_OK;
+}
+
+aaac_status check_ws(void* ws, size_t have, size_t need) {
+  if (!ws) return fail(AAAC_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+  if (!aligned16(ws)) return fail(AAAC_ERR_ALIGN, "workspace is not 16-byte aligned");
+  if (have < need) return fail(AAAC_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", have, need);
+  return AAAC_OK;
+}
+
+aaac_status from_cuda(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return ok();
+  return fail(AAAC_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+size_t weight_side_bytes(const aaac_config* cfg, int64_t N, int64_t K) {
+  if (!cfg || N <= 0 || K <= 0 || cfg->S <= 0) return 0;
+  size_t fit = aaac::fit_ws_bytes(N, K);
+  size_t pack = fit + aaac::pack_extra_bytes(N, K, cfg->S);
+  size_t init = aaac::init_ctl_bytes();
+  size_t m = fit > pack ? fit : pack;
+  return m > init ? m : init;
+}
+
+#define CHECK(x)                         \
+  do {                                   \
+    aaac_status _s = (x);                \
+    if (_s != AAAC_OK) return _s;        \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* aaac_last_error(void) { return g_last_error.c_str(); }
+
+const char* aaac_version(void) { return "libaaac 0.1 (sm_100a)"; }
+
+uint64_t aaac_kernel_launches(void) { return aaac::g_launches.load(std::memory_order_relaxed); }
+
+size_t aaac_workspace_size(const aaac_config* cfg, int64_t N, int64_t K, int64_t T) {
+  size_t need = weight_side_bytes(cfg, N, K);
+  if (T > 0 && K > 0) {
+    size_t imp = aaac::plan_importance(T, K).total;
+    if (imp > need) need = imp;
+  }
+  return need < 256 ? 256 : need;
+}
+
+aaac_status aaac_importance(const void* X, int64_t T, int64_t K, int64_t ldx, uint32_t flags,
+                            float* I, void* ws, size_t ws_bytes, void* stream) {
+  CHECK(check_ptr(X, "X"));
+  CHECK(check_ptr(I, "I"));
+  if (T <= 0 || K <= 0) return fail(AAAC_ERR_SHAPE, "T and K must be positive");
+  if (K % 8 || ldx % 8) return fail(AAAC_ERR_ALIGN, "K and ldx must be multiples of 8");
+  if (ldx < K) return fail(AAAC_ERR_SHAPE, "ldx (%lld) < K (%lld)", (long long)ldx, (long long)K);
+  if (K > INT32_MAX || T > ((int64_t)1 << 40))
+    return fail(AAAC_ERR_SHAPE, "K or T out of range");
+  if (flags & ~3u) return fail(AAAC_ERR_INVALID_ARG, "unknown importance flags 0x%x", flags);
+  CHECK(check_ws(ws, ws_bytes, aaac::plan_importance(T, K).total));
+  return from_cuda(aaac::launch_importance(reinterpret_cast<const uint16_t*>(X), T, K, ldx, flags,
+                                           I, ws, (cudaStream_t)stream),
+                   "aaac_importance");
+}
+
+aaac_status aaac_init_codebooks(const void* W, int64_t N, int64_t K, const aaac_config* cfg,
+                                void* scales, float* T, void* ws, size_t ws_bytes,
+                                void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  CHECK(check_ptr(W, "W"));
+  CHECK(check_ptr(scales, "scales"));
+  CHECK(check_ptr(T, "T"));
+  CHECK(check_ws(ws, ws_bytes, aaac::init_ctl_bytes()));
+  return from_cuda(aaac::launch_init(reinterpret_cast<const uint16_t*>(W), N, K, cfg->fmt, cfg->g,
+                                     scales, T, ws, (cudaStream_t)stream),
+                   "aaac_init_codebooks");
+}
+
+aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
+                           const void* scales, const aaac_config* cfg, float* T,
+                           double* err_hist, aaac_stats* stats, void* ws, size_t ws_bytes,
+                           void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  CHECK(check_ptr(W, "W"));
+  CHECK(check_ptr(I, "I"));
+  CHECK(check_ptr(scales, "scales"));
+  CHECK(check_ptr(T, "T"));
+  CHECK(check_ptr(err_hist, "err_hist", false));
+  CHECK(check_ptr(stats, "stats", false));
+  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K)));
+  return from_cuda(aaac::launch_fit(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
+                                    cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T, err_hist,
+                                    stats, ws, (cudaStream_t)stream),
+                   "aaac_fit_layer");
+}
+
+aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const void* scales,
+                      const aaac_config* cfg, const float* T, uint16_t* T_bf16, uint8_t* codes,
+                      void* scales_tagged, uint8_t* choice_bits, double* err_final, void* ws,
+                      size_t ws_bytes, void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  CHECK(check_ptr(W, "W"));
+  CHECK(check_ptr(I, "I"));
+  CHECK(check_ptr(scales, "scales"));
+  CHECK(check_ptr(T, "T"));
+  CHECK(check_ptr(T_bf16, "T_bf16"));
+  CHECK(check_ptr(codes, "codes"));
+  CHECK(check_ptr(scales_tagged, "scales_tagged"));
+  CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
+  CHECK(check_ptr(err_final, "err_final", false));
+  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K) + aaac::pack_extra_bytes(N, K, cfg->S)));
+  return from_cuda(aaac::launch_pack(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
+                                     cfg->fmt, cfg->g, cfg->S, cfg->flags, T, T_bf16, codes,
+                                     scales_tagged, choice_bits, err_final, ws,
+                                     (cudaStream_t)stream),
+                   "aaac_pack");
+}
+
+}  // extern "C"

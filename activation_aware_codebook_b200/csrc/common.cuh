@@ -1,0 +1,131 @@
+// common.cuh -- device helpers shared by the libaaac kernels (sm_100a).
+//
+// Number formats, IEEE total-order keys, and the per-codebook assignment
+// tables: sorted codebook -> distinct values -> exact midpoint thresholds.
+// "Technical summary: AAAC" section 2, core mechanism 4 (assign each weight to
+// its nearest entry; 1-D Voronoi cells).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "aaac.h"
+
+namespace aaac {
+
+constexpr int kInt4 = 0;
+constexpr int kNvfp4 = 1;
+constexpr int kWarps = 8;             // warps per block of the streaming kernels
+constexpr int kThreads = kWarps * 32;
+constexpr int kSegCols = 256;         // columns a warp covers per row (32 lanes x 8)
+constexpr double kMagic = 6755399441055744.0;  // 1.5 * 2^52: x + magic rounds x to an integer
+
+__host__ __device__ inline int ncodes(int fmt) { return fmt == kInt4 ? 16 : 15; }
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// E4M3 ("fn"): bias 7, 3 mantissa bits, S.1111.111 is NaN; subnormal m/8 * 2^-6.
+__device__ __forceinline__ float e4m3_mag(uint32_t v) {
+  uint32_t e = (v >> 3) & 15u, m = v & 7u;
+  if (e == 0) return __uint2float_rn(m) * 0.001953125f;  // m * 2^-9, exact
+  if (e == 15 && m == 7) return __uint_as_float(0x7fc00000u);
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// Decoded magnitude of a stored scale (the sign bit, a choice tag, ignored).
+template <int FMT>
+__device__ __forceinline__ float load_scale(const void* scales, int64_t idx) {
+  if (FMT == kInt4) {
+    uint32_t h = __ldg(reinterpret_cast<const unsigned short*>(scales) + idx);
+    return __uint_as_float((h & 0x7fffu) << 16);
+  } else {
+    uint32_t v = __ldg(reinterpret_cast<const unsigned char*>(scales) + idx);
+    return e4m3_mag(v & 0x7fu);
+  }
+}
+
+// r = fp32_RN(1/s); a group is live when s > 0 and r is finite.
+__device__ __forceinline__ bool scale_live(float s, float* r) {
+  if (!(s > 0.0f)) { *r = 0.0f; return false; }
+  float rc = __frcp_rn(s);
+  if (!(rc < __uint_as_float(0x7f800000u))) { *r = 0.0f; return false; }
+  *r = rc;
+  return true;
+}
+
+__host__ __device__ __forceinline__ uint32_t order_key_bits(uint32_t b) {
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ uint32_t order_key(float f) { return order_key_bits(__float_as_uint(f)); }
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Assignment tables of one codebook.  With the codebook sorted ascending and
+// v_0 < v_1 < ... < v_{m-1} its distinct values, the nearest entry of u (lowest
+// index on a tie) is idx[c] where c = #{i : u >= thr_i} and thr_i is the
+// smallest fp32 strictly above the exact midpoint (v_i + v_{i+1}) / 2.  Slots
+// past m-1 thresholds hold +inf; idx/val past m-1 repeat the last value.
+struct Book {
+  float thr[16];
+  float val[16];
+  int32_t idx[16];
+};
+
+struct Books {
+  Book b[2];
+};
+
+// Smallest fp32 strictly greater than (a + b) / 2, exactly (a, b finite fp32).
+__device__ inline float midpoint_threshold(float a, float b) {
+  double x = a, y = b;
+  double s = __dadd_rn(x, y);                // two-sum: s + e == a + b exactly
+  double bb = __dsub_rn(s, x);
+  double e = __dadd_rn(__dsub_rn(x, __dsub_rn(s, bb)), __dsub_rn(y, bb));
+  double h = s * 0.5, l = e * 0.5;           // exact halving
+  float f = __double2float_rn(h);
+  double d = __dsub_rn((double)f, h);        // exact: f is within an ulp of h
+  if (d <= l) f = nextafterf(f, __uint_as_float(0x7f800000u));
+  return f;
+}
+
+// Insertion sort of t[0..n) in IEEE total order (one thread).
+__device__ inline void sort_book(float* t, int n) {
+  for (int i = 1; i < n; i++) {
+    float v = t[i];
+    uint32_t kv = order_key(v);
+    int j = i - 1;
+    while (j >= 0 && order_key(t[j]) > kv) { t[j + 1] = t[j]; j--; }
+    t[j + 1] = v;
+  }
+}
+
+// Build the tables of a sorted codebook t[0..n) (one thread).
+__device__ inline void build_book(const float* t, int n, Book* bk) {
+  int m = 0;
+  for (int j = 0; j < n; j++) {
+    if (m == 0 || !(t[j] == bk->val[m - 1])) {  // -0 == +0: one value
+      bk->val[m] = t[j];
+      bk->idx[m] = j;
+      m++;
+    }
+  }
+  for (int i = 0; i < 16; i++) bk->thr[i] = __uint_as_float(0x7f800000u);
+  for (int i = 0; i + 1 < m; i++) bk->thr[i] = midpoint_threshold(bk->val[i], bk->val[i + 1]);
+  for (int i = m; i < 16; i++) { bk->val[i] = bk->val[m - 1]; bk->idx[i] = bk->idx[m - 1]; }
+}
+
+// Count of thresholds <= u (branchless search over 15 sorted thresholds).
+__device__ __forceinline__ int book_count(const Book& bk, float u) {
+  int c = 0;
+  c += (bk.thr[c + 7] <= u) ? 8 : 0;
+  c += (bk.thr[c + 3] <= u) ? 4 : 0;
+  c += (bk.thr[c + 1] <= u) ? 2 : 0;
+  c += (bk.thr[c] <= u) ? 1 : 0;
+  return c;
+}
+
+}  // namespace aaac

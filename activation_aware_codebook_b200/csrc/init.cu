@@ -1,0 +1,240 @@
+// init.cu -- per-group absmax scales and the quantile initialisation.
+//
+// "Technical summary: AAAC", section 1 and section 4 (the 4-bit format fixes
+// the per-group scale structure: g=128 INT4, g=16 NVFP4) and section 2, core
+// mechanism 4, initialisation (T0 and T1 from evenly spaced quantiles of the
+// normalised weights, T1 shifted by half a step).
+//
+//   scales_kernel   one pass over W: absmax of each group (max of the bf16
+//                   magnitude bits, reduced over the group's lanes with warp
+//                   shuffles), then INT4 s = bf16_RN(fp32_RN(a/7)) or NVFP4
+//                   s = e4m3_RN_satfinite(a).
+//   radix_pass      histogram of one 8-bit digit of the IEEE total-order key
+//                   of u = fp32_RN(w * fp32_RN(1/s)), restricted to the keys
+//                   whose higher digits match one of the (at most 32) prefixes
+//                   still being resolved; block-private shared-memory counts
+//                   flushed to global once per block.
+//   radix_select    one thread per target rank walks its prefix's histogram
+//                   and fixes the next digit (4 passes of 8 bits resolve the
+//                   32-bit key exactly, ties included).
+#include "common.cuh"
+#include "internal.h"
+
+namespace aaac {
+
+struct InitCtl {
+  int64_t rank[32];
+  int64_t resid[32];
+  uint32_t prefix[32];
+  uint32_t slot_prefix[32];
+  int32_t nslots;
+  int32_t nranks;
+  int32_t n;
+  int32_t pad;
+  uint32_t hist[32][256];
+};
+
+size_t init_ctl_bytes() { return align256(sizeof(InitCtl)); }
+
+PassPlan plan_pass(int64_t N, int64_t K) {
+  PassPlan p;
+  p.ncb = (int)((K + kSegCols - 1) / kSegCols);
+  int target = 148 * 4;
+  int64_t nrc = (target + p.ncb - 1) / p.ncb;
+  if (nrc > N) nrc = N;
+  if (nrc < 1) nrc = 1;
+  p.rows_per_chunk = (int)((N + nrc - 1) / nrc);
+  p.nrc = (int)((N + p.rows_per_chunk - 1) / p.rows_per_chunk);
+  p.blocks = p.ncb * p.nrc;
+  return p;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads)
+scales_kernel(const uint16_t* __restrict__ W, int N, int K, int g, void* __restrict__ scales,
+              int ncb, int rows_per_chunk) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cb = blockIdx.x % ncb, rc = blockIdx.x / ncb;
+  const int col0 = cb * kSegCols + lane * 8;
+  const bool active = col0 < K;
+  const int lanes_g = g >> 3;
+  const int G = K / g;
+  const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
+  for (int r = r0 + warp; r < r1; r += kWarps) {
+    uint32_t mx = 0;
+    if (active) {
+      uint4 v = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)r * K + col0));
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        mx = max(mx, w[i] & 0x7fffu);
+        mx = max(mx, (w[i] >> 16) & 0x7fffu);
+      }
+    }
+    for (int o = 1; o < lanes_g; o <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (active && (lane & (lanes_g - 1)) == 0) {
+      const float a = __uint_as_float(mx << 16);
+      const int64_t idx = (int64_t)r * G + col0 / g;
+      if (FMT == kInt4) {
+        __nv_bfloat16 s = __float2bfloat16_rn(__fdiv_rn(a, 7.0f));
+        reinterpret_cast<unsigned short*>(scales)[idx] = __bfloat16_as_ushort(s);
+      } else {
+        reinterpret_cast<unsigned char*>(scales)[idx] =
+            (unsigned char)__nv_cvt_float_to_fp8(a, __NV_SATFINITE, __NV_E4M3);
+      }
+    }
+  }
+}
+
+struct RankInit {
+  int64_t rank[32];
+};
+
+__global__ void init_setup(InitCtl* c, RankInit ri, int nranks, int n) {
+  for (int i = threadIdx.x; i < 32 * 256; i += blockDim.x) (&c->hist[0][0])[i] = 0u;
+  if (threadIdx.x < 32) {
+    int i = threadIdx.x;
+    c->rank[i] = i < nranks ? ri.rank[i] : 0;
+    c->resid[i] = c->rank[i];
+    c->prefix[i] = 0u;
+    c->slot_prefix[i] = 0u;
+  }
+  if (threadIdx.x == 0) {
+    c->nslots = 1;
+    c->nranks = nranks;
+    c->n = n;
+  }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads)
+radix_pass(const uint16_t* __restrict__ W, int N, int K, int g, const void* __restrict__ scales,
+           InitCtl* c, int pass, int ncb, int rows_per_chunk) {
+  __shared__ uint32_t sh[32][256];
+  __shared__ uint32_t sp[32];
+  __shared__ int ns;
+  for (int i = threadIdx.x; i < 32 * 256; i += blockDim.x) (&sh[0][0])[i] = 0u;
+  if (threadIdx.x < 32) sp[threadIdx.x] = c->slot_prefix[threadIdx.x];
+  if (threadIdx.x == 0) ns = c->nslots;
+  __syncthreads();
+  const int nslots = ns;
+  const int shift = 24 - 8 * pass;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cb = blockIdx.x % ncb, rc = blockIdx.x / ncb;
+  const int col0 = cb * kSegCols + lane * 8;
+  const bool active = col0 < K;
+  const int G = K / g;
+  const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
+  if (active) {
+    for (int r = r0 + warp; r < r1; r += kWarps) {
+      uint4 v = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)r * K + col0));
+      const float s = load_scale<FMT>(scales, (int64_t)r * G + col0 / g);
+      float rcp;
+      const bool live = scale_live(s, &rcp);
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const float wf = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+        const float u = live ? __fmul_rn(wf, rcp) : 0.0f;
+        const uint32_t key = order_key(u);
+        int slot = 0;
+        if (pass > 0) {
+          const uint32_t pre = key >> (shift + 8);
+          int lo = 0, hi = nslots;  // sorted distinct prefixes
+          while (lo < hi) {
+            int mid = (lo + hi) >> 1;
+            if (sp[mid] < pre) lo = mid + 1; else hi = mid;
+          }
+          slot = (lo < nslots && sp[lo] == pre) ? lo : -1;
+        }
+        if (slot >= 0) atomicAdd(&sh[slot][(key >> shift) & 255u], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nslots * 256; i += blockDim.x) {
+    const uint32_t v = (&sh[0][0])[i];
+    if (v) atomicAdd(&c->hist[0][0] + i, v);
+  }
+}
+
+__global__ void radix_select(InitCtl* c, int pass, float* T) {
+  __shared__ uint32_t newp[32];
+  const int i = threadIdx.x;  // 32 threads
+  const int nr = c->nranks;
+  if (i < nr) {
+    int slot = 0;
+    if (pass > 0) {
+      for (int s = 0; s < c->nslots; s++)
+        if (c->slot_prefix[s] == c->prefix[i]) slot = s;
+    }
+    int64_t want = c->resid[i], cum = 0;
+    int d = 0;
+    for (; d < 255; d++) {
+      const int64_t h = c->hist[slot][d];
+      if (cum + h > want) break;
+      cum += h;
+    }
+    c->resid[i] = want - cum;
+    c->prefix[i] = (pass == 0) ? (uint32_t)d : ((c->prefix[i] << 8) | (uint32_t)d);
+    newp[i] = c->prefix[i];
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < 32 * 256; j += blockDim.x) (&c->hist[0][0])[j] = 0u;
+  if (i == 0) {
+    // sorted distinct prefixes for the next pass (T0's and T1's ranks
+    // interleave, so sort first)
+    for (int a = 1; a < nr; a++) {
+      const uint32_t v = newp[a];
+      int b = a - 1;
+      while (b >= 0 && newp[b] > v) { newp[b + 1] = newp[b]; b--; }
+      newp[b + 1] = v;
+    }
+    int m = 0;
+    for (int r = 0; r < nr; r++)
+      if (m == 0 || c->slot_prefix[m - 1] != newp[r]) c->slot_prefix[m++] = newp[r];
+    c->nslots = m;
+    if (pass == 3) {
+      const int n = c->n;
+      for (int j = 0; j < 16; j++) {
+        T[j] = j < n ? key_to_float(c->prefix[j]) : 0.0f;
+        T[16 + j] = j < n ? key_to_float(c->prefix[n + j]) : 0.0f;
+      }
+    }
+  }
+}
+
+cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* scales,
+                        float* T, void* ws, cudaStream_t st) {
+  const PassPlan pp = plan_pass(N, K);
+  InitCtl* c = reinterpret_cast<InitCtl*>(ws);
+  const int n = ncodes(fmt);
+  const int64_t M = N * K;
+  RankInit ri;
+  for (int j = 0; j < n; j++) {
+    ri.rank[j] = (int64_t)(((__int128)(2 * j + 1) * M) / (2 * n));
+    int64_t r1 = (int64_t)(((__int128)(j + 1) * M) / n);
+    ri.rank[n + j] = r1 > M - 1 ? M - 1 : r1;
+  }
+  for (int j = 2 * n; j < 32; j++) ri.rank[j] = 0;
+  if (fmt == kInt4)
+    scales_kernel<kInt4><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, g, scales, pp.ncb,
+                                                         pp.rows_per_chunk);
+  else
+    scales_kernel<kNvfp4><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, g, scales, pp.ncb,
+                                                          pp.rows_per_chunk);
+  init_setup<<<1, 256, 0, st>>>(c, ri, 2 * n, n);
+  for (int pass = 0; pass < 4; pass++) {
+    if (fmt == kInt4)
+      radix_pass<kInt4><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, g, scales, c, pass,
+                                                        pp.ncb, pp.rows_per_chunk);
+    else
+      radix_pass<kNvfp4><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, g, scales, c, pass,
+                                                         pp.ncb, pp.rows_per_chunk);
+    radix_select<<<1, 32, 0, st>>>(c, pass, T);
+  }
+  count_launches(10);
+  return cudaGetLastError();
+}
+
+}  // namespace aaac

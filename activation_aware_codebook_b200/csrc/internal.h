@@ -1,0 +1,55 @@
+// internal.h -- host-side launchers and workspace layout shared by the
+// translation units of libaaac.so.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "aaac.h"
+
+namespace aaac {
+
+// ---- workspace sections (byte offsets, each 256-aligned) -----------------
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct ImportancePlan {
+  int ncb;        // 256-column strips
+  int rb;         // row blocks
+  int64_t rows_per_rb;
+  size_t partial_bytes;  // double [rb][K]
+  size_t list_bytes;     // int32 [K] flagged columns + counter
+  size_t total;
+};
+ImportancePlan plan_importance(int64_t T, int64_t K);
+
+struct PassPlan {
+  int ncb;        // 256-column strips
+  int nrc;        // row chunks
+  int rows_per_chunk;
+  int blocks;     // ncb * nrc
+};
+PassPlan plan_pass(int64_t N, int64_t K);
+
+size_t fit_ctl_bytes();
+size_t init_ctl_bytes();
+size_t pack_extra_bytes(int64_t N, int64_t K, int S);
+size_t fit_ws_bytes(int64_t N, int64_t K);
+
+// ---- launch accounting (aaac_kernel_launches) ------------------------------
+void count_launches(int n);
+
+// ---- launchers (return cudaGetLastError() of their launches) --------------
+cudaError_t launch_importance(const uint16_t* X, int64_t T, int64_t K, int64_t ldx, uint32_t flags,
+                              float* I, void* ws, cudaStream_t st);
+cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* scales,
+                        float* T, void* ws, cudaStream_t st);
+cudaError_t launch_fit(const uint16_t* W, int64_t N, int64_t K, const float* I,
+                       const void* scales, int fmt, int g, int S, int iters, uint32_t flags,
+                       float* T, double* err_hist, aaac_stats* stats, void* ws, cudaStream_t st);
+cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const float* I,
+                        const void* scales, int fmt, int g, int S, uint32_t flags, const float* T,
+                        uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
+                        uint8_t* choice_bits, double* err_final, void* ws, cudaStream_t st);
+
+}  // namespace aaac

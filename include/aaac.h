@@ -1,0 +1,169 @@
+/*
+ * aaac.h -- C ABI of libaaac.so, the B200 (sm_100a) implementation of the
+ * per-layer codebook fit of AAAC (activation-aware adaptive codebooks) for
+ * 4-bit group-scaled weights.
+ *
+ * Source of the method: "Technical summary: AAAC (activation-aware adaptive
+ * codebooks)", gist.science/ko/paper/2605.08692.  Section references below
+ * are to that page.
+ *
+ * Conventions shared by every call
+ *  - All tensors are caller-allocated DEVICE memory on the current CUDA device,
+ *    except the aaac_config struct, which is host memory read during the call.
+ *    The library allocates nothing: scratch memory is the caller's workspace
+ *    (ws, ws_bytes), sized by aaac_workspace_size().
+ *  - W is the weight, row-major [N][K] bf16 (N output rows, K input columns);
+ *    groups of g (scale) and S (codebook choice) weights run along K.
+ *    X is the calibration activation, row-major [T][ldx] bf16 (T tokens).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Outputs are valid once that stream has synchronised.
+ *  - Pointers must be 16-byte aligned; K and ldx must be multiples of 8.
+ *  - On an invalid argument a call returns an error BEFORE launching anything
+ *    and leaves every output untouched.  A CUDA launch error maps to
+ *    AAAC_ERR_CUDA.  aaac_last_error() gives a message for the calling thread.
+ *  - Calls on one stream may share a workspace; concurrent calls on different
+ *    streams need different workspaces.
+ *  - NaN or infinite weights / activations are outside the contract: results
+ *    are then unspecified, but every memory access stays in bounds.
+ */
+#ifndef AAAC_H
+#define AAAC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AAAC_OK = 0,
+    AAAC_ERR_INVALID_ARG = 1, /* null pointer, bad flag, iters < 0            */
+    AAAC_ERR_SHAPE = 2,       /* K % g, g % S, S % 8, sizes out of range      */
+    AAAC_ERR_ALIGN = 3,       /* pointer or leading dimension not aligned     */
+    AAAC_ERR_UNSUPPORTED = 4, /* format / group size this build does not do  */
+    AAAC_ERR_CUDA = 5,        /* a CUDA runtime error (see aaac_last_error)    */
+    AAAC_ERR_WORKSPACE = 6,   /* ws is NULL or smaller than required           */
+    AAAC_ERR_TIMEOUT = 7      /* reserved: a bounded device wait ran out       */
+} aaac_status;
+
+/* Section 1 / 4: the two 4-bit layouts evaluated on the page.
+ *   AAAC_INT4  : g = 128 (any multiple of 8 up to 256 accepted), codebooks of
+ *                16 entries, scale stored as bf16.
+ *   AAAC_NVFP4 : g = 16, codebooks of 15 entries, scale stored as FP8 E4M3. */
+typedef enum { AAAC_INT4 = 0, AAAC_NVFP4 = 1 } aaac_format;
+
+/* flags of aaac_config */
+#define AAAC_FREEZE_T0 1u         /* never refine T0                            */
+#define AAAC_FREEZE_T1 2u         /* never refine T1                            */
+#define AAAC_SINGLE_CODEBOOK 4u   /* every group takes T0                       */
+
+typedef struct {
+    int32_t fmt;     /* aaac_format                                            */
+    int32_t g;       /* scale group size along K                               */
+    int32_t S;       /* selection group size: S % 8 == 0, g % S == 0           */
+    int32_t iters;   /* assign+refine rounds of aaac_fit_layer, >= 0           */
+    uint32_t flags;  /* AAAC_FREEZE_T0 | AAAC_FREEZE_T1 | AAAC_SINGLE_CODEBOOK */
+} aaac_config;
+
+/* flags of aaac_importance */
+#define AAAC_IMPORTANCE_ACCUMULATE 1u /* I_out = fp32_RN(I_in + sum), I_in read from I */
+#define AAAC_IMPORTANCE_EXACT 2u      /* take the exact path for every column          */
+
+/* Device-side statistics written by aaac_fit_layer (one struct, device memory). */
+typedef struct {
+    int64_t near_ties;      /* groups with |D1-D0| < 1e-6 max(D0,D1), last round  */
+    int64_t groups_t1;      /* selection groups on T1, last round                 */
+    int64_t empty_cells;    /* unfrozen entries left unchanged at the last refine */
+    int64_t dead_groups;    /* scale groups with s == 0 or non-finite 1/s         */
+    int64_t exact_groups;   /* groups whose choice took the exact fp64 path, all rounds */
+    int32_t L;              /* fixed-point exponent of the centroid sums          */
+    int32_t reserved;
+} aaac_stats;
+
+/* Bytes of workspace that a call with this configuration needs.  T is the
+ * token count of aaac_importance (0 when only the weight-side calls are used);
+ * N, K describe the layer (0 when only aaac_importance is used).  One
+ * workspace of the returned size serves every call on these sizes. */
+size_t aaac_workspace_size(const aaac_config* cfg, int64_t N, int64_t K, int64_t T);
+
+/* Column importance, section 2 core mechanism 2:  I_k = sum_t X[t,k]^2.
+ *   X      device bf16 [T][ldx]; only the first K columns are read.
+ *   I      device fp32 [K]; written, and read first when ACCUMULATE is set.
+ *   flags  AAAC_IMPORTANCE_ACCUMULATE, AAAC_IMPORTANCE_EXACT.
+ * The result is the exact sum rounded once to fp32 (nearest, ties to even):
+ * an fp64 pass with a rigorous error bound decides every column whose bound
+ * does not straddle an fp32 rounding boundary; the rest are summed exactly.
+ * Requires 0 < T, 0 < K, K % 8 == 0, ldx % 8 == 0, ldx >= K. */
+aaac_status aaac_importance(const void* X, int64_t T, int64_t K, int64_t ldx, uint32_t flags,
+                            float* I, void* ws, size_t ws_bytes, void* stream);
+
+/* Scales and quantile initialisation, section 2 core mechanism 4
+ * (initialisation: evenly spaced quantiles of the normalised weights, T1
+ * shifted by half a step), with the scale of section 1 / 4 read as
+ *   INT4 : s = bf16_RN(fp32_RN(max|w| / 7))      NVFP4 : s = e4m3_RN_sat(max|w|)
+ *   u = fp32_RN(w * fp32_RN(1/s)); groups with s == 0 or 1/s = inf have u = 0.
+ *   T0[j] = u_(floor((2j+1)M / 2n)),  T1[j] = u_(min(M-1, floor((j+1)M/n)))
+ * over the ascending IEEE total order of all M = N*K values, n = 16 (INT4) or
+ * 15 (NVFP4).
+ *   W       device bf16 [N][K]
+ *   scales  device, written: bf16 [N][K/g] (INT4) or uint8 E4M3 [N][K/g] (NVFP4)
+ *   T       device fp32 [2][16], written; entries j >= n are 0.
+ * Requires N*K < 2^31. */
+aaac_status aaac_init_codebooks(const void* W, int64_t N, int64_t K, const aaac_config* cfg,
+                                void* scales, float* T, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/* The alternating fit, section 2 core mechanisms 2 and 4: cfg->iters rounds of
+ *   assign : u's nearest entry in each codebook (exact distance, lowest index
+ *            on a tie); per selection group of S weights
+ *            D_c = sum I_k (u - T_c[q])^2, choice = (D_1 < D_0) decided exactly
+ *            as by sequential fp64 arithmetic;
+ *   refine : each unfrozen entry becomes the I*s^2-weighted centroid of its
+ *            cell, T = sum A u / sum A with A = I_k s^2, both sums exact
+ *            integer fixed point; an empty cell keeps its value; each
+ *            codebook is then sorted ascending.
+ *   W, scales  as written by aaac_init_codebooks (sign bits ignored)
+ *   I          device fp32 [K]
+ *   T          device fp32 [2][16]: in the start codebooks, out the fitted ones
+ *   err_hist   device fp64 [iters]: sum over groups of s^2 * D_choice at the
+ *              assign of each round (may be NULL)
+ *   stats      device aaac_stats (may be NULL)
+ * Requires N*K < 2^31. */
+aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
+                           const void* scales, const aaac_config* cfg, float* T,
+                           double* err_hist, aaac_stats* stats, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Storage, section 2 core mechanism 3 and section 4: T is sorted and rounded
+ * to bf16, a last assign (as in the fit) runs with the bf16 tables, then
+ *   T_bf16        device uint16 [2][16] (64 bytes; entries j >= n are 0)
+ *   codes         device uint8 [N][K/2]: entry index, low nibble = even k
+ *   scales_tagged device, like scales: the scale with its sign bit set to the
+ *                 group's choice when S == g (0 when S < g)
+ *   choice_bits   device uint8 [N][ceil(K/S/8)], bit j%8 of byte j/8 = choice
+ *                 of selection group j (LSB first); required when S < g,
+ *                 ignored (may be NULL) when S == g
+ *   err_final     device fp64 [1]: sum over weights of I_k (w - s T[c][q])^2
+ *                 (may be NULL) */
+aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const void* scales,
+                      const aaac_config* cfg, const float* T, uint16_t* T_bf16, uint8_t* codes,
+                      void* scales_tagged, uint8_t* choice_bits, double* err_final, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/* Message describing the last failed call on the calling thread ("" after a
+ * successful call).  Valid until the next call on the thread. */
+const char* aaac_last_error(void);
+
+/* Library version string. */
+const char* aaac_version(void);
+
+/* Number of CUDA kernels this library has launched in the process so far
+ * (all threads, all devices).  A measurement aid: the difference across a
+ * region counts the library's kernel launches in it. */
+uint64_t aaac_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* AAAC_H */

@@ -1,0 +1,210 @@
+"""GPU parity: libaaac (through the C ABI) against the CPU oracle, element by
+element, on seeded synthetic inputs.
+
+Bar (AAAC fit contract): importance, scales, initial codebooks, fitted
+codebooks, codes, choice bits and tagged scales bit-exact; err_hist and
+err_final within 1e-5 relative (the GPU sums them in a different order and
+takes clear-cut codebook choices from fp32 sums).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_aware_codebook_b200 import binding as bb
+from activation_aware_codebook_b200 import synth
+
+pytestmark = pytest.mark.gpu
+RTOL = 1e-5
+
+
+def u16(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def npbits(t):
+    a = t.detach().cpu().contiguous().numpy()
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
+def cfg_of(fmt, g, S, iters, flags=0):
+    return bb.Config(fmt, g, S, iters, flags)
+
+
+def layer(N, K, seed, T=64, heavy=True, dist="normal"):
+    W, X = synth.small_layer(N, K, seed, T=T, heavy=heavy, dist=dist)
+    return W.cuda(), X.cuda()
+
+
+# --------------------------------------------------------------------------
+# importance
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("T,K", [(128, 512), (1000, 520), (7, 8), (3000, 4096)])
+def test_importance_bit_exact(T, K):
+    X = synth.make_activations(T, K, seed=T + K, heavy=True).cuda()
+    I = bb.importance(X)
+    ref = oracle.importance(u16(X))
+    assert np.array_equal(npbits(I), ref.view(np.uint32))
+    Ie = bb.importance(X, exact=True)
+    assert np.array_equal(npbits(Ie), ref.view(np.uint32))
+
+
+def test_importance_accumulate_strided_and_boundary():
+    X = synth.make_activations(300, 264, seed=5, heavy=False)
+    wide = torch.zeros(300, 272, dtype=torch.bfloat16)
+    wide[:, :264] = X
+    wide = wide.cuda()
+    I = bb.importance(wide[:120], ncols=264)
+    I = bb.importance(wide[120:], I=I, accumulate=True, ncols=264)
+    Xb = u16(X)
+    ref = oracle.importance(Xb[120:], I_in=oracle.importance(Xb[:120]))
+    assert np.array_equal(npbits(I), ref.view(np.uint32))
+    # columns whose fp64 sum sits on an fp32 rounding boundary
+    cols = [[4096.0, 1.0, 2.0 ** -60, 0.0], [4096.0, 1.0, 0.0, 0.0],
+            [4096.0, 1.0, -(2.0 ** -60), 2.0 ** -61], [1e-39, -1e-39, 2.0 ** -130, 0.0],
+            [2.0 ** 64, 0.0, 0.0, 0.0], [3.0, 5.0, 7.0, 11.0], [0, 0, 0, 0], [1, 1, 1, 1]]
+    Xc = torch.tensor(cols, dtype=torch.float32).t().contiguous().to(torch.bfloat16)
+    Ig = bb.importance(Xc.cuda())
+    assert np.array_equal(npbits(Ig), oracle.importance(u16(Xc)).view(np.uint32))
+    assert float(Ig[0]) == 2.0 ** 24 + 2 and float(Ig[1]) == 2.0 ** 24
+
+
+# --------------------------------------------------------------------------
+# scales, init, fit, pack
+# --------------------------------------------------------------------------
+CASES = [(bb.INT4, 128, 128, 256, 512), (bb.INT4, 128, 16, 37, 640), (bb.NVFP4, 16, 16, 64, 512),
+         (bb.INT4, 32, 8, 48, 256), (bb.NVFP4, 16, 16, 33, 1040)]
+
+
+@pytest.mark.parametrize("fmt,g,S,N,K", CASES)
+def test_init_bit_exact(fmt, g, S, N, K):
+    W, _ = layer(N, K, seed=N * K + g)
+    cfg = cfg_of(fmt, g, S, 0)
+    scl, T = bb.init_codebooks(W, cfg)
+    rscl, rT = oracle.init_codebooks(u16(W), fmt, g)
+    assert np.array_equal(scl.cpu().numpy().view(rscl.dtype), rscl)
+    assert np.array_equal(npbits(T), rT.view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt,g,S,N,K", CASES)
+@pytest.mark.parametrize("iters", [1, 6])
+def test_fit_and_pack_bit_exact(fmt, g, S, N, K, iters):
+    W, X = layer(N, K, seed=3 * N + K + iters, dist="student_t4" if fmt == bb.NVFP4 else "normal")
+    cfg = cfg_of(fmt, g, S, iters)
+    out = bb.run_layer(W, X, cfg)
+    ref = oracle.run_layer(u16(W), u16(X), fmt, g, S, iters)
+    check_against_oracle(out, ref, cfg)
+
+
+def check_against_oracle(out, ref, cfg, label=""):
+    torch.cuda.synchronize()
+    assert np.array_equal(npbits(out["I"]), ref["I"].view(np.uint32)), label
+    assert np.array_equal(out["scales"].cpu().numpy().view(ref["scales"].dtype), ref["scales"])
+    assert np.array_equal(npbits(out["T_init"]), ref["T_init"].view(np.uint32)), label
+    T, rT = out["T"].cpu().numpy(), ref["T"]
+    assert np.array_equal(T.view(np.uint32), rT.view(np.uint32)), (label, T, rT)
+    st = bb.decode_stats(out["stats"])
+    assert st["L"] == ref["stats"].L
+    if cfg.iters:
+        assert st["groups_t1"] == ref["stats"].groups_t1
+        assert st["empty_cells"] == ref["stats"].empty_cells
+        assert st["dead_groups"] == ref["stats"].dead_groups
+        eh = out["err_hist"].cpu().numpy()
+        np.testing.assert_allclose(eh, ref["err_hist"], rtol=RTOL, atol=0)
+    assert np.array_equal(out["T_bf16"].cpu().numpy().view(np.uint16), ref["T_bf16"])
+    assert np.array_equal(out["codes"].cpu().numpy(), ref["codes"]), label
+    assert np.array_equal(out["scales_tagged"].cpu().numpy().view(ref["scales_tagged"].dtype),
+                          ref["scales_tagged"])
+    if cfg.S != cfg.g:
+        assert np.array_equal(out["choice_bits"].cpu().numpy(), ref["choice_bits"])
+    np.testing.assert_allclose(float(out["err_final"][0]), ref["err_final"], rtol=RTOL)
+
+
+def test_single_256x512_int4_workload():
+    """The 256x512 INT4 g=128 S=128 layer, X[128, 512], 10 iterations, seed 0."""
+    wl = synth.WORKLOADS["single-256x512-int4"]
+    lin = wl.linears[0]
+    W = synth.make_weight(lin.N, lin.K, synth.seed_of(wl.name, 0, lin.name, "W"))
+    X = synth.make_activations(wl.tokens, lin.K, synth.seed_of(wl.name, 0, lin.name, "X"),
+                               wl.heavy)
+    cfg = cfg_of(wl.fmt, wl.g, wl.S, wl.iters)
+    out = bb.run_layer(W.cuda(), X.cuda(), cfg)
+    ref = oracle.run_layer(u16(W), u16(X), wl.fmt, wl.g, wl.S, wl.iters)
+    check_against_oracle(out, ref, cfg)
+    eh = out["err_hist"].cpu().numpy()
+    assert np.all(eh[1:] <= eh[:-1] * (1 + 1e-6))
+
+
+# --------------------------------------------------------------------------
+# degenerate inputs
+# --------------------------------------------------------------------------
+def test_dead_groups_constant_weights_and_duplicates():
+    N, K, g = 40, 256, 16
+    W = synth.make_weight(N, K, seed=90)
+    W[0] = 0                      # every group of row 0 has s = 0
+    W[1, :64] = 1e-4              # NVFP4: scale underflows to 0
+    W[2:10] = 0.5                 # constant groups: heavy duplicate u values
+    X = synth.make_activations(32, K, seed=91, heavy=True)
+    X[:, 10:20] = 0               # columns with zero importance
+    for fmt, S in ((bb.NVFP4, 16), (bb.INT4, 16)):
+        cfg = cfg_of(fmt, g, S, 5)
+        out = bb.run_layer(W.cuda(), X.cuda(), cfg)
+        ref = oracle.run_layer(u16(W), u16(X), fmt, g, S, 5)
+        check_against_oracle(out, ref, cfg, label=f"fmt{fmt}")
+        assert bb.decode_stats(out["stats"])["dead_groups"] > 0
+
+
+def test_all_equal_weights():
+    W = torch.full((16, 256), 0.25, dtype=torch.bfloat16)
+    X = synth.make_activations(16, 256, seed=92, heavy=False)
+    cfg = cfg_of(bb.INT4, 128, 128, 3)
+    out = bb.run_layer(W.cuda(), X.cuda(), cfg)
+    ref = oracle.run_layer(u16(W), u16(X), bb.INT4, 128, 128, 3)
+    check_against_oracle(out, ref, cfg)
+
+
+@pytest.mark.parametrize("flags", [bb.FREEZE_T0 | bb.FREEZE_T1, bb.SINGLE_CODEBOOK, bb.FREEZE_T1])
+def test_flags_rtn_single_frozen(flags):
+    N, K, g = 64, 512, 128
+    W, X = layer(N, K, seed=93 + flags)
+    cfg = cfg_of(bb.INT4, g, 16, 4, flags)
+    I = bb.importance(X)
+    scl, _ = bb.init_codebooks(W, cfg)
+    grid = torch.arange(-8, 8, dtype=torch.float32)
+    T0 = torch.stack([grid, grid + 0.5]).cuda()
+    T, eh, st = bb.fit_layer(W, I, scl, T0.clone(), cfg)
+    out = bb.pack(W, I, scl, T, cfg)
+    Wb, Ib, sb = u16(W), I.cpu().numpy(), scl.cpu().numpy()
+    rT, reh, rst = oracle.fit(Wb, Ib, sb, T0.cpu().numpy(), bb.INT4, g, 16, 4, flags)
+    assert np.array_equal(npbits(T), rT.view(np.uint32))
+    np.testing.assert_allclose(eh.cpu().numpy()[:4], reh, rtol=RTOL)
+    rp = oracle.pack(Wb, Ib, sb, rT, bb.INT4, g, 16, flags)
+    assert np.array_equal(out["codes"].cpu().numpy(), rp["codes"])
+    assert np.array_equal(out["choice_bits"].cpu().numpy(), rp["choice_bits"])
+    if flags & bb.SINGLE_CODEBOOK:
+        assert not out["choice_bits"].any()
+
+
+def test_deterministic_bits():
+    W, X = layer(512, 1024, seed=95)
+    cfg = cfg_of(bb.INT4, 128, 16, 8)
+    a = bb.run_layer(W, X, cfg)
+    b = bb.run_layer(W, X, cfg)
+    for k in ("I", "T", "codes", "scales_tagged", "choice_bits", "err_final", "err_hist"):
+        assert torch.equal(a[k].view(torch.uint8), b[k].view(torch.uint8)), k
+
+
+# --------------------------------------------------------------------------
+# full-size layers (the oracle still finishes in seconds on these)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("name,idx,iters", [("llama1b-nvfp4", 0, 20), ("llama8b-int4-s16", 1, 20)])
+def test_full_size_layer(name, idx, iters):
+    wl = synth.WORKLOADS[name]
+    lin = wl.linears[idx]
+    W = synth.make_weight(lin.N, lin.K, synth.seed_of(wl.name, 0, lin.name, "W"), wl.w_dist)
+    tokens = 4096  # importance parity at full token count is tested separately
+    X = synth.make_activations(tokens, lin.K, synth.seed_of(wl.name, 0, lin.x_key, "X"), wl.heavy)
+    cfg = cfg_of(wl.fmt, wl.g, wl.S, iters)
+    out = bb.run_layer(W.cuda(), X.cuda(), cfg)
+    ref = oracle.run_layer(u16(W), u16(X), wl.fmt, wl.g, wl.S, iters)
+    check_against_oracle(out, ref, cfg, label=name)
