@@ -73,6 +73,8 @@ struct Book {
   float thr[16];
   float val[16];
   int32_t idx[16];
+  int32_t m;        // number of distinct values
+  int32_t pad[3];
 };
 
 struct Books {
@@ -116,6 +118,7 @@ __device__ inline void build_book(const float* t, int n, Book* bk) {
   for (int i = 0; i < 16; i++) bk->thr[i] = __uint_as_float(0x7f800000u);
   for (int i = 0; i + 1 < m; i++) bk->thr[i] = midpoint_threshold(bk->val[i], bk->val[i + 1]);
   for (int i = m; i < 16; i++) { bk->val[i] = bk->val[m - 1]; bk->idx[i] = bk->idx[m - 1]; }
+  bk->m = m;
 }
 
 // Count of thresholds <= u (branchless search over 15 sorted thresholds).

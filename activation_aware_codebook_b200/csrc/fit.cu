@@ -9,25 +9,55 @@
 //   core mechanism 4  alternating assign (nearest entry, Voronoi cells) and
 //                     refine (activation-weighted centroid of each cell).
 //
-// One fit round = assign_pass<false> (one streaming pass over W) + fit_finalize
-// (one block).  assign_pass: a warp covers 256 columns of a row (a 16-byte
-// load per lane, 8 weights), keeps the codebook tables in shared memory,
-// finds each weight's nearest entry in both codebooks by a branchless search
-// over exact midpoint thresholds, sums the per-group errors in fp32 and
-// reduces them over the group's lanes with shuffles.  A choice the fp32 sums
-// cannot decide under their rounding-error bound is recomputed by the group's
-// leader lane with the sequential fp64 rule.  The refine sums are exact
-// integers, rint(A 2^L u) and rint(A 2^L) with A = I_k s^2, accumulated as
-// 64-bit integers in shared-memory bins and flushed once per block, so the
-// result does not depend on the order of the additions.
+// One fit round is ONE launch of fit_pass<false>: a streaming pass over W whose
+// last block to finish (atomic ticket, no waiting) does the refine, sorts the
+// books, rebuilds the tables and records the error.  Per block: 4 warps; a warp
+// covers 256 columns of a row (16 bytes per lane) and walks the rows of its
+// chunk with a 6-deep cp.async ring, so several rows per warp are in flight.
+//
+// Nearest entry, per weight and book (exact):
+//   bucket b = rint(u * la + 64) (one FFMA), lut[b] = the count c of distinct-
+//   value thresholds below the bucket (and a flag when two or more thresholds
+//   fall inside it);  pair[c] = (v_c, v_{c+1});  with A = fl(u-v_c)^2 and
+//   B = fl(u-v_{c+1})^2 the count is c+1 when B < A and c when A < B -- both
+//   exact, because rounding is monotone -- and the rare A == B or flagged
+//   buckets take the exact threshold search.  min(A, B) is the squared error.
+// Choice: fp32 group sums when their gap exceeds the rounding bound, else the
+//   sequential fp64 rule (the group's leader lane recomputes it).
+// Refine sums: per weight rint(A 2^L u) and rint(A 2^L), A = I_k s^2, as the
+//   raw bit patterns of fp64 FMA/ADD results with magic constants; summed in
+//   lane-private shared-memory bins modulo 2^64, which keeps num exact modulo
+//   2^51 and den modulo 2^52 -- exact because every lane's partial sum is far
+//   below those bounds.  Integer sums make the result independent of order.
 #include "common.cuh"
 #include "internal.h"
 
 namespace aaac {
 
+constexpr int kNB = 128;                  // bucket LUT entries
+constexpr int kFitWarps = 2;
+constexpr int kFitThreads = kFitWarps * 32;
+constexpr int kStages = 6;                // rows per warp in flight
+constexpr int kFitBlocksPerSM = 5;
+constexpr float kBucketMagic = 12582912.0f;           // 1.5 * 2^23
+constexpr double kDenMagic = 4503599627370496.0;      // 2^52
+#define kInf __int_as_float(0x7f800000)
+
+// lut[c][b] = 8 * (distinct-value count below bucket b) for book c, or 128
+// (the NaN pair, which forces the exact search) when two or more of the
+// book's thresholds fall strictly inside the bucket.  pair[c][j] =
+// (v_j, v_{j+1}); pair[c][16] = (NaN, NaN).
+struct Tables {
+  Book bk[2];
+  float2 pair[2][17];
+  uint8_t lut[2][kNB];
+  float la;
+  int32_t pad[3];
+};
+
 struct FitCtl {
+  Tables tb;
   float T[2][16];
-  Books bk;
   int32_t n;
   int32_t L;
   double twoL;
@@ -35,17 +65,21 @@ struct FitCtl {
   uint32_t Umax_bits;
   unsigned long long S2max_bits;
   unsigned long long dead_groups;
-  unsigned long long bins[2][16][2];
+  long long bins[2][16][2];
   unsigned long long near_ties;
   unsigned long long groups_t1;
   unsigned long long exact_groups;
   unsigned long long empty_cells;
+  unsigned int ticket;
+  int32_t pad2;
 };
 
 size_t fit_ctl_bytes() { return align256(sizeof(FitCtl)); }
 
+static PassPlan fit_plan(int64_t N, int64_t K) { return plan_pass(N, K, 148 * kFitBlocksPerSM); }
+
 size_t fit_ws_bytes(int64_t N, int64_t K) {
-  const PassPlan pp = plan_pass(N, K);
+  const PassPlan pp = fit_plan(N, K);
   return fit_ctl_bytes() + align256((size_t)pp.blocks * sizeof(double));
 }
 
@@ -53,15 +87,62 @@ size_t pack_extra_bytes(int64_t N, int64_t K, int S) {
   return align256((size_t)N * (size_t)(K / S));
 }
 
+static size_t smem_bytes(bool pack) {
+  size_t b = (sizeof(Tables) + 15) & ~(size_t)15;
+  b += (size_t)kFitWarps * kStages * 32 * sizeof(uint4);
+  if (!pack) b += (size_t)kFitWarps * 32 * 32 * sizeof(ulonglong2);
+  return b;
+}
+
 // ---------------------------------------------------------------------------
-// prep: the exact maxima that fix the refine's fixed-point exponent
+// buckets and tables
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bucket_t(float u, float la) {
+  return __fmaf_rn(u, la, kBucketMagic + (float)(kNB / 2));
+}
+
+// rint(x * la + 64) without wrap-around, clamped to [-1, kNB] (table builder).
+__device__ inline int bucket_raw(float x, float la) {
+  if (!(fabsf(x) * la < 4.0e6f)) return (x < 0.0f) ? -1 : kNB;
+  const int r = (int)(__float_as_uint(bucket_t(x, la)) - __float_as_uint(kBucketMagic));
+  return min(max(r, -1), kNB);
+}
+
+// Entry of bucket b for book c: 8 * #(thresholds <= every u of the bucket),
+// or 128 when two or more thresholds fall strictly inside it.
+__device__ uint8_t lut_entry(const Tables& tb, int c, int b) {
+  const Book& bk = tb.bk[c];
+  int base = 0, inner = 0;
+  for (int i = 0; i + 1 < bk.m; i++) {
+    const float th = bk.thr[i];
+    const int rb = bucket_raw(th, tb.la);
+    if (rb < b) {
+      base++;
+    } else if (rb == b) {
+      const int rp = bucket_raw(nextafterf(th, -kInf), tb.la);
+      if (rp < b) base++;   // th is the bucket's smallest value
+      else inner++;
+    }
+  }
+  return (uint8_t)(inner > 1 ? 128 : 8 * base);
+}
+
+__device__ void fill_pairs(Tables& tb, int c) {
+  const Book& bk = tb.bk[c];
+  for (int j = 0; j < 16; j++)
+    tb.pair[c][j] = make_float2(bk.val[j], (j + 1 < bk.m) ? bk.val[j + 1] : kInf);
+  tb.pair[c][16] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+}
+
+// ---------------------------------------------------------------------------
+// prep: the exact maxima that fix the refine's fixed-point exponent and the
+// bucket scale
 // ---------------------------------------------------------------------------
 template <int FMT>
 __global__ void __launch_bounds__(kThreads)
 fit_prep(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
          const void* __restrict__ scales, int g, FitCtl* ctl, int ncb, int rows_per_chunk) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // I_max over all columns
   uint32_t im = 0;
   for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < K; k += gridDim.x * blockDim.x)
     im = max(im, __float_as_uint(I[k]));
@@ -123,56 +204,191 @@ __device__ void write_stats(const FitCtl* ctl, aaac_stats* st) {
   st->reserved = 0;
 }
 
+__device__ float bucket_scale(const FitCtl* ctl) {
+  const float Umax = __uint_as_float(ctl->Umax_bits);
+  return Umax > 0.0f ? __fdiv_rn(62.5f, Umax) : 0.0f;  // |u| * la < 63: buckets 1..127
+}
+
+// Tables of both books from ctl->T (sorted first), all threads of one block.
+__device__ void publish_tables(FitCtl* ctl, Tables& tb, int n, bool sort_in_place) {
+  if (threadIdx.x < 2) {
+    const int c = threadIdx.x;
+    if (sort_in_place) sort_book(ctl->T[c], n);
+    build_book(ctl->T[c], n, &tb.bk[c]);
+    fill_pairs(tb, c);
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < 2 * kNB; b += blockDim.x) tb.lut[b / kNB][b % kNB] = lut_entry(tb, b / kNB, b % kNB);
+  __syncthreads();
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(&tb);
+  uint32_t* dst = reinterpret_cast<uint32_t*>(&ctl->tb);
+  for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
+}
+
 // L = B - E(I_max) - E(S2_max) - max(0, E(U_max)), B = min(40, 61 - ceil(log2 M))
-__global__ void fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st) {
-  if (threadIdx.x != 0) return;
-  int c = 0;
-  while (((int64_t)1 << c) < M) c++;
-  int B = 61 - c;
-  if (B > 40) B = 40;
-  const double Imax = (double)__uint_as_float(ctl->Imax_bits);
-  const double S2max = __longlong_as_double((long long)ctl->S2max_bits);
-  const double Umax = (double)__uint_as_float(ctl->Umax_bits);
-  int L = 0;
-  if (Imax > 0.0 && S2max > 0.0) {
-    int eU = Umax > 0.0 ? frexp_exponent(Umax) : 0;
-    if (eU < 0) eU = 0;
-    L = B - frexp_exponent(Imax) - frexp_exponent(S2max) - eU;
+__global__ void __launch_bounds__(kFitThreads)
+fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st) {
+  __shared__ Tables tb;
+  if (threadIdx.x == 0) {
+    int c = 0;
+    while (((int64_t)1 << c) < M) c++;
+    int B = 61 - c;
+    if (B > 40) B = 40;
+    const double Imax = (double)__uint_as_float(ctl->Imax_bits);
+    const double S2max = __longlong_as_double((long long)ctl->S2max_bits);
+    const double Umax = (double)__uint_as_float(ctl->Umax_bits);
+    int L = 0;
+    if (Imax > 0.0 && S2max > 0.0) {
+      int eU = Umax > 0.0 ? frexp_exponent(Umax) : 0;
+      if (eU < 0) eU = 0;
+      L = B - frexp_exponent(Imax) - frexp_exponent(S2max) - eU;
+    }
+    ctl->L = L;
+    ctl->twoL = ldexp(1.0, L);
+    ctl->n = n;
+    tb.la = bucket_scale(ctl);
   }
-  ctl->L = L;
-  ctl->twoL = ldexp(1.0, L);
-  ctl->n = n;
-  for (int b = 0; b < 2; b++) {
-    for (int j = 0; j < 16; j++) ctl->T[b][j] = T_user[b * 16 + j];
-    sort_book(ctl->T[b], n);
-    build_book(ctl->T[b], n, &ctl->bk.b[b]);
-    for (int j = 0; j < 16; j++) T_user[b * 16 + j] = ctl->T[b][j];
+  if (threadIdx.x < 32) {
+    const int c = threadIdx.x >> 4, j = threadIdx.x & 15;
+    ctl->T[c][j] = T_user[threadIdx.x];
   }
-  write_stats(ctl, st);
+  __syncthreads();
+  publish_tables(ctl, tb, n, true);
+  __syncthreads();
+  if (threadIdx.x < 32) T_user[threadIdx.x] = ctl->T[threadIdx.x >> 4][threadIdx.x & 15];
+  if (threadIdx.x == 0) write_stats(ctl, st);
 }
 
 // ---------------------------------------------------------------------------
-// the streaming assign pass (fit: + refine sums; pack: + outputs)
+// the streaming pass (fit: + refine sums; pack: + outputs)
 // ---------------------------------------------------------------------------
 struct PackOut {
   uint8_t* codes;
   void* tagged;
   uint8_t* choice_bytes;
+  double* err_final;
 };
 
+struct RoundOut {
+  double* err_hist;
+  float* T_user;
+  aaac_stats* stats;
+  int it;
+};
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+// Packed pairs of fp32 (Blackwell f32x2 arithmetic, each lane rounded to nearest).
+__device__ __forceinline__ unsigned long long f2pack(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2unpack(unsigned long long p) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p));
+  return make_float2(a, b);
+}
+__device__ __forceinline__ unsigned long long f2sub(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2mul(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// The refine of one round, run by the last block of the pass.
+__device__ void round_finalize(FitCtl* ctl, Tables& tb, const double* errp, int nb,
+                               uint32_t flags, const RoundOut& ro, double* sred) {
+  const int tid = threadIdx.x;
+  double part = 0.0;
+  for (int b = tid; b < nb; b += blockDim.x) part = __dadd_rn(part, __ldcg(errp + b));
+  sred[tid] = part;
+  __syncthreads();
+  if (tid == 0) {
+    double e = 0.0;
+    for (int i = 0; i < (int)blockDim.x; i++) e = __dadd_rn(e, sred[i]);
+    if (ro.err_hist) ro.err_hist[ro.it] = e;
+  }
+  const int n = ctl->n;
+  __shared__ int s_empty[2];
+  if (tid < 2) {
+    const int c = tid;
+    const bool frozen = (c == 0) ? (flags & AAAC_FREEZE_T0) : (flags & AAAC_FREEZE_T1);
+    int updated = 0;
+    if (!frozen) {
+      const Book& bk = tb.bk[c];  // tables of the round that just ran
+      for (int j = 0; j < bk.m; j++) {
+        const long long num = __ldcg(&ctl->bins[c][j][0]);
+        const long long den = __ldcg(&ctl->bins[c][j][1]);
+        if (den > 0) {
+          ctl->T[c][bk.idx[j]] =
+              __double2float_rn(__ddiv_rn(__ll2double_rn(num), __ll2double_rn(den)));
+          updated++;
+        }
+      }
+    }
+    s_empty[c] = frozen ? 0 : n - updated;
+  }
+  __syncthreads();
+  publish_tables(ctl, tb, n, true);
+  __syncthreads();
+  if (tid < 32) ro.T_user[tid] = ctl->T[tid >> 4][tid & 15];
+  if (tid < 64) (&ctl->bins[0][0][0])[tid] = 0;
+  if (tid == 0) {
+    // counters other blocks updated with atomics: read them from L2
+    const unsigned long long empty = (unsigned long long)(s_empty[0] + s_empty[1]);
+    ctl->empty_cells = empty;
+    if (ro.stats) {
+      ro.stats->near_ties = (int64_t)__ldcg(&ctl->near_ties);
+      ro.stats->groups_t1 = (int64_t)__ldcg(&ctl->groups_t1);
+      ro.stats->empty_cells = (int64_t)empty;
+      ro.stats->dead_groups = (int64_t)__ldcg(&ctl->dead_groups);
+      ro.stats->exact_groups = (int64_t)__ldcg(&ctl->exact_groups);
+      ro.stats->L = ctl->L;
+      ro.stats->reserved = 0;
+    }
+    ctl->near_ties = 0;
+    ctl->groups_t1 = 0;
+    ctl->ticket = 0;
+  }
+}
+
 template <int FMT, bool PACK>
-__global__ void __launch_bounds__(kThreads, 2)
-assign_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
-            const void* __restrict__ scales, int g, int S, uint32_t flags, FitCtl* ctl,
-            double* __restrict__ errp, int ncb, int rows_per_chunk, float tau, PackOut po) {
-  __shared__ Books sbk;
-  __shared__ unsigned long long sbins[64];
-  __shared__ double sred[kThreads];
+__global__ void __launch_bounds__(kFitThreads, kFitBlocksPerSM)
+fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
+         const void* __restrict__ scales, int g, int S, uint32_t flags, FitCtl* ctl,
+         double* __restrict__ errp, int ncb, int rows_per_chunk, float tau, PackOut po,
+         RoundOut ro) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  Tables& tb = *reinterpret_cast<Tables*>(smem);
+  uint4* ring = reinterpret_cast<uint4*>(smem + ((sizeof(Tables) + 15) & ~(size_t)15));
+  ulonglong2* bins = reinterpret_cast<ulonglong2*>(ring + kFitWarps * kStages * 32);
+  __shared__ double sred[kFitThreads];
+  __shared__ int s_last;
+
   {
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(&ctl->bk);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(&sbk);
-    for (int i = threadIdx.x; i < (int)(sizeof(Books) / 4); i += blockDim.x) dst[i] = src[i];
-    if (!PACK && threadIdx.x < 64) sbins[threadIdx.x] = 0ull;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(&ctl->tb);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(&tb);
+    for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
+    if (!PACK)
+      for (int i = threadIdx.x; i < kFitWarps * 32 * 32; i += blockDim.x)
+        bins[i] = make_ulonglong2(0ull, 0ull);
   }
   const double twoL = ctl->twoL;
   __syncthreads();
@@ -186,6 +402,9 @@ assign_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restric
   const int leader_lane = lane & ~(lanes_s - 1);
   const bool s_leader = lane == leader_lane;
   const bool single = (flags & AAAC_SINGLE_CODEBOOK) != 0;
+  const float la = tb.la;
+  uint4* myring = ring + warp * kStages * 32 + lane;
+  ulonglong2* mybins = bins + warp * 32 * 32 + lane;
 
   float Ik[8];
   double I2L[8];
@@ -201,36 +420,72 @@ assign_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restric
 #pragma unroll
   for (int i = 0; i < 8; i++) I2L[i] = (double)Ik[i] * twoL;
 
+  const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
+  const uint16_t* wcol = W + col0;
+  // ring prologue
+#pragma unroll
+  for (int k = 0; k < kStages; k++) {
+    const int rr = r0 + warp + kFitWarps * k;
+    if (active && rr < r1) cp_async16(myring + k * 32, wcol + (int64_t)rr * K);
+    cp_async_commit();
+  }
+  float s_next = 0.0f;
+  if (active && r0 + warp < r1) s_next = load_scale<FMT>(scales, (int64_t)(r0 + warp) * G + col0 / g);
+
   double err_acc = 0.0;
   unsigned long long n_near = 0, n_exact = 0, n_t1 = 0;
-  const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
-  for (int r = r0 + warp; r < r1; r += kWarps) {  // warp-uniform trip count
-    uint4 v = make_uint4(0, 0, 0, 0);
-    float s = 0.0f;
-    if (active) {
-      v = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)r * K + col0));
-      s = load_scale<FMT>(scales, (int64_t)r * G + col0 / g);
-    }
+  int slot = 0;
+  for (int r = r0 + warp; r < r1; r += kFitWarps) {  // warp-uniform trip count
+    cp_async_wait<kStages - 1>();
+    const uint4 v = active ? myring[slot * 32] : make_uint4(0, 0, 0, 0);
+    const float s = s_next;
+    if (active && r + kFitWarps < r1)
+      s_next = load_scale<FMT>(scales, (int64_t)(r + kFitWarps) * G + col0 / g);
     float rcp;
     const bool live = active && scale_live(s, &rcp);
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-    float u[8], t0v[8], t1v[8];
-    int q0[8], q1[8];
-    float d0 = 0.0f, d1 = 0.0f;
+    float u[8];
+    uint32_t kk[8];  // 8 * distinct count: book 0 in bits 0..7, book 1 in bits 8..15
+    unsigned long long dd = 0ull;  // (D0, D1) partial sums
+    const unsigned long long rcp2 = f2pack(rcp, rcp);
+#pragma unroll
+    for (int h = 0; h < 4; h++) {
+      const float2 up = f2unpack(f2mul(f2pack(bf16_lo(wv[h]), bf16_hi(wv[h])), rcp2));
+      u[2 * h] = live ? up.x : 0.0f;
+      u[2 * h + 1] = live ? up.y : 0.0f;
+    }
 #pragma unroll
     for (int i = 0; i < 8; i++) {
-      const float wf = (i & 1) ? bf16_hi(wv[i >> 1]) : bf16_lo(wv[i >> 1]);
-      u[i] = live ? __fmul_rn(wf, rcp) : 0.0f;
-      const int c0 = book_count(sbk.b[0], u[i]);
-      const int c1 = book_count(sbk.b[1], u[i]);
-      q0[i] = sbk.b[0].idx[c0];
-      q1[i] = sbk.b[1].idx[c1];
-      t0v[i] = sbk.b[0].val[c0];
-      t1v[i] = sbk.b[1].val[c1];
-      const float e0 = __fsub_rn(u[i], t0v[i]);
-      const float e1 = __fsub_rn(u[i], t1v[i]);
-      d0 = __fmaf_rn(Ik[i], __fmul_rn(e0, e0), d0);
-      d1 = __fmaf_rn(Ik[i], __fmul_rn(e1, e1), d1);
+      const uint32_t bi = __float_as_uint(bucket_t(u[i], la)) & (kNB - 1);
+      const uint32_t c0 = tb.lut[0][bi], c1 = tb.lut[1][bi];
+      const unsigned long long p0 = *reinterpret_cast<const unsigned long long*>(
+          reinterpret_cast<const unsigned char*>(&tb.pair[0][0]) + c0);
+      const unsigned long long p1 = *reinterpret_cast<const unsigned long long*>(
+          reinterpret_cast<const unsigned char*>(&tb.pair[1][0]) + c1);
+      const unsigned long long uu = f2pack(u[i], u[i]);
+      const unsigned long long e0 = f2sub(uu, p0), e1 = f2sub(uu, p1);
+      const float2 s0 = f2unpack(f2mul(e0, e0)), s1 = f2unpack(f2mul(e1, e1));
+      const bool up0 = s0.y < s0.x, dn0 = s0.x < s0.y;
+      const bool up1 = s1.y < s1.x, dn1 = s1.x < s1.y;
+      uint32_t k0 = c0 + (up0 ? 8u : 0u), k1 = c1 + (up1 ? 8u : 0u);
+      float m0 = up0 ? s0.y : s0.x, m1 = up1 ? s1.y : s1.x;
+      if (!(up0 | dn0) | !(up1 | dn1)) {  // rare: tie, or a crowded bucket
+        const int x0 = book_count(tb.bk[0], u[i]), x1 = book_count(tb.bk[1], u[i]);
+        const float f0 = __fsub_rn(u[i], tb.bk[0].val[x0]);
+        const float f1 = __fsub_rn(u[i], tb.bk[1].val[x1]);
+        k0 = 8u * (uint32_t)x0;
+        k1 = 8u * (uint32_t)x1;
+        m0 = __fmul_rn(f0, f0);
+        m1 = __fmul_rn(f1, f1);
+      }
+      kk[i] = k0 | (k1 << 8);
+      dd = f2fma(f2pack(Ik[i], Ik[i]), f2pack(m0, m1), dd);
+    }
+    float d0, d1;
+    {
+      const float2 dv = f2unpack(dd);
+      d0 = dv.x;
+      d1 = dv.y;
     }
     for (int o = 1; o < lanes_s; o <<= 1) {
       d0 = __fadd_rn(d0, __shfl_xor_sync(0xffffffffu, d0, o));
@@ -256,8 +511,8 @@ assign_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restric
         const float wf = __uint_as_float((uint32_t)wrow[j] << 16);
         const float uj = __fmul_rn(wf, rcp);
         const double Ij = (double)I[kbase + j];
-        const double ea = __dsub_rn((double)uj, (double)sbk.b[0].val[book_count(sbk.b[0], uj)]);
-        const double eb = __dsub_rn((double)uj, (double)sbk.b[1].val[book_count(sbk.b[1], uj)]);
+        const double ea = __dsub_rn((double)uj, (double)tb.bk[0].val[book_count(tb.bk[0], uj)]);
+        const double eb = __dsub_rn((double)uj, (double)tb.bk[1].val[book_count(tb.bk[1], uj)]);
         E0 = __dadd_rn(E0, __dmul_rn(Ij, __dmul_rn(ea, ea)));
         E1 = __dadd_rn(E1, __dmul_rn(Ij, __dmul_rn(eb, eb)));
       }
@@ -278,24 +533,32 @@ assign_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restric
     if (!PACK) {
       if (live) {
         const double s2 = (double)s * (double)s;
+        const int shift = choice ? 8 : 0;
+        ulonglong2* cb_bins = mybins + choice * 16 * 32;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-          const int q = choice ? q1[i] : q0[i];
+          const uint32_t q = ((kk[i] >> shift) >> 3) & 15u;
           const double A = __dmul_rn(I2L[i], s2);  // exact: 24 + 16 bits
-          const double num = __dsub_rn(__fma_rn(A, (double)u[i], kMagic), kMagic);
-          const double den = __dsub_rn(__dadd_rn(A, kMagic), kMagic);
-          atomicAdd(&sbins[(choice * 16 + q) * 2 + 0], (unsigned long long)(long long)num);
-          atomicAdd(&sbins[(choice * 16 + q) * 2 + 1], (unsigned long long)(long long)den);
+          const unsigned long long num =
+              (unsigned long long)__double_as_longlong(__fma_rn(A, (double)u[i], kMagic));
+          const unsigned long long den =
+              (unsigned long long)__double_as_longlong(__dadd_rn(A, kDenMagic));
+          ulonglong2 x = cb_bins[q * 32];
+          x.x += num;
+          x.y += den;
+          cb_bins[q * 32] = x;
         }
       }
     } else if (active) {
+      const Book& bc = tb.bk[choice];
+      const int shift = choice ? 8 : 0;
       uint32_t packed = 0;
 #pragma unroll
       for (int i = 0; i < 8; i++) {
-        const int q = choice ? q1[i] : q0[i];
-        packed |= (uint32_t)q << (4 * i);
+        const uint32_t q = ((kk[i] >> shift) >> 3) & 15u;
+        packed |= (uint32_t)bc.idx[q] << (4 * i);
         const float wf = (i & 1) ? bf16_hi(wv[i >> 1]) : bf16_lo(wv[i >> 1]);
-        const double wh = (double)s * (double)(choice ? t1v[i] : t0v[i]);
+        const double wh = (double)s * (double)bc.val[q];
         const double d = __dsub_rn((double)wf, wh);
         err_acc = __fma_rn((double)Ik[i], __dmul_rn(d, d), err_acc);
       }
@@ -314,10 +577,16 @@ assign_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restric
       }
       if (S != g && s_leader) po.choice_bytes[(int64_t)r * KS + col0 / S] = (uint8_t)choice;
     }
+    // refill this slot with the row kStages steps ahead
+    {
+      const int rr = r + kFitWarps * kStages;
+      if (active && rr < r1) cp_async16(myring + slot * 32, wcol + (int64_t)rr * K);
+      cp_async_commit();
+    }
+    slot = (slot + 1 == kStages) ? 0 : slot + 1;
   }
+  cp_async_wait<0>();
 
-  // fixed-order block reduction of the error partials
-  sred[threadIdx.x] = err_acc;
   for (int o = 16; o > 0; o >>= 1) {
     n_near += __shfl_xor_sync(0xffffffffu, n_near, o);
     n_exact += __shfl_xor_sync(0xffffffffu, n_exact, o);
@@ -328,50 +597,51 @@ assign_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restric
     if (n_exact) atomicAdd(&ctl->exact_groups, n_exact);
     if (n_t1) atomicAdd(&ctl->groups_t1, n_t1);
   }
+  sred[threadIdx.x] = err_acc;
   __syncthreads();
   if (threadIdx.x == 0) {
     double t = 0.0;
-    for (int i = 0; i < kThreads; i++) t = __dadd_rn(t, sred[i]);
+    for (int i = 0; i < kFitThreads; i++) t = __dadd_rn(t, sred[i]);
     errp[blockIdx.x] = t;
   }
   if (!PACK && threadIdx.x < 64) {
-    const unsigned long long b = sbins[threadIdx.x];
-    if (b) atomicAdd(&ctl->bins[0][0][0] + threadIdx.x, b);
-  }
-}
-
-// refine (section 2, core mechanism 4): T = fp32(fp64(num) / fp64(den)) when
-// den > 0, else unchanged; then sort and rebuild the tables.
-__global__ void fit_finalize(FitCtl* ctl, const double* __restrict__ errp, int nblocks,
-                             double* err_hist, int it, uint32_t flags, float* T_user,
-                             aaac_stats* st) {
-  if (threadIdx.x != 0) return;
-  double e = 0.0;
-  for (int b = 0; b < nblocks; b++) e = __dadd_rn(e, errp[b]);
-  if (err_hist) err_hist[it] = e;
-  const int n = ctl->n;
-  unsigned long long empty = 0;
-  for (int c = 0; c < 2; c++) {
-    const bool frozen = (c == 0) ? (flags & AAAC_FREEZE_T0) : (flags & AAAC_FREEZE_T1);
-    if (frozen) continue;
-    for (int j = 0; j < n; j++) {
-      const long long num = (long long)ctl->bins[c][j][0];
-      const long long den = (long long)ctl->bins[c][j][1];
-      if (den > 0)
-        ctl->T[c][j] = __double2float_rn(__ddiv_rn(__ll2double_rn(num), __ll2double_rn(den)));
-      else
-        empty++;
+    // lane-private raw sums -> exact integers: num is exact modulo 2^51, den
+    // modulo 2^52, and every lane's partial is far inside those ranges.
+    const int cell = threadIdx.x >> 1, which = threadIdx.x & 1;
+    long long sum = 0;
+    for (int w = 0; w < kFitWarps; w++) {
+      const ulonglong2* p = bins + (w * 32 + cell) * 32;
+      for (int l = 0; l < 32; l++) {
+        const unsigned long long raw = which ? p[l].y : p[l].x;
+        sum += which ? (long long)(raw & ((1ull << 52) - 1))
+                     : ((long long)(raw << 13) >> 13);
+      }
     }
-    sort_book(ctl->T[c], n);
-    build_book(ctl->T[c], n, &ctl->bk.b[c]);
+    if (sum) atomicAdd(reinterpret_cast<unsigned long long*>(&ctl->bins[0][0][0]) + threadIdx.x,
+                       (unsigned long long)sum);
   }
-  ctl->empty_cells = empty;
-  for (int c = 0; c < 2; c++)
-    for (int j = 0; j < 16; j++) T_user[c * 16 + j] = ctl->T[c][j];
-  write_stats(ctl, st);
-  for (int i = 0; i < 64; i++) (&ctl->bins[0][0][0])[i] = 0ull;
-  ctl->near_ties = 0;
-  ctl->groups_t1 = 0;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&ctl->ticket, 1u) == gridDim.x - 1) ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (!PACK) {
+    round_finalize(ctl, tb, errp, gridDim.x, flags, ro, sred);
+  } else {
+    double part = 0.0;
+    for (int b = threadIdx.x; b < (int)gridDim.x; b += blockDim.x)
+      part = __dadd_rn(part, __ldcg(errp + b));
+    __syncthreads();
+    sred[threadIdx.x] = part;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double e = 0.0;
+      for (int i = 0; i < kFitThreads; i++) e = __dadd_rn(e, sred[i]);
+      if (po.err_final) *po.err_final = e;
+      ctl->ticket = 0;
+    }
+  }
 }
 
 static float choice_tau(int S) {
@@ -380,44 +650,61 @@ static float choice_tau(int S) {
   return (float)((12 + lg) * ldexp(1.0, -22));
 }
 
+template <int FMT, bool PACK>
+static cudaError_t set_smem() {
+  return cudaFuncSetAttribute(fit_pass<FMT, PACK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)smem_bytes(PACK));
+}
+
 template <int FMT>
-static void launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const float* I,
-                         const void* scales, int g, int S, int iters, uint32_t flags, float* T,
-                         double* err_hist, aaac_stats* stats, void* ws, cudaStream_t st) {
-  const PassPlan pp = plan_pass(N, K);
+static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const float* I,
+                                const void* scales, int g, int S, int iters, uint32_t flags,
+                                float* T, double* err_hist, aaac_stats* stats, void* ws,
+                                cudaStream_t st) {
+  static cudaError_t attr = set_smem<FMT, false>();
+  if (attr != cudaSuccess) return attr;
+  const PassPlan pp = fit_plan(N, K);
+  const PassPlan pprep = plan_pass(N, K);
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
   double* errp = reinterpret_cast<double*>(reinterpret_cast<char*>(ws) + fit_ctl_bytes());
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
-  fit_prep<FMT><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl, pp.ncb,
-                                                pp.rows_per_chunk);
-  fit_setup<<<1, 32, 0, st>>>(ctl, T, N * K, ncodes(FMT), stats);
+  fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
+                                                   pprep.ncb, pprep.rows_per_chunk);
+  fit_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), stats);
   const float tau = choice_tau(S);
   for (int it = 0; it < iters; it++) {
-    assign_pass<FMT, false><<<pp.blocks, kThreads, 0, st>>>(
+    fit_pass<FMT, false><<<pp.blocks, kFitThreads, smem_bytes(false), st>>>(
         W, (int)N, (int)K, I, scales, g, S, flags, ctl, errp, pp.ncb, pp.rows_per_chunk, tau,
-        PackOut{nullptr, nullptr, nullptr});
-    fit_finalize<<<1, 32, 0, st>>>(ctl, errp, pp.blocks, err_hist, it, flags, T, stats);
+        PackOut{nullptr, nullptr, nullptr, nullptr}, RoundOut{err_hist, T, stats, it});
   }
-  count_launches(2 + 2 * iters);
+  count_launches(2 + iters);
+  return cudaSuccess;
 }
 
 cudaError_t launch_fit(const uint16_t* W, int64_t N, int64_t K, const float* I,
                        const void* scales, int fmt, int g, int S, int iters, uint32_t flags,
                        float* T, double* err_hist, aaac_stats* stats, void* ws, cudaStream_t st) {
-  if (fmt == kInt4)
-    launch_fit_t<kInt4>(W, N, K, I, scales, g, S, iters, flags, T, err_hist, stats, ws, st);
-  else
-    launch_fit_t<kNvfp4>(W, N, K, I, scales, g, S, iters, flags, T, err_hist, stats, ws, st);
+  cudaError_t e = (fmt == kInt4)
+                      ? launch_fit_t<kInt4>(W, N, K, I, scales, g, S, iters, flags, T, err_hist,
+                                            stats, ws, st)
+                      : launch_fit_t<kNvfp4>(W, N, K, I, scales, g, S, iters, flags, T, err_hist,
+                                             stats, ws, st);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
 // pack
 // ---------------------------------------------------------------------------
-__global__ void pack_setup(FitCtl* ctl, const float* T_user, int n, uint16_t* T_bf16) {
-  if (threadIdx.x != 0) return;
-  ctl->n = n;
-  for (int b = 0; b < 2; b++) {
+__global__ void __launch_bounds__(kFitThreads)
+pack_setup(FitCtl* ctl, const float* T_user, int n, uint16_t* T_bf16) {
+  __shared__ Tables tb;
+  if (threadIdx.x == 0) {
+    ctl->n = n;
+    tb.la = bucket_scale(ctl);
+  }
+  if (threadIdx.x < 2) {
+    const int b = threadIdx.x;
     float t[16];
     for (int j = 0; j < 16; j++) t[j] = T_user[b * 16 + j];
     sort_book(t, n);
@@ -426,15 +713,9 @@ __global__ void pack_setup(FitCtl* ctl, const float* T_user, int n, uint16_t* T_
       T_bf16[b * 16 + j] = h;
       ctl->T[b][j] = __uint_as_float((uint32_t)h << 16);
     }
-    build_book(ctl->T[b], n, &ctl->bk.b[b]);
   }
-}
-
-__global__ void pack_finalize(const double* __restrict__ errp, int nblocks, double* err_final) {
-  if (threadIdx.x != 0) return;
-  double e = 0.0;
-  for (int b = 0; b < nblocks; b++) e = __dadd_rn(e, errp[b]);
-  if (err_final) *err_final = e;
+  __syncthreads();
+  publish_tables(ctl, tb, n, false);
 }
 
 // choice bytes [N][K/S] -> bits [N][ceil(K/S/8)], LSB first
@@ -449,31 +730,49 @@ __global__ void pack_bits(const uint8_t* __restrict__ cb, int64_t N, int KS, uin
   bits[i] = (uint8_t)byte;
 }
 
-cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const float* I,
-                        const void* scales, int fmt, int g, int S, uint32_t flags, const float* T,
-                        uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
-                        uint8_t* choice_bits, double* err_final, void* ws, cudaStream_t st) {
-  const PassPlan pp = plan_pass(N, K);
+template <int FMT>
+static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const float* I,
+                                 const void* scales, int g, int S, uint32_t flags, const float* T,
+                                 uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
+                                 uint8_t* choice_bits, double* err_final, void* ws,
+                                 cudaStream_t st) {
+  static cudaError_t attr = set_smem<FMT, true>();
+  if (attr != cudaSuccess) return attr;
+  const PassPlan pp = fit_plan(N, K);
+  const PassPlan pprep = plan_pass(N, K);
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
   double* errp = reinterpret_cast<double*>(reinterpret_cast<char*>(ws) + fit_ctl_bytes());
   uint8_t* cbytes = reinterpret_cast<uint8_t*>(ws) + fit_ws_bytes(N, K);
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
-  pack_setup<<<1, 32, 0, st>>>(ctl, T, ncodes(fmt), T_bf16);
+  fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
+                                                   pprep.ncb, pprep.rows_per_chunk);
+  pack_setup<<<1, kFitThreads, 0, st>>>(ctl, T, ncodes(FMT), T_bf16);
   const float tau = choice_tau(S);
-  const PackOut po{codes, scales_tagged, cbytes};
-  if (fmt == kInt4)
-    assign_pass<kInt4, true><<<pp.blocks, kThreads, 0, st>>>(
-        W, (int)N, (int)K, I, scales, g, S, flags, ctl, errp, pp.ncb, pp.rows_per_chunk, tau, po);
-  else
-    assign_pass<kNvfp4, true><<<pp.blocks, kThreads, 0, st>>>(
-        W, (int)N, (int)K, I, scales, g, S, flags, ctl, errp, pp.ncb, pp.rows_per_chunk, tau, po);
-  pack_finalize<<<1, 32, 0, st>>>(errp, pp.blocks, err_final);
+  const PackOut po{codes, scales_tagged, cbytes, err_final};
+  fit_pass<FMT, true><<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
+      W, (int)N, (int)K, I, scales, g, S, flags, ctl, errp, pp.ncb, pp.rows_per_chunk, tau, po,
+      RoundOut{nullptr, nullptr, nullptr, 0});
+  int launches = 3;
   if (S != g) {
     const int KS = (int)(K / S);
     const int64_t total = N * ((KS + 7) / 8);
     pack_bits<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(cbytes, N, KS, choice_bits);
+    launches++;
   }
-  count_launches(S != g ? 4 : 3);
+  count_launches(launches);
+  return cudaSuccess;
+}
+
+cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const float* I,
+                        const void* scales, int fmt, int g, int S, uint32_t flags, const float* T,
+                        uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
+                        uint8_t* choice_bits, double* err_final, void* ws, cudaStream_t st) {
+  cudaError_t e = (fmt == kInt4)
+                      ? launch_pack_t<kInt4>(W, N, K, I, scales, g, S, flags, T, T_bf16, codes,
+                                             scales_tagged, choice_bits, err_final, ws, st)
+                      : launch_pack_t<kNvfp4>(W, N, K, I, scales, g, S, flags, T, T_bf16, codes,
+                                              scales_tagged, choice_bits, err_final, ws, st);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

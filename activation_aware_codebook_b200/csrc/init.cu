@@ -36,10 +36,9 @@ struct InitCtl {
 
 size_t init_ctl_bytes() { return align256(sizeof(InitCtl)); }
 
-PassPlan plan_pass(int64_t N, int64_t K) {
+PassPlan plan_pass(int64_t N, int64_t K, int target) {
   PassPlan p;
   p.ncb = (int)((K + kSegCols - 1) / kSegCols);
-  int target = 148 * 4;
   int64_t nrc = (target + p.ncb - 1) / p.ncb;
   if (nrc > N) nrc = N;
   if (nrc < 1) nrc = 1;

@@ -29,7 +29,7 @@ struct PassPlan {
   int rows_per_chunk;
   int blocks;     // ncb * nrc
 };
-PassPlan plan_pass(int64_t N, int64_t K);
+PassPlan plan_pass(int64_t N, int64_t K, int target_blocks = 148 * 4);
 
 size_t fit_ctl_bytes();
 size_t init_ctl_bytes();

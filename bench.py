@@ -1,0 +1,480 @@
+#!/usr/bin/env python
+"""AAAC layer-fit benchmark: weights assigned+refined per second per iteration.
+
+One step = the whole hot path over one transformer block of Llama-3-8B-shaped
+linears (q, k, v, o, gate, up, down; INT4 g=128, selection groups S=16, 20
+assign/refine iterations) with seeded synthetic weights and calibration
+activations X[262144, K]:
+    importance (once per distinct activation) -> scales + quantile init -> fit
+    -> 4-bit pack,
+all through the C ABI of libaaac.so with the inputs resident in HBM.
+value = sum over linears of N*K*iters / step time (whole job, all ranks).
+
+Multi-GPU: one process per GPU (torchrun); layers are independent, so rank r
+fits block r of the sweep and no collective touches the data path (weak
+scaling).  Timing: CUDA events on the launching stream, barrier +
+synchronize on both sides, max over ranks.
+
+--impl reference times the CPU oracle (test infrastructure) on a bounded
+sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("AAAC fit: weights assigned+refined/s per iteration; "
+          "achieved HBM GB/s vs 8 TB/s")
+UNIT = "weights/s per iteration"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="llama8b-int4-s16")
+    p.add_argument("--tokens", type=int, default=0, help="override calibration tokens")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    return p.parse_args()
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def blocks_for_rank(rank, world, nblocks):
+    """Independent layer blocks of a sweep, dealt round-robin to the ranks."""
+    return [b for b in range(nblocks) if b % world == rank]
+
+
+def max_over_ranks(value, world, device="cpu"):
+    """The slowest rank's time: every rank's value is replaced by the max."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "activation_aware_codebook_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel_src_hash):
+    """DRAM bytes per fit pass from the committed ncu summary, when it was taken
+    on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "fit_pass_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("source_hash") != kernel_src_hash:
+        return None
+    return d
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def build_block(wl, block, tokens, dev):
+    import torch
+
+    from activation_aware_codebook_b200 import synth
+    Xs, Ws = {}, {}
+    for lin in wl.linears:
+        if lin.x_key not in Xs:
+            Xs[lin.x_key] = synth.make_activations(
+                tokens, lin.K, synth.seed_of(wl.name, block, lin.x_key, "X"), wl.heavy,
+                device=dev)
+        Ws[lin.name] = synth.make_weight(
+            lin.N, lin.K, synth.seed_of(wl.name, block, lin.name, "W"), wl.w_dist, device=dev)
+    torch.cuda.synchronize()
+    return Xs, Ws
+
+
+class Block:
+    """Device buffers and the step of one block of linears."""
+
+    def __init__(self, wl, Xs, Ws, dev):
+        import torch
+
+        from activation_aware_codebook_b200 import binding as bb
+        self.bb, self.wl, self.Xs, self.Ws = bb, wl, Xs, Ws
+        self.cfg = bb.Config(wl.fmt, wl.g, wl.S, wl.iters)
+        tokens = next(iter(Xs.values())).shape[0]
+        self.ws = torch.empty(max(bb.workspace_size(self.cfg, l.N, l.K, tokens)
+                                  for l in wl.linears), dtype=torch.uint8, device=dev)
+        self.I = {k: torch.zeros(x.shape[1], dtype=torch.float32, device=dev)
+                  for k, x in Xs.items()}
+        sdt = torch.int16 if wl.fmt == bb.INT4 else torch.uint8
+        self.scales, self.T, self.eh, self.st, self.out = {}, {}, {}, {}, {}
+        for l in wl.linears:
+            self.scales[l.name] = torch.empty(l.N, l.K // wl.g, dtype=sdt, device=dev)
+            self.T[l.name] = torch.zeros(2, 16, dtype=torch.float32, device=dev)
+            self.eh[l.name] = torch.zeros(wl.iters, dtype=torch.float64, device=dev)
+            self.st[l.name] = torch.zeros(bb.STATS_BYTES, dtype=torch.uint8, device=dev)
+            nb = (l.K // wl.S + 7) // 8
+            self.out[l.name] = dict(
+                T_bf16=torch.zeros(2, 16, dtype=torch.int16, device=dev),
+                codes=torch.empty(l.N, l.K // 2, dtype=torch.uint8, device=dev),
+                scales_tagged=torch.empty(l.N, l.K // wl.g, dtype=sdt, device=dev),
+                choice_bits=(torch.empty(l.N, nb, dtype=torch.uint8, device=dev)
+                             if wl.S != wl.g else None),
+                err_final=torch.zeros(1, dtype=torch.float64, device=dev))
+        self.weight_iters = sum(l.N * l.K for l in wl.linears) * wl.iters
+
+    def step(self, fit_events=None, probe=None):
+        bb, cfg = self.bb, self.cfg
+        for k, X in self.Xs.items():
+            bb.importance(X, I=self.I[k], ws=self.ws)
+        for l in self.wl.linears:
+            W = self.Ws[l.name]
+            bb.init_codebooks(W, cfg, ws=self.ws, scales=self.scales[l.name], T=self.T[l.name])
+            if fit_events is not None and l.name == probe:
+                fit_events[0].record()
+            bb.fit_layer(W, self.I[l.x_key], self.scales[l.name], self.T[l.name], cfg,
+                         ws=self.ws, err_hist=self.eh[l.name], stats=self.st[l.name])
+            if fit_events is not None and l.name == probe:
+                fit_events[1].record()
+            bb.pack(W, self.I[l.x_key], self.scales[l.name], self.T[l.name], cfg, ws=self.ws,
+                    out=self.out[l.name])
+
+    def output_bytes(self):
+        tot = 0
+        for l in self.wl.linears:
+            for v in self.out[l.name].values():
+                if v is not None:
+                    tot += v.numel() * v.element_size()
+        return tot
+
+
+def fit_setup_ms(blk, lin, reps=5):
+    """Time of a fit call with zero rounds (prep + setup) on the probe layer."""
+    import torch
+    bb = blk.bb
+    cfg0 = bb.Config(blk.cfg.fmt, blk.cfg.g, blk.cfg.S, 0)
+    W = blk.Ws[lin.name]
+    T = blk.T[lin.name].clone()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    for _ in range(reps + 1):
+        e0.record()
+        bb.fit_layer(W, blk.I[lin.x_key], blk.scales[lin.name], T, cfg0, ws=blk.ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times[1:])
+
+
+def run_ours(args, rank, local_rank, world):
+    import torch
+    import torch.distributed as dist
+
+    from activation_aware_codebook_b200 import binding as bb
+    from activation_aware_codebook_b200 import synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    bb.load()
+    wl = synth.WORKLOADS[args.workload]
+    tokens = args.tokens or wl.tokens
+    block = blocks_for_rank(rank, world, max(world, wl.layers))[0]
+    Xs, Ws = build_block(wl, block, tokens, dev)
+    blk = Block(wl, Xs, Ws, dev)
+    probe = max(wl.linears, key=lambda l: l.N * l.K)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        blk.step()
+    torch.cuda.synchronize()
+    setup_ms = fit_setup_ms(blk, probe)
+
+    n_fit = args.steps
+    fit_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_fit)]
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    launches0 = bb.kernel_launches()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(args.steps):
+        blk.step(fit_events=fit_ev[i], probe=probe.name)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    launches = bb.kernel_launches() - launches0
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    fit_ms = statistics.median(a.elapsed_time(b) for a, b in fit_ev)
+    ms_max = max_over_ranks(ms, world, dev)
+
+    # roofline of the fit round (assign pass + one-block finalize) on the probe layer
+    iter_ms = (fit_ms - setup_ms) / wl.iters
+    scale_bytes = 2 if wl.fmt == bb.INT4 else 1
+    bytes_per_iter = (probe.N * probe.K * 2 + probe.N * (probe.K // wl.g) * scale_bytes
+                      + probe.K * 4)
+    achieved = bytes_per_iter / (iter_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    traffic = None
+    tr = committed_traffic(source_hash("fit.cu", "common.cuh"))
+    if tr is not None and tr.get("N") and tr.get("K"):
+        traffic = tr["dram_bytes_per_launch"] * (probe.N * probe.K) / (tr["N"] * tr["K"])
+
+    # end to end through the C ABI with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(blk, args.e2e_steps, dev)
+
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": world * blk.weight_iters / (ms_max * 1e-3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32+i64", "impl": "ours",
+            "data": "synthetic: seeded N(0,0.02) weights with 0.1% x10 outliers, "
+                    "lognormal-channel activations with 5 heavy channels",
+            "config": {"workload": wl.name, "linears": [f"{l.name} {l.N}x{l.K}"
+                                                        for l in wl.linears],
+                       "weights_per_block": sum(l.N * l.K for l in wl.linears),
+                       "tokens": tokens, "format": "INT4" if wl.fmt == bb.INT4 else "NVFP4",
+                       "g": wl.g, "S": wl.S, "iters": wl.iters,
+                       "blocks": world, "parallelism": f"layer-parallel x{world} (no collective)",
+                       "l2": "inputs larger than L2 (activations %.1f GiB per step)" % (
+                           sum(x.numel() * 2 for x in Xs.values()) / 2 ** 30)},
+            "roofline": {"kernel": "assign_pass<INT4,fit> + fit_finalize (one fit round)",
+                         "layer": f"{probe.name} {probe.N}x{probe.K}",
+                         "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "bytes_per_launch": bytes_per_iter,
+                         "round_ms": iter_ms},
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+        }
+        if e2e is not None:
+            out["e2e"] = e2e
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+def run_e2e(blk, steps, dev):
+    """Same step through the public API with host-resident inputs: pinned H2D
+    of every activation and weight, the four calls, D2H of every output."""
+    import torch
+    hostX = {k: torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for k, x in blk.Xs.items()}
+    hostW = {k: torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for k, w in blk.Ws.items()}
+    for k in hostX:
+        hostX[k].copy_(blk.Xs[k])
+    for k in hostW:
+        hostW[k].copy_(blk.Ws[k])
+    hostOut = {l.name: {k: (torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                            if v is not None else None) for k, v in blk.out[l.name].items()}
+               for l in blk.wl.linears}
+    h2d = sum(v.numel() * v.element_size() for v in list(hostX.values()) + list(hostW.values()))
+    d2h = blk.output_bytes()
+
+    def one():
+        for k in hostX:
+            blk.Xs[k].copy_(hostX[k], non_blocking=True)
+        for k in hostW:
+            blk.Ws[k].copy_(hostW[k], non_blocking=True)
+        blk.step()
+        for l in blk.wl.linears:
+            for k, v in blk.out[l.name].items():
+                if v is not None:
+                    hostOut[l.name][k].copy_(v, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"value": blk.weight_iters / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(wl, tokens_sample=16384, layers=("k_proj", "v_proj")):
+    """A bounded sample of the workload for the CPU oracle: the named linears
+    of block 0 with a token subsample for the importance."""
+    from activation_aware_codebook_b200 import synth
+    lins = [l for l in wl.linears if l.name in layers] or [min(wl.linears,
+                                                                key=lambda l: l.N * l.K)]
+    data = []
+    Xc = {}
+    for l in lins:
+        if l.x_key not in Xc:
+            Xc[l.x_key] = synth.bits_u16(synth.make_activations(
+                tokens_sample, l.K, synth.seed_of(wl.name, 0, l.x_key, "X"), wl.heavy))
+        W = synth.bits_u16(synth.make_weight(l.N, l.K, synth.seed_of(wl.name, 0, l.name, "W"),
+                                             wl.w_dist))
+        data.append((l, W, Xc[l.x_key]))
+    desc = (f"{'+'.join(l.name for l in lins)} of block 0 ({sum(l.N * l.K for l in lins)} "
+            f"weights, {wl.iters} iterations), importance on {tokens_sample} tokens")
+    return data, desc
+
+
+def oracle_step(wl, data):
+    import oracle
+    for l, W, X in data:
+        oracle.run_layer(W, X, wl.fmt, wl.g, wl.S, wl.iters)
+
+
+def cores_used():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
+                             else os.cpu_count())
+
+
+def cpu_baseline(wl):
+    data, desc = oracle_sample(wl)
+    w_it = sum(l.N * l.K for l, _, _ in data) * wl.iters
+    t0 = time.perf_counter()
+    oracle_step(wl, data)
+    dt = time.perf_counter() - t0
+    return {"value": w_it / dt, "unit": UNIT, "cores": cores_used(), "kind": "oracle",
+            "sample": desc, "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from activation_aware_codebook_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    data, desc = oracle_sample(wl)
+    w_it = sum(l.N * l.K for l, _, _ in data) * wl.iters
+    for _ in range(args.warmup):
+        oracle_step(wl, data)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(wl, data)
+    ms = (time.perf_counter() - t0) / args.steps * 1e3
+    v = w_it / (ms * 1e-3)
+    return {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64+i64", "impl": "reference",
+            "data": "synthetic (same generator and seeds as our arm, bounded sample)",
+            "config": {"workload": wl.name, "sample": desc},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores_used(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank, local_rank, world = env_rank()
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+    else:
+        out = run_ours(args, rank, local_rank, world)
+        if out is not None and world == 1 and not args.no_cpu_baseline:
+            from activation_aware_codebook_b200 import synth
+            out["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[args.workload])
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()
