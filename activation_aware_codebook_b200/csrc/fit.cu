@@ -661,7 +661,8 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
                                 const void* scales, int g, int S, int iters, uint32_t flags,
                                 float* T, double* err_hist, aaac_stats* stats, void* ws,
                                 cudaStream_t st) {
-  static cudaError_t attr = set_smem<FMT, false>();
+  // per call: the attribute belongs to the current device's copy of the kernel
+  const cudaError_t attr = set_smem<FMT, false>();
   if (attr != cudaSuccess) return attr;
   const PassPlan pp = fit_plan(N, K);
   const PassPlan pprep = plan_pass(N, K);
@@ -736,7 +737,7 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
                                  uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
                                  uint8_t* choice_bits, double* err_final, void* ws,
                                  cudaStream_t st) {
-  static cudaError_t attr = set_smem<FMT, true>();
+  const cudaError_t attr = set_smem<FMT, true>();
   if (attr != cudaSuccess) return attr;
   const PassPlan pp = fit_plan(N, K);
   const PassPlan pprep = plan_pass(N, K);
