@@ -28,7 +28,8 @@ STATUS = {0: "AAAC_OK", 1: "AAAC_ERR_INVALID_ARG", 2: "AAAC_ERR_SHAPE", 3: "AAAC
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaaac.so")
 
 EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaac_fit_layer",
-           "aaac_pack", "aaac_last_error", "aaac_version", "aaac_kernel_launches")
+           "aaac_pack", "aaac_last_error", "aaac_version", "aaac_kernel_launches",
+           "aaac_fit_layer_fixed_scratch")
 
 
 class AaacError(RuntimeError):
@@ -95,6 +96,8 @@ def load(path: str = LIB_PATH):
     L.aaac_last_error.argtypes = []
     L.aaac_version.restype = ctypes.c_char_p
     L.aaac_version.argtypes = []
+    L.aaac_fit_layer_fixed_scratch.restype = ctypes.c_int
+    L.aaac_fit_layer_fixed_scratch.argtypes = [P, i64, i64, P, P, P, P, P, P, P]
     L.aaac_kernel_launches.restype = ctypes.c_uint64
     L.aaac_kernel_launches.argtypes = []
     _lib = L
@@ -204,6 +207,25 @@ def fit_layer(W: torch.Tensor, I: torch.Tensor, scales: torch.Tensor, T: torch.T
     _check(load().aaac_fit_layer(_ptr(W), N, K, _ptr(I), _ptr(scales), ctypes.byref(c), _ptr(T),
                                  _ptr(err_hist), _ptr(stats), _ptr(ws), ws.numel(),
                                  _stream(stream)))
+    return T, err_hist, stats
+
+
+def fit_layer_fixed_scratch(W: torch.Tensor, I: torch.Tensor, scales: torch.Tensor,
+                            T: torch.Tensor, cfg: Config, err_hist: Optional[torch.Tensor] = None,
+                            stats: Optional[torch.Tensor] = None, stream=None):
+    """fit_layer for callers that cannot allocate: the library's own fixed
+    scratch replaces the workspace (see aaac_fit_layer_fixed_scratch)."""
+    _need_cuda()
+    W = _bits16(W)
+    N, K = W.shape
+    if err_hist is None:
+        err_hist = torch.zeros(max(cfg.iters, 1), dtype=torch.float64, device=W.device)
+    if stats is None:
+        stats = torch.zeros(STATS_BYTES, dtype=torch.uint8, device=W.device)
+    c = cfg.c()
+    _check(load().aaac_fit_layer_fixed_scratch(_ptr(W), N, K, _ptr(I), _ptr(scales),
+                                               ctypes.byref(c), _ptr(T), _ptr(err_hist),
+                                               _ptr(stats), _stream(stream)))
     return T, err_hist, stats
 
 

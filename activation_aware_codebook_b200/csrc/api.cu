@@ -167,6 +167,32 @@ aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
                    "aaac_fit_layer");
 }
 
+aaac_status aaac_fit_layer_fixed_scratch(const void* W, int64_t N, int64_t K, const float* I,
+                                         const void* scales, const aaac_config* cfg, float* T,
+                                         double* err_hist, aaac_stats* stats, void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  CHECK(check_ptr(W, "W"));
+  CHECK(check_ptr(I, "I"));
+  CHECK(check_ptr(scales, "scales"));
+  CHECK(check_ptr(T, "T"));
+  CHECK(check_ptr(err_hist, "err_hist", false));
+  CHECK(check_ptr(stats, "stats", false));
+  const size_t need = aaac::fit_ws_bytes(N, K);
+  if (need > aaac::fixed_scratch_bytes())
+    return fail(AAAC_ERR_WORKSPACE,
+                "this layer (N=%lld K=%lld) needs %zu bytes of scratch but the library's fixed "
+                "scratch holds %zu; call aaac_fit_layer with a workspace instead",
+                (long long)N, (long long)K, need, aaac::fixed_scratch_bytes());
+  void* ws = nullptr;
+  cudaError_t e = aaac::fixed_scratch_ptr(&ws);
+  if (e != cudaSuccess) return from_cuda(e, "aaac_fit_layer_fixed_scratch: scratch address");
+  return from_cuda(aaac::launch_fit(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
+                                    cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T, err_hist,
+                                    stats, ws, (cudaStream_t)stream),
+                   "aaac_fit_layer_fixed_scratch");
+}
+
 aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const void* scales,
                       const aaac_config* cfg, const float* T, uint16_t* T_bf16, uint8_t* codes,
                       void* scales_tagged, uint8_t* choice_bits, double* err_final, void* ws,

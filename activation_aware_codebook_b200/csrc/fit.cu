@@ -29,6 +29,8 @@
 //   lane-private shared-memory bins modulo 2^64, which keeps num exact modulo
 //   2^51 and den modulo 2^52 -- exact because every lane's partial sum is far
 //   below those bounds.  Integer sums make the result independent of order.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -692,6 +694,39 @@ cudaError_t launch_fit(const uint16_t* W, int64_t N, int64_t K, const float* I,
                                              stats, ws, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// library-owned scratch for aaac_fit_layer_fixed_scratch
+// ---------------------------------------------------------------------------
+// The fit's scratch (control block + one fp64 per block) in a file-scope device
+// array: every GPU that loads the library holds it until the process exits.
+// All calls share it, so calls whose work overlaps on the GPU would race.
+constexpr size_t kFixedScratchBytes = 256 * 1024;
+static __device__ __align__(256) unsigned char g_fit_scratch[kFixedScratchBytes];
+
+size_t fixed_scratch_bytes() { return kFixedScratchBytes; }
+
+// In host code g_fit_scratch names a host-side stand-in, not device memory:
+// the device address is looked up with cudaGetSymbolAddress, once per device,
+// with that device current, and cached.
+cudaError_t fixed_scratch_ptr(void** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fit_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
 }
 
 // ---------------------------------------------------------------------------

@@ -36,6 +36,10 @@ size_t init_ctl_bytes();
 size_t pack_extra_bytes(int64_t N, int64_t K, int S);
 size_t fit_ws_bytes(int64_t N, int64_t K);
 
+// ---- the fit's library-owned scratch (fit.cu) -----------------------------
+size_t fixed_scratch_bytes();
+cudaError_t fixed_scratch_ptr(void** out);
+
 // ---- launch accounting (aaac_kernel_launches) ------------------------------
 void count_launches(int n);
 

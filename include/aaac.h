@@ -135,6 +135,29 @@ aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
                            double* err_hist, aaac_stats* stats, void* ws, size_t ws_bytes,
                            void* stream);
 
+/* The same fit as aaac_fit_layer, for callers that cannot allocate device
+ * memory -- for example code that runs where cudaMalloc is not permitted, or
+ * a plugin that has no access to its host framework's allocator and so cannot
+ * provide a workspace.  The paper has no counterpart to this call; it exists
+ * for integration only.
+ *   Arguments and results are those of aaac_fit_layer, without ws/ws_bytes.
+ *   Scratch: a 256 KiB array inside the library (every GPU that loads the
+ *   library holds it until the process exits).  Layers whose scratch need,
+ *   aaac_workspace_size's fit share, exceeds it are rejected with
+ *   AAAC_ERR_WORKSPACE before anything is launched (in practice only layers
+ *   with K above about 8 million).
+ *   The first call on a device looks up the array's device address with that
+ *   device current; make that first call before any stream capture.
+ *   All calls share the one array and it keeps the previous call's contents
+ *   (the call clears what must start at zero).  Calls whose work overlaps on
+ *   the GPU -- concurrent streams, or concurrent host threads -- race on it:
+ *   serialise them.
+ *   The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *   library routine. */
+aaac_status aaac_fit_layer_fixed_scratch(const void* W, int64_t N, int64_t K, const float* I,
+                                         const void* scales, const aaac_config* cfg, float* T,
+                                         double* err_hist, aaac_stats* stats, void* stream);
+
 /* Storage, section 2 core mechanism 3 and section 4: T is sorted and rounded
  * to bf16, a last assign (as in the fit) runs with the bf16 tables, then
  *   T_bf16        device uint16 [2][16] (64 bytes; entries j >= n are 0)
