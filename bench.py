@@ -302,7 +302,7 @@ def run_ours(args, rank, local_rank, world):
     fit_ms = statistics.median(a.elapsed_time(b) for a, b in fit_ev)
     ms_max = max_over_ranks(ms, world, dev)
 
-    # roofline of the fit round (assign pass + one-block finalize) on the probe layer
+    # roofline of one fit round (one fit_pass launch) on the probe layer
     iter_ms = (fit_ms - setup_ms) / wl.iters
     scale_bytes = 2 if wl.fmt == bb.INT4 else 1
     bytes_per_iter = (probe.N * probe.K * 2 + probe.N * (probe.K // wl.g) * scale_bytes
@@ -336,7 +336,7 @@ def run_ours(args, rank, local_rank, world):
                        "blocks": world, "parallelism": f"layer-parallel x{world} (no collective)",
                        "l2": "inputs larger than L2 (activations %.1f GiB per step)" % (
                            sum(x.numel() * 2 for x in Xs.values()) / 2 ** 30)},
-            "roofline": {"kernel": "assign_pass<INT4,fit> + fit_finalize (one fit round)",
+            "roofline": {"kernel": "fit_pass (one fit round; refine fused in its last block)",
                          "layer": f"{probe.name} {probe.N}x{probe.K}",
                          "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
