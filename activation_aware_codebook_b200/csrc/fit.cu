@@ -15,13 +15,14 @@
 // covers 256 columns of a row (16 bytes per lane) and walks the rows of its
 // chunk with a 6-deep cp.async ring, so several rows per warp are in flight.
 //
-// Nearest entry, per weight and book (exact):
-//   bucket b = rint(u * la + 64) (one FFMA), lut[b] = the count c of distinct-
-//   value thresholds below the bucket (and a flag when two or more thresholds
-//   fall inside it);  pair[c] = (v_c, v_{c+1});  with A = fl(u-v_c)^2 and
-//   B = fl(u-v_{c+1})^2 the count is c+1 when B < A and c when A < B -- both
-//   exact, because rounding is monotone -- and the rare A == B or flagged
-//   buckets take the exact threshold search.  min(A, B) is the squared error.
+// Nearest entry in both books at once (exact):
+//   the midpoint thresholds of both books, merged and deduplicated (at most
+//   30), split the u line into merged cells; cell m fixes both books' nearest
+//   entries, mval[m] = (v0, v1).  bucket b = rint(u * la + 64) (one FFMA);
+//   mlut[b] = the number c of merged thresholds at or below every u of the
+//   bucket (255 when two or more fall inside it: the exact search takes over);
+//   then m = c + (u >= mthr[c]) -- exact, because every threshold is the
+//   smallest fp32 above an exact midpoint.
 // Choice: fp32 group sums when their gap exceeds the rounding bound, else the
 //   sequential fp64 rule (the group's leader lane recomputes it).
 // Refine sums: per weight rint(A 2^L u) and rint(A 2^L), A = I_k s^2, as the
@@ -45,16 +46,18 @@ constexpr float kBucketMagic = 12582912.0f;           // 1.5 * 2^23
 constexpr double kDenMagic = 4503599627370496.0;      // 2^52
 #define kInf __int_as_float(0x7f800000)
 
-// lut[c][b] = 8 * (distinct-value count below bucket b) for book c, or 128
-// (the NaN pair, which forces the exact search) when two or more of the
-// book's thresholds fall strictly inside the bucket.  pair[c][j] =
-// (v_j, v_{j+1}); pair[c][16] = (NaN, NaN).
+// Merged tables of both books (see the header comment).  Entries from 31 on
+// are padding (mthr = +inf), so a lookup at 255 stays in bounds.
+constexpr int kMerged = 256;
 struct Tables {
   Book bk[2];
-  float2 pair[2][17];
-  uint8_t lut[2][kNB];
+  float mthr[kMerged];     // merged thresholds, ascending, +inf padded
+  float2 mval[kMerged];    // (v0[count0], v1[count1]) of merged cell m
+  uint8_t mcell[kMerged];  // count0 | count1 << 4 of merged cell m
+  uint8_t mlut[kNB];       // bucket -> merged base count, 255 = crowded bucket
   float la;
-  int32_t pad[3];
+  int32_t nm;              // number of merged thresholds
+  int32_t pad[2];
 };
 
 struct FitCtl {
@@ -110,13 +113,12 @@ __device__ inline int bucket_raw(float x, float la) {
   return min(max(r, -1), kNB);
 }
 
-// Entry of bucket b for book c: 8 * #(thresholds <= every u of the bucket),
-// or 128 when two or more thresholds fall strictly inside it.
-__device__ uint8_t lut_entry(const Tables& tb, int c, int b) {
-  const Book& bk = tb.bk[c];
+// Entry of bucket b: the number of merged thresholds <= every u of the
+// bucket, or 255 when two or more fall strictly inside it.
+__device__ uint8_t mlut_entry(const Tables& tb, int b) {
   int base = 0, inner = 0;
-  for (int i = 0; i + 1 < bk.m; i++) {
-    const float th = bk.thr[i];
+  for (int i = 0; i < tb.nm; i++) {
+    const float th = tb.mthr[i];
     const int rb = bucket_raw(th, tb.la);
     if (rb < b) {
       base++;
@@ -126,14 +128,36 @@ __device__ uint8_t lut_entry(const Tables& tb, int c, int b) {
       else inner++;
     }
   }
-  return (uint8_t)(inner > 1 ? 128 : 8 * base);
+  return (uint8_t)(inner > 1 ? 255 : base);
 }
 
-__device__ void fill_pairs(Tables& tb, int c) {
-  const Book& bk = tb.bk[c];
-  for (int j = 0; j < 16; j++)
-    tb.pair[c][j] = make_float2(bk.val[j], (j + 1 < bk.m) ? bk.val[j + 1] : kInf);
-  tb.pair[c][16] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+// Merge both books' thresholds (one thread).
+__device__ void merge_thresholds(Tables& tb) {
+  const Book& a = tb.bk[0];
+  const Book& b = tb.bk[1];
+  int i = 0, j = 0, n = 0;
+  const int na = a.m - 1, nb = b.m - 1;
+  while (i < na || j < nb) {
+    float t;
+    if (j >= nb || (i < na && a.thr[i] < b.thr[j])) t = a.thr[i++];
+    else if (i >= na || b.thr[j] < a.thr[i]) t = b.thr[j++];
+    else { t = a.thr[i++]; j++; }  // equal thresholds: one cell boundary
+    tb.mthr[n++] = t;
+  }
+  tb.nm = n;
+  for (int k = n; k < kMerged; k++) tb.mthr[k] = kInf;
+}
+
+// Cell m of the merged tables (thread per cell).
+__device__ void merged_cell(Tables& tb, int m) {
+  int c0 = 0, c1 = 0;
+  if (m >= 1 && m <= tb.nm) {
+    const float lo = tb.mthr[m - 1];  // smallest u of the cell
+    for (int i = 0; i + 1 < tb.bk[0].m; i++) c0 += (tb.bk[0].thr[i] <= lo) ? 1 : 0;
+    for (int i = 0; i + 1 < tb.bk[1].m; i++) c1 += (tb.bk[1].thr[i] <= lo) ? 1 : 0;
+  }
+  tb.mcell[m] = (uint8_t)(c0 | (c1 << 4));
+  tb.mval[m] = make_float2(tb.bk[0].val[c0], tb.bk[1].val[c1]);
 }
 
 // ---------------------------------------------------------------------------
@@ -213,14 +237,20 @@ __device__ float bucket_scale(const FitCtl* ctl) {
 
 // Tables of both books from ctl->T (sorted first), all threads of one block.
 __device__ void publish_tables(FitCtl* ctl, Tables& tb, int n, bool sort_in_place) {
+  __shared__ float sT[2][16];  // sort and scan in shared memory, not in L2
+  if (threadIdx.x < 32) sT[threadIdx.x >> 4][threadIdx.x & 15] = ctl->T[threadIdx.x >> 4][threadIdx.x & 15];
+  __syncthreads();
   if (threadIdx.x < 2) {
     const int c = threadIdx.x;
-    if (sort_in_place) sort_book(ctl->T[c], n);
-    build_book(ctl->T[c], n, &tb.bk[c]);
-    fill_pairs(tb, c);
+    if (sort_in_place) sort_book(sT[c], n);
+    build_book(sT[c], n, &tb.bk[c]);
   }
   __syncthreads();
-  for (int b = threadIdx.x; b < 2 * kNB; b += blockDim.x) tb.lut[b / kNB][b % kNB] = lut_entry(tb, b / kNB, b % kNB);
+  if (threadIdx.x < 32) ctl->T[threadIdx.x >> 4][threadIdx.x & 15] = sT[threadIdx.x >> 4][threadIdx.x & 15];
+  if (threadIdx.x == 0) merge_thresholds(tb);
+  __syncthreads();
+  for (int m = threadIdx.x; m < kMerged; m += blockDim.x) merged_cell(tb, m);
+  for (int b = threadIdx.x; b < kNB; b += blockDim.x) tb.mlut[b] = mlut_entry(tb, b);
   __syncthreads();
   const uint32_t* src = reinterpret_cast<const uint32_t*>(&tb);
   uint32_t* dst = reinterpret_cast<uint32_t*>(&ctl->tb);
@@ -421,6 +451,9 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   }
 #pragma unroll
   for (int i = 0; i < 8; i++) I2L[i] = (double)Ik[i] * twoL;
+  unsigned long long I2[8];
+#pragma unroll
+  for (int i = 0; i < 8; i++) I2[i] = f2pack(Ik[i], Ik[i]);
 
   const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
   const uint16_t* wcol = W + col0;
@@ -431,8 +464,11 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     if (active && rr < r1) cp_async16(myring + k * 32, wcol + (int64_t)rr * K);
     cp_async_commit();
   }
-  float s_next = 0.0f;
+  // scales prefetched two rows ahead
+  float s_next = 0.0f, s_next2 = 0.0f;
   if (active && r0 + warp < r1) s_next = load_scale<FMT>(scales, (int64_t)(r0 + warp) * G + col0 / g);
+  if (active && r0 + warp + kFitWarps < r1)
+    s_next2 = load_scale<FMT>(scales, (int64_t)(r0 + warp + kFitWarps) * G + col0 / g);
 
   double err_acc = 0.0;
   unsigned long long n_near = 0, n_exact = 0, n_t1 = 0;
@@ -441,14 +477,16 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     cp_async_wait<kStages - 1>();
     const uint4 v = active ? myring[slot * 32] : make_uint4(0, 0, 0, 0);
     const float s = s_next;
-    if (active && r + kFitWarps < r1)
-      s_next = load_scale<FMT>(scales, (int64_t)(r + kFitWarps) * G + col0 / g);
+    s_next = s_next2;
+    if (active && r + 2 * kFitWarps < r1)
+      s_next2 = load_scale<FMT>(scales, (int64_t)(r + 2 * kFitWarps) * G + col0 / g);
     float rcp;
     const bool live = active && scale_live(s, &rcp);
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
     float u[8];
-    uint32_t kk[8];  // 8 * distinct count: book 0 in bits 0..7, book 1 in bits 8..15
+    uint32_t mm[8];  // merged cell of each weight
     unsigned long long dd = 0ull;  // (D0, D1) partial sums
+    bool crowded = false;
     const unsigned long long rcp2 = f2pack(rcp, rcp);
 #pragma unroll
     for (int h = 0; h < 4; h++) {
@@ -458,30 +496,29 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     }
 #pragma unroll
     for (int i = 0; i < 8; i++) {
-      const uint32_t bi = __float_as_uint(bucket_t(u[i], la)) & (kNB - 1);
-      const uint32_t c0 = tb.lut[0][bi], c1 = tb.lut[1][bi];
-      const unsigned long long p0 = *reinterpret_cast<const unsigned long long*>(
-          reinterpret_cast<const unsigned char*>(&tb.pair[0][0]) + c0);
-      const unsigned long long p1 = *reinterpret_cast<const unsigned long long*>(
-          reinterpret_cast<const unsigned char*>(&tb.pair[1][0]) + c1);
-      const unsigned long long uu = f2pack(u[i], u[i]);
-      const unsigned long long e0 = f2sub(uu, p0), e1 = f2sub(uu, p1);
-      const float2 s0 = f2unpack(f2mul(e0, e0)), s1 = f2unpack(f2mul(e1, e1));
-      const bool up0 = s0.y < s0.x, dn0 = s0.x < s0.y;
-      const bool up1 = s1.y < s1.x, dn1 = s1.x < s1.y;
-      uint32_t k0 = c0 + (up0 ? 8u : 0u), k1 = c1 + (up1 ? 8u : 0u);
-      float m0 = up0 ? s0.y : s0.x, m1 = up1 ? s1.y : s1.x;
-      if (!(up0 | dn0) | !(up1 | dn1)) {  // rare: tie, or a crowded bucket
-        const int x0 = book_count(tb.bk[0], u[i]), x1 = book_count(tb.bk[1], u[i]);
-        const float f0 = __fsub_rn(u[i], tb.bk[0].val[x0]);
-        const float f1 = __fsub_rn(u[i], tb.bk[1].val[x1]);
-        k0 = 8u * (uint32_t)x0;
-        k1 = 8u * (uint32_t)x1;
-        m0 = __fmul_rn(f0, f0);
-        m1 = __fmul_rn(f1, f1);
+      const uint32_t c = tb.mlut[__float_as_uint(bucket_t(u[i], la)) & (kNB - 1)];
+      crowded |= (c == 255u);
+      const uint32_t m = c + (u[i] >= tb.mthr[c] ? 1u : 0u);
+      mm[i] = m;
+      const unsigned long long vv = *reinterpret_cast<const unsigned long long*>(&tb.mval[m]);
+      const unsigned long long e = f2sub(f2pack(u[i], u[i]), vv);
+      dd = f2fma(I2[i], f2mul(e, e), dd);
+    }
+    if (crowded) {  // rare: a bucket with two or more thresholds; redo the lane exactly
+      dd = 0ull;
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        int m = 0;
+        m += (tb.mthr[m + 15] <= u[i]) ? 16 : 0;
+        m += (tb.mthr[m + 7] <= u[i]) ? 8 : 0;
+        m += (tb.mthr[m + 3] <= u[i]) ? 4 : 0;
+        m += (tb.mthr[m + 1] <= u[i]) ? 2 : 0;
+        m += (tb.mthr[m] <= u[i]) ? 1 : 0;
+        mm[i] = (uint32_t)m;
+        const unsigned long long vv = *reinterpret_cast<const unsigned long long*>(&tb.mval[m]);
+        const unsigned long long e = f2sub(f2pack(u[i], u[i]), vv);
+        dd = f2fma(I2[i], f2mul(e, e), dd);
       }
-      kk[i] = k0 | (k1 << 8);
-      dd = f2fma(f2pack(Ik[i], Ik[i]), f2pack(m0, m1), dd);
     }
     float d0, d1;
     {
@@ -523,23 +560,25 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     choice = __shfl_sync(0xffffffffu, choice, leader_lane);
 
     if (s_leader && live) {
-      double D0 = exact ? E0 : (double)d0, D1 = exact ? E1 : (double)d1;
-      if (single) D1 = D0 + fabs(D0) + 1.0;  // no near-tie count when T1 is off
-      const double mx = fmax(D0, D1);
-      if (fabs(D1 - D0) < 1e-6 * mx) n_near++;
-      n_exact += exact ? 1 : 0;
+      if (exact) {
+        n_exact++;
+        if (fabs(E1 - E0) < 1e-6 * fmax(E0, E1)) n_near++;
+        if (!PACK) err_acc += (double)(s * s) * (choice ? E1 : E0);  // s*s exact in fp32
+      } else {
+        if (!single && fabsf(d1 - d0) < 1e-6f * fmaxf(d0, d1)) n_near++;
+        if (!PACK) err_acc += (double)(s * s) * (double)(choice ? d1 : d0);
+      }
       n_t1 += choice;
-      if (!PACK) err_acc += (double)s * (double)s * (choice ? D1 : D0);
     }
 
     if (!PACK) {
       if (live) {
         const double s2 = (double)s * (double)s;
-        const int shift = choice ? 8 : 0;
+        const int shift = choice ? 4 : 0;
         ulonglong2* cb_bins = mybins + choice * 16 * 32;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-          const uint32_t q = ((kk[i] >> shift) >> 3) & 15u;
+          const uint32_t q = ((uint32_t)tb.mcell[mm[i]] >> shift) & 15u;
           const double A = __dmul_rn(I2L[i], s2);  // exact: 24 + 16 bits
           const unsigned long long num =
               (unsigned long long)__double_as_longlong(__fma_rn(A, (double)u[i], kMagic));
@@ -553,11 +592,11 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
       }
     } else if (active) {
       const Book& bc = tb.bk[choice];
-      const int shift = choice ? 8 : 0;
+      const int shift = choice ? 4 : 0;
       uint32_t packed = 0;
 #pragma unroll
       for (int i = 0; i < 8; i++) {
-        const uint32_t q = ((kk[i] >> shift) >> 3) & 15u;
+        const uint32_t q = ((uint32_t)tb.mcell[mm[i]] >> shift) & 15u;
         packed |= (uint32_t)bc.idx[q] << (4 * i);
         const float wf = (i & 1) ? bf16_hi(wv[i >> 1]) : bf16_lo(wv[i >> 1]);
         const double wh = (double)s * (double)bc.val[q];

@@ -39,7 +39,7 @@ size_t init_ctl_bytes() { return align256(sizeof(InitCtl)); }
 PassPlan plan_pass(int64_t N, int64_t K, int target) {
   PassPlan p;
   p.ncb = (int)((K + kSegCols - 1) / kSegCols);
-  int64_t nrc = (target + p.ncb - 1) / p.ncb;
+  int64_t nrc = target / p.ncb;  // at most `target` blocks: one full wave
   if (nrc > N) nrc = N;
   if (nrc < 1) nrc = 1;
   p.rows_per_chunk = (int)((N + nrc - 1) / nrc);
