@@ -157,30 +157,42 @@ radix_pass(const uint16_t* __restrict__ W, int N, int K, int g, const void* __re
   }
 }
 
-__global__ void radix_select(InitCtl* c, int pass, float* T) {
+// 256 threads: the histograms are read into shared memory once, then one
+// thread per target rank walks its prefix's 256 counts there.
+__global__ void __launch_bounds__(256) radix_select(InitCtl* c, int pass, float* T) {
+  __shared__ uint32_t hist[32][256];
+  __shared__ uint32_t sp[32];
   __shared__ uint32_t newp[32];
-  const int i = threadIdx.x;  // 32 threads
+  __shared__ int ns;
+  const int tid = threadIdx.x;
   const int nr = c->nranks;
-  if (i < nr) {
+  if (tid == 0) ns = c->nslots;
+  if (tid < 32) sp[tid] = c->slot_prefix[tid];
+  __syncthreads();
+  const int nslots = ns;
+  for (int j = tid; j < nslots * 256; j += blockDim.x) {
+    (&hist[0][0])[j] = (&c->hist[0][0])[j];
+    (&c->hist[0][0])[j] = 0u;  // ready for the next pass
+  }
+  __syncthreads();
+  if (tid < nr) {
     int slot = 0;
-    if (pass > 0) {
-      for (int s = 0; s < c->nslots; s++)
-        if (c->slot_prefix[s] == c->prefix[i]) slot = s;
-    }
-    int64_t want = c->resid[i], cum = 0;
+    if (pass > 0)
+      for (int s = 0; s < nslots; s++)
+        if (sp[s] == c->prefix[tid]) slot = s;
+    int64_t want = c->resid[tid], cum = 0;
     int d = 0;
     for (; d < 255; d++) {
-      const int64_t h = c->hist[slot][d];
+      const int64_t h = hist[slot][d];
       if (cum + h > want) break;
       cum += h;
     }
-    c->resid[i] = want - cum;
-    c->prefix[i] = (pass == 0) ? (uint32_t)d : ((c->prefix[i] << 8) | (uint32_t)d);
-    newp[i] = c->prefix[i];
+    c->resid[tid] = want - cum;
+    c->prefix[tid] = (pass == 0) ? (uint32_t)d : ((c->prefix[tid] << 8) | (uint32_t)d);
+    newp[tid] = c->prefix[tid];
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < 32 * 256; j += blockDim.x) (&c->hist[0][0])[j] = 0u;
-  if (i == 0) {
+  if (tid == 0) {
     // sorted distinct prefixes for the next pass (T0's and T1's ranks
     // interleave, so sort first)
     for (int a = 1; a < nr; a++) {
@@ -191,15 +203,15 @@ __global__ void radix_select(InitCtl* c, int pass, float* T) {
     }
     int m = 0;
     for (int r = 0; r < nr; r++)
-      if (m == 0 || c->slot_prefix[m - 1] != newp[r]) c->slot_prefix[m++] = newp[r];
+      if (m == 0 || sp[m - 1] != newp[r]) sp[m++] = newp[r];
     c->nslots = m;
-    if (pass == 3) {
-      const int n = c->n;
-      for (int j = 0; j < 16; j++) {
-        T[j] = j < n ? key_to_float(c->prefix[j]) : 0.0f;
-        T[16 + j] = j < n ? key_to_float(c->prefix[n + j]) : 0.0f;
-      }
-    }
+  }
+  __syncthreads();
+  if (tid < 32) c->slot_prefix[tid] = sp[tid];
+  if (pass == 3 && tid < 32) {
+    const int n = c->n;
+    const int j = tid & 15, b = tid >> 4;
+    T[tid] = j < n ? key_to_float(c->prefix[b * n + j]) : 0.0f;
   }
 }
 
@@ -230,7 +242,7 @@ cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g,
     else
       radix_pass<kNvfp4><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, g, scales, c, pass,
                                                          pp.ncb, pp.rows_per_chunk);
-    radix_select<<<1, 32, 0, st>>>(c, pass, T);
+    radix_select<<<1, 256, 0, st>>>(c, pass, T);
   }
   count_launches(10);
   return cudaGetLastError();
