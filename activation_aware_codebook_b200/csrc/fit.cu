@@ -27,9 +27,11 @@
 //   sequential fp64 rule (the group's leader lane recomputes it).
 // Refine sums: per weight rint(A 2^L u) and rint(A 2^L), A = I_k s^2, as the
 //   raw bit patterns of fp64 FMA/ADD results with magic constants; summed in
-//   lane-private shared-memory bins modulo 2^64, which keeps num exact modulo
-//   2^51 and den modulo 2^52 -- exact because every lane's partial sum is far
-//   below those bounds.  Integer sums make the result independent of order.
+//   shared-memory bins modulo 2^64, which keeps num exact modulo 2^51 and den
+//   modulo 2^52 -- exact because every bin's partial sum stays far below those
+//   bounds.  Each pair of lanes owns one set of bins and the two lanes update it
+//   in turn (read-modify-write, no atomics); halving the bins' shared memory
+//   lets 16 warps share an SM.  Integer sums make the result order-free.
 #include <mutex>
 
 #include "common.cuh"
@@ -41,7 +43,7 @@ constexpr int kNB = 128;                  // bucket LUT entries
 constexpr int kFitWarps = 2;
 constexpr int kFitThreads = kFitWarps * 32;
 constexpr int kStages = 6;                // rows per warp in flight
-constexpr int kFitBlocksPerSM = 5;
+constexpr int kFitBlocksPerSM = 8;
 constexpr float kBucketMagic = 12582912.0f;           // 1.5 * 2^23
 constexpr double kDenMagic = 4503599627370496.0;      // 2^52
 #define kInf __int_as_float(0x7f800000)
@@ -95,7 +97,7 @@ size_t pack_extra_bytes(int64_t N, int64_t K, int S) {
 static size_t smem_bytes(bool pack) {
   size_t b = (sizeof(Tables) + 15) & ~(size_t)15;
   b += (size_t)kFitWarps * kStages * 32 * sizeof(uint4);
-  if (!pack) b += (size_t)kFitWarps * 32 * 32 * sizeof(ulonglong2);
+  if (!pack) b += (size_t)kFitWarps * 32 * 16 * sizeof(ulonglong2);
   return b;
 }
 
@@ -419,7 +421,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     uint32_t* dst = reinterpret_cast<uint32_t*>(&tb);
     for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
     if (!PACK)
-      for (int i = threadIdx.x; i < kFitWarps * 32 * 32; i += blockDim.x)
+      for (int i = threadIdx.x; i < kFitWarps * 32 * 16; i += blockDim.x)
         bins[i] = make_ulonglong2(0ull, 0ull);
   }
   const double twoL = ctl->twoL;
@@ -436,7 +438,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   const bool single = (flags & AAAC_SINGLE_CODEBOOK) != 0;
   const float la = tb.la;
   uint4* myring = ring + warp * kStages * 32 + lane;
-  ulonglong2* mybins = bins + warp * 32 * 32 + lane;
+  ulonglong2* mybins = bins + warp * 32 * 16 + (lane >> 1);
 
   float Ik[8];
   double I2L[8];
@@ -572,23 +574,31 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     }
 
     if (!PACK) {
-      if (live) {
-        const double s2 = (double)s * (double)s;
-        const int shift = choice ? 4 : 0;
-        ulonglong2* cb_bins = mybins + choice * 16 * 32;
+      const double s2 = (double)s * (double)s;
+      const int shift = choice ? 4 : 0;
+      ulonglong2* cb_bins = mybins + choice * 16 * 16;
+      unsigned long long nums[8], dens[8];
+      uint32_t qs[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-          const uint32_t q = ((uint32_t)tb.mcell[mm[i]] >> shift) & 15u;
-          const double A = __dmul_rn(I2L[i], s2);  // exact: 24 + 16 bits
-          const unsigned long long num =
-              (unsigned long long)__double_as_longlong(__fma_rn(A, (double)u[i], kMagic));
-          const unsigned long long den =
-              (unsigned long long)__double_as_longlong(__dadd_rn(A, kDenMagic));
-          ulonglong2 x = cb_bins[q * 32];
-          x.x += num;
-          x.y += den;
-          cb_bins[q * 32] = x;
+      for (int i = 0; i < 8; i++) {
+        qs[i] = ((uint32_t)tb.mcell[mm[i]] >> shift) & 15u;
+        const double A = __dmul_rn(I2L[i], s2);  // exact: 24 + 16 bits
+        nums[i] = (unsigned long long)__double_as_longlong(__fma_rn(A, (double)u[i], kMagic));
+        dens[i] = (unsigned long long)__double_as_longlong(__dadd_rn(A, kDenMagic));
+      }
+      // the two lanes of a pair share bins: update them one lane at a time
+#pragma unroll
+      for (int half = 0; half < 2; half++) {
+        if (live && (lane & 1) == half) {
+#pragma unroll
+          for (int i = 0; i < 8; i++) {
+            ulonglong2 x = cb_bins[qs[i] * 16];
+            x.x += nums[i];
+            x.y += dens[i];
+            cb_bins[qs[i] * 16] = x;
+          }
         }
+        __syncwarp();
       }
     } else if (active) {
       const Book& bc = tb.bk[choice];
@@ -651,8 +661,8 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     const int cell = threadIdx.x >> 1, which = threadIdx.x & 1;
     long long sum = 0;
     for (int w = 0; w < kFitWarps; w++) {
-      const ulonglong2* p = bins + (w * 32 + cell) * 32;
-      for (int l = 0; l < 32; l++) {
+      const ulonglong2* p = bins + (w * 32 + cell) * 16;
+      for (int l = 0; l < 16; l++) {
         const unsigned long long raw = which ? p[l].y : p[l].x;
         sum += which ? (long long)(raw & ((1ull << 52) - 1))
                      : ((long long)(raw << 13) >> 13);
