@@ -13,7 +13,7 @@
 // last block to finish (atomic ticket, no waiting) does the refine, sorts the
 // books, rebuilds the tables and records the error.  Per block: 4 warps; a warp
 // covers 256 columns of a row (16 bytes per lane) and walks the rows of its
-// chunk with a 6-deep cp.async ring, so several rows per warp are in flight.
+// chunk with a 3-deep cp.async ring, so several rows per warp are in flight.
 //
 // Nearest entry in both books at once (exact):
 //   the midpoint thresholds of both books, merged and deduplicated (at most
@@ -42,15 +42,16 @@ namespace aaac {
 constexpr int kNB = 128;                  // bucket LUT entries
 constexpr int kFitWarps = 2;
 constexpr int kFitThreads = kFitWarps * 32;
-constexpr int kStages = 6;                // rows per warp in flight
-constexpr int kFitBlocksPerSM = 8;
+constexpr int kStages = 3;                // rows per warp in flight
+constexpr int kFitBlocksPerSM = 10;
 constexpr float kBucketMagic = 12582912.0f;           // 1.5 * 2^23
 constexpr double kDenMagic = 4503599627370496.0;      // 2^52
 #define kInf __int_as_float(0x7f800000)
 
-// Merged tables of both books (see the header comment).  Entries from 31 on
-// are padding (mthr = +inf), so a lookup at 255 stays in bounds.
-constexpr int kMerged = 256;
+// Merged tables of both books (see the header comment).  Entries past the
+// last cell are padding (mthr = +inf); 33 entries keep every lookup in bounds.
+constexpr int kMerged = 33;
+constexpr uint32_t kCrowded = 31;  // lut value of a crowded bucket (base counts are <= 30)
 struct Tables {
   Book bk[2];
   float mthr[kMerged];     // merged thresholds, ascending, +inf padded
@@ -130,7 +131,7 @@ __device__ uint8_t mlut_entry(const Tables& tb, int b) {
       else inner++;
     }
   }
-  return (uint8_t)(inner > 1 ? 255 : base);
+  return (uint8_t)(inner > 1 ? kCrowded : base);
 }
 
 // Merge both books' thresholds (one thread).
@@ -441,7 +442,6 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   ulonglong2* mybins = bins + warp * 32 * 16 + (lane >> 1);
 
   float Ik[8];
-  double I2L[8];
   if (active) {
     const float4 a = __ldg(reinterpret_cast<const float4*>(I + col0));
     const float4 b = __ldg(reinterpret_cast<const float4*>(I + col0 + 4));
@@ -451,11 +451,6 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
 #pragma unroll
     for (int i = 0; i < 8; i++) Ik[i] = 0.0f;
   }
-#pragma unroll
-  for (int i = 0; i < 8; i++) I2L[i] = (double)Ik[i] * twoL;
-  unsigned long long I2[8];
-#pragma unroll
-  for (int i = 0; i < 8; i++) I2[i] = f2pack(Ik[i], Ik[i]);
 
   const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
   const uint16_t* wcol = W + col0;
@@ -499,12 +494,12 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
 #pragma unroll
     for (int i = 0; i < 8; i++) {
       const uint32_t c = tb.mlut[__float_as_uint(bucket_t(u[i], la)) & (kNB - 1)];
-      crowded |= (c == 255u);
+      crowded |= (c == kCrowded);
       const uint32_t m = c + (u[i] >= tb.mthr[c] ? 1u : 0u);
       mm[i] = m;
       const unsigned long long vv = *reinterpret_cast<const unsigned long long*>(&tb.mval[m]);
       const unsigned long long e = f2sub(f2pack(u[i], u[i]), vv);
-      dd = f2fma(I2[i], f2mul(e, e), dd);
+      dd = f2fma(f2pack(Ik[i], Ik[i]), f2mul(e, e), dd);
     }
     if (crowded) {  // rare: a bucket with two or more thresholds; redo the lane exactly
       dd = 0ull;
@@ -519,7 +514,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
         mm[i] = (uint32_t)m;
         const unsigned long long vv = *reinterpret_cast<const unsigned long long*>(&tb.mval[m]);
         const unsigned long long e = f2sub(f2pack(u[i], u[i]), vv);
-        dd = f2fma(I2[i], f2mul(e, e), dd);
+        dd = f2fma(f2pack(Ik[i], Ik[i]), f2mul(e, e), dd);
       }
     }
     float d0, d1;
@@ -574,7 +569,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     }
 
     if (!PACK) {
-      const double s2 = (double)s * (double)s;
+      const double s2L = (double)s * (double)s * twoL;  // exact: s^2 has 16 bits
       const int shift = choice ? 4 : 0;
       ulonglong2* cb_bins = mybins + choice * 16 * 16;
       unsigned long long nums[8], dens[8];
@@ -582,7 +577,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
 #pragma unroll
       for (int i = 0; i < 8; i++) {
         qs[i] = ((uint32_t)tb.mcell[mm[i]] >> shift) & 15u;
-        const double A = __dmul_rn(I2L[i], s2);  // exact: 24 + 16 bits
+        const double A = __dmul_rn((double)Ik[i], s2L);  // exact: 24 + 16 bits
         nums[i] = (unsigned long long)__double_as_longlong(__fma_rn(A, (double)u[i], kMagic));
         dens[i] = (unsigned long long)__double_as_longlong(__dadd_rn(A, kDenMagic));
       }

@@ -208,3 +208,40 @@ def test_full_size_layer(name, idx, iters):
     out = bb.run_layer(W.cuda(), X.cuda(), cfg)
     ref = oracle.run_layer(u16(W), u16(X), wl.fmt, wl.g, wl.S, iters)
     check_against_oracle(out, ref, cfg, label=name)
+
+
+# --------------------------------------------------------------------------
+# full bench sizes: importance on 262144 tokens (sampled columns), and the
+# largest (Qwen-32B-shaped, NVFP4) layer for a few rounds
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("K", [4096, 14336])
+def test_importance_full_tokens_sampled_columns(K):
+    wl = synth.WORKLOADS["llama8b-int4-s16"]
+    X = synth.make_activations(wl.tokens, K, synth.seed_of(wl.name, 0, f"probe{K}", "X"), wl.heavy,
+                               device="cuda")
+    I = bb.importance(X)
+    Ie = bb.importance(X, exact=True)
+    rng = np.random.default_rng(K)
+    cols = np.sort(rng.choice(K, 48, replace=False))
+    heavy = torch.topk(synth.channel_scales(K, synth.seed_of(wl.name, 0, f"probe{K}", "X") ^ 0,
+                                            wl.heavy, device="cuda"), 3).indices.cpu().numpy()
+    cols = np.unique(np.concatenate([cols, heavy, [0, K - 1]]))
+    sub = u16(X[:, torch.from_numpy(cols).cuda()].contiguous())
+    ref = oracle.importance(sub)
+    got = I.cpu().numpy()[cols]
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    assert torch.equal(I.view(torch.int32), Ie.view(torch.int32))  # fast path == exact path
+    del X
+
+
+def test_qwen32b_nvfp4_full_layer_few_rounds():
+    wl = synth.WORKLOADS["qwen32b-nvfp4"]
+    lin = wl.linears[0]  # gate 27648x5120, Student-t weights
+    W = synth.make_weight(lin.N, lin.K, synth.seed_of(wl.name, 0, lin.name, "W"), wl.w_dist,
+                          device="cuda")
+    X = synth.make_activations(2048, lin.K, synth.seed_of(wl.name, 0, lin.x_key, "X"), wl.heavy,
+                               device="cuda")
+    cfg = cfg_of(wl.fmt, wl.g, wl.S, 2)
+    out = bb.run_layer(W, X, cfg)
+    ref = oracle.run_layer(u16(W), u16(X), wl.fmt, wl.g, wl.S, 2)
+    check_against_oracle(out, ref, cfg, label="qwen32b gate")
