@@ -77,10 +77,6 @@ struct Book {
   int32_t pad[3];
 };
 
-struct Books {
-  Book b[2];
-};
-
 // Smallest fp32 strictly greater than (a + b) / 2, exactly (a, b finite fp32).
 __device__ inline float midpoint_threshold(float a, float b) {
   double x = a, y = b;
@@ -103,22 +99,6 @@ __device__ inline void sort_book(float* t, int n) {
     while (j >= 0 && order_key(t[j]) > kv) { t[j + 1] = t[j]; j--; }
     t[j + 1] = v;
   }
-}
-
-// Build the tables of a sorted codebook t[0..n) (one thread).
-__device__ inline void build_book(const float* t, int n, Book* bk) {
-  int m = 0;
-  for (int j = 0; j < n; j++) {
-    if (m == 0 || !(t[j] == bk->val[m - 1])) {  // -0 == +0: one value
-      bk->val[m] = t[j];
-      bk->idx[m] = j;
-      m++;
-    }
-  }
-  for (int i = 0; i < 16; i++) bk->thr[i] = __uint_as_float(0x7f800000u);
-  for (int i = 0; i + 1 < m; i++) bk->thr[i] = midpoint_threshold(bk->val[i], bk->val[i + 1]);
-  for (int i = m; i < 16; i++) { bk->val[i] = bk->val[m - 1]; bk->idx[i] = bk->idx[m - 1]; }
-  bk->m = m;
 }
 
 // Count of thresholds <= u (branchless search over 15 sorted thresholds).

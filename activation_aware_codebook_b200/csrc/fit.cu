@@ -11,16 +11,18 @@
 //
 // One fit round is ONE launch of fit_pass<false>: a streaming pass over W whose
 // last block to finish (atomic ticket, no waiting) does the refine, sorts the
-// books, rebuilds the tables and records the error.  Per block: 4 warps; a warp
+// books, rebuilds the tables and records the error.  Per block: 2 warps; a warp
 // covers 256 columns of a row (16 bytes per lane) and walks the rows of its
 // chunk with a 3-deep cp.async ring, so several rows per warp are in flight.
+// The grid is one wave (10 blocks per SM).
 //
 // Nearest entry in both books at once (exact):
 //   the midpoint thresholds of both books, merged and deduplicated (at most
 //   30), split the u line into merged cells; cell m fixes both books' nearest
 //   entries, mval[m] = (v0, v1).  bucket b = rint(u * la + 64) (one FFMA);
 //   mlut[b] = the number c of merged thresholds at or below every u of the
-//   bucket (255 when two or more fall inside it: the exact search takes over);
+//   bucket (kCrowded when two or more fall inside it: a binary search takes
+//   over);
 //   then m = c + (u >= mthr[c]) -- exact, because every threshold is the
 //   smallest fp32 above an exact midpoint.
 // Choice: fp32 group sums when their gap exceeds the rounding bound, else the
@@ -57,7 +59,7 @@ struct Tables {
   float mthr[kMerged];     // merged thresholds, ascending, +inf padded
   float2 mval[kMerged];    // (v0[count0], v1[count1]) of merged cell m
   uint8_t mcell[kMerged];  // count0 | count1 << 4 of merged cell m
-  uint8_t mlut[kNB];       // bucket -> merged base count, 255 = crowded bucket
+  uint8_t mlut[kNB];       // bucket -> merged base count, kCrowded = crowded bucket
   float la;
   int32_t nm;              // number of merged thresholds
   int32_t pad[2];
@@ -116,24 +118,6 @@ __device__ inline int bucket_raw(float x, float la) {
   return min(max(r, -1), kNB);
 }
 
-// Entry of bucket b: the number of merged thresholds <= every u of the
-// bucket, or 255 when two or more fall strictly inside it.
-__device__ uint8_t mlut_entry(const Tables& tb, int b) {
-  int base = 0, inner = 0;
-  for (int i = 0; i < tb.nm; i++) {
-    const float th = tb.mthr[i];
-    const int rb = bucket_raw(th, tb.la);
-    if (rb < b) {
-      base++;
-    } else if (rb == b) {
-      const int rp = bucket_raw(nextafterf(th, -kInf), tb.la);
-      if (rp < b) base++;   // th is the bucket's smallest value
-      else inner++;
-    }
-  }
-  return (uint8_t)(inner > 1 ? kCrowded : base);
-}
-
 // Merge both books' thresholds (one thread).
 __device__ void merge_thresholds(Tables& tb) {
   const Book& a = tb.bk[0];
@@ -161,6 +145,64 @@ __device__ void merged_cell(Tables& tb, int m) {
   }
   tb.mcell[m] = (uint8_t)(c0 | (c1 << 4));
   tb.mval[m] = make_float2(tb.bk[0].val[c0], tb.bk[1].val[c1]);
+}
+
+// All tables from the codebooks sT[2][16] (shared memory), by every thread of
+// one block (blockDim >= 64): sort (optional), distinct values, exact midpoint
+// thresholds, merged thresholds, merged cells, and the bucket table (bucket b
+// counts the merged thresholds at or below its smallest u, or kCrowded when
+// two or more fall strictly inside it).
+__device__ void build_tables(Tables& tb, float (*sT)[16], int n, bool sort_first) {
+  __shared__ int s_rb[32], s_first[32];
+  const int tid = threadIdx.x;
+  if (tid < 2) {
+    const int c = tid;
+    if (sort_first) sort_book(sT[c], n);
+    Book& bk = tb.bk[c];
+    int m = 0;
+    for (int j = 0; j < n; j++) {
+      if (m == 0 || !(sT[c][j] == bk.val[m - 1])) {  // -0 == +0: one value
+        bk.val[m] = sT[c][j];
+        bk.idx[m] = j;
+        m++;
+      }
+    }
+    for (int i = m; i < 16; i++) { bk.val[i] = bk.val[m - 1]; bk.idx[i] = bk.idx[m - 1]; }
+    bk.m = m;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    Book& bk = tb.bk[tid >> 4];
+    const int i = tid & 15;
+    bk.thr[i] = (i + 1 < bk.m) ? midpoint_threshold(bk.val[i], bk.val[i + 1]) : kInf;
+  }
+  __syncthreads();
+  if (tid == 0) merge_thresholds(tb);
+  __syncthreads();
+  if (tid < tb.nm) {
+    const float th = tb.mthr[tid];
+    const int rb = bucket_raw(th, tb.la);
+    s_rb[tid] = rb;
+    s_first[tid] = bucket_raw(nextafterf(th, -kInf), tb.la) < rb;  // th opens its bucket
+  }
+  __syncthreads();
+  for (int m = tid; m < kMerged; m += blockDim.x) merged_cell(tb, m);
+  for (int b = tid; b < kNB; b += blockDim.x) {
+    int base = 0, inner = 0;
+    for (int i = 0; i < tb.nm; i++) {
+      const int rb = s_rb[i];
+      if (rb < b || (rb == b && s_first[i])) base++;
+      else if (rb == b) inner++;
+    }
+    tb.mlut[b] = (uint8_t)(inner > 1 ? kCrowded : base);
+  }
+  __syncthreads();
+}
+
+__device__ void store_tables(FitCtl* ctl, const Tables& tb) {
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(&tb);
+  uint32_t* dst = reinterpret_cast<uint32_t*>(&ctl->tb);
+  for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
 }
 
 // ---------------------------------------------------------------------------
@@ -238,28 +280,6 @@ __device__ float bucket_scale(const FitCtl* ctl) {
   return Umax > 0.0f ? __fdiv_rn(62.5f, Umax) : 0.0f;  // |u| * la < 63: buckets 1..127
 }
 
-// Tables of both books from ctl->T (sorted first), all threads of one block.
-__device__ void publish_tables(FitCtl* ctl, Tables& tb, int n, bool sort_in_place) {
-  __shared__ float sT[2][16];  // sort and scan in shared memory, not in L2
-  if (threadIdx.x < 32) sT[threadIdx.x >> 4][threadIdx.x & 15] = ctl->T[threadIdx.x >> 4][threadIdx.x & 15];
-  __syncthreads();
-  if (threadIdx.x < 2) {
-    const int c = threadIdx.x;
-    if (sort_in_place) sort_book(sT[c], n);
-    build_book(sT[c], n, &tb.bk[c]);
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) ctl->T[threadIdx.x >> 4][threadIdx.x & 15] = sT[threadIdx.x >> 4][threadIdx.x & 15];
-  if (threadIdx.x == 0) merge_thresholds(tb);
-  __syncthreads();
-  for (int m = threadIdx.x; m < kMerged; m += blockDim.x) merged_cell(tb, m);
-  for (int b = threadIdx.x; b < kNB; b += blockDim.x) tb.mlut[b] = mlut_entry(tb, b);
-  __syncthreads();
-  const uint32_t* src = reinterpret_cast<const uint32_t*>(&tb);
-  uint32_t* dst = reinterpret_cast<uint32_t*>(&ctl->tb);
-  for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
-}
-
 // L = B - E(I_max) - E(S2_max) - max(0, E(U_max)), B = min(40, 61 - ceil(log2 M))
 __global__ void __launch_bounds__(kFitThreads)
 fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st) {
@@ -283,14 +303,16 @@ fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st) {
     ctl->n = n;
     tb.la = bucket_scale(ctl);
   }
+  __shared__ float sT[2][16];
+  if (threadIdx.x < 32) sT[threadIdx.x >> 4][threadIdx.x & 15] = T_user[threadIdx.x];
+  __syncthreads();
+  build_tables(tb, sT, n, true);
+  store_tables(ctl, tb);
   if (threadIdx.x < 32) {
-    const int c = threadIdx.x >> 4, j = threadIdx.x & 15;
-    ctl->T[c][j] = T_user[threadIdx.x];
+    const float t = sT[threadIdx.x >> 4][threadIdx.x & 15];
+    ctl->T[threadIdx.x >> 4][threadIdx.x & 15] = t;
+    T_user[threadIdx.x] = t;
   }
-  __syncthreads();
-  publish_tables(ctl, tb, n, true);
-  __syncthreads();
-  if (threadIdx.x < 32) T_user[threadIdx.x] = ctl->T[threadIdx.x >> 4][threadIdx.x & 15];
   if (threadIdx.x == 0) write_stats(ctl, st);
 }
 
@@ -347,13 +369,22 @@ __device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsign
   return r;
 }
 
-// The refine of one round, run by the last block of the pass.
+// The refine of one round, run by the last block of the pass: centroids from
+// the integer sums (section 2, core mechanism 4), T = fp32(fp64(num) /
+// fp64(den)) when den > 0, else unchanged; then sorted books and new tables.
+// Everything is staged in shared memory and spread over the block's threads.
 __device__ void round_finalize(FitCtl* ctl, Tables& tb, const double* errp, int nb,
                                uint32_t flags, const RoundOut& ro, double* sred) {
+  __shared__ float sT[2][16];
+  __shared__ long long sb[64];
+  __shared__ int s_upd[2];
   const int tid = threadIdx.x;
   double part = 0.0;
   for (int b = tid; b < nb; b += blockDim.x) part = __dadd_rn(part, __ldcg(errp + b));
   sred[tid] = part;
+  if (tid < 64) sb[tid] = __ldcg(&ctl->bins[0][0][0] + tid);
+  if (tid < 32) sT[tid >> 4][tid & 15] = ctl->T[tid >> 4][tid & 15];
+  if (tid < 2) s_upd[tid] = 0;
   __syncthreads();
   if (tid == 0) {
     double e = 0.0;
@@ -361,34 +392,32 @@ __device__ void round_finalize(FitCtl* ctl, Tables& tb, const double* errp, int 
     if (ro.err_hist) ro.err_hist[ro.it] = e;
   }
   const int n = ctl->n;
-  __shared__ int s_empty[2];
-  if (tid < 2) {
-    const int c = tid;
+  if (tid < 32) {
+    const int c = tid >> 4, j = tid & 15;
     const bool frozen = (c == 0) ? (flags & AAAC_FREEZE_T0) : (flags & AAAC_FREEZE_T1);
-    int updated = 0;
-    if (!frozen) {
-      const Book& bk = tb.bk[c];  // tables of the round that just ran
-      for (int j = 0; j < bk.m; j++) {
-        const long long num = __ldcg(&ctl->bins[c][j][0]);
-        const long long den = __ldcg(&ctl->bins[c][j][1]);
-        if (den > 0) {
-          ctl->T[c][bk.idx[j]] =
-              __double2float_rn(__ddiv_rn(__ll2double_rn(num), __ll2double_rn(den)));
-          updated++;
-        }
+    const Book& bk = tb.bk[c];  // tables of the round that just ran
+    if (!frozen && j < bk.m) {
+      const long long num = sb[(c * 16 + j) * 2], den = sb[(c * 16 + j) * 2 + 1];
+      if (den > 0) {
+        sT[c][bk.idx[j]] = __double2float_rn(__ddiv_rn(__ll2double_rn(num), __ll2double_rn(den)));
+        atomicAdd(&s_upd[c], 1);
       }
     }
-    s_empty[c] = frozen ? 0 : n - updated;
   }
   __syncthreads();
-  publish_tables(ctl, tb, n, true);
-  __syncthreads();
-  if (tid < 32) ro.T_user[tid] = ctl->T[tid >> 4][tid & 15];
+  const bool f0 = (flags & AAAC_FREEZE_T0) != 0, f1 = (flags & AAAC_FREEZE_T1) != 0;
+  const int empty = (f0 ? 0 : n - s_upd[0]) + (f1 ? 0 : n - s_upd[1]);
+  build_tables(tb, sT, n, true);
+  store_tables(ctl, tb);
+  if (tid < 32) {
+    const float t = sT[tid >> 4][tid & 15];
+    ctl->T[tid >> 4][tid & 15] = t;
+    ro.T_user[tid] = t;
+  }
   if (tid < 64) (&ctl->bins[0][0][0])[tid] = 0;
   if (tid == 0) {
     // counters other blocks updated with atomics: read them from L2
-    const unsigned long long empty = (unsigned long long)(s_empty[0] + s_empty[1]);
-    ctl->empty_cells = empty;
+    ctl->empty_cells = (unsigned long long)empty;
     if (ro.stats) {
       ro.stats->near_ties = (int64_t)__ldcg(&ctl->near_ties);
       ro.stats->groups_t1 = (int64_t)__ldcg(&ctl->groups_t1);
@@ -779,23 +808,25 @@ cudaError_t fixed_scratch_ptr(void** out) {
 __global__ void __launch_bounds__(kFitThreads)
 pack_setup(FitCtl* ctl, const float* T_user, int n, uint16_t* T_bf16) {
   __shared__ Tables tb;
+  __shared__ float sT[2][16];
   if (threadIdx.x == 0) {
     ctl->n = n;
     tb.la = bucket_scale(ctl);
   }
-  if (threadIdx.x < 2) {
-    const int b = threadIdx.x;
-    float t[16];
-    for (int j = 0; j < 16; j++) t[j] = T_user[b * 16 + j];
-    sort_book(t, n);
-    for (int j = 0; j < 16; j++) {
-      const unsigned short h = j < n ? __bfloat16_as_ushort(__float2bfloat16_rn(t[j])) : 0;
-      T_bf16[b * 16 + j] = h;
-      ctl->T[b][j] = __uint_as_float((uint32_t)h << 16);
-    }
+  if (threadIdx.x < 32) sT[threadIdx.x >> 4][threadIdx.x & 15] = T_user[threadIdx.x];
+  __syncthreads();
+  if (threadIdx.x < 2) sort_book(sT[threadIdx.x], n);
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int b = threadIdx.x >> 4, j = threadIdx.x & 15;
+    const unsigned short h = j < n ? __bfloat16_as_ushort(__float2bfloat16_rn(sT[b][j])) : 0;
+    T_bf16[threadIdx.x] = h;
+    sT[b][j] = __uint_as_float((uint32_t)h << 16);
   }
   __syncthreads();
-  publish_tables(ctl, tb, n, false);
+  build_tables(tb, sT, n, false);
+  store_tables(ctl, tb);
+  if (threadIdx.x < 32) ctl->T[threadIdx.x >> 4][threadIdx.x & 15] = sT[threadIdx.x >> 4][threadIdx.x & 15];
 }
 
 // choice bytes [N][K/S] -> bits [N][ceil(K/S/8)], LSB first
