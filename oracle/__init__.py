@@ -23,8 +23,9 @@ paper/2605.08692) and what pins it (tests/test_oracle_*.py):
                     duplicates, signed zeros.
   group_error       section 2 mech. 2 (lower activation-weighted error).
                     Pinned by exact rational errors and brute-force choice.
-  rint_mul          exact fixed-point terms of the refine sums.  Pinned by
-                    exact rational rounding (half to even).
+  round_mul         exact fixed-point terms of the refine sums (floor in even
+                    columns, ceil in odd ones).  Pinned by exact rational
+                    floor / ceil.
   fit               section 2 mech. 4 (alternating assign / refine).  Pinned
                     by: the RTN special case (fixed uniform INT4 grid), the
                     plain 1-D k-means special case (equal importance, one
@@ -93,8 +94,8 @@ def lib():
         L.orc_assign.argtypes = [P, i32, P, i64, P]
         L.orc_group_error.restype = ctypes.c_double
         L.orc_group_error.argtypes = [P, P, P, P, i32]
-        L.orc_rint_mul.restype = i64
-        L.orc_rint_mul.argtypes = [ctypes.c_double, ctypes.c_float]
+        L.orc_round_mul.restype = i64
+        L.orc_round_mul.argtypes = [ctypes.c_double, ctypes.c_float, i32]
         L.orc_fixed_point_L.restype = i32
         L.orc_fixed_point_L.argtypes = [i64, ctypes.c_double, ctypes.c_double, ctypes.c_double]
         L.orc_fit.restype = i32
@@ -224,8 +225,9 @@ def group_error(u, Ik, Tc, q):
     return lib().orc_group_error(_p(u), _p(Ik), _p(Tc), _p(q), u.size)
 
 
-def rint_mul(a, u):
-    return lib().orc_rint_mul(float(a), float(u))
+def round_mul(a, u, up):
+    """floor(a*u) (up=False) or ceil(a*u) (up=True) of the exact product."""
+    return lib().orc_round_mul(float(a), float(u), 1 if up else 0)
 
 
 def fixed_point_L(M, I_max, S2_max, U_max):

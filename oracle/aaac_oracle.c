@@ -453,15 +453,18 @@ double orc_group_error(const float* u, const float* Ik, const float* Tc, const u
 /* R6: refine -- activation-weighted centroid of each Voronoi cell           */
 /*     (section 2, core mechanism 4, refine), in the normalised domain u:    */
 /*       T_c[q] = sum A u / sum A over the cell, A = I_k * s^2,              */
-/*     summed as exact integers: num += rint(A 2^L u), den += rint(A 2^L),   */
+/*     summed as exact integers: num += R_k(A 2^L u), den += R_k(A 2^L),     */
+/*     where R_k rounds the exact product down (floor) in even columns k and */
+/*     up (ceil) in odd columns -- no ties, no bias on average.              */
 /*     L = B - E(I_max) - E(S2_max) - max(0, E(U_max)),                       */
 /*     B = min(40, 61 - ceil(log2 M)), E(x) = frexp exponent (x < 2^E(x)).   */
 /*     T = fp32(fp64(num) / fp64(den)) when den > 0, else unchanged; then the */
-/*     codebook is re-sorted.  rint is round-half-even on the exact product. */
+/*     codebook is re-sorted.                                                 */
 /* ------------------------------------------------------------------------ */
 
-/* rint(a * u) of the exact product, ties to even; |result| < 2^62 assumed. */
-int64_t orc_rint_mul(double a, float u)
+/* floor(a * u) (up == 0) or ceil(a * u) (up != 0) of the exact product;
+ * |result| < 2^62 assumed. */
+int64_t orc_round_mul(double a, float u, int up)
 {
     if (a == 0.0 || u == 0.0f) return 0;
     int ea, eu;
@@ -473,22 +476,25 @@ int64_t orc_rint_mul(double a, float u)
     i128 p = (i128)ma * (i128)mu;
     int neg = p < 0;
     u128 m = neg ? (u128)(-p) : (u128)p;
+    /* |a u| = m 2^sh; q = floor(|a u|), inexact = fractional part != 0 */
     u128 q;
+    int inexact = 0;
     if (sh >= 0) {
         q = m << sh;
     } else {
         int rs = -sh;
         if (rs > 120) {
             q = 0;
+            inexact = m != 0;
         } else {
             q = m >> rs;
-            u128 rem = m - (q << rs);
-            u128 half = (u128)1 << (rs - 1);
-            if (rem > half || (rem == half && (q & 1u))) q++;
+            inexact = (m - (q << rs)) != 0;
         }
     }
+    /* floor(x) = q for x >= 0, -q - inexact for x < 0; ceil mirrors it */
     int64_t v = (int64_t)q;
-    return neg ? -v : v;
+    if (!neg) return (up && inexact) ? v + 1 : v;
+    return (!up && inexact) ? -v - 1 : -v;
 }
 
 static int clog2_i64(int64_t M)
@@ -586,8 +592,9 @@ static void assign_pass(const layer_t* Ly, const float* T, int L, uint8_t* choic
                     double s2 = (double)s * (double)s;
                     for (int i = 0; i < S; i++) {
                         double A2L = ldexp((double)Ik[i] * s2, L); /* exact */
-                        my[c][qc[i]][0] += orc_rint_mul(A2L, u[i]);
-                        my[c][qc[i]][1] += orc_rint_mul(A2L, 1.0f);
+                        int up = (int)((k0 + i) & 1); /* column parity */
+                        my[c][qc[i]][0] += orc_round_mul(A2L, u[i], up);
+                        my[c][qc[i]][1] += orc_round_mul(A2L, 1.0f, up);
                     }
                 }
             }

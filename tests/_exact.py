@@ -40,16 +40,6 @@ def f32_rn(x: Fraction) -> np.float32:
     return np.float32(sign * best[1])
 
 
-def rint_half_even(x: Fraction) -> int:
-    fl = x.numerator // x.denominator
-    rem = x - fl
-    if rem > Fraction(1, 2):
-        return fl + 1
-    if rem < Fraction(1, 2):
-        return fl
-    return fl if fl % 2 == 0 else fl + 1
-
-
 def argmin_nearest(T, u) -> int:
     """Lowest index j minimising |u - T_j| exactly."""
     uf = frac_f32(u)

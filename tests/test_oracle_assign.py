@@ -7,13 +7,14 @@ codebook with the lower activation-weighted error).  Readings R4 (nearest by
 exact distance, lowest index on a tie) and R5 (fp64 sequential error, T0 wins
 a tie) are pinned by brute-force exact rational enumeration.
 """
+import math
 from fractions import Fraction
 
 import numpy as np
 import pytest
 
 import oracle
-from tests._exact import argmin_nearest, frac_f32, rint_half_even
+from tests._exact import argmin_nearest, frac_f32
 
 
 def _check(T, us):
@@ -109,21 +110,27 @@ def test_choice_and_codes_bruteforce_on_tiny_layer():
     assert ch.sum() > 0 and ch.sum() < ch.size  # both books used
 
 
-def test_rint_mul_exact():
+def test_round_mul_exact():
+    """Refine terms: floor of the exact product in even columns, ceil in odd."""
     rng = np.random.default_rng(9)
     for _ in range(2000):
         I = np.float32(abs(rng.standard_normal()) * 10.0 ** rng.integers(-3, 4))
         s = np.float32(abs(rng.standard_normal()))
         a = float(np.ldexp(np.float64(I) * np.float64(s) * np.float64(s), int(rng.integers(0, 30))))
         u = np.float32(rng.standard_normal() * 4)
-        exact = rint_half_even(Fraction(a) * frac_f32(u))
-        assert oracle.rint_mul(a, u) == exact
-    # exact ties round to even
-    assert oracle.rint_mul(2.5, np.float32(1.0)) == 2
-    assert oracle.rint_mul(3.5, np.float32(1.0)) == 4
-    assert oracle.rint_mul(-2.5, np.float32(1.0)) == -2
-    assert oracle.rint_mul(1.25, np.float32(-2.0)) == -2
-    assert oracle.rint_mul(1.25, np.float32(6.0)) == 8  # 7.5 -> 8
+        x = Fraction(a) * frac_f32(u)
+        assert oracle.round_mul(a, u, False) == math.floor(x)
+        assert oracle.round_mul(a, u, True) == math.ceil(x)
+    # halves, exact integers, products below one, signs, zero
+    cases = [(2.5, 1.0), (-2.5, 1.0), (1.25, -2.0), (1.25, 6.0), (3.0, 2.0), (-3.0, 2.0),
+             (2.0 ** -40, 1.5), (2.0 ** -40, -1.5), (0.0, 3.0), (5.0, 0.0), (2.0 ** 50, 1.0)]
+    for a, u in cases:
+        x = Fraction(a) * Fraction(u)
+        assert oracle.round_mul(a, np.float32(u), False) == math.floor(x), (a, u)
+        assert oracle.round_mul(a, np.float32(u), True) == math.ceil(x), (a, u)
+    assert oracle.round_mul(2.5, np.float32(1.0), False) == 2
+    assert oracle.round_mul(-2.5, np.float32(1.0), False) == -3
+    assert oracle.round_mul(-2.5, np.float32(1.0), True) == -2
 
 
 @pytest.mark.parametrize("M", [1, 1000, 2 ** 20, 58720256, 141557760])
