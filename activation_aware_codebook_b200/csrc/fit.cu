@@ -12,28 +12,33 @@
 // One fit round is ONE launch of fit_pass<false>: a streaming pass over W whose
 // last block to finish (atomic ticket, no waiting) does the refine, sorts the
 // books, rebuilds the tables and records the error.  Per block: 2 warps; a warp
-// covers 256 columns of a row (16 bytes per lane) and walks the rows of its
-// chunk with a 3-deep cp.async ring, so several rows per warp are in flight.
-// The grid is one wave (10 blocks per SM).
+// covers 512 columns of a row, 16 per lane (32 bytes), and walks the rows of
+// its chunk with a 3-deep cp.async ring.  The grid is one wave (5 blocks per
+// SM, bounded by the refine bins' shared memory).
 //
 // Nearest entry in both books at once (exact):
 //   the midpoint thresholds of both books, merged and deduplicated (at most
 //   30), split the u line into merged cells; cell m fixes both books' nearest
-//   entries, mval[m] = (v0, v1).  bucket b = rint(u * la + 64) (one FFMA);
-//   mlut[b] = the number c of merged thresholds at or below every u of the
-//   bucket (kCrowded when two or more fall inside it: a binary search takes
-//   over);
-//   then m = c + (u >= mthr[c]) -- exact, because every threshold is the
-//   smallest fp32 above an exact midpoint.
+//   values mv0[m], mv1[m] and bin offsets moff[m].  bucket b = rint(u * la +
+//   64) (one FMA); mlut[b] = the number c of merged thresholds at or below
+//   every u of the bucket, then m = c + (u >= mthr[c]) -- exact, because every
+//   threshold is the smallest fp32 above an exact midpoint.  A bucket holding
+//   two or more thresholds maps to the sentinel cell kCrowded whose values are
+//   NaN: the NaN reaches the lane's error sums and the lane redoes its 16
+//   weights with a binary search.  Every lookup array is 4 bytes per entry and
+//   at most 33 entries long, so each warp-wide lookup is one shared-memory
+//   wavefront.
 // Choice: fp32 group sums when their gap exceeds the rounding bound, else the
 //   sequential fp64 rule (the group's leader lane recomputes it).
-// Refine sums: per weight rint(A 2^L u) and rint(A 2^L), A = I_k s^2, as the
-//   raw bit patterns of fp64 FMA/ADD results with magic constants; summed in
-//   shared-memory bins modulo 2^64, which keeps num exact modulo 2^51 and den
-//   modulo 2^52 -- exact because every bin's partial sum stays far below those
-//   bounds.  Each pair of lanes owns one set of bins and the two lanes update it
-//   in turn (read-modify-write, no atomics); halving the bins' shared memory
-//   lets 16 warps share an SM.  Integer sums make the result order-free.
+// Refine sums: per weight R_k(A 2^L u) and R_k(A 2^L), A = I_k s^2, R_k = floor
+//   for even columns k and ceil for odd ones.  Each lane owns 32 bins (book,
+//   entry) of (num, den) held as fp64 with biases 1.5 * 2^52 and 2^52, where
+//   every value is an integer and the spacing is 1: one FMA / ADD rounded
+//   toward -inf (+inf) adds floor (ceil) of the exact term, so every partial
+//   sum is exact whatever the order, as long as it stays below 2^51 -- the
+//   launch plan bounds the rows per lane to keep it there.  Bins are laid out
+//   [book*16 + entry][lane] in 16-byte cells: a warp's read-modify-write of
+//   its bins touches 32 distinct bank quads, with no conflicts.
 #include <mutex>
 
 #include "common.cuh"
@@ -45,9 +50,15 @@ constexpr int kNB = 128;                  // bucket LUT entries
 constexpr int kFitWarps = 2;
 constexpr int kFitThreads = kFitWarps * 32;
 constexpr int kStages = 3;                // rows per warp in flight
-constexpr int kFitBlocksPerSM = 10;
+constexpr int kFitBlocksPerSM = 5;
+constexpr int kLaneCols = 16;             // columns per lane
+constexpr int kWarpCols = 32 * kLaneCols; // columns per warp (one row segment)
+constexpr int kRingRowBytes = kWarpCols * 2;
+constexpr int kCellBytes = 32 * 16;       // one (book, entry) row of a warp's bins
+constexpr int kWarpBinBytes = 32 * kCellBytes;
 constexpr float kBucketMagic = 12582912.0f;           // 1.5 * 2^23
-constexpr double kDenMagic = 4503599627370496.0;      // 2^52
+constexpr double kNumBias = 6755399441055744.0;       // 1.5 * 2^52
+constexpr double kDenBias = 4503599627370496.0;       // 2^52
 #define kInf __int_as_float(0x7f800000)
 
 // Merged tables of both books (see the header comment).  Entries past the
@@ -55,15 +66,17 @@ constexpr double kDenMagic = 4503599627370496.0;      // 2^52
 constexpr int kMerged = 33;
 constexpr uint32_t kCrowded = 31;  // lut value of a crowded bucket (base counts are <= 30)
 struct Tables {
-  Book bk[2];
   float mthr[kMerged];     // merged thresholds, ascending, +inf padded
-  float2 mval[kMerged];    // (v0[count0], v1[count1]) of merged cell m
-  uint8_t mcell[kMerged];  // count0 | count1 << 4 of merged cell m
+  float mv0[kMerged];      // book-0 value of merged cell m (NaN at kCrowded)
+  float mv1[kMerged];      // book-1 value of merged cell m (NaN at kCrowded)
+  uint32_t moff[kMerged];  // bin offsets of cell m: book 0 low 16 bits, book 1 high
   uint8_t mlut[kNB];       // bucket -> merged base count, kCrowded = crowded bucket
+  Book bk[2];
   float la;
   int32_t nm;              // number of merged thresholds
   int32_t pad[2];
 };
+constexpr int kTablesBytes = (int)((sizeof(Tables) + 127) & ~(size_t)127);
 
 struct FitCtl {
   Tables tb;
@@ -86,7 +99,21 @@ struct FitCtl {
 
 size_t fit_ctl_bytes() { return align256(sizeof(FitCtl)); }
 
-static PassPlan fit_plan(int64_t N, int64_t K) { return plan_pass(N, K, 148 * kFitBlocksPerSM); }
+// One wave of 512-column strips x row chunks; rows per warp are capped so a
+// lane's refine partials (16 terms a row, each below 2^B) stay below 2^50.
+static PassPlan fit_plan(int64_t N, int64_t K) {
+  PassPlan pp = plan_pass(N, K, 148 * kFitBlocksPerSM, kWarpCols);
+  int c = 0;
+  while (((int64_t)1 << c) < N * K) c++;
+  const int Bmax = (61 - c) < 40 ? (61 - c) : 40;
+  const int64_t max_rows = ((int64_t)1 << (50 - Bmax)) / kLaneCols * kFitWarps;
+  if (pp.rows_per_chunk > max_rows) {
+    pp.rows_per_chunk = (int)max_rows;
+    pp.nrc = (int)((N + max_rows - 1) / max_rows);
+    pp.blocks = pp.ncb * pp.nrc;
+  }
+  return pp;
+}
 
 size_t fit_ws_bytes(int64_t N, int64_t K) {
   const PassPlan pp = fit_plan(N, K);
@@ -98,9 +125,8 @@ size_t pack_extra_bytes(int64_t N, int64_t K, int S) {
 }
 
 static size_t smem_bytes(bool pack) {
-  size_t b = (sizeof(Tables) + 15) & ~(size_t)15;
-  b += (size_t)kFitWarps * kStages * 32 * sizeof(uint4);
-  if (!pack) b += (size_t)kFitWarps * 32 * 16 * sizeof(ulonglong2);
+  size_t b = kTablesBytes + (size_t)kFitWarps * kStages * kRingRowBytes;
+  if (!pack) b += (size_t)kFitWarps * kWarpBinBytes;
   return b;
 }
 
@@ -137,14 +163,21 @@ __device__ void merge_thresholds(Tables& tb) {
 
 // Cell m of the merged tables (thread per cell).
 __device__ void merged_cell(Tables& tb, int m) {
+  if (m == (int)kCrowded) {
+    tb.mv0[m] = __int_as_float(0x7fc00000);
+    tb.mv1[m] = __int_as_float(0x7fc00000);
+    tb.moff[m] = 0;
+    return;
+  }
   int c0 = 0, c1 = 0;
   if (m >= 1 && m <= tb.nm) {
     const float lo = tb.mthr[m - 1];  // smallest u of the cell
     for (int i = 0; i + 1 < tb.bk[0].m; i++) c0 += (tb.bk[0].thr[i] <= lo) ? 1 : 0;
     for (int i = 0; i + 1 < tb.bk[1].m; i++) c1 += (tb.bk[1].thr[i] <= lo) ? 1 : 0;
   }
-  tb.mcell[m] = (uint8_t)(c0 | (c1 << 4));
-  tb.mval[m] = make_float2(tb.bk[0].val[c0], tb.bk[1].val[c1]);
+  tb.mv0[m] = tb.bk[0].val[c0];
+  tb.mv1[m] = tb.bk[1].val[c1];
+  tb.moff[m] = (uint32_t)(c0 * kCellBytes) | ((uint32_t)((16 + c1) * kCellBytes) << 16);
 }
 
 // All tables from the codebooks sT[2][16] (shared memory), by every thread of
@@ -433,16 +466,89 @@ __device__ void round_finalize(FitCtl* ctl, Tables& tb, const double* errp, int 
   }
 }
 
+// Chunk j (16 bytes) of a warp's 1 KB row segment sits at ring slot j ^ bit 3
+// of j: the lanes of a quarter warp then read eight distinct bank quads.
+__device__ __forceinline__ int ring_slot(int j) { return j ^ ((j >> 3) & 1); }
+
+// fp32 errors of one pair of weights against both books: dd0 += I (u - v0)^2,
+// dd1 += I (u - v1)^2, lane x of each pair the even column, lane y the odd one.
+__device__ __forceinline__ void pair_errors(unsigned long long u2, unsigned long long I2,
+                                            float v0x, float v0y, float v1x, float v1y,
+                                            unsigned long long& dd0, unsigned long long& dd1) {
+  const unsigned long long e0 = f2sub(u2, f2pack(v0x, v0y));
+  const unsigned long long e1 = f2sub(u2, f2pack(v1x, v1y));
+  dd0 = f2fma(I2, f2mul(e0, e0), dd0);
+  dd1 = f2fma(I2, f2mul(e1, e1), dd1);
+}
+
+// Merged cell of u by binary search over the merged thresholds (crowded buckets).
+__device__ __forceinline__ uint32_t merged_search(const Tables& tb, float u) {
+  uint32_t m = 0;
+  m += (tb.mthr[m + 15] <= u) ? 16 : 0;
+  m += (tb.mthr[m + 7] <= u) ? 8 : 0;
+  m += (tb.mthr[m + 3] <= u) ? 4 : 0;
+  m += (tb.mthr[m + 1] <= u) ? 2 : 0;
+  m += (tb.mthr[m] <= u) ? 1 : 0;
+  return m;
+}
+
+// The sequential fp64 errors of one group (section 2, core mechanism 2; the
+// oracle's rule): E_c = sum_j I_j (u_j - T_c[nearest])^2 in column order.
+__device__ void exact_group_errors(const uint16_t* __restrict__ wrow, const float* __restrict__ Ig,
+                                   int n, float rcp, const Tables& tb, double* E0, double* E1) {
+  double a = 0.0, b = 0.0;
+  for (int j = 0; j < n; j++) {
+    const float wf = __uint_as_float((uint32_t)wrow[j] << 16);
+    const float uj = __fmul_rn(wf, rcp);
+    const double Ij = (double)Ig[j];
+    const double ea = __dsub_rn((double)uj, (double)tb.bk[0].val[book_count(tb.bk[0], uj)]);
+    const double eb = __dsub_rn((double)uj, (double)tb.bk[1].val[book_count(tb.bk[1], uj)]);
+    a = __dadd_rn(a, __dmul_rn(Ij, __dmul_rn(ea, ea)));
+    b = __dadd_rn(b, __dmul_rn(Ij, __dmul_rn(eb, eb)));
+  }
+  *E0 = a;
+  *E1 = b;
+}
+
+// fp32 choice when the gap clears the rounding bound; else `exact` is set.
+__device__ __forceinline__ int fast_choice(float d0, float d1, float tau, bool* exact) {
+  const float sum = __fadd_rn(d0, d1);
+  const float gap = fabsf(__fsub_rn(d1, d0));
+  const bool decided = (sum >= 8.673617379884035e-19f) && (sum < 3.0e38f) &&
+                       (gap > __fmul_rn(tau, sum));
+  *exact = !decided;
+  return (decided && d1 < d0) ? 1 : 0;
+}
+
+struct GroupStats {
+  unsigned int near, exact, t1;
+  double err;
+};
+
+// Counters of one live group: near ties, exact decisions, T1 groups, s^2 D.
+__device__ __forceinline__ void count_group(GroupStats& gs, bool exact, double E0, double E1,
+                                            float d0, float d1, int ch, bool single, float s) {
+  if (exact) {
+    gs.exact++;
+    if (fabs(E1 - E0) < 1e-6 * fmax(E0, E1)) gs.near++;
+    gs.err += (double)(s * s) * (ch ? E1 : E0);  // s*s exact in fp32
+  } else {
+    if (!single && fabsf(d1 - d0) < 1e-6f * fmaxf(d0, d1)) gs.near++;
+    gs.err += (double)(s * s) * (double)(ch ? d1 : d0);
+  }
+  gs.t1 += ch;
+}
+
 template <int FMT, bool PACK>
 __global__ void __launch_bounds__(kFitThreads, kFitBlocksPerSM)
 fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
          const void* __restrict__ scales, int g, int S, uint32_t flags, FitCtl* ctl,
          double* __restrict__ errp, int ncb, int rows_per_chunk, float tau, PackOut po,
          RoundOut ro) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem[];
   Tables& tb = *reinterpret_cast<Tables*>(smem);
-  uint4* ring = reinterpret_cast<uint4*>(smem + ((sizeof(Tables) + 15) & ~(size_t)15));
-  ulonglong2* bins = reinterpret_cast<ulonglong2*>(ring + kFitWarps * kStages * 32);
+  unsigned char* ring = smem + kTablesBytes;
+  unsigned char* bins = ring + kFitWarps * kStages * kRingRowBytes;
   __shared__ double sred[kFitThreads];
   __shared__ int s_last;
 
@@ -450,44 +556,59 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     const uint32_t* src = reinterpret_cast<const uint32_t*>(&ctl->tb);
     uint32_t* dst = reinterpret_cast<uint32_t*>(&tb);
     for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
-    if (!PACK)
-      for (int i = threadIdx.x; i < kFitWarps * 32 * 16; i += blockDim.x)
-        bins[i] = make_ulonglong2(0ull, 0ull);
+    if (!PACK) {
+      double2* b = reinterpret_cast<double2*>(bins);
+      for (int i = threadIdx.x; i < kFitWarps * kWarpBinBytes / 16; i += blockDim.x)
+        b[i] = make_double2(kNumBias, kDenBias);
+    }
   }
   const double twoL = ctl->twoL;
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cb = blockIdx.x % ncb, rc = blockIdx.x / ncb;
-  const int col0 = cb * kSegCols + lane * 8;
+  const int seg = cb * kWarpCols;           // first column of the warp's row segment
+  const int col0 = seg + lane * kLaneCols;  // first of this lane's 16 columns
   const bool active = col0 < K;
   const int G = K / g, KS = K / S;
-  const int lanes_s = S >> 3, lanes_g = g >> 3;
-  const int leader_lane = lane & ~(lanes_s - 1);
-  const bool s_leader = lane == leader_lane;
+  const int lanes_s = S >> 4;               // lanes per choice group when S >= 16
+  const int leader_lane = S >= 16 ? (lane & ~(lanes_s - 1)) : lane;
   const bool single = (flags & AAAC_SINGLE_CODEBOOK) != 0;
   const float la = tb.la;
-  uint4* myring = ring + warp * kStages * 32 + lane;
-  ulonglong2* mybins = bins + warp * 32 * 16 + (lane >> 1);
+  unsigned char* wring = ring + warp * kStages * kRingRowBytes;
+  const int wr0 = ring_slot(lane) * 16, wr1 = ring_slot(32 + lane) * 16;
+  const int rd0 = ring_slot(2 * lane) * 16, rd1 = ring_slot(2 * lane + 1) * 16;
+  const bool cp0 = seg + lane * 8 < K, cp1 = seg + 256 + lane * 8 < K;
+  unsigned char* mybins = bins + warp * kWarpBinBytes + lane * 16;
 
-  float Ik[8];
-  if (active) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(I + col0));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(I + col0 + 4));
-    Ik[0] = a.x; Ik[1] = a.y; Ik[2] = a.z; Ik[3] = a.w;
-    Ik[4] = b.x; Ik[5] = b.y; Ik[6] = b.z; Ik[7] = b.w;
-  } else {
+  // importance of the lane's columns: fp32 pairs (choice) and fp64 (refine)
+  unsigned long long I2[8];
+  double Id[16];
+  {
+    float Iv[16];
 #pragma unroll
-    for (int i = 0; i < 8; i++) Ik[i] = 0.0f;
+    for (int q = 0; q < 4; q++) {
+      const float4 a = active ? __ldg(reinterpret_cast<const float4*>(I + col0) + q)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      Iv[4 * q] = a.x; Iv[4 * q + 1] = a.y; Iv[4 * q + 2] = a.z; Iv[4 * q + 3] = a.w;
+    }
+#pragma unroll
+    for (int p = 0; p < 8; p++) I2[p] = f2pack(Iv[2 * p], Iv[2 * p + 1]);
+#pragma unroll
+    for (int i = 0; i < 16; i++) Id[i] = (double)Iv[i];
   }
 
   const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
-  const uint16_t* wcol = W + col0;
-  // ring prologue
+  const uint16_t* wseg = W + seg;
+  // ring prologue: each lane copies chunks lane and 32 + lane of the segment
 #pragma unroll
   for (int k = 0; k < kStages; k++) {
     const int rr = r0 + warp + kFitWarps * k;
-    if (active && rr < r1) cp_async16(myring + k * 32, wcol + (int64_t)rr * K);
+    if (rr < r1) {
+      const uint16_t* src = wseg + (int64_t)rr * K + lane * 8;
+      if (cp0) cp_async16(wring + k * kRingRowBytes + wr0, src);
+      if (cp1) cp_async16(wring + k * kRingRowBytes + wr1, src + 256);
+    }
     cp_async_commit();
   }
   // scales prefetched two rows ahead
@@ -496,200 +617,224 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   if (active && r0 + warp + kFitWarps < r1)
     s_next2 = load_scale<FMT>(scales, (int64_t)(r0 + warp + kFitWarps) * G + col0 / g);
 
-  double err_acc = 0.0;
-  unsigned long long n_near = 0, n_exact = 0, n_t1 = 0;
+  GroupStats gs{0u, 0u, 0u, 0.0};
+  double err_w = 0.0;  // pack: weight-space error
   int slot = 0;
+  const unsigned long long la2 = f2pack(la, la);
+  const unsigned long long cc2 = f2pack(kBucketMagic + (float)(kNB / 2), kBucketMagic + (float)(kNB / 2));
   for (int r = r0 + warp; r < r1; r += kFitWarps) {  // warp-uniform trip count
     cp_async_wait<kStages - 1>();
-    const uint4 v = active ? myring[slot * 32] : make_uint4(0, 0, 0, 0);
+    __syncwarp();  // the row's chunks were copied by other lanes
+    const unsigned char* srow = wring + slot * kRingRowBytes;
+    const uint4 va = *reinterpret_cast<const uint4*>(srow + rd0);
+    const uint4 vb = *reinterpret_cast<const uint4*>(srow + rd1);
+    __syncwarp();  // every lane has read the slot before it is refilled
+    {
+      const int rr = r + kFitWarps * kStages;
+      if (rr < r1) {
+        const uint16_t* src = wseg + (int64_t)rr * K + lane * 8;
+        if (cp0) cp_async16(wring + slot * kRingRowBytes + wr0, src);
+        if (cp1) cp_async16(wring + slot * kRingRowBytes + wr1, src + 256);
+      }
+      cp_async_commit();
+    }
+    slot = (slot + 1 == kStages) ? 0 : slot + 1;
+
     const float s = s_next;
     s_next = s_next2;
     if (active && r + 2 * kFitWarps < r1)
       s_next2 = load_scale<FMT>(scales, (int64_t)(r + 2 * kFitWarps) * G + col0 / g);
     float rcp;
-    const bool live = active && scale_live(s, &rcp);
-    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-    float u[8];
-    uint32_t mm[8];  // merged cell of each weight
-    unsigned long long dd = 0ull;  // (D0, D1) partial sums
-    bool crowded = false;
-    const unsigned long long rcp2 = f2pack(rcp, rcp);
+    const bool live = active && scale_live(s, &rcp);  // dead: rcp = 0, u = +-0
+    const uint32_t wv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+    const unsigned long long rr2 = f2pack(rcp, rcp);
+    unsigned long long u2[8];
 #pragma unroll
-    for (int h = 0; h < 4; h++) {
-      const float2 up = f2unpack(f2mul(f2pack(bf16_lo(wv[h]), bf16_hi(wv[h])), rcp2));
-      u[2 * h] = live ? up.x : 0.0f;
-      u[2 * h + 1] = live ? up.y : 0.0f;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const uint32_t c = tb.mlut[__float_as_uint(bucket_t(u[i], la)) & (kNB - 1)];
-      crowded |= (c == kCrowded);
-      const uint32_t m = c + (u[i] >= tb.mthr[c] ? 1u : 0u);
-      mm[i] = m;
-      const unsigned long long vv = *reinterpret_cast<const unsigned long long*>(&tb.mval[m]);
-      const unsigned long long e = f2sub(f2pack(u[i], u[i]), vv);
-      dd = f2fma(f2pack(Ik[i], Ik[i]), f2mul(e, e), dd);
-    }
-    if (crowded) {  // rare: a bucket with two or more thresholds; redo the lane exactly
-      dd = 0ull;
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        int m = 0;
-        m += (tb.mthr[m + 15] <= u[i]) ? 16 : 0;
-        m += (tb.mthr[m + 7] <= u[i]) ? 8 : 0;
-        m += (tb.mthr[m + 3] <= u[i]) ? 4 : 0;
-        m += (tb.mthr[m + 1] <= u[i]) ? 2 : 0;
-        m += (tb.mthr[m] <= u[i]) ? 1 : 0;
-        mm[i] = (uint32_t)m;
-        const unsigned long long vv = *reinterpret_cast<const unsigned long long*>(&tb.mval[m]);
-        const unsigned long long e = f2sub(f2pack(u[i], u[i]), vv);
-        dd = f2fma(f2pack(Ik[i], Ik[i]), f2mul(e, e), dd);
-      }
-    }
-    float d0, d1;
-    {
-      const float2 dv = f2unpack(dd);
-      d0 = dv.x;
-      d1 = dv.y;
-    }
-    for (int o = 1; o < lanes_s; o <<= 1) {
-      d0 = __fadd_rn(d0, __shfl_xor_sync(0xffffffffu, d0, o));
-      d1 = __fadd_rn(d1, __shfl_xor_sync(0xffffffffu, d1, o));
-    }
-    // The choice (section 2, core mechanism 2): decided in fp32 when the gap
-    // exceeds the fp32 error bound, else by the sequential fp64 rule.
-    int choice = 0;
-    bool exact = false;
-    if (live && !single) {
-      const float sum = __fadd_rn(d0, d1);
-      const float gap = fabsf(__fsub_rn(d1, d0));
-      const bool decided = (sum >= 8.673617379884035e-19f) && (sum < 3.0e38f) &&
-                           (gap > __fmul_rn(tau, sum));
-      if (decided) choice = (d1 < d0) ? 1 : 0;
-      else exact = true;
-    }
-    double E0 = 0.0, E1 = 0.0;
-    if (exact && s_leader) {
-      const int kbase = col0 - (lane - leader_lane) * 8;  // first column of the group
-      const uint16_t* wrow = W + (int64_t)r * K + kbase;
-      for (int j = 0; j < S; j++) {
-        const float wf = __uint_as_float((uint32_t)wrow[j] << 16);
-        const float uj = __fmul_rn(wf, rcp);
-        const double Ij = (double)I[kbase + j];
-        const double ea = __dsub_rn((double)uj, (double)tb.bk[0].val[book_count(tb.bk[0], uj)]);
-        const double eb = __dsub_rn((double)uj, (double)tb.bk[1].val[book_count(tb.bk[1], uj)]);
-        E0 = __dadd_rn(E0, __dmul_rn(Ij, __dmul_rn(ea, ea)));
-        E1 = __dadd_rn(E1, __dmul_rn(Ij, __dmul_rn(eb, eb)));
-      }
-      choice = (E1 < E0) ? 1 : 0;
-    }
-    choice = __shfl_sync(0xffffffffu, choice, leader_lane);
+    for (int p = 0; p < 8; p++) u2[p] = f2mul(f2pack(bf16_lo(wv[p]), bf16_hi(wv[p])), rr2);
 
-    if (s_leader && live) {
-      if (exact) {
-        n_exact++;
-        if (fabs(E1 - E0) < 1e-6 * fmax(E0, E1)) n_near++;
-        if (!PACK) err_acc += (double)(s * s) * (choice ? E1 : E0);  // s*s exact in fp32
-      } else {
-        if (!single && fabsf(d1 - d0) < 1e-6f * fmaxf(d0, d1)) n_near++;
-        if (!PACK) err_acc += (double)(s * s) * (double)(choice ? d1 : d0);
-      }
-      n_t1 += choice;
+    // nearest entries of both books, and the fp32 group errors
+    uint32_t moffs[16];
+    unsigned long long dd0[2] = {0ull, 0ull}, dd1[2] = {0ull, 0ull};
+#pragma unroll
+    for (int p = 0; p < 8; p++) {
+      const float2 uf = f2unpack(u2[p]);
+      const float2 bf = f2unpack(f2fma(u2[p], la2, cc2));
+      const uint32_t cx = tb.mlut[__float_as_uint(bf.x) & (kNB - 1)];
+      const uint32_t cy = tb.mlut[__float_as_uint(bf.y) & (kNB - 1)];
+      const uint32_t mx = cx + (uf.x >= tb.mthr[cx] ? 1u : 0u);
+      const uint32_t my = cy + (uf.y >= tb.mthr[cy] ? 1u : 0u);
+      moffs[2 * p] = tb.moff[mx];
+      moffs[2 * p + 1] = tb.moff[my];
+      pair_errors(u2[p], I2[p], tb.mv0[mx], tb.mv0[my], tb.mv1[mx], tb.mv1[my], dd0[p >> 2],
+                  dd1[p >> 2]);
     }
+    float D0[2], D1[2];
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      const float2 a = f2unpack(dd0[h]), b = f2unpack(dd1[h]);
+      D0[h] = __fadd_rn(a.x, a.y);
+      D1[h] = __fadd_rn(b.x, b.y);
+    }
+    if (active && isnan(__fadd_rn(D0[0], D0[1]))) {
+      // a crowded bucket (rare): redo the lane's weights with the binary search
+      dd0[0] = dd0[1] = dd1[0] = dd1[1] = 0ull;
+#pragma unroll
+      for (int p = 0; p < 8; p++) {
+        const float2 uf = f2unpack(u2[p]);
+        const uint32_t mx = merged_search(tb, uf.x), my = merged_search(tb, uf.y);
+        moffs[2 * p] = tb.moff[mx];
+        moffs[2 * p + 1] = tb.moff[my];
+        pair_errors(u2[p], I2[p], tb.mv0[mx], tb.mv0[my], tb.mv1[mx], tb.mv1[my], dd0[p >> 2],
+                    dd1[p >> 2]);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const float2 a = f2unpack(dd0[h]), b = f2unpack(dd1[h]);
+        D0[h] = __fadd_rn(a.x, a.y);
+        D1[h] = __fadd_rn(b.x, b.y);
+      }
+    }
+
+    // The choice (section 2, core mechanism 2): decided in fp32 when the gap
+    // exceeds the fp32 error bound, else by the sequential fp64 rule.  S = 8:
+    // the lane holds two groups; S >= 16: a group spans S/16 lanes.
+    int ch[2] = {0, 0};
+    bool ex[2] = {false, false};
+    float g0[2] = {D0[0], D0[1]}, g1[2] = {D1[0], D1[1]};
+    if (S == 8) {
+#pragma unroll
+      for (int h = 0; h < 2; h++)
+        if (live && !single) ch[h] = fast_choice(D0[h], D1[h], tau, &ex[h]);
+    } else {
+      float d0 = __fadd_rn(D0[0], D0[1]), d1 = __fadd_rn(D1[0], D1[1]);
+      for (int o = 1; o < lanes_s; o <<= 1) {
+        d0 = __fadd_rn(d0, __shfl_xor_sync(0xffffffffu, d0, o));
+        d1 = __fadd_rn(d1, __shfl_xor_sync(0xffffffffu, d1, o));
+      }
+      g0[0] = g0[1] = d0;
+      g1[0] = g1[1] = d1;
+      if (live && !single) ch[0] = fast_choice(d0, d1, tau, &ex[0]);
+      ch[1] = ch[0];
+      ex[1] = ex[0];
+    }
+    double E0[2] = {0.0, 0.0}, E1[2] = {0.0, 0.0};
+    if (__any_sync(0xffffffffu, ex[0] || ex[1])) {
+      const uint16_t* wrow = W + (int64_t)r * K + col0;
+      if (S == 8) {
+#pragma unroll
+        for (int h = 0; h < 2; h++)
+          if (ex[h]) {
+            exact_group_errors(wrow + 8 * h, I + col0 + 8 * h, 8, rcp, tb, &E0[h], &E1[h]);
+            ch[h] = (E1[h] < E0[h]) ? 1 : 0;
+          }
+      } else {
+        if (ex[0] && lane == leader_lane) {
+          exact_group_errors(wrow, I + col0, S, rcp, tb, &E0[0], &E1[0]);
+          ch[0] = (E1[0] < E0[0]) ? 1 : 0;
+        }
+        ch[0] = __shfl_sync(0xffffffffu, ch[0], leader_lane);
+        ch[1] = ch[0];
+      }
+    }
+    if (live) {
+      if (S == 8) {
+        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], single, s);
+        count_group(gs, ex[1], E0[1], E1[1], g0[1], g1[1], ch[1], single, s);
+      } else if (lane == leader_lane) {
+        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], single, s);
+      }
+    }
+    const uint32_t sel0 = ch[0] ? 0x4432u : 0x4410u;  // book-1 or book-0 half of moff
+    const uint32_t sel1 = ch[1] ? 0x4432u : 0x4410u;
 
     if (!PACK) {
-      const double s2L = (double)s * (double)s * twoL;  // exact: s^2 has 16 bits
-      const int shift = choice ? 4 : 0;
-      ulonglong2* cb_bins = mybins + choice * 16 * 16;
-      unsigned long long nums[8], dens[8];
-      uint32_t qs[8];
+      if (live) {
+        const double s2L = (double)s * (double)s * twoL;  // exact: s^2 has at most 16 bits
 #pragma unroll
-      for (int i = 0; i < 8; i++) {
-        qs[i] = ((uint32_t)tb.mcell[mm[i]] >> shift) & 15u;
-        const double A = __dmul_rn((double)Ik[i], s2L);  // exact: 24 + 16 bits
-        nums[i] = (unsigned long long)__double_as_longlong(__fma_rn(A, (double)u[i], kMagic));
-        dens[i] = (unsigned long long)__double_as_longlong(__dadd_rn(A, kDenMagic));
-      }
-      // the two lanes of a pair share bins: update them one lane at a time
-#pragma unroll
-      for (int half = 0; half < 2; half++) {
-        if (live && (lane & 1) == half) {
-#pragma unroll
-          for (int i = 0; i < 8; i++) {
-            ulonglong2 x = cb_bins[qs[i] * 16];
-            x.x += nums[i];
-            x.y += dens[i];
-            cb_bins[qs[i] * 16] = x;
+        for (int i = 0; i < 16; i++) {
+          const uint32_t off = __byte_perm(moffs[i], 0u, i < 8 ? sel0 : sel1);
+          double2* bp = reinterpret_cast<double2*>(mybins + off);
+          const float2 uf = f2unpack(u2[i >> 1]);
+          const double ud = (double)((i & 1) ? uf.y : uf.x);
+          const double A = __dmul_rn(Id[i], s2L);  // exact: 24 + 16 bits
+          double2 b = *bp;
+          if (i & 1) {  // odd column: ceil
+            b.x = __fma_ru(A, ud, b.x);
+            b.y = __dadd_ru(b.y, A);
+          } else {      // even column: floor
+            b.x = __fma_rd(A, ud, b.x);
+            b.y = __dadd_rd(b.y, A);
           }
+          *bp = b;
         }
-        __syncwarp();
       }
     } else if (active) {
-      const Book& bc = tb.bk[choice];
-      const int shift = choice ? 4 : 0;
-      uint32_t packed = 0;
+      unsigned long long packed = 0ull;
 #pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const uint32_t q = ((uint32_t)tb.mcell[mm[i]] >> shift) & 15u;
-        packed |= (uint32_t)bc.idx[q] << (4 * i);
+      for (int i = 0; i < 16; i++) {
+        const int h = i >> 3;
+        const uint32_t off = __byte_perm(moffs[i], 0u, h ? sel1 : sel0);
+        const uint32_t q = (off / kCellBytes) & 15u;
+        const Book& bc = tb.bk[ch[h]];
+        packed |= (unsigned long long)bc.idx[q] << (4 * i);
         const float wf = (i & 1) ? bf16_hi(wv[i >> 1]) : bf16_lo(wv[i >> 1]);
         const double wh = (double)s * (double)bc.val[q];
         const double d = __dsub_rn((double)wf, wh);
-        err_acc = __fma_rn((double)Ik[i], __dmul_rn(d, d), err_acc);
+        err_w = __fma_rn(Id[i], __dmul_rn(d, d), err_w);
       }
-      *reinterpret_cast<uint32_t*>(po.codes + ((int64_t)r * K + col0) / 2) = packed;
-      if ((lane & (lanes_g - 1)) == 0) {
+      *reinterpret_cast<unsigned long long*>(po.codes + ((int64_t)r * K + col0) / 2) = packed;
+      if ((lane & ((g >> 4) - 1)) == 0) {
         const int64_t gi = (int64_t)r * G + col0 / g;
-        const uint32_t tag = (S == g) ? (uint32_t)choice : 0u;
+        const uint32_t tag = (S == g) ? (uint32_t)ch[0] : 0u;
         if (FMT == kInt4) {
-          const uint32_t h = reinterpret_cast<const unsigned short*>(scales)[gi];
+          const uint32_t hs = reinterpret_cast<const unsigned short*>(scales)[gi];
           reinterpret_cast<unsigned short*>(po.tagged)[gi] =
-              (unsigned short)((h & 0x7fffu) | (tag << 15));
+              (unsigned short)((hs & 0x7fffu) | (tag << 15));
         } else {
-          const uint32_t b = reinterpret_cast<const unsigned char*>(scales)[gi];
-          reinterpret_cast<unsigned char*>(po.tagged)[gi] = (unsigned char)((b & 0x7fu) | (tag << 7));
+          const uint32_t bs = reinterpret_cast<const unsigned char*>(scales)[gi];
+          reinterpret_cast<unsigned char*>(po.tagged)[gi] = (unsigned char)((bs & 0x7fu) | (tag << 7));
         }
       }
-      if (S != g && s_leader) po.choice_bytes[(int64_t)r * KS + col0 / S] = (uint8_t)choice;
+      if (S != g) {
+        if (S == 8) {
+          po.choice_bytes[(int64_t)r * KS + col0 / 8] = (uint8_t)ch[0];
+          po.choice_bytes[(int64_t)r * KS + col0 / 8 + 1] = (uint8_t)ch[1];
+        } else if (lane == leader_lane) {
+          po.choice_bytes[(int64_t)r * KS + col0 / S] = (uint8_t)ch[0];
+        }
+      }
     }
-    // refill this slot with the row kStages steps ahead
-    {
-      const int rr = r + kFitWarps * kStages;
-      if (active && rr < r1) cp_async16(myring + slot * 32, wcol + (int64_t)rr * K);
-      cp_async_commit();
-    }
-    slot = (slot + 1 == kStages) ? 0 : slot + 1;
   }
   cp_async_wait<0>();
 
   for (int o = 16; o > 0; o >>= 1) {
-    n_near += __shfl_xor_sync(0xffffffffu, n_near, o);
-    n_exact += __shfl_xor_sync(0xffffffffu, n_exact, o);
-    n_t1 += __shfl_xor_sync(0xffffffffu, n_t1, o);
+    gs.near += __shfl_xor_sync(0xffffffffu, gs.near, o);
+    gs.exact += __shfl_xor_sync(0xffffffffu, gs.exact, o);
+    gs.t1 += __shfl_xor_sync(0xffffffffu, gs.t1, o);
   }
   if (lane == 0) {
-    if (n_near) atomicAdd(&ctl->near_ties, n_near);
-    if (n_exact) atomicAdd(&ctl->exact_groups, n_exact);
-    if (n_t1) atomicAdd(&ctl->groups_t1, n_t1);
+    if (gs.near) atomicAdd(&ctl->near_ties, (unsigned long long)gs.near);
+    if (gs.exact) atomicAdd(&ctl->exact_groups, (unsigned long long)gs.exact);
+    if (gs.t1) atomicAdd(&ctl->groups_t1, (unsigned long long)gs.t1);
   }
-  sred[threadIdx.x] = err_acc;
+  sred[threadIdx.x] = PACK ? err_w : gs.err;
   __syncthreads();
   if (threadIdx.x == 0) {
     double t = 0.0;
     for (int i = 0; i < kFitThreads; i++) t = __dadd_rn(t, sred[i]);
     errp[blockIdx.x] = t;
   }
-  if (!PACK && threadIdx.x < 64) {
-    // lane-private raw sums -> exact integers: num is exact modulo 2^51, den
-    // modulo 2^52, and every lane's partial is far inside those ranges.
-    const int cell = threadIdx.x >> 1, which = threadIdx.x & 1;
+  if (!PACK) {
+    // lane bins -> exact integer partials (bias removed exactly), one
+    // (book, entry, num | den) per thread, summed over the block's lanes
+    const int bc = threadIdx.x >> 1, which = threadIdx.x & 1;
+    const double bias = which ? kDenBias : kNumBias;
     long long sum = 0;
     for (int w = 0; w < kFitWarps; w++) {
-      const ulonglong2* p = bins + (w * 32 + cell) * 16;
-      for (int l = 0; l < 16; l++) {
-        const unsigned long long raw = which ? p[l].y : p[l].x;
-        sum += which ? (long long)(raw & ((1ull << 52) - 1))
-                     : ((long long)(raw << 13) >> 13);
+      const unsigned char* p = bins + w * kWarpBinBytes + bc * kCellBytes + which * 8;
+      for (int j = 0; j < 32; j++) {
+        const int l = (j + bc) & 31;  // staggered: fewer bank conflicts
+        sum += __double2ll_rn(__dsub_rn(*reinterpret_cast<const double*>(p + l * 16), bias));
       }
     }
     if (sum) atomicAdd(reinterpret_cast<unsigned long long*>(&ctl->bins[0][0][0]) + threadIdx.x,

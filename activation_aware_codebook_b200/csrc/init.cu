@@ -36,9 +36,9 @@ struct InitCtl {
 
 size_t init_ctl_bytes() { return align256(sizeof(InitCtl)); }
 
-PassPlan plan_pass(int64_t N, int64_t K, int target) {
+PassPlan plan_pass(int64_t N, int64_t K, int target, int seg_cols) {
   PassPlan p;
-  p.ncb = (int)((K + kSegCols - 1) / kSegCols);
+  p.ncb = (int)((K + seg_cols - 1) / seg_cols);
   int64_t nrc = target / p.ncb;  // at most `target` blocks: one full wave
   if (nrc > N) nrc = N;
   if (nrc < 1) nrc = 1;

@@ -14,7 +14,7 @@ namespace aaac {
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct ImportancePlan {
-  int ncb;        // 256-column strips
+  int ncb;        // column strips (seg_cols wide)
   int rb;         // row blocks
   int64_t rows_per_rb;
   size_t partial_bytes;  // double [rb][K]
@@ -24,12 +24,12 @@ struct ImportancePlan {
 ImportancePlan plan_importance(int64_t T, int64_t K);
 
 struct PassPlan {
-  int ncb;        // 256-column strips
+  int ncb;        // column strips (seg_cols wide)
   int nrc;        // row chunks
   int rows_per_chunk;
   int blocks;     // ncb * nrc
 };
-PassPlan plan_pass(int64_t N, int64_t K, int target_blocks = 148 * 4);
+PassPlan plan_pass(int64_t N, int64_t K, int target_blocks = 148 * 4, int seg_cols = 256);
 
 size_t fit_ctl_bytes();
 size_t init_ctl_bytes();
