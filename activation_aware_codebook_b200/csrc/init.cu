@@ -67,6 +67,8 @@ __device__ __forceinline__ float group_scale(uint32_t mx, uint32_t* stored) {
   }
 }
 
+constexpr int kRadixRows = 4;  // rows per lane loaded ahead in a radix pass
+
 struct RankInit {
   int64_t rank[32];
 };
@@ -88,26 +90,98 @@ __global__ void init_setup(InitCtl* c, RankInit ri, int nranks, int n) {
   }
 }
 
-// Slot of a prefix: the bucket's two entries are compared (hash table), or a
-// binary search over the sorted prefixes when no hash was found.
-__device__ __forceinline__ int prefix_slot(uint32_t pre, const uint4* tab, uint32_t mult,
-                                           const uint32_t* sp, int nslots) {
-  if (mult) {
-    const uint4 e = tab[(pre * mult) >> 24];
-    return e.x == pre ? (int)e.y : (e.z == pre ? (int)e.w : -1);
+struct RadixArgs {
+  const uint16_t* W;
+  int N, K, g;
+  void* scales;
+  int pass, ncb, rows_per_chunk;
+};
+
+// The rows of one warp.  MODE 0: the first pass (scales, top digit); 1: later
+// passes with the prefix hash; 2: later passes with the binary search.
+template <int FMT, int MODE>
+__device__ __forceinline__ void radix_rows(const RadixArgs& a, uint32_t (*sh)[256], const uint4* tab,
+                                           uint32_t mult, const uint32_t* sp, int nslots) {
+  const int shift = 24 - 8 * a.pass;
+  const int K = a.K, g = a.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cb = blockIdx.x % a.ncb, rc = blockIdx.x / a.ncb;
+  const int col0 = cb * kSegCols + lane * 8;
+  const bool active = col0 < K;
+  const int lanes_g = g >> 3;
+  const int G = K / g;
+  const int r0 = rc * a.rows_per_chunk, r1 = min(a.N, r0 + a.rows_per_chunk);
+  if (MODE != 0 && !active) return;  // no warp collectives in later passes
+  // kRadixRows rows per lane are loaded before any is processed (loads in flight)
+  for (int rb = r0 + warp; rb < r1; rb += kWarps * kRadixRows) {  // warp-uniform
+    uint4 vr[kRadixRows];
+    float sr[kRadixRows];
+#pragma unroll
+    for (int k = 0; k < kRadixRows; k++) {
+      const int r = rb + k * kWarps;
+      const bool ok = active && r < r1;
+      vr[k] = ok ? __ldg(reinterpret_cast<const uint4*>(a.W + (int64_t)r * K + col0))
+                 : make_uint4(0u, 0u, 0u, 0u);
+      sr[k] = (MODE != 0 && ok) ? load_scale<FMT>(a.scales, (int64_t)r * G + col0 / g) : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < kRadixRows; k++) {
+      const int r = rb + k * kWarps;
+      if (r >= r1) break;  // warp-uniform
+      const uint32_t w[4] = {vr[k].x, vr[k].y, vr[k].z, vr[k].w};
+      float s = sr[k];
+      if (MODE == 0) {
+        uint32_t mx = 0;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+          mx = max(mx, w[i] & 0x7fffu);
+          mx = max(mx, (w[i] >> 16) & 0x7fffu);
+        }
+        for (int o = 1; o < lanes_g; o <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        uint32_t stored;
+        s = group_scale<FMT>(mx, &stored);
+        if (active && (lane & (lanes_g - 1)) == 0) {
+          const int64_t gi = (int64_t)r * G + col0 / g;
+          if (FMT == kInt4) reinterpret_cast<unsigned short*>(a.scales)[gi] = (unsigned short)stored;
+          else reinterpret_cast<unsigned char*>(a.scales)[gi] = (unsigned char)stored;
+        }
+      }
+      float rcp;
+      const bool live = scale_live(s, &rcp);
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const float wf = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+        const float u = live ? __fmul_rn(wf, rcp) : 0.0f;
+        const uint32_t key = order_key(u);
+        if (MODE == 0) {
+          // lanes holding the same top digit add once (fewer same-address atomics)
+          const uint32_t d = active ? (key >> 24) : 0x100u;
+          const uint32_t peers = __match_any_sync(0xffffffffu, d);
+          if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&sh[warp][d], (uint32_t)__popc(peers));
+        } else {
+          const uint32_t pre = key >> (shift + 8);
+          int slot;
+          if (MODE == 1) {
+            const uint4 e = tab[(pre * mult) >> 24];
+            slot = e.x == pre ? (int)e.y : (e.z == pre ? (int)e.w : -1);
+          } else {
+            int lo = 0, hi = nslots;  // sorted distinct prefixes
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if (sp[mid] < pre) lo = mid + 1; else hi = mid;
+            }
+            slot = (lo < nslots && sp[lo] == pre) ? lo : -1;
+          }
+          if (slot >= 0) atomicAdd(&sh[slot][(key >> shift) & 255u], 1u);
+        }
+      }
+    }
   }
-  int lo = 0, hi = nslots;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (sp[mid] < pre) lo = mid + 1; else hi = mid;
-  }
-  return (lo < nslots && sp[lo] == pre) ? lo : -1;
 }
 
 template <int FMT, bool FIRST>
 __global__ void __launch_bounds__(kThreads)
-radix_pass(const uint16_t* __restrict__ W, int N, int K, int g, void* __restrict__ scales,
-           InitCtl* c, int pass, int ncb, int rows_per_chunk) {
+radix_pass(RadixArgs a, InitCtl* c) {
   __shared__ uint32_t sh[32][256];  // first pass: per-warp counts; else per-slot counts
   __shared__ uint4 tab[256];
   __shared__ uint32_t sp[32];
@@ -124,56 +198,9 @@ radix_pass(const uint16_t* __restrict__ W, int N, int K, int g, void* __restrict
   }
   __syncthreads();
   const int nslots = FIRST ? 1 : ns;
-  const uint32_t mult = FIRST ? 0u : smult;
-  const int shift = 24 - 8 * pass;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cb = blockIdx.x % ncb, rc = blockIdx.x / ncb;
-  const int col0 = cb * kSegCols + lane * 8;
-  const bool active = col0 < K;
-  const int lanes_g = g >> 3;
-  const int G = K / g;
-  const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
-  for (int r = r0 + warp; r < r1; r += kWarps) {  // warp-uniform: every lane takes part
-    const uint4 v = active ? __ldg(reinterpret_cast<const uint4*>(W + (int64_t)r * K + col0))
-                           : make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    const int64_t gi = (int64_t)r * G + col0 / g;
-    float s;
-    if (FIRST) {
-      uint32_t mx = 0;
-#pragma unroll
-      for (int i = 0; i < 4; i++) {
-        mx = max(mx, w[i] & 0x7fffu);
-        mx = max(mx, (w[i] >> 16) & 0x7fffu);
-      }
-      for (int o = 1; o < lanes_g; o <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      uint32_t stored;
-      s = group_scale<FMT>(mx, &stored);
-      if (active && (lane & (lanes_g - 1)) == 0) {
-        if (FMT == kInt4) reinterpret_cast<unsigned short*>(scales)[gi] = (unsigned short)stored;
-        else reinterpret_cast<unsigned char*>(scales)[gi] = (unsigned char)stored;
-      }
-    } else {
-      s = active ? load_scale<FMT>(scales, gi) : 0.0f;
-    }
-    float rcp;
-    const bool live = scale_live(s, &rcp);
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const float wf = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
-      const float u = live ? __fmul_rn(wf, rcp) : 0.0f;
-      const uint32_t key = order_key(u);
-      if (FIRST) {
-        // lanes holding the same top digit add once (fewer same-address atomics)
-        const uint32_t d = active ? (key >> 24) : 0x100u;
-        const uint32_t peers = __match_any_sync(0xffffffffu, d);
-        if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&sh[warp][d], (uint32_t)__popc(peers));
-      } else {
-        const int slot = prefix_slot(key >> (shift + 8), tab, mult, sp, nslots);
-        if (active && slot >= 0) atomicAdd(&sh[slot][(key >> shift) & 255u], 1u);
-      }
-    }
-  }
+  if (FIRST) radix_rows<FMT, 0>(a, sh, tab, 0u, sp, 1);
+  else if (smult) radix_rows<FMT, 1>(a, sh, tab, smult, sp, nslots);
+  else radix_rows<FMT, 2>(a, sh, tab, 0u, sp, nslots);
   __syncthreads();
   if (FIRST) {
     for (int d = threadIdx.x; d < 256; d += blockDim.x) {
@@ -189,87 +216,151 @@ radix_pass(const uint16_t* __restrict__ W, int N, int K, int g, void* __restrict
   }
 }
 
-// 256 threads: the histograms are read into shared memory once, then one
-// thread per target rank walks its prefix's 256 counts there.
+// 256 threads.  The histograms are read into shared memory; warp w resolves
+// target ranks w, w + 8, ...: a warp scan over its prefix's 256 counts finds
+// the digit.  Warp 0 then sorts and deduplicates the new prefixes and builds
+// the next pass's prefix hash table (bucket (p * mult) >> 24 of 256, two
+// entries each; multipliers are tried until no bucket receives three).
 __global__ void __launch_bounds__(256) radix_select(InitCtl* c, int pass, float* T) {
   __shared__ uint32_t hist[32][256];
   __shared__ uint32_t sp[32];
   __shared__ uint32_t newp[32];
+  __shared__ uint32_t sorted[32];
+  __shared__ uint4 stab[256];
   __shared__ int ns;
-  __shared__ int bcnt[256];
   __shared__ uint32_t smult;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const unsigned full = 0xffffffffu;
   const int nr = c->nranks;
   if (tid == 0) ns = c->nslots;
   if (tid < 32) sp[tid] = c->slot_prefix[tid];
   __syncthreads();
   const int nslots = ns;
-  for (int j = tid; j < nslots * 256; j += blockDim.x) {
-    (&hist[0][0])[j] = (&c->hist[0][0])[j];
-    (&c->hist[0][0])[j] = 0u;  // ready for the next pass
+  const int nh = nslots * 256;
+  uint32_t* gh = &c->hist[0][0];
+  for (int j0 = 0; j0 < nh; j0 += 256 * 8) {  // 8 loads in flight per thread
+    uint32_t v[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      const int j = j0 + k * 256 + tid;
+      v[k] = j < nh ? __ldcg(gh + j) : 0u;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      const int j = j0 + k * 256 + tid;
+      if (j < nh) (&hist[0][0])[j] = v[k];
+    }
   }
+  for (int j = tid; j < nh; j += 256) gh[j] = 0u;  // ready for the next pass (own entries)
   __syncthreads();
-  if (tid < nr) {
+
+  for (int t = warp; t < nr; t += 8) {  // warp-uniform
     int slot = 0;
-    if (pass > 0)
-      for (int s = 0; s < nslots; s++)
-        if (sp[s] == c->prefix[tid]) slot = s;
-    int64_t want = c->resid[tid], cum = 0;
-    int d = 0;
-    for (; d < 255; d++) {
-      const int64_t h = hist[slot][d];
-      if (cum + h > want) break;
-      cum += h;
+    const uint32_t pre = c->prefix[t];
+    if (pass > 0) {
+      const unsigned m = __ballot_sync(full, lane < nslots && sp[lane] == pre);
+      slot = m ? __ffs(m) - 1 : 0;
     }
-    c->resid[tid] = want - cum;
-    c->prefix[tid] = (pass == 0) ? (uint32_t)d : ((c->prefix[tid] << 8) | (uint32_t)d);
-    newp[tid] = c->prefix[tid];
+    const int64_t want = c->resid[t];
+    uint32_t h[8];
+    int64_t loc = 0;
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      h[k] = hist[slot][lane * 8 + k];
+      loc += h[k];
+    }
+    int64_t incl = loc;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(full, incl, o);
+      if (lane >= o) incl += y;
+    }
+    // first digit d < 255 with (count below d) + h[d] > want, else 255
+    int64_t cum = incl - loc, cd = 0;
+    int dl = 256;
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      const int d = lane * 8 + k;
+      if (dl == 256 && d < 255 && cum + (int64_t)h[k] > want) {
+        dl = d;
+        cd = cum;
+      }
+      cum += h[k];
+    }
+    const unsigned hit = __ballot_sync(full, dl < 256);
+    int d;
+    int64_t below;
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      d = __shfl_sync(full, dl, src);
+      below = __shfl_sync(full, cd, src);
+    } else {
+      d = 255;
+      below = __shfl_sync(full, incl, 31) - (int64_t)__shfl_sync(full, h[7], 31);
+    }
+    if (lane == 0) {
+      c->resid[t] = want - below;
+      const uint32_t p = (pass == 0) ? (uint32_t)d : ((pre << 8) | (uint32_t)d);
+      c->prefix[t] = p;
+      newp[t] = p;
+    }
   }
   __syncthreads();
-  if (tid == 0) {
-    // sorted distinct prefixes for the next pass (T0's and T1's ranks
-    // interleave, so sort first)
-    for (int a = 1; a < nr; a++) {
-      const uint32_t v = newp[a];
-      int b = a - 1;
-      while (b >= 0 && newp[b] > v) { newp[b + 1] = newp[b]; b--; }
-      newp[b + 1] = v;
+
+  if (warp == 0) {
+    // sorted distinct prefixes (T0's and T1's ranks interleave): stable rank
+    const uint32_t v = lane < nr ? newp[lane] : 0xffffffffu;
+    int rk = 0;
+    for (int j = 0; j < nr; j++) {
+      const uint32_t x = __shfl_sync(full, v, j);
+      rk += (x < v || (x == v && j < lane)) ? 1 : 0;
     }
-    int m = 0;
-    for (int r = 0; r < nr; r++)
-      if (m == 0 || sp[m - 1] != newp[r]) sp[m++] = newp[r];
-    c->nslots = m;
-    // the next pass's prefix hash: bucket (p * mult) >> 24 of 256, two entries
-    // each; multipliers are tried until no bucket receives three prefixes
+    if (lane < nr) sorted[rk] = v;
+    __syncwarp();
+    const uint32_t sv = lane < nr ? sorted[lane] : 0u;
+    const uint32_t prev = __shfl_up_sync(full, sv, 1);
+    const bool first = lane < nr && (lane == 0 || prev != sv);
+    const unsigned fm = __ballot_sync(full, first);
+    const int m = __popc(fm);
+    if (first) sp[__popc(fm & ((1u << lane) - 1u))] = sv;
+    __syncwarp();
     uint32_t mult = 0u;
     if (pass < 3) {
-      for (int att = 0; att < 64 && mult == 0u; att++) {
+      for (int att = 0; att < 64; att++) {
         const uint32_t mu = (0x9E3779B1u + 0x6A09E667u * (uint32_t)att) | 1u;
-        for (int b = 0; b < 256; b++) bcnt[b] = 0;
-        bool ok = true;
-        for (int i = 0; i < m && ok; i++) ok = ++bcnt[(sp[i] * mu) >> 24] <= 2;
-        if (ok) mult = mu;
+        const uint32_t bk = lane < m ? (sp[lane] * mu) >> 24 : 0x100u + (uint32_t)lane;
+        const uint32_t peers = __match_any_sync(full, bk);
+        if (__all_sync(full, __popc(peers) <= 2)) {
+          mult = mu;
+          break;
+        }
       }
     }
-    smult = mult;
+    if (lane == 0) {
+      c->nslots = m;
+      smult = mult;
+    }
+  }
+  stab[tid] = make_uint4(~0u, ~0u, ~0u, ~0u);
+  __syncthreads();
+  const uint32_t mult = smult;
+  if (warp == 0 && pass < 3 && mult) {
+    const int m = c->nslots;
+    const uint32_t bk = lane < m ? (sp[lane] * mult) >> 24 : 0x100u + (uint32_t)lane;
+    const uint32_t peers = __match_any_sync(full, bk);
+    if (lane < m) {
+      if (__popc(peers & ((1u << lane) - 1u)) == 0) {
+        stab[bk].x = sp[lane];
+        stab[bk].y = (uint32_t)lane;
+      } else {
+        stab[bk].z = sp[lane];
+        stab[bk].w = (uint32_t)lane;
+      }
+    }
   }
   __syncthreads();
   if (tid < 32) c->slot_prefix[tid] = sp[tid];
   if (pass < 3) {
-    const uint32_t mult = smult;
-    // bucket tid: its prefixes in slot order, empty entries ~0
-    uint4 e = make_uint4(~0u, ~0u, ~0u, ~0u);
-    if (mult) {
-      int k = 0;
-      const int m = c->nslots;
-      for (int i = 0; i < m; i++)
-        if ((int)((sp[i] * mult) >> 24) == tid) {
-          if (k == 0) { e.x = sp[i]; e.y = (uint32_t)i; }
-          else { e.z = sp[i]; e.w = (uint32_t)i; }
-          k++;
-        }
-    }
-    c->htab[tid] = e;
+    c->htab[tid] = stab[tid];
     if (tid == 0) c->hmult = mult;
   }
   if (pass == 3 && tid < 32) {
@@ -294,20 +385,13 @@ cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g,
   for (int j = 2 * n; j < 32; j++) ri.rank[j] = 0;
   init_setup<<<1, 256, 0, st>>>(c, ri, 2 * n, n);
   for (int pass = 0; pass < 4; pass++) {
+    const RadixArgs a{W, (int)N, (int)K, g, scales, pass, pp.ncb, pp.rows_per_chunk};
     if (fmt == kInt4) {
-      if (pass == 0)
-        radix_pass<kInt4, true><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, g, scales, c,
-                                                                pass, pp.ncb, pp.rows_per_chunk);
-      else
-        radix_pass<kInt4, false><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, g, scales, c,
-                                                                 pass, pp.ncb, pp.rows_per_chunk);
+      if (pass == 0) radix_pass<kInt4, true><<<pp.blocks, kThreads, 0, st>>>(a, c);
+      else radix_pass<kInt4, false><<<pp.blocks, kThreads, 0, st>>>(a, c);
     } else {
-      if (pass == 0)
-        radix_pass<kNvfp4, true><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, g, scales, c,
-                                                                 pass, pp.ncb, pp.rows_per_chunk);
-      else
-        radix_pass<kNvfp4, false><<<pp.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, g, scales,
-                                                                  c, pass, pp.ncb, pp.rows_per_chunk);
+      if (pass == 0) radix_pass<kNvfp4, true><<<pp.blocks, kThreads, 0, st>>>(a, c);
+      else radix_pass<kNvfp4, false><<<pp.blocks, kThreads, 0, st>>>(a, c);
     }
     radix_select<<<1, 256, 0, st>>>(c, pass, T);
   }
