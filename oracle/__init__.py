@@ -35,6 +35,12 @@ paper/2605.08692) and what pins it (tests/test_oracle_*.py):
                     choice, S=16 at 0.0625 bpw).  Pinned by the printed
                     storage arithmetic (tests/golden/storage_arithmetic.txt)
                     and by a round trip that recomputes err_final.
+  dequant_bf16      section 1 (dequantised values used at inference, W4A16)
+                    and section 2 mech. 3.  Pinned by a hand-built packed
+                    layer with its values worked out by hand, and by the RTN
+                    special case against numpy's textbook INT4 dequantisation.
+  linear            Y = X W_hat^T in fp64.  Pinned by one-hot rows of X
+                    (Y is a column of W_hat exactly) and by numpy's matmul.
   Final fitted values of a whole run: parity unpinned by the pages (they print
   no worked example); held only by the pins above.
 """
@@ -103,6 +109,10 @@ def lib():
         L.orc_pack.restype = i32
         L.orc_pack.argtypes = [P, i64, i64, P, P, i32, i32, i32, ctypes.c_uint, P, P, P, P, P,
                                P, P]
+        L.orc_dequant_bf16.restype = None
+        L.orc_dequant_bf16.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P]
+        L.orc_linear.restype = None
+        L.orc_linear.argtypes = [P, i64, i64, P, i64, i64, P]
         L.orc_unpack.restype = None
         L.orc_unpack.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, P]
         _lib = L
@@ -278,6 +288,29 @@ def unpack(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S):
     lib().orc_unpack(_p(codes), _p(tagged), _p(bits), _p(T_bf16), N, K, fmt, g, S, _p(w_hat),
                      _p(ch))
     return w_hat, ch
+
+
+def dequant_bf16(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S):
+    """bf16 bits of bf16_RN(s * T_bf16[c][code]) per weight, [N, K] uint16."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    tagged = np.ascontiguousarray(scales_tagged, dtype=scale_dtype(fmt))
+    bits = None if choice_bits is None else np.ascontiguousarray(choice_bits, dtype=np.uint8)
+    T_bf16 = np.ascontiguousarray(T_bf16, dtype=np.uint16)
+    w_hat = np.empty((N, K), dtype=np.uint16)
+    lib().orc_dequant_bf16(_p(codes), _p(tagged), _p(bits), _p(T_bf16), N, K, fmt, g, S,
+                           _p(w_hat))
+    return w_hat
+
+
+def linear(X_u16, w_hat_u16):
+    """Y = X @ w_hat^T in fp64 (k order), X [M, K] and w_hat [N, K] bf16 bits."""
+    X = np.ascontiguousarray(X_u16, dtype=np.uint16)
+    Wh = np.ascontiguousarray(w_hat_u16, dtype=np.uint16)
+    M, K = X.shape
+    N = Wh.shape[0]
+    Y = np.empty((M, N), dtype=np.float64)
+    lib().orc_linear(_p(X), M, K, _p(Wh), N, K, _p(Y))
+    return Y
 
 
 def run_layer(W_u16, X_u16, fmt, g, S, iters, flags=0):

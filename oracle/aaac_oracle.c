@@ -782,3 +782,39 @@ void orc_unpack(const uint8_t* codes, const void* scales_tagged, const uint8_t* 
             w_hat[r * K + k] = (float)((double)s * (double)orc_bf16_to_f32(T_bf16[c * 16 + qv]));
         }
 }
+
+/* ------------------------------------------------------------------------ */
+/* R15: inference dequantisation (section 1: the dequantised values that    */
+/*      decide the weights used at inference, W4A16; section 2 mech. 3:     */
+/*      BF16 tables, choice in the scale's sign bit or in a bitmask).        */
+/*      w_hat[n][k] = bf16_RN(s[n][k/g] * T_bf16[c][code[n][k]]): the exact  */
+/*      product (at most 16 significant bits, exact in fp32) rounded once   */
+/*      to the 16-bit activation type.                                       */
+/* ------------------------------------------------------------------------ */
+void orc_dequant_bf16(const uint8_t* codes, const void* scales_tagged, const uint8_t* choice_bits,
+                      const uint16_t* T_bf16, int64_t N, int64_t K, int fmt, int g, int S,
+                      uint16_t* w_hat)
+{
+    float* wf = (float*)malloc(sizeof(float) * (size_t)(N * K));
+    uint8_t* ch = (uint8_t*)malloc((size_t)(N * (K / S)));
+    orc_unpack(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S, wf, ch);
+    for (int64_t i = 0; i < N * K; i++) w_hat[i] = orc_f32_to_bf16_rn(wf[i]);
+    free(wf);
+    free(ch);
+}
+
+/* W4A16 linear: Y[m][n] = sum_k X[m][k] * w_hat[n][k], summed in fp64 in k  */
+/* order (X bf16 [M][ldx], w_hat bf16 [N][K]).                               */
+void orc_linear(const uint16_t* X, int64_t M, int64_t ldx, const uint16_t* w_hat, int64_t N,
+                int64_t K, double* Y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += (double)orc_bf16_to_f32(X[m * ldx + k]) *
+                       (double)orc_bf16_to_f32(w_hat[n * K + k]);
+            Y[m * N + n] = acc;
+        }
+}
