@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaaac.so"
 
 EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaac_fit_layer",
            "aaac_pack", "aaac_last_error", "aaac_version", "aaac_kernel_launches",
-           "aaac_fit_layer_fixed_scratch")
+           "aaac_fit_layer_fixed_scratch", "aaac_dequant", "aaac_linear")
 
 
 class AaacError(RuntimeError):
@@ -98,6 +98,10 @@ def load(path: str = LIB_PATH):
     L.aaac_version.argtypes = []
     L.aaac_fit_layer_fixed_scratch.restype = ctypes.c_int
     L.aaac_fit_layer_fixed_scratch.argtypes = [P, i64, i64, P, P, P, P, P, P, P]
+    L.aaac_dequant.restype = ctypes.c_int
+    L.aaac_dequant.argtypes = [P, P, P, P, i64, i64, P, P, P]
+    L.aaac_linear.restype = ctypes.c_int
+    L.aaac_linear.argtypes = [P, i64, i64, P, P, P, P, i64, i64, P, P, P]
     L.aaac_kernel_launches.restype = ctypes.c_uint64
     L.aaac_kernel_launches.argtypes = []
     _lib = L
@@ -257,6 +261,38 @@ def pack(W: torch.Tensor, I: torch.Tensor, scales: torch.Tensor, T: torch.Tensor
                             _ptr(out["T_bf16"]), _ptr(out["codes"]), _ptr(out["scales_tagged"]),
                             _ptr(out["choice_bits"]), _ptr(out["err_final"]), _ptr(ws),
                             ws.numel(), _stream(stream)))
+    return out
+
+
+def dequant(packed: dict, cfg: Config, N: int, K: int, out: Optional[torch.Tensor] = None,
+            stream=None) -> torch.Tensor:
+    """bf16 weights of a packed layer (the dict pack() returns), [N, K] bf16 bits (int16)."""
+    _need_cuda()
+    dev = packed["codes"].device
+    if out is None:
+        out = torch.empty(N, K, dtype=torch.int16, device=dev)
+    c = cfg.c()
+    _check(load().aaac_dequant(_ptr(packed["codes"]), _ptr(packed["scales_tagged"]),
+                               _ptr(packed.get("choice_bits")), _ptr(packed["T_bf16"]), N, K,
+                               ctypes.byref(c), _ptr(out), _stream(stream)))
+    return out
+
+
+def linear(X: torch.Tensor, packed: dict, cfg: Config, N: int, K: int,
+           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """W4A16 linear on a packed layer: Y[M, N] = X[M, K] @ W_hat^T, fp32."""
+    _need_cuda()
+    assert X.dtype in (torch.bfloat16, torch.int16, torch.uint16), X.dtype
+    if X.stride(1) != 1 or X.stride(0) % 8:
+        X = X.contiguous()
+    M, ldx = X.shape[0], X.stride(0)
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float32, device=X.device)
+    c = cfg.c()
+    _check(load().aaac_linear(_ptr(X), M, ldx, _ptr(packed["codes"]),
+                              _ptr(packed["scales_tagged"]), _ptr(packed.get("choice_bits")),
+                              _ptr(packed["T_bf16"]), N, K, ctypes.byref(c), _ptr(out),
+                              _stream(stream)))
     return out
 
 

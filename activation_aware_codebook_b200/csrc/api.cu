@@ -216,4 +216,44 @@ aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const
                    "aaac_pack");
 }
 
+aaac_status aaac_dequant(const uint8_t* codes, const void* scales_tagged,
+                         const uint8_t* choice_bits, const uint16_t* T_bf16, int64_t N, int64_t K,
+                         const aaac_config* cfg, uint16_t* W_hat, void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  CHECK(check_ptr(codes, "codes"));
+  CHECK(check_ptr(scales_tagged, "scales_tagged"));
+  CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
+  CHECK(check_ptr(T_bf16, "T_bf16"));
+  CHECK(check_ptr(W_hat, "W_hat"));
+  return from_cuda(aaac::launch_dequant(codes, scales_tagged, choice_bits, T_bf16, N, K, cfg->fmt,
+                                        cfg->g, cfg->S, W_hat, (cudaStream_t)stream),
+                   "aaac_dequant");
+}
+
+aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                        const void* scales_tagged, const uint8_t* choice_bits,
+                        const uint16_t* T_bf16, int64_t N, int64_t K, const aaac_config* cfg,
+                        float* Y, void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  if (M < 1 || M > ((int64_t)1 << 20))
+    return fail(AAAC_ERR_SHAPE, "M=%lld must be in [1, 2^20]", (long long)M);
+  if (ldx < K) return fail(AAAC_ERR_SHAPE, "ldx=%lld < K=%lld", (long long)ldx, (long long)K);
+  if (ldx % 8) return fail(AAAC_ERR_ALIGN, "ldx=%lld is not a multiple of 8", (long long)ldx);
+  if (M * ldx >= ((int64_t)1 << 40))
+    return fail(AAAC_ERR_SHAPE, "M*ldx is too large (M=%lld ldx=%lld)", (long long)M,
+                (long long)ldx);
+  CHECK(check_ptr(X, "X"));
+  CHECK(check_ptr(codes, "codes"));
+  CHECK(check_ptr(scales_tagged, "scales_tagged"));
+  CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
+  CHECK(check_ptr(T_bf16, "T_bf16"));
+  CHECK(check_ptr(Y, "Y"));
+  return from_cuda(aaac::launch_linear(reinterpret_cast<const uint16_t*>(X), M, ldx, codes,
+                                       scales_tagged, choice_bits, T_bf16, N, K, cfg->fmt,
+                                       cfg->g, cfg->S, Y, (cudaStream_t)stream),
+                   "aaac_linear");
+}
+
 }  // extern "C"

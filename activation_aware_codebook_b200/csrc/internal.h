@@ -56,4 +56,11 @@ cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const float* I,
                         uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
                         uint8_t* choice_bits, double* err_final, void* ws, cudaStream_t st);
 
+cudaError_t launch_dequant(const uint8_t* codes, const void* tagged, const uint8_t* cbits,
+                           const uint16_t* Tb, int64_t N, int64_t K, int fmt, int g, int S,
+                           uint16_t* W_hat, cudaStream_t st);
+cudaError_t launch_linear(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                          const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
+                          int64_t K, int fmt, int g, int S, float* Y, cudaStream_t st);
+
 }  // namespace aaac

@@ -174,6 +174,37 @@ aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const
                       void* scales_tagged, uint8_t* choice_bits, double* err_final, void* ws,
                       size_t ws_bytes, void* stream);
 
+/* Inference dequantisation (section 1: the dequantised values from the
+ * table decide the weights used at inference, W4A16; section 2 core mechanism
+ * 3: BF16 tables, choice in the scale's sign bit or in a bitmask).  The packed
+ * layer of aaac_pack back to bf16 weights:
+ *   W_hat[n][k] = bf16_RN(s[n][k/g] * T_bf16[c][code[n][k]])
+ * where s is the magnitude of the stored scale and c is its sign bit (S == g)
+ * or bit (k/S)%8 of choice_bits[n][(k/S)/8] (S < g).  The product has at most
+ * 16 significant bits, so it is exact in fp32 and rounded once.
+ *   codes, scales_tagged, choice_bits, T_bf16: as aaac_pack writes them
+ *                 (choice_bits may be NULL when S == g)
+ *   cfg           fmt, g and S of the packed layer (iters and flags ignored)
+ *   W_hat         device uint16 (bf16 bits) [N][K]
+ * No workspace.  An NVFP4 code 15 (never written by aaac_pack) reads entry 15
+ * of the table, which aaac_pack sets to 0. */
+aaac_status aaac_dequant(const uint8_t* codes, const void* scales_tagged,
+                         const uint8_t* choice_bits, const uint16_t* T_bf16, int64_t N, int64_t K,
+                         const aaac_config* cfg, uint16_t* W_hat, void* stream);
+
+/* The W4A16 linear layer on the packed format (section 1, W4A16 inference):
+ *   Y[m][n] = sum_k X[m][k] * W_hat[n][k]      (W_hat as in aaac_dequant)
+ *   X   device bf16 [M][ldx] (M tokens; ldx >= K, a multiple of 8)
+ *   Y   device fp32 [M][N]
+ * The dequantised weights never reach memory: each kernel expands its codes
+ * on the fly.  Accumulation is fp32 in the library's order; every result is
+ * within K * 2^-24 * sum_k |X[m][k] W_hat[n][k]| of the exact sum.
+ * M in [1, 2^20].  No workspace. */
+aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                        const void* scales_tagged, const uint8_t* choice_bits,
+                        const uint16_t* T_bf16, int64_t N, int64_t K, const aaac_config* cfg,
+                        float* Y, void* stream);
+
 /* Message describing the last failed call on the calling thread ("" after a
  * successful call).  Valid until the next call on the thread. */
 const char* aaac_last_error(void);

@@ -1,0 +1,109 @@
+"""GPU parity of the inference path on the packed format (reading R15):
+aaac_dequant bit-exact against the oracle's bf16 dequantisation, and
+aaac_linear within the fp32 summation bound K * 2^-24 * sum_k |x w_hat| of the
+oracle's fp64 linear.  Packed layers come from the oracle's own pack, so the
+inputs are independent of the CUDA fit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_aware_codebook_b200 import binding as bb
+from activation_aware_codebook_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def u16(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def f32_of_bf16(h):
+    return (np.asarray(h, dtype=np.uint32) << 16).view(np.float32)
+
+
+def packed_layer(N, K, fmt, g, S, seed, iters=3, dist="normal"):
+    """A layer fitted and packed by the oracle; returns (host dict, device dict)."""
+    W, X = synth.small_layer(N, K, seed, T=64, heavy=True, dist=dist)
+    host = oracle.run_layer(u16(W), u16(X), fmt, g, S, iters)
+    dev = {}
+    for key in ("codes", "scales_tagged", "choice_bits", "T_bf16"):
+        a = host[key]
+        dev[key] = None if a is None else torch.from_numpy(
+            np.ascontiguousarray(a).view(np.int16 if a.dtype == np.uint16 else a.dtype)).cuda()
+    return host, dev
+
+
+CASES = [(oracle.INT4, 128, 16), (oracle.INT4, 128, 128), (oracle.INT4, 64, 8),
+         (oracle.NVFP4, 16, 16)]
+
+
+@pytest.mark.parametrize("fmt,g,S", CASES)
+@pytest.mark.parametrize("N,K", [(96, 512), (33, 384)])
+def test_dequant_bit_exact(fmt, g, S, N, K):
+    host, dev = packed_layer(N, K, fmt, g, S, seed=N + K + S)
+    cfg = bb.Config(fmt, g, S, 0)
+    W_hat = bb.dequant(dev, cfg, N, K)
+    ref = oracle.dequant_bf16(host["codes"], host["scales_tagged"], host["choice_bits"],
+                              host["T_bf16"], N, K, fmt, g, S)
+    assert np.array_equal(u16(W_hat), ref)
+
+
+def check_linear(Y, Xb, Wh):
+    ref = oracle.linear(Xb, Wh)
+    K = Xb.shape[1]
+    mag = np.abs(f32_of_bf16(Xb).astype(np.float64)) @ np.abs(f32_of_bf16(Wh).astype(np.float64)).T
+    bound = K * 2.0 ** -24 * mag + 1e-30
+    err = np.abs(Y.cpu().numpy().astype(np.float64) - ref)
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+@pytest.mark.parametrize("fmt,g,S", CASES)
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 13])
+def test_linear_within_bound(fmt, g, S, M):
+    N, K = 70, 640
+    host, dev = packed_layer(N, K, fmt, g, S, seed=7 + M)
+    cfg = bb.Config(fmt, g, S, 0)
+    X = synth.make_activations(M, K, seed=100 + M, heavy=True).cuda()
+    Y = bb.linear(X, dev, cfg, N, K)
+    Wh = oracle.dequant_bf16(host["codes"], host["scales_tagged"], host["choice_bits"],
+                             host["T_bf16"], N, K, fmt, g, S)
+    check_linear(Y, u16(X), Wh)
+
+
+def test_linear_strided_x_and_one_hot():
+    N, K = 40, 256
+    host, dev = packed_layer(N, K, oracle.INT4, 128, 16, seed=3)
+    cfg = bb.Config(oracle.INT4, 128, 16, 0)
+    wide = torch.zeros(4, K + 24, dtype=torch.bfloat16)
+    cols = [0, 9, 130, 255]
+    for i, c in enumerate(cols):
+        wide[i, c] = 1.0
+    Y = bb.linear(wide.cuda()[:, :K], dev, cfg, N, K)  # ldx = K + 24
+    Wh = f32_of_bf16(oracle.dequant_bf16(host["codes"], host["scales_tagged"],
+                                         host["choice_bits"], host["T_bf16"], N, K,
+                                         oracle.INT4, 128, 16))
+    for i, c in enumerate(cols):
+        assert np.array_equal(Y[i].cpu().numpy(), Wh[:, c])
+
+
+def test_dequant_and_linear_full_size_gate():
+    """A 14336 x 4096 layer fitted and packed on the GPU; dequantisation
+    bit-exact against the oracle on the same packed bits, and the M = 1 linear
+    within the bound on every output."""
+    N, K = 14336, 4096
+    W = synth.make_weight(N, K, 91, device="cuda")
+    X = synth.make_activations(2048, K, 92, True, device="cuda")
+    cfg = bb.Config(oracle.INT4, 128, 16, 2)
+    out = bb.run_layer(W, X, cfg)
+    W_hat = bb.dequant(out, cfg, N, K)
+    host = {k: (None if out[k] is None else out[k].cpu().numpy())
+            for k in ("codes", "scales_tagged", "choice_bits", "T_bf16")}
+    ref = oracle.dequant_bf16(host["codes"], host["scales_tagged"].view(np.uint16),
+                              host["choice_bits"], host["T_bf16"].view(np.uint16), N, K,
+                              oracle.INT4, 128, 16)
+    assert np.array_equal(u16(W_hat), ref)
+    x = synth.make_activations(1, K, 93, True, device="cuda")
+    Y = bb.linear(x, out, cfg, N, K)
+    check_linear(Y, u16(x), ref)
