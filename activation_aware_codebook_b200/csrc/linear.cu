@@ -10,13 +10,14 @@
 // bits; the bf16x2 multiply rounds the exact product once, which is that
 // definition.
 //
-//   dequant_kernel  16 weights per thread: 8 bytes of codes in, 32 bytes of
-//                   bf16 out; the 32-entry table sits in shared memory.
-//   gemv_kernel     small M: a warp owns R output rows and walks K, 8 columns
-//                   per lane per step; each lane expands its 8 codes (table
-//                   lookup, bf16x2 scale multiply) and accumulates with fp32x2
-//                   FMAs against the token tile's activations held in
-//                   registers.  MT tokens x R rows = 8 accumulator pairs.
+//   dequant_kernel  one warp per row, 16 weights per lane per step: 8 bytes
+//                   of codes in, 32 bytes of bf16 out; the 32-entry table
+//                   sits in shared memory.
+//   gemv_kernel     small M: a warp owns R output rows and MT tokens and walks
+//                   K, 16 columns per lane per step; each lane expands its
+//                   codes (table lookup, bf16x2 scale multiply) and
+//                   accumulates with fp32x2 FMAs against the token tile's
+//                   activations held in registers.
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,27 +25,17 @@ namespace aaac {
 
 namespace {
 
-// Stored scale of group gi: bf16 bits of its magnitude, and its sign bit.
+// A stored scale (bf16 bits for INT4, an E4M3 byte for NVFP4): bf16 bits of
+// its magnitude, and its sign bit in *tag.  E4M3 magnitudes are exact in bf16
+// (3 mantissa bits, exponents 2^-9 .. 2^8).
 template <int FMT>
-__device__ __forceinline__ uint32_t scale_bf16(const void* tagged, int64_t gi, uint32_t* tag) {
+__device__ __forceinline__ uint32_t decode_scale(uint32_t v, uint32_t* tag) {
   if (FMT == kInt4) {
-    const uint32_t h = __ldg(reinterpret_cast<const unsigned short*>(tagged) + gi);
-    *tag = h >> 15;
-    return h & 0x7fffu;
-  } else {
-    const uint32_t v = __ldg(reinterpret_cast<const unsigned char*>(tagged) + gi);
-    *tag = v >> 7;
-    // E4M3 magnitudes are exact in bf16 (3 mantissa bits, exponents 2^-9..2^8)
-    return __float_as_uint(e4m3_mag(v & 0x7fu)) >> 16;
+    *tag = v >> 15;
+    return v & 0x7fffu;
   }
-}
-
-// Choice of the selection group holding column k of row n.
-__device__ __forceinline__ uint32_t group_choice(uint32_t tag, const uint8_t* cbits, int64_t n,
-                                                 int nb, int k, int g, int S) {
-  if (S == g) return tag;
-  const int j = k / S;
-  return (__ldg(cbits + n * nb + (j >> 3)) >> (j & 7)) & 1u;
+  *tag = v >> 7;
+  return __float_as_uint(e4m3_mag(v & 0x7fu)) >> 16;
 }
 
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
@@ -70,97 +61,132 @@ __device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsign
   return r;
 }
 
-// Eight dequantised weights (bf16x2 pairs, even column low) of one lane.
+// Eight dequantised weights (bf16x2 pairs, even column low) from one word of
+// codes: the table offsets of four even and four odd nibbles are formed at
+// once (byte j of ev / od = 2 * code + 32 * c, a byte offset into sT), then
+// one 16-bit table load per weight and one bf16x2 multiply per pair.
 __device__ __forceinline__ void expand8(uint32_t cw, uint32_t sbf, uint32_t c,
                                         const unsigned short* sT, uint32_t out[4]) {
   const uint32_t s2 = sbf | (sbf << 16);
-  const unsigned short* t = sT + c * 16;
+  const uint32_t cb = c ? 0x20202020u : 0u;
+  const uint32_t ev = ((cw << 1) & 0x1e1e1e1eu) | cb;
+  const uint32_t od = ((cw >> 3) & 0x1e1e1e1eu) | cb;
+  const unsigned char* tb = reinterpret_cast<const unsigned char*>(sT);
 #pragma unroll
   for (int p = 0; p < 4; p++) {
-    const uint32_t lo = t[(cw >> (8 * p)) & 15u];
-    const uint32_t hi = t[(cw >> (8 * p + 4)) & 15u];
-    out[p] = bf16x2_mul(lo | (hi << 16), s2);
+    const uint32_t lo = *reinterpret_cast<const unsigned short*>(tb + __byte_perm(ev, 0u, 0x4440u + p));
+    const uint32_t hi = *reinterpret_cast<const unsigned short*>(tb + __byte_perm(od, 0u, 0x4440u + p));
+    out[p] = bf16x2_mul(__byte_perm(lo, hi, 0x5410u), s2);
   }
 }
 
+// Sixteen weights of one lane and row: codes (8 bytes), the scale of the
+// group (g >= 16 holds all 16), the choice byte (S >= 8: both 8-column halves
+// fall in one byte), expanded to 8 bf16x2 pairs.
 template <int FMT>
-__global__ void __launch_bounds__(256)
-dequant_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ tagged,
-               const uint8_t* __restrict__ cbits, const uint16_t* __restrict__ Tb, int64_t N,
-               int K, int g, int S, uint16_t* __restrict__ W_hat) {
-  __shared__ unsigned short sT[32];
-  if (threadIdx.x < 32) sT[threadIdx.x] = Tb[threadIdx.x];
-  __syncthreads();
-  const int G = K / g, nb = (K / S + 7) / 8, per_row = K / 16;
-  const int64_t total = N * per_row;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t n = i / per_row;
-    const int k0 = (int)(i - n * per_row) * 16;
-    const uint2 cw = __ldg(reinterpret_cast<const uint2*>(codes + (n * K + k0) / 2));
-    uint32_t out[8];
-#pragma unroll
-    for (int h = 0; h < 2; h++) {
-      const int k = k0 + 8 * h;
-      uint32_t tag;
-      const uint32_t sbf = scale_bf16<FMT>(tagged, n * G + k / g, &tag);
-      const uint32_t c = group_choice(tag, cbits, n, nb, k, g, S);
-      expand8(h ? cw.y : cw.x, sbf, c, sT, out + 4 * h);
-    }
-    uint4* dst = reinterpret_cast<uint4*>(W_hat + n * K + k0);
-    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-  }
+__device__ __forceinline__ void expand16(uint2 cw, uint32_t sv, uint32_t cbyte, int k0, int ls,
+                                         bool sign_choice, const unsigned short* sT,
+                                         uint32_t out[8]) {
+  uint32_t tag;
+  const uint32_t sbf = decode_scale<FMT>(sv, &tag);
+  const uint32_t c0 = sign_choice ? tag : ((cbyte >> ((k0 >> ls) & 7)) & 1u);
+  const uint32_t c1 = sign_choice ? tag : ((cbyte >> (((k0 + 8) >> ls) & 7)) & 1u);
+  expand8(cw.x, sbf, c0, sT, out);
+  expand8(cw.y, sbf, c1, sT, out + 4);
 }
 
-constexpr int kGemvWarps = 4;
+constexpr int kLinWarps = 8;
 
-template <int FMT, int MT, int R>
-__global__ void __launch_bounds__(kGemvWarps * 32)
-gemv_kernel(const uint16_t* __restrict__ X, int M, int ldx, const uint8_t* __restrict__ codes,
-            const void* __restrict__ tagged, const uint8_t* __restrict__ cbits,
-            const uint16_t* __restrict__ Tb, int N, int K, int g, int S, float* __restrict__ Y) {
+// One warp per row (rows strided over the grid); lane l covers columns
+// [16 l + 512 i, +16).  Loads of a step are issued before use.
+template <int FMT>
+__global__ void __launch_bounds__(kLinWarps * 32)
+dequant_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ tagged,
+               const uint8_t* __restrict__ cbits, const uint16_t* __restrict__ Tb, int N, int K,
+               int lg, int ls, uint16_t* __restrict__ W_hat) {
   __shared__ unsigned short sT[32];
   if (threadIdx.x < 32) sT[threadIdx.x] = Tb[threadIdx.x];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = (blockIdx.y * kGemvWarps + warp) * R;  // grid: x = token tiles, y = rows
+  const int G = K >> lg, nb = ((K >> ls) + 7) >> 3;
+  const bool sign_choice = lg == ls;
+  for (int n = blockIdx.x * kLinWarps + warp; n < N; n += gridDim.x * kLinWarps) {
+    const uint8_t* crow = codes + (int64_t)n * (K >> 1);
+    const int64_t grow = (int64_t)n * G;
+    const uint8_t* brow = cbits + (int64_t)n * nb;
+    uint16_t* wrow = W_hat + (int64_t)n * K;
+    for (int k0 = lane * 16; k0 < K; k0 += 512) {
+      const uint2 cw = __ldg(reinterpret_cast<const uint2*>(crow + (k0 >> 1)));
+      const uint32_t sv = (FMT == kInt4)
+          ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(tagged) + grow + (k0 >> lg))
+          : (uint32_t)__ldg(reinterpret_cast<const unsigned char*>(tagged) + grow + (k0 >> lg));
+      const uint32_t cbyte = sign_choice ? 0u : (uint32_t)__ldg(brow + (k0 >> (ls + 3)));
+      uint32_t out[8];
+      expand16<FMT>(cw, sv, cbyte, k0, ls, sign_choice, sT, out);
+      uint4* dst = reinterpret_cast<uint4*>(wrow + k0);
+      dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+      dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    }
+  }
+}
+
+// Small M: a warp owns R rows and MT tokens and walks all of K, 16 columns
+// per lane per step; activations for the step sit in registers (fp32 pairs)
+// and feed fp32x2 FMAs with the expanded weights.  Lane partials meet in a
+// shuffle tree.
+template <int FMT, int MT, int R>
+__global__ void __launch_bounds__(kLinWarps * 32)
+gemv_kernel(const uint16_t* __restrict__ X, int M, int ldx, const uint8_t* __restrict__ codes,
+            const void* __restrict__ tagged, const uint8_t* __restrict__ cbits,
+            const uint16_t* __restrict__ Tb, int N, int K, int lg, int ls, float* __restrict__ Y) {
+  __shared__ unsigned short sT[32];
+  if (threadIdx.x < 32) sT[threadIdx.x] = Tb[threadIdx.x];
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = (blockIdx.y * kLinWarps + warp) * R;  // grid: x = token tiles, y = row tiles
   const int m0 = blockIdx.x * MT;
   if (n0 >= N) return;  // warp-uniform
-  const int G = K / g, nb = (K / S + 7) / 8;
+  const int G = K >> lg, nb = ((K >> ls) + 7) >> 3;
+  const bool sign_choice = lg == ls;
   unsigned long long acc[R][MT];
 #pragma unroll
   for (int r = 0; r < R; r++)
 #pragma unroll
     for (int m = 0; m < MT; m++) acc[r][m] = 0ull;
 
-  for (int k0 = lane * 8; k0 < K; k0 += 256) {
-    unsigned long long x2[MT][4];
+  for (int k0 = lane * 16; k0 < K; k0 += 512) {
+    uint4 xv[MT][2];
+    uint2 cw[R];
+    uint32_t sv[R], cbyte[R];
 #pragma unroll
     for (int m = 0; m < MT; m++) {
-      uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-      if (m0 + m < M) xv = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)(m0 + m) * ldx + k0));
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-      for (int p = 0; p < 4; p++) x2[m][p] = f2pack(bf16_lo(xw[p]), bf16_hi(xw[p]));
+      const uint4* xp = reinterpret_cast<const uint4*>(X + (int64_t)min(m0 + m, M - 1) * ldx + k0);
+      xv[m][0] = __ldg(xp);
+      xv[m][1] = __ldg(xp + 1);
     }
-    uint32_t cw[R];
-#pragma unroll
-    for (int r = 0; r < R; r++)
-      cw[r] = (n0 + r < N)
-                  ? __ldg(reinterpret_cast<const uint32_t*>(codes + ((int64_t)(n0 + r) * K + k0) / 2))
-                  : 0u;
 #pragma unroll
     for (int r = 0; r < R; r++) {
-      const int n = n0 + r;
-      if (n >= N) break;  // warp-uniform
-      uint32_t tag;
-      const uint32_t sbf = scale_bf16<FMT>(tagged, (int64_t)n * G + k0 / g, &tag);
-      const uint32_t c = group_choice(tag, cbits, n, nb, k0, g, S);
-      uint32_t w[4];
-      expand8(cw[r], sbf, c, sT, w);
+      const int n = min(n0 + r, N - 1);  // rows past N repeat the last row; never stored
+      cw[r] = __ldg(reinterpret_cast<const uint2*>(codes + (((int64_t)n * K + k0) >> 1)));
+      const int64_t gi = (int64_t)n * G + (k0 >> lg);
+      sv[r] = (FMT == kInt4) ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(tagged) + gi)
+                             : (uint32_t)__ldg(reinterpret_cast<const unsigned char*>(tagged) + gi);
+      cbyte[r] = sign_choice ? 0u : (uint32_t)__ldg(cbits + (int64_t)n * nb + (k0 >> (ls + 3)));
+    }
+    unsigned long long x2[MT][8];
 #pragma unroll
-      for (int p = 0; p < 4; p++) {
+    for (int m = 0; m < MT; m++) {
+      const uint32_t xw[8] = {xv[m][0].x, xv[m][0].y, xv[m][0].z, xv[m][0].w,
+                              xv[m][1].x, xv[m][1].y, xv[m][1].z, xv[m][1].w};
+#pragma unroll
+      for (int p = 0; p < 8; p++) x2[m][p] = f2pack(bf16_lo(xw[p]), bf16_hi(xw[p]));
+    }
+#pragma unroll
+    for (int r = 0; r < R; r++) {
+      uint32_t w[8];
+      expand16<FMT>(cw[r], sv[r], cbyte[r], k0, ls, sign_choice, sT, w);
+#pragma unroll
+      for (int p = 0; p < 8; p++) {
         const unsigned long long wf = f2pack(bf16_lo(w[p]), bf16_hi(w[p]));
 #pragma unroll
         for (int m = 0; m < MT; m++) acc[r][m] = f2fma(x2[m][p], wf, acc[r][m]);
@@ -181,39 +207,44 @@ gemv_kernel(const uint16_t* __restrict__ X, int M, int ldx, const uint8_t* __res
 template <int FMT, int MT, int R>
 void launch_gemv_t(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                    const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
-                   int64_t K, int g, int S, float* Y, cudaStream_t st) {
-  const unsigned rows_per_block = kGemvWarps * R;
+                   int64_t K, int lg, int ls, float* Y, cudaStream_t st) {
   // token tiles along x (consecutive blocks reuse the same codes from L2)
+  const unsigned rows_per_block = kLinWarps * R;
   const dim3 grid((unsigned)((M + MT - 1) / MT), (unsigned)((N + rows_per_block - 1) / rows_per_block));
-  gemv_kernel<FMT, MT, R><<<grid, kGemvWarps * 32, 0, st>>>(X, (int)M, (int)ldx, codes, tagged,
-                                                            cbits, Tb, (int)N, (int)K, g, S, Y);
+  gemv_kernel<FMT, MT, R><<<grid, kLinWarps * 32, 0, st>>>(X, (int)M, (int)ldx, codes, tagged,
+                                                           cbits, Tb, (int)N, (int)K, lg, ls, Y);
 }
 
 template <int FMT>
 void launch_gemv(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                  const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
-                 int64_t K, int g, int S, float* Y, cudaStream_t st) {
-  if (M == 1) launch_gemv_t<FMT, 1, 8>(X, M, ldx, codes, tagged, cbits, Tb, N, K, g, S, Y, st);
-  else if (M == 2) launch_gemv_t<FMT, 2, 4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, g, S, Y, st);
-  else if (M <= 4) launch_gemv_t<FMT, 4, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, g, S, Y, st);
-  else launch_gemv_t<FMT, 8, 1>(X, M, ldx, codes, tagged, cbits, Tb, N, K, g, S, Y, st);
+                 int64_t K, int lg, int ls, float* Y, cudaStream_t st) {
+  if (M == 1) launch_gemv_t<FMT, 1, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
+  else if (M == 2) launch_gemv_t<FMT, 2, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
+  else if (M <= 4) launch_gemv_t<FMT, 4, 1>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
+  else launch_gemv_t<FMT, 8, 1>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
 }
 
 }  // namespace
 
+static int log2_of(int v) {
+  int l = 0;
+  while ((1 << l) < v) l++;
+  return l;
+}
+
 cudaError_t launch_dequant(const uint8_t* codes, const void* tagged, const uint8_t* cbits,
                            const uint16_t* Tb, int64_t N, int64_t K, int fmt, int g, int S,
                            uint16_t* W_hat, cudaStream_t st) {
-  const int64_t chunks = N * (K / 16);
-  int64_t blocks = (chunks + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  if (blocks < 1) blocks = 1;
+  const int lg = log2_of(g), ls = log2_of(S);
+  const int64_t want = (N + kLinWarps - 1) / kLinWarps;
+  const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
   if (fmt == kInt4)
-    dequant_kernel<kInt4><<<(unsigned)blocks, 256, 0, st>>>(codes, tagged, cbits, Tb, N, (int)K,
-                                                            g, S, W_hat);
+    dequant_kernel<kInt4><<<blocks, kLinWarps * 32, 0, st>>>(codes, tagged, cbits, Tb, (int)N, (int)K, lg, ls,
+                                                  W_hat);
   else
-    dequant_kernel<kNvfp4><<<(unsigned)blocks, 256, 0, st>>>(codes, tagged, cbits, Tb, N, (int)K,
-                                                             g, S, W_hat);
+    dequant_kernel<kNvfp4><<<blocks, kLinWarps * 32, 0, st>>>(codes, tagged, cbits, Tb, (int)N, (int)K, lg,
+                                                   ls, W_hat);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -221,8 +252,9 @@ cudaError_t launch_dequant(const uint8_t* codes, const void* tagged, const uint8
 cudaError_t launch_linear(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                           const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
                           int64_t K, int fmt, int g, int S, float* Y, cudaStream_t st) {
-  if (fmt == kInt4) launch_gemv<kInt4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, g, S, Y, st);
-  else launch_gemv<kNvfp4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, g, S, Y, st);
+  const int lg = log2_of(g), ls = log2_of(S);
+  if (fmt == kInt4) launch_gemv<kInt4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
+  else launch_gemv<kNvfp4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
   count_launches(1);
   return cudaGetLastError();
 }
