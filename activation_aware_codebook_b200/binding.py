@@ -29,7 +29,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaaac.so"
 
 EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaac_fit_layer",
            "aaac_pack", "aaac_last_error", "aaac_version", "aaac_kernel_launches",
-           "aaac_fit_layer_fixed_scratch", "aaac_dequant", "aaac_linear")
+           "aaac_fit_layer_fixed_scratch", "aaac_dequant", "aaac_linear",
+           "aaac_device_timeouts")
 
 
 class AaacError(RuntimeError):
@@ -102,6 +103,8 @@ def load(path: str = LIB_PATH):
     L.aaac_dequant.argtypes = [P, P, P, P, i64, i64, P, P, P]
     L.aaac_linear.restype = ctypes.c_int
     L.aaac_linear.argtypes = [P, i64, i64, P, P, P, P, i64, i64, P, P, P]
+    L.aaac_device_timeouts.restype = ctypes.c_int
+    L.aaac_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     L.aaac_kernel_launches.restype = ctypes.c_uint64
     L.aaac_kernel_launches.argtypes = []
     _lib = L
@@ -262,6 +265,14 @@ def pack(W: torch.Tensor, I: torch.Tensor, scales: torch.Tensor, T: torch.Tensor
                             _ptr(out["choice_bits"]), _ptr(out["err_final"]), _ptr(ws),
                             ws.numel(), _stream(stream)))
     return out
+
+
+def device_timeouts() -> int:
+    """1 when a bounded device wait of the library's kernels has run out since
+    the library was loaded on the current device, else 0."""
+    v = ctypes.c_uint32(0)
+    _check(load().aaac_device_timeouts(ctypes.byref(v)))
+    return int(v.value)
 
 
 def dequant(packed: dict, cfg: Config, N: int, K: int, out: Optional[torch.Tensor] = None,

@@ -256,4 +256,13 @@ aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* co
                    "aaac_linear");
 }
 
+aaac_status aaac_device_timeouts(uint32_t* flag) {
+  if (!flag) return fail(AAAC_ERR_INVALID_ARG, "flag is NULL");
+  unsigned int v = 0;
+  const cudaError_t e = aaac::gemm_timeout_flag(&v);
+  if (e != cudaSuccess) return from_cuda(e, "aaac_device_timeouts");
+  *flag = v ? 1u : 0u;
+  return AAAC_OK;
+}
+
 }  // extern "C"

@@ -63,4 +63,9 @@ cudaError_t launch_linear(const uint16_t* X, int64_t M, int64_t ldx, const uint8
                           const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
                           int64_t K, int fmt, int g, int S, float* Y, cudaStream_t st);
 
+cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                        const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
+                        int64_t K, int fmt, int lg, int ls, float* Y, cudaStream_t st);
+cudaError_t gemm_timeout_flag(unsigned int* out);
+
 }  // namespace aaac

@@ -221,11 +221,12 @@ void launch_gemv(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes
                  int64_t K, int lg, int ls, float* Y, cudaStream_t st) {
   if (M == 1) launch_gemv_t<FMT, 1, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
   else if (M == 2) launch_gemv_t<FMT, 2, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
-  else if (M <= 4) launch_gemv_t<FMT, 4, 1>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
-  else launch_gemv_t<FMT, 8, 1>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
+  else launch_gemv_t<FMT, 4, 1>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
 }
 
 }  // namespace
+
+constexpr int64_t kGemvMaxM = 4;  // token counts above this go to the tensor-core kernel
 
 static int log2_of(int v) {
   int l = 0;
@@ -253,6 +254,11 @@ cudaError_t launch_linear(const uint16_t* X, int64_t M, int64_t ldx, const uint8
                           const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
                           int64_t K, int fmt, int g, int S, float* Y, cudaStream_t st) {
   const int lg = log2_of(g), ls = log2_of(S);
+  if (M > kGemvMaxM) {  // tensor cores: dequantised tiles in shared memory
+    const cudaError_t e = launch_gemm(X, M, ldx, codes, tagged, cbits, Tb, N, K, fmt, lg, ls, Y, st);
+    if (e == cudaSuccess) count_launches(1);
+    return e;
+  }
   if (fmt == kInt4) launch_gemv<kInt4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
   else launch_gemv<kNvfp4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
   count_launches(1);

@@ -205,6 +205,13 @@ aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* co
                         const uint16_t* T_bf16, int64_t N, int64_t K, const aaac_config* cfg,
                         float* Y, void* stream);
 
+/* Device-side wait status of the current device: *flag = 1 when a bounded
+ * wait inside one of the library's kernels (the tensor-core aaac_linear path)
+ * has run out since the library was loaded, else 0.  A kernel whose wait ran
+ * out writes NaN to its output tile and still releases its tensor memory.
+ * Synchronises with the device (reads a device variable). */
+aaac_status aaac_device_timeouts(uint32_t* flag);
+
 /* Message describing the last failed call on the calling thread ("" after a
  * successful call).  Valid until the next call on the thread. */
 const char* aaac_last_error(void);

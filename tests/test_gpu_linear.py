@@ -107,3 +107,39 @@ def test_dequant_and_linear_full_size_gate():
     x = synth.make_activations(1, K, 93, True, device="cuda")
     Y = bb.linear(x, out, cfg, N, K)
     check_linear(Y, u16(x), ref)
+
+
+GEMM_CASES = [(oracle.INT4, 128, 16, 200, 640), (oracle.INT4, 128, 128, 130, 384),
+              (oracle.NVFP4, 16, 16, 70, 208), (oracle.INT4, 32, 8, 256, 96)]
+
+
+@pytest.mark.parametrize("fmt,g,S,N,K", GEMM_CASES)
+@pytest.mark.parametrize("M", [5, 9, 64, 100, 257, 600])
+def test_linear_tensor_core_path(fmt, g, S, N, K, M):
+    """Token counts above 8 take the tcgen05 kernel: partial weight-row tiles
+    (N not a multiple of 128), partial token tiles, and a last K block that
+    is only partly inside K (K = 208, 96)."""
+    host, dev = packed_layer(N, K, fmt, g, S, seed=M + N)
+    cfg = bb.Config(fmt, g, S, 0)
+    X = synth.make_activations(M, K, seed=200 + M, heavy=True).cuda()
+    Y = bb.linear(X, dev, cfg, N, K)
+    torch.cuda.synchronize()
+    assert bb.device_timeouts() == 0
+    Wh = oracle.dequant_bf16(host["codes"], host["scales_tagged"], host["choice_bits"],
+                             host["T_bf16"], N, K, fmt, g, S)
+    check_linear(Y, u16(X), Wh)
+
+
+def test_linear_tensor_core_many_tiles():
+    """150 weight-row tiles (at least one per SM): the unsplit path, each CTA
+    over all of K."""
+    N, K, M = 128 * 150, 128, 100
+    host, dev = packed_layer(N, K, oracle.INT4, 128, 16, seed=11, iters=1)
+    cfg = bb.Config(oracle.INT4, 128, 16, 0)
+    X = synth.make_activations(M, K, seed=12, heavy=True).cuda()
+    Y = bb.linear(X, dev, cfg, N, K)
+    torch.cuda.synchronize()
+    assert bb.device_timeouts() == 0
+    Wh = oracle.dequant_bf16(host["codes"], host["scales_tagged"], host["choice_bits"],
+                             host["T_bf16"], N, K, oracle.INT4, 128, 16)
+    check_linear(Y, u16(X), Wh)
