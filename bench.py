@@ -51,6 +51,10 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--linear", action="store_true",
+                   help="time the W4A16 linear on a packed 14336x4096 layer instead of the fit")
+    p.add_argument("--tokens-list", default="1,16,256,4096",
+                   help="token counts for --linear")
     return p.parse_args()
 
 
@@ -462,10 +466,111 @@ def run_reference(args, rank, world):
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+
+# ---------------------------------------------------------------------------
+# --linear: the inference consumer of the packed format (W4A16)
+# ---------------------------------------------------------------------------
+LINEAR_N, LINEAR_K = 14336, 4096
+
+
+def run_linear(args):
+    """Y = X W_hat^T through aaac_linear on a gate_proj-shaped packed layer.
+    Each timed launch is preceded by an L2 flush (a 256 MiB write outside the
+    timed region); one CUDA-event pair per launch on the launching stream."""
+    import torch
+    from activation_aware_codebook_b200 import binding as bb, synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    N, K = LINEAR_N, LINEAR_K
+    cfg = bb.Config(bb.INT4, 128, 16, 1)
+    W = synth.make_weight(N, K, 91, device=dev)
+    X = synth.make_activations(2048, K, 92, True, device=dev)
+    packed = bb.run_layer(W, X, cfg)
+    del W, X
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.int8, device=dev)
+    hbm, hbm_kind = measured_peak()
+    tflops_peak, tf_kind = measured_tensor_peak()
+    code_bytes = N * K // 2 + N * (K // 128) * 2 + N * (K // 16 // 8)
+    points = []
+    launches0 = bb.kernel_launches()
+    sampler = ClockSampler(0)
+    sampler.start()
+    for M in [int(t) for t in args.tokens_list.split(",") if t]:
+        x = synth.make_activations(M, K, 93 + M, True, device=dev)
+        Y = torch.empty(M, N, dtype=torch.float32, device=dev)
+        st = torch.cuda.current_stream()
+        for _ in range(args.warmup):
+            bb.linear(x, packed, cfg, N, K, out=Y)
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            bb.linear(x, packed, cfg, N, K, out=Y)
+            e1.record(st)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        byts = code_bytes + M * K * 2 + M * N * 4
+        flops = 2.0 * M * N * K
+        if M <= 64:
+            roof = {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": hbm,
+                    "peak_kind": hbm_kind, "unit": "GB/s"}
+        else:
+            roof = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": tflops_peak,
+                    "peak_kind": tf_kind, "unit": "TFLOP/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        points.append({"tokens": M, "us": ms * 1e3, "tokens_per_s": M / (ms * 1e-3),
+                       "path": "gemv" if M <= 4 else "tcgen05", "roofline": roof})
+    clocks = sampler.stop()
+    launches = bb.kernel_launches() - launches0
+    head = points[0]
+    out = {"metric": "W4A16 linear on AAAC-packed weights (gate_proj 14336x4096, INT4 g=128 S=16): tokens/s",
+           "value": head["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": head["us"] / 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x bf16 -> f32",
+           "data": "synthetic: packed layer fitted on seeded synthetic weights and activations",
+           "config": {"workload": "w4a16-linear-14336x4096", "tokens": [p["tokens"] for p in points],
+                      "l2": "256 MiB write between timed launches"},
+           "points": points, "gpu_launches": int(launches), "clocks": clocks}
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = linear_cpu_baseline(packed)
+    return out
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (burst)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def linear_cpu_baseline(packed):
+    """The oracle (dequantisation + fp64 linear) on a 512-row slice, 16 tokens."""
+    import numpy as np
+    import oracle
+    from activation_aware_codebook_b200 import synth
+    rows, M, K = 512, 16, LINEAR_K
+    host = {k: packed[k][:rows].cpu().numpy() for k in ("codes", "scales_tagged", "choice_bits")}
+    Tb = packed["T_bf16"].cpu().numpy().view(np.uint16)
+    x = synth.bits_u16(synth.make_activations(M, K, 109, True))
+    t = time.time()
+    Wh = oracle.dequant_bf16(host["codes"], host["scales_tagged"].view(np.uint16),
+                             host["choice_bits"], Tb, rows, K, oracle.INT4, 128, 16)
+    oracle.linear(x, Wh)
+    dt = time.time() - t
+    return {"value": M / dt, "unit": "tokens/s (512 of 14336 rows)", "cores": os.cpu_count(),
+            "kind": "oracle", "sample": f"{rows} rows x {K} x {M} tokens", "seconds": dt}
+
 def main():
     args = parse()
     rank, local_rank, world = env_rank()
-    if args.impl == "reference":
+    if args.linear:
+        out = run_linear(args) if rank == 0 else None
+    elif args.impl == "reference":
         out = run_reference(args, rank, world)
     else:
         out = run_ours(args, rank, local_rank, world)
