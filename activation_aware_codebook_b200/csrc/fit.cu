@@ -144,90 +144,157 @@ __device__ inline int bucket_raw(float x, float la) {
   return min(max(r, -1), kNB);
 }
 
-// Merge both books' thresholds (one thread).
-__device__ void merge_thresholds(Tables& tb) {
-  const Book& a = tb.bk[0];
-  const Book& b = tb.bk[1];
-  int i = 0, j = 0, n = 0;
-  const int na = a.m - 1, nb = b.m - 1;
-  while (i < na || j < nb) {
-    float t;
-    if (j >= nb || (i < na && a.thr[i] < b.thr[j])) t = a.thr[i++];
-    else if (i >= na || b.thr[j] < a.thr[i]) t = b.thr[j++];
-    else { t = a.thr[i++]; j++; }  // equal thresholds: one cell boundary
-    tb.mthr[n++] = t;
-  }
-  tb.nm = n;
-  for (int k = n; k < kMerged; k++) tb.mthr[k] = kInf;
-}
-
-// Cell m of the merged tables (thread per cell).
-__device__ void merged_cell(Tables& tb, int m) {
-  if (m == (int)kCrowded) {
-    tb.mv0[m] = __int_as_float(0x7fc00000);
-    tb.mv1[m] = __int_as_float(0x7fc00000);
-    tb.moff[m] = 0;
-    return;
-  }
-  int c0 = 0, c1 = 0;
-  if (m >= 1 && m <= tb.nm) {
-    const float lo = tb.mthr[m - 1];  // smallest u of the cell
-    for (int i = 0; i + 1 < tb.bk[0].m; i++) c0 += (tb.bk[0].thr[i] <= lo) ? 1 : 0;
-    for (int i = 0; i + 1 < tb.bk[1].m; i++) c1 += (tb.bk[1].thr[i] <= lo) ? 1 : 0;
-  }
-  tb.mv0[m] = tb.bk[0].val[c0];
-  tb.mv1[m] = tb.bk[1].val[c1];
-  tb.moff[m] = (uint32_t)(c0 * kCellBytes) | ((uint32_t)((16 + c1) * kCellBytes) << 16);
-}
-
-// All tables from the codebooks sT[2][16] (shared memory), by every thread of
-// one block (blockDim >= 64): sort (optional), distinct values, exact midpoint
-// thresholds, merged thresholds, merged cells, and the bucket table (bucket b
-// counts the merged thresholds at or below its smallest u, or kCrowded when
-// two or more fall strictly inside it).
+// All tables from the codebooks sT[2][16] (shared memory), by the threads of
+// one block (blockDim >= 64; warp 0 does the per-entry work, lane = book * 16
+// + entry):
+//   1. sort (optional; stable ranks in IEEE total order), then the distinct
+//      values (-0 == +0) by ballot, and their exact midpoint thresholds;
+//   2. merge: each threshold takes a unique slot (book 0 before an equal
+//      book-1 value), equal neighbours collapse to one merged threshold, and
+//      the counts of each book's thresholds at or below it come from prefix
+//      masks of the slots' sources;
+//   3. merged cells: nearest values and bin offsets of both books; the
+//      sentinel cell kCrowded holds NaN;
+//   4. bucket table: a histogram of the thresholds' buckets and a warp scan;
+//      bucket b counts the thresholds below it or opening it, and is crowded
+//      when two or more fall strictly inside.
+// When sort_first, sT is left sorted (the callers write it back as T).
 __device__ void build_tables(Tables& tb, float (*sT)[16], int n, bool sort_first) {
-  __shared__ int s_rb[32], s_first[32];
-  const int tid = threadIdx.x;
-  if (tid < 2) {
-    const int c = tid;
-    if (sort_first) sort_book(sT[c], n);
-    Book& bk = tb.bk[c];
-    int m = 0;
-    for (int j = 0; j < n; j++) {
-      if (m == 0 || !(sT[c][j] == bk.val[m - 1])) {  // -0 == +0: one value
-        bk.val[m] = sT[c][j];
-        bk.idx[m] = j;
-        m++;
+  __shared__ float s_sorted[2][16];
+  __shared__ float s_slot[32];
+  __shared__ int s_src[32];
+  __shared__ int s_cc[2][kMerged];
+  __shared__ int s_A[kNB + 2], s_F[kNB + 2];
+  const int tid = threadIdx.x, lane = tid & 31;
+  const unsigned full = 0xffffffffu;
+  for (int i = tid; i < kNB + 2; i += blockDim.x) {
+    s_A[i] = 0;
+    s_F[i] = 0;
+  }
+  if (tid < 32) {
+    const int c = lane >> 4, j = lane & 15;
+    // 1. sort and distinct values
+    const float v = sT[c][j];
+    if (sort_first) {
+      const uint32_t kv = order_key(v);
+      int rk = 0;
+      for (int i = 0; i < n; i++) {
+        const uint32_t ki = order_key(sT[c][i]);
+        rk += (ki < kv || (ki == kv && i < j)) ? 1 : 0;
       }
+      if (j < n) s_sorted[c][rk] = v;
+    } else if (j < n) {
+      s_sorted[c][j] = v;
     }
-    for (int i = m; i < 16; i++) { bk.val[i] = bk.val[m - 1]; bk.idx[i] = bk.idx[m - 1]; }
-    bk.m = m;
+    __syncwarp();
+    const float w = j < n ? s_sorted[c][j] : 0.0f;
+    if (sort_first && j < n) sT[c][j] = w;
+    const bool distinct = j < n && (j == 0 || !(w == s_sorted[c][j - 1]));
+    const unsigned mine = (__ballot_sync(full, distinct) >> (16 * c)) & 0xffffu;
+    const int m = __popc(mine);
+    Book& bk = tb.bk[c];
+    if (distinct) {
+      const int pos = __popc(mine & ((1u << j) - 1u));
+      bk.val[pos] = w;
+      bk.idx[pos] = j;
+    }
+    __syncwarp();
+    if (j >= m) {
+      bk.val[j] = bk.val[m - 1];
+      bk.idx[j] = bk.idx[m - 1];
+    }
+    if (j == 0) bk.m = m;
+    __syncwarp();
+    bk.thr[j] = (j + 1 < m) ? midpoint_threshold(bk.val[j], bk.val[j + 1]) : kInf;
+    __syncwarp();
+    // 2. merge
+    const int na = tb.bk[0].m - 1, nb = tb.bk[1].m - 1;
+    const bool have = (c == 0) ? (j < na) : (j < nb);
+    if (have) {
+      const float t = bk.thr[j];
+      int slot = j;
+      if (c == 0) {
+        for (int q = 0; q < nb; q++) slot += (tb.bk[1].thr[q] < t) ? 1 : 0;
+      } else {
+        for (int q = 0; q < na; q++) slot += (tb.bk[0].thr[q] <= t) ? 1 : 0;
+      }
+      s_slot[slot] = t;
+      s_src[slot] = c;
+    }
+    __syncwarp();
+    const int ns = na + nb;  // <= 30
+    const bool in = lane < ns;
+    const float t = in ? s_slot[lane] : 0.0f;
+    const bool keep = in && (lane == 0 || !(t == s_slot[lane - 1]));
+    const bool dup_next = in && lane + 1 < ns && t == s_slot[lane + 1];
+    const unsigned kb = __ballot_sync(full, keep);
+    const unsigned from0 = __ballot_sync(full, in && s_src[lane] == 0);
+    const unsigned from1 = __ballot_sync(full, in && s_src[lane] == 1);
+    const int nm = __popc(kb);
+    if (keep) {
+      const int idx = __popc(kb & ((1u << lane) - 1u));
+      const int end = lane + (dup_next ? 1 : 0);  // last slot equal to t
+      const unsigned upto = (end >= 31) ? full : ((2u << end) - 1u);
+      tb.mthr[idx] = t;
+      s_cc[0][idx + 1] = __popc(from0 & upto);
+      s_cc[1][idx + 1] = __popc(from1 & upto);
+    }
+    if (lane == 0) {
+      tb.nm = nm;
+      s_cc[0][0] = 0;
+      s_cc[1][0] = 0;
+    }
+  }
+  __syncthreads();
+  // 3. cells
+  const int nm = tb.nm;
+  for (int m = tid; m < kMerged; m += blockDim.x) {
+    if (m >= nm) tb.mthr[m] = kInf;
+    if (m == (int)kCrowded) {
+      tb.mv0[m] = __int_as_float(0x7fc00000);
+      tb.mv1[m] = __int_as_float(0x7fc00000);
+      tb.moff[m] = 0;
+    } else {
+      const int c0 = m <= nm ? s_cc[0][m] : 0, c1 = m <= nm ? s_cc[1][m] : 0;
+      tb.mv0[m] = tb.bk[0].val[c0];
+      tb.mv1[m] = tb.bk[1].val[c1];
+      tb.moff[m] = (uint32_t)(c0 * kCellBytes) | ((uint32_t)((16 + c1) * kCellBytes) << 16);
+    }
+  }
+  // 4. bucket table
+  if (tid < nm) {
+    const float th = tb.mthr[tid];
+    const int rb = bucket_raw(th, tb.la);                                  // -1 .. kNB
+    const bool first = bucket_raw(nextafterf(th, -kInf), tb.la) < rb;     // th opens its bucket
+    atomicAdd(&s_A[rb + 1], 1);
+    if (first) atomicAdd(&s_F[rb + 1], 1);
   }
   __syncthreads();
   if (tid < 32) {
-    Book& bk = tb.bk[tid >> 4];
-    const int i = tid & 15;
-    bk.thr[i] = (i + 1 < bk.m) ? midpoint_threshold(bk.val[i], bk.val[i + 1]) : kInf;
-  }
-  __syncthreads();
-  if (tid == 0) merge_thresholds(tb);
-  __syncthreads();
-  if (tid < tb.nm) {
-    const float th = tb.mthr[tid];
-    const int rb = bucket_raw(th, tb.la);
-    s_rb[tid] = rb;
-    s_first[tid] = bucket_raw(nextafterf(th, -kInf), tb.la) < rb;  // th opens its bucket
-  }
-  __syncthreads();
-  for (int m = tid; m < kMerged; m += blockDim.x) merged_cell(tb, m);
-  for (int b = tid; b < kNB; b += blockDim.x) {
-    int base = 0, inner = 0;
-    for (int i = 0; i < tb.nm; i++) {
-      const int rb = s_rb[i];
-      if (rb < b || (rb == b && s_first[i])) base++;
-      else if (rb == b) inner++;
+    // exclusive prefix P[k] = sum of A[k' < k], 5 entries per lane
+    int v[5], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 5; i++) {
+      const int k = lane * 5 + i;
+      v[i] = k < kNB + 2 ? s_A[k] : 0;
+      sum += v[i];
     }
-    tb.mlut[b] = (uint8_t)(inner > 1 ? kCrowded : base);
+    int incl = sum;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(full, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 5; i++) {
+      const int k = lane * 5 + i;  // k = b + 1 for bucket b
+      if (k >= 1 && k <= kNB) {
+        const int base = run + s_F[k];
+        const int inner = v[i] - s_F[k];
+        tb.mlut[k - 1] = (uint8_t)(inner > 1 ? kCrowded : base);
+      }
+      run += v[i];
+    }
   }
   __syncthreads();
 }
@@ -413,7 +480,16 @@ __device__ void round_finalize(FitCtl* ctl, Tables& tb, const double* errp, int 
   __shared__ int s_upd[2];
   const int tid = threadIdx.x;
   double part = 0.0;
-  for (int b = tid; b < nb; b += blockDim.x) part = __dadd_rn(part, __ldcg(errp + b));
+  for (int b0 = tid; b0 < nb; b0 += 8 * (int)blockDim.x) {  // 8 loads in flight per thread
+    double v[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      const int b = b0 + k * (int)blockDim.x;
+      v[k] = b < nb ? __ldcg(errp + b) : 0.0;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; k++) part = __dadd_rn(part, v[k]);
+  }
   sred[tid] = part;
   if (tid < 64) sb[tid] = __ldcg(&ctl->bins[0][0][0] + tid);
   if (tid < 32) sT[tid >> 4][tid & 15] = ctl->T[tid >> 4][tid & 15];

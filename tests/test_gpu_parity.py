@@ -185,6 +185,30 @@ def test_flags_rtn_single_frozen(flags):
         assert not out["choice_bits"].any()
 
 
+def test_crowded_buckets_duplicates_and_signed_zeros():
+    """Codebooks with entries 0.02 apart (several midpoint thresholds inside
+    one lookup bucket: the exact binary search takes over), equal entries
+    (one cell), and -0 / +0 (equal values, one cell)."""
+    N, K, g = 96, 512, 128
+    W, X = layer(N, K, seed=97)
+    cfg = cfg_of(bb.INT4, g, 16, 2)
+    I = bb.importance(X)
+    scl, _ = bb.init_codebooks(W, cfg)
+    b0 = [-3, -2, -1, 0.50, 0.52, 0.54, 0.56, 1, 2, 3, 4, 5, 6, -4, -5, 7]
+    b1 = [-7.5, -6.5, -0.0, 0.0, 0.031, 0.033, 0.035, 1.5, 1.5, 2.5, 3.5, 4.5, 5.5, 6.5, -1.5, -2.5]
+    T0 = torch.tensor([b0, b1], dtype=torch.float32).cuda()
+    for iters in (1, 2):
+        c = cfg_of(bb.INT4, g, 16, iters)
+        T, eh, st = bb.fit_layer(W, I, scl, T0.clone(), c)
+        Wb, Ib, sb = u16(W), I.cpu().numpy(), scl.cpu().numpy()
+        rT, reh, rst = oracle.fit(Wb, Ib, sb, T0.cpu().numpy(), bb.INT4, g, 16, iters)
+        assert np.array_equal(npbits(T), rT.view(np.uint32))
+    out = bb.pack(W, I, scl, T0, cfg)
+    rp = oracle.pack(u16(W), I.cpu().numpy(), scl.cpu().numpy(), T0.cpu().numpy(), bb.INT4, g, 16)
+    assert np.array_equal(out["codes"].cpu().numpy(), rp["codes"])
+    assert np.array_equal(out["choice_bits"].cpu().numpy(), rp["choice_bits"])
+
+
 def test_deterministic_bits():
     W, X = layer(512, 1024, seed=95)
     cfg = cfg_of(bb.INT4, 128, 16, 8)
