@@ -52,6 +52,8 @@ constexpr int kFitThreads = kFitWarps * 32;
 constexpr int kStages = 3;                // rows per warp in flight
 constexpr int kFitBlocksPerSM = 5;
 constexpr int kLaneCols = 16;             // columns per lane
+constexpr int kItemRows = 4;              // rows of one work item
+constexpr int kMaxStrips = 256;           // per-strip work counters (more strips: one counter)
 constexpr int kWarpCols = 32 * kLaneCols; // columns per warp (one row segment)
 constexpr int kRingRowBytes = kWarpCols * 2;
 constexpr int kCellBytes = 32 * 16;       // one (book, entry) row of a warp's bins
@@ -94,30 +96,46 @@ struct FitCtl {
   unsigned long long exact_groups;
   unsigned long long empty_cells;
   unsigned int ticket;
-  int32_t pad2;
+  unsigned int next_item;  // work-item counter of the running pass (many strips)
+  unsigned int strip_next[kMaxStrips];  // per-strip item counters of the running pass
+  double twoLe;            // fixed-point scale of the objective sums
+  unsigned long long err_acc;  // sum of rint(s^2 D 2^Le) of the running pass
 };
 
 size_t fit_ctl_bytes() { return align256(sizeof(FitCtl)); }
 
-// One wave of 512-column strips x row chunks; rows per warp are capped so a
-// lane's refine partials (16 terms a row, each below 2^B) stay below 2^50.
-static PassPlan fit_plan(int64_t N, int64_t K) {
-  PassPlan pp = plan_pass(N, K, 148 * kFitBlocksPerSM, kWarpCols);
+// Work items: kItemRows rows of one 512-column strip; warps claim them from
+// a global counter.  A lane's refine partial over its rows (16 terms a row,
+// each below 2^B) must stay below 2^50, which caps the items a warp may
+// claim; the grid is one wave, or more when the caps need more warps.
+struct FitPlan {
+  int ncb, cpc, items, max_items, blocks;
+};
+
+static FitPlan fit_plan(int64_t N, int64_t K) {
+  FitPlan p;
+  p.ncb = (int)((K + kWarpCols - 1) / kWarpCols);
+  p.cpc = (int)((N + kItemRows - 1) / kItemRows);
+  p.items = p.ncb * p.cpc;
   int c = 0;
   while (((int64_t)1 << c) < N * K) c++;
   const int Bmax = (61 - c) < 40 ? (61 - c) : 40;
-  const int64_t max_rows = ((int64_t)1 << (50 - Bmax)) / kLaneCols * kFitWarps;
-  if (pp.rows_per_chunk > max_rows) {
-    pp.rows_per_chunk = (int)max_rows;
-    pp.nrc = (int)((N + max_rows - 1) / max_rows);
-    pp.blocks = pp.ncb * pp.nrc;
-  }
-  return pp;
+  const int64_t cap_rows = ((int64_t)1 << (50 - Bmax)) / kLaneCols;  // >= 64
+  p.max_items = (int)(cap_rows / kItemRows);
+  const int64_t per_block = (int64_t)kFitWarps * p.max_items;
+  const int64_t need = (p.items + per_block - 1) / per_block;
+  const int64_t useful = (p.items + kFitWarps - 1) / kFitWarps;
+  int64_t blocks = 148 * kFitBlocksPerSM;
+  if (blocks > useful) blocks = useful;
+  if (blocks < need) blocks = need;
+  p.blocks = (int)blocks;
+  return p;
 }
 
 size_t fit_ws_bytes(int64_t N, int64_t K) {
-  const PassPlan pp = fit_plan(N, K);
-  return fit_ctl_bytes() + align256((size_t)pp.blocks * sizeof(double));
+  (void)N;
+  (void)K;
+  return fit_ctl_bytes();  // the control block: work counter, sums, tables
 }
 
 size_t pack_extra_bytes(int64_t N, int64_t K, int S) {
@@ -364,6 +382,23 @@ __device__ inline int frexp_exponent(double x) {
   return e;
 }
 
+// 2^Le for the objective sums: every contribution is a group's s^2 D (or a
+// row's weight-space error), rounded to an integer after scaling by 2^Le.
+// Both are below M * I_max * S2_max * (2 U_max)^2 in total (|u - T| <= 2 U_max,
+// |w - s T| <= 2 sqrt(S2_max) U_max), and Le keeps that bound below 2^61, so
+// the int64 sums cannot overflow and do not depend on the order of addition.
+__device__ double objective_scale(const FitCtl* ctl, int64_t M) {
+  const double Imax = (double)__uint_as_float(ctl->Imax_bits);
+  const double S2max = __longlong_as_double((long long)ctl->S2max_bits);
+  const double Umax = (double)__uint_as_float(ctl->Umax_bits);
+  const double bound = (double)M * Imax * S2max * 4.0 * Umax * Umax;
+  if (!(bound > 0.0)) return 1.0;
+  int Le = 61 - frexp_exponent(bound);
+  if (Le > 1000) Le = 1000;
+  if (Le < -1000) Le = -1000;
+  return ldexp(1.0, Le);
+}
+
 __device__ void write_stats(const FitCtl* ctl, aaac_stats* st) {
   if (!st) return;
   st->near_ties = (int64_t)ctl->near_ties;
@@ -400,6 +435,8 @@ fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st) {
     }
     ctl->L = L;
     ctl->twoL = ldexp(1.0, L);
+    ctl->twoLe = objective_scale(ctl, M);
+    ctl->err_acc = 0ull;
     ctl->n = n;
     tb.la = bucket_scale(ctl);
   }
@@ -473,33 +510,20 @@ __device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsign
 // the integer sums (section 2, core mechanism 4), T = fp32(fp64(num) /
 // fp64(den)) when den > 0, else unchanged; then sorted books and new tables.
 // Everything is staged in shared memory and spread over the block's threads.
-__device__ void round_finalize(FitCtl* ctl, Tables& tb, const double* errp, int nb,
-                               uint32_t flags, const RoundOut& ro, double* sred) {
+__device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const RoundOut& ro) {
   __shared__ float sT[2][16];
   __shared__ long long sb[64];
   __shared__ int s_upd[2];
   const int tid = threadIdx.x;
-  double part = 0.0;
-  for (int b0 = tid; b0 < nb; b0 += 8 * (int)blockDim.x) {  // 8 loads in flight per thread
-    double v[8];
-#pragma unroll
-    for (int k = 0; k < 8; k++) {
-      const int b = b0 + k * (int)blockDim.x;
-      v[k] = b < nb ? __ldcg(errp + b) : 0.0;
-    }
-#pragma unroll
-    for (int k = 0; k < 8; k++) part = __dadd_rn(part, v[k]);
-  }
-  sred[tid] = part;
   if (tid < 64) sb[tid] = __ldcg(&ctl->bins[0][0][0] + tid);
   if (tid < 32) sT[tid >> 4][tid & 15] = ctl->T[tid >> 4][tid & 15];
   if (tid < 2) s_upd[tid] = 0;
-  __syncthreads();
   if (tid == 0) {
-    double e = 0.0;
-    for (int i = 0; i < (int)blockDim.x; i++) e = __dadd_rn(e, sred[i]);
-    if (ro.err_hist) ro.err_hist[ro.it] = e;
+    const long long acc = (long long)__ldcg(&ctl->err_acc);
+    if (ro.err_hist) ro.err_hist[ro.it] = (double)acc / ctl->twoLe;
+    ctl->err_acc = 0ull;
   }
+  __syncthreads();
   const int n = ctl->n;
   if (tid < 32) {
     const int c = tid >> 4, j = tid & 15;
@@ -538,8 +562,10 @@ __device__ void round_finalize(FitCtl* ctl, Tables& tb, const double* errp, int 
     }
     ctl->near_ties = 0;
     ctl->groups_t1 = 0;
+    ctl->next_item = 0;
     ctl->ticket = 0;
   }
+  for (int i = tid; i < kMaxStrips; i += blockDim.x) ctl->strip_next[i] = 0u;
 }
 
 // Chunk j (16 bytes) of a warp's 1 KB row segment sits at ring slot j ^ bit 3
@@ -598,20 +624,24 @@ __device__ __forceinline__ int fast_choice(float d0, float d1, float tau, bool* 
 
 struct GroupStats {
   unsigned int near, exact, t1;
-  double err;
+  unsigned long long err;  // sum of rint(contribution * 2^Le), modulo 2^64
 };
 
-// Counters of one live group: near ties, exact decisions, T1 groups, s^2 D.
+// Counters of one live group: near ties, exact decisions, T1 groups, and
+// its objective s^2 D in fixed point (scale twoLe).
 __device__ __forceinline__ void count_group(GroupStats& gs, bool exact, double E0, double E1,
-                                            float d0, float d1, int ch, bool single, float s) {
+                                            float d0, float d1, int ch, bool single, float s,
+                                            double twoLe) {
+  double e;
   if (exact) {
     gs.exact++;
     if (fabs(E1 - E0) < 1e-6 * fmax(E0, E1)) gs.near++;
-    gs.err += (double)(s * s) * (ch ? E1 : E0);  // s*s exact in fp32
+    e = (double)(s * s) * (ch ? E1 : E0);  // s*s exact in fp32
   } else {
     if (!single && fabsf(d1 - d0) < 1e-6f * fmaxf(d0, d1)) gs.near++;
-    gs.err += (double)(s * s) * (double)(ch ? d1 : d0);
+    e = (double)(s * s) * (double)(ch ? d1 : d0);
   }
+  gs.err += (unsigned long long)__double2ll_rn(e * twoLe);
   gs.t1 += ch;
 }
 
@@ -619,13 +649,12 @@ template <int FMT, bool PACK>
 __global__ void __launch_bounds__(kFitThreads, kFitBlocksPerSM)
 fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
          const void* __restrict__ scales, int g, int S, uint32_t flags, FitCtl* ctl,
-         double* __restrict__ errp, int ncb, int rows_per_chunk, float tau, PackOut po,
+         int cpc, int n_items, int max_items, float tau, PackOut po,
          RoundOut ro) {
   extern __shared__ __align__(128) unsigned char smem[];
   Tables& tb = *reinterpret_cast<Tables*>(smem);
   unsigned char* ring = smem + kTablesBytes;
   unsigned char* bins = ring + kFitWarps * kStages * kRingRowBytes;
-  __shared__ double sred[kFitThreads];
   __shared__ int s_last;
 
   {
@@ -639,13 +668,11 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     }
   }
   const double twoL = ctl->twoL;
+  const double twoLe = ctl->twoLe;
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cb = blockIdx.x % ncb, rc = blockIdx.x / ncb;
-  const int seg = cb * kWarpCols;           // first column of the warp's row segment
-  const int col0 = seg + lane * kLaneCols;  // first of this lane's 16 columns
-  const bool active = col0 < K;
+  const unsigned full = 0xffffffffu;
   const int G = K / g, KS = K / S;
   const int lanes_s = S >> 4;               // lanes per choice group when S >= 16
   const int leader_lane = S >= 16 ? (lane & ~(lanes_s - 1)) : lane;
@@ -654,72 +681,156 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   unsigned char* wring = ring + warp * kStages * kRingRowBytes;
   const int wr0 = ring_slot(lane) * 16, wr1 = ring_slot(32 + lane) * 16;
   const int rd0 = ring_slot(2 * lane) * 16, rd1 = ring_slot(2 * lane + 1) * 16;
-  const bool cp0 = seg + lane * 8 < K, cp1 = seg + 256 + lane * 8 < K;
   unsigned char* mybins = bins + warp * kWarpBinBytes + lane * 16;
 
-  // importance of the lane's columns: fp32 pairs (choice) and fp64 (refine)
-  unsigned long long I2[8];
-  double Id[16];
-  {
-    float Iv[16];
-#pragma unroll
-    for (int q = 0; q < 4; q++) {
-      const float4 a = active ? __ldg(reinterpret_cast<const float4*>(I + col0) + q)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-      Iv[4 * q] = a.x; Iv[4 * q + 1] = a.y; Iv[4 * q + 2] = a.z; Iv[4 * q + 3] = a.w;
+  // ---- the warp's rows: work items (kItemRows rows of one 512-column strip)
+  // claimed from a global counter, one claim in flight ahead of its use, in a
+  // small FIFO that the W prefetch fills and the row loop drains.
+  __shared__ int s_fifo[kFitWarps][8];
+  int* fifo = s_fifo[warp];
+  // Strips: each warp starts on its home strip and moves to the next strip
+  // when one runs dry (per-strip counters keep a warp on one strip, so its
+  // importance registers rarely change); with more than kMaxStrips strips a
+  // single counter hands out items in order.
+  const int ncb = n_items / cpc;
+  const bool per_strip = ncb <= kMaxStrips;
+  int cur_strip = (int)((blockIdx.x * kFitWarps + warp) % (unsigned)ncb), tried = 0;
+  unsigned pend = 0u;
+  bool pend_ok = false, no_more = false;
+  int claimed = 0, tail = 0;
+  auto claim = [&]() {  // warp-uniform: start one claim
+    pend_ok = !no_more && claimed < max_items;
+    if (pend_ok) {
+      if (lane == 0)
+        pend = per_strip ? atomicAdd(&ctl->strip_next[cur_strip], 1u) : atomicAdd(&ctl->next_item, 1u);
+      claimed++;
     }
-#pragma unroll
-    for (int p = 0; p < 8; p++) I2[p] = f2pack(Iv[2 * p], Iv[2 * p + 1]);
-#pragma unroll
-    for (int i = 0; i < 16; i++) Id[i] = (double)Iv[i];
-  }
+  };
+  auto land_push = [&]() {  // the pending claim's item (or -1) into the FIFO, next claim
+    int it = -1;
+    while (pend_ok) {
+      const int v = __shfl_sync(full, (int)pend, 0);
+      if (!per_strip) {
+        if (v < n_items) it = v;
+        break;
+      }
+      if (v < cpc) {
+        it = cur_strip * cpc + v;
+        break;
+      }
+      claimed--;  // this strip has run dry: try the next one
+      if (++tried >= ncb) break;
+      cur_strip = cur_strip + 1 == ncb ? 0 : cur_strip + 1;
+      claim();
+    }
+    if (it < 0) no_more = true;
+    if (lane == 0) fifo[tail & 7] = it;
+    tail++;
+    __syncwarp();
+    claim();
+  };
+  claim();
+  land_push();
 
-  const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
-  const uint16_t* wseg = W + seg;
-  // ring prologue: each lane copies chunks lane and 32 + lane of the segment
-#pragma unroll
-  for (int k = 0; k < kStages; k++) {
-    const int rr = r0 + warp + kFitWarps * k;
-    if (rr < r1) {
-      const uint16_t* src = wseg + (int64_t)rr * K + lane * 8;
-      if (cp0) cp_async16(wring + k * kRingRowBytes + wr0, src);
-      if (cp1) cp_async16(wring + k * kRingRowBytes + wr1, src + 256);
+  // prefetch cursor: FIFO position pq, next row pr and end pe of that item,
+  // and the item's strip values (set when the cursor enters the item)
+  int pq = 0, pr = 0, pe = 0, pgi = 0;
+  const uint16_t* psrc = W;
+  bool pc0 = false, pc1 = false, pact = false;
+  auto enter = [&](int it) {
+    if (it < 0) return;
+    const int pseg = (it / cpc) * kWarpCols;
+    pr = (it % cpc) * kItemRows;
+    pe = min(N, pr + kItemRows);
+    psrc = W + pseg + lane * 8;
+    pc0 = pseg + lane * 8 < K;
+    pc1 = pseg + 256 + lane * 8 < K;
+    const int pcol0 = pseg + lane * kLaneCols;
+    pact = pcol0 < K;
+    pgi = pact ? pcol0 / g : 0;
+  };
+  enter(fifo[0]);
+  float sq0 = 0.0f, sq1 = 0.0f, sq2 = 0.0f;  // scales of the rows in flight
+  // issue the row at the prefetch cursor into ring slot ps; returns its scale
+  auto prefetch = [&](int ps) -> float {
+    float sc = 0.0f;
+    if (fifo[pq & 7] >= 0) {
+      const uint16_t* src = psrc + (int64_t)pr * K;
+      if (pc0) cp_async16(wring + ps * kRingRowBytes + wr0, src);
+      if (pc1) cp_async16(wring + ps * kRingRowBytes + wr1, src + 256);
+      if (pact) sc = load_scale<FMT>(scales, (int64_t)pr * G + pgi);
+      if (++pr >= pe) {
+        pq++;
+        if (pq == tail) land_push();
+        enter(fifo[pq & 7]);
+      }
     }
     cp_async_commit();
-  }
-  // scales prefetched two rows ahead
-  float s_next = 0.0f, s_next2 = 0.0f;
-  if (active && r0 + warp < r1) s_next = load_scale<FMT>(scales, (int64_t)(r0 + warp) * G + col0 / g);
-  if (active && r0 + warp + kFitWarps < r1)
-    s_next2 = load_scale<FMT>(scales, (int64_t)(r0 + warp + kFitWarps) * G + col0 / g);
+    return sc;
+  };
+  sq0 = prefetch(0);
+  sq1 = prefetch(1);
+  sq2 = prefetch(2);
 
-  GroupStats gs{0u, 0u, 0u, 0.0};
-  double err_w = 0.0;  // pack: weight-space error
+  // consumer cursor: FIFO position cq, row cr, item end ce, strip ccb; and
+  // the strip whose importance is loaded
+  int cq = 0, cr = 0, ce = 0, ccb = 0;
+  auto centre = [&](int it) {
+    if (it < 0) return;
+    ccb = it / cpc;
+    cr = (it % cpc) * kItemRows;
+    ce = min(N, cr + kItemRows);
+  };
+  centre(fifo[0]);
+  int cur_cb = -1, col0 = 0;
+  bool active = false;
+  unsigned long long I2[8];
+  double Id[16];
+#pragma unroll
+  for (int p = 0; p < 8; p++) I2[p] = 0ull;
+#pragma unroll
+  for (int i = 0; i < 16; i++) Id[i] = 0.0;
+
+  GroupStats gs{0u, 0u, 0u, 0ull};
   int slot = 0;
   const unsigned long long la2 = f2pack(la, la);
   const unsigned long long cc2 = f2pack(kBucketMagic + (float)(kNB / 2), kBucketMagic + (float)(kNB / 2));
-  for (int r = r0 + warp; r < r1; r += kFitWarps) {  // warp-uniform trip count
+  while (true) {  // warp-uniform
+    if (fifo[cq & 7] < 0) break;
+    const int r = cr;
+    const int cb = ccb;
+    if (cb != cur_cb) {  // importance of the lane's columns: fp32 pairs and fp64
+      cur_cb = cb;
+      col0 = cb * kWarpCols + lane * kLaneCols;
+      active = col0 < K;
+      float Iv[16];
+#pragma unroll
+      for (int q = 0; q < 4; q++) {
+        const float4 a = active ? __ldg(reinterpret_cast<const float4*>(I + col0) + q)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        Iv[4 * q] = a.x; Iv[4 * q + 1] = a.y; Iv[4 * q + 2] = a.z; Iv[4 * q + 3] = a.w;
+      }
+#pragma unroll
+      for (int p = 0; p < 8; p++) I2[p] = f2pack(Iv[2 * p], Iv[2 * p + 1]);
+#pragma unroll
+      for (int i = 0; i < 16; i++) Id[i] = (double)Iv[i];
+    }
+    if (++cr >= ce) {
+      cq++;
+      centre(fifo[cq & 7]);  // already pushed: the prefetch runs ahead
+    }
     cp_async_wait<kStages - 1>();
     __syncwarp();  // the row's chunks were copied by other lanes
     const unsigned char* srow = wring + slot * kRingRowBytes;
     const uint4 va = *reinterpret_cast<const uint4*>(srow + rd0);
     const uint4 vb = *reinterpret_cast<const uint4*>(srow + rd1);
     __syncwarp();  // every lane has read the slot before it is refilled
-    {
-      const int rr = r + kFitWarps * kStages;
-      if (rr < r1) {
-        const uint16_t* src = wseg + (int64_t)rr * K + lane * 8;
-        if (cp0) cp_async16(wring + slot * kRingRowBytes + wr0, src);
-        if (cp1) cp_async16(wring + slot * kRingRowBytes + wr1, src + 256);
-      }
-      cp_async_commit();
-    }
+    const float s = sq0;
+    sq0 = sq1;
+    sq1 = sq2;
+    sq2 = prefetch(slot);  // the row kStages positions ahead into this slot
     slot = (slot + 1 == kStages) ? 0 : slot + 1;
 
-    const float s = s_next;
-    s_next = s_next2;
-    if (active && r + 2 * kFitWarps < r1)
-      s_next2 = load_scale<FMT>(scales, (int64_t)(r + 2 * kFitWarps) * G + col0 / g);
     float rcp;
     const bool live = active && scale_live(s, &rcp);  // dead: rcp = 0, u = +-0
     const uint32_t wv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
@@ -814,10 +925,10 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     }
     if (live) {
       if (S == 8) {
-        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], single, s);
-        count_group(gs, ex[1], E0[1], E1[1], g0[1], g1[1], ch[1], single, s);
+        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], single, s, PACK ? 0.0 : twoLe);
+        count_group(gs, ex[1], E0[1], E1[1], g0[1], g1[1], ch[1], single, s, PACK ? 0.0 : twoLe);
       } else if (lane == leader_lane) {
-        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], single, s);
+        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], single, s, PACK ? 0.0 : twoLe);
       }
     }
     const uint32_t sel0 = ch[0] ? 0x4432u : 0x4410u;  // book-1 or book-0 half of moff
@@ -845,6 +956,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
         }
       }
     } else if (active) {
+      double err_w = 0.0;  // weight-space error of this row's 16 weights
       unsigned long long packed = 0ull;
 #pragma unroll
       for (int i = 0; i < 16; i++) {
@@ -858,6 +970,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
         const double d = __dsub_rn((double)wf, wh);
         err_w = __fma_rn(Id[i], __dmul_rn(d, d), err_w);
       }
+      gs.err += (unsigned long long)__double2ll_rn(err_w * twoLe);
       *reinterpret_cast<unsigned long long*>(po.codes + ((int64_t)r * K + col0) / 2) = packed;
       if ((lane & ((g >> 4) - 1)) == 0) {
         const int64_t gi = (int64_t)r * G + col0 / g;
@@ -893,13 +1006,10 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     if (gs.exact) atomicAdd(&ctl->exact_groups, (unsigned long long)gs.exact);
     if (gs.t1) atomicAdd(&ctl->groups_t1, (unsigned long long)gs.t1);
   }
-  sred[threadIdx.x] = PACK ? err_w : gs.err;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double t = 0.0;
-    for (int i = 0; i < kFitThreads; i++) t = __dadd_rn(t, sred[i]);
-    errp[blockIdx.x] = t;
-  }
+  // objective: integer sums, the same whatever the order
+  for (int o = 16; o > 0; o >>= 1) gs.err += __shfl_xor_sync(0xffffffffu, gs.err, o);
+  if (lane == 0 && gs.err) atomicAdd(&ctl->err_acc, gs.err);
+  __syncthreads();  // every lane's bins are complete
   if (!PACK) {
     // lane bins -> exact integer partials (bias removed exactly), one
     // (book, entry, num | den) per thread, summed over the block's lanes
@@ -923,20 +1033,16 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   if (!s_last) return;
   __threadfence();
   if (!PACK) {
-    round_finalize(ctl, tb, errp, gridDim.x, flags, ro, sred);
+    round_finalize(ctl, tb, flags, ro);
   } else {
-    double part = 0.0;
-    for (int b = threadIdx.x; b < (int)gridDim.x; b += blockDim.x)
-      part = __dadd_rn(part, __ldcg(errp + b));
-    __syncthreads();
-    sred[threadIdx.x] = part;
-    __syncthreads();
     if (threadIdx.x == 0) {
-      double e = 0.0;
-      for (int i = 0; i < kFitThreads; i++) e = __dadd_rn(e, sred[i]);
-      if (po.err_final) *po.err_final = e;
+      const long long acc = (long long)__ldcg(&ctl->err_acc);
+      if (po.err_final) *po.err_final = (double)acc / ctl->twoLe;
+      ctl->err_acc = 0ull;
+      ctl->next_item = 0;
       ctl->ticket = 0;
     }
+    for (int i = threadIdx.x; i < kMaxStrips; i += blockDim.x) ctl->strip_next[i] = 0u;
   }
 }
 
@@ -960,10 +1066,9 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
   // per call: the attribute belongs to the current device's copy of the kernel
   const cudaError_t attr = set_smem<FMT, false>();
   if (attr != cudaSuccess) return attr;
-  const PassPlan pp = fit_plan(N, K);
+  const FitPlan pp = fit_plan(N, K);
   const PassPlan pprep = plan_pass(N, K);
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
-  double* errp = reinterpret_cast<double*>(reinterpret_cast<char*>(ws) + fit_ctl_bytes());
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
                                                    pprep.ncb, pprep.rows_per_chunk);
@@ -971,7 +1076,7 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
   const float tau = choice_tau(S);
   for (int it = 0; it < iters; it++) {
     fit_pass<FMT, false><<<pp.blocks, kFitThreads, smem_bytes(false), st>>>(
-        W, (int)N, (int)K, I, scales, g, S, flags, ctl, errp, pp.ncb, pp.rows_per_chunk, tau,
+        W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items, tau,
         PackOut{nullptr, nullptr, nullptr, nullptr}, RoundOut{err_hist, T, stats, it});
   }
   count_launches(2 + iters);
@@ -1027,11 +1132,13 @@ cudaError_t fixed_scratch_ptr(void** out) {
 // pack
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kFitThreads)
-pack_setup(FitCtl* ctl, const float* T_user, int n, uint16_t* T_bf16) {
+pack_setup(FitCtl* ctl, const float* T_user, int64_t M, int n, uint16_t* T_bf16) {
   __shared__ Tables tb;
   __shared__ float sT[2][16];
   if (threadIdx.x == 0) {
     ctl->n = n;
+    ctl->twoLe = objective_scale(ctl, M);
+    ctl->err_acc = 0ull;
     tb.la = bucket_scale(ctl);
   }
   if (threadIdx.x < 32) sT[threadIdx.x >> 4][threadIdx.x & 15] = T_user[threadIdx.x];
@@ -1070,19 +1177,18 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
                                  cudaStream_t st) {
   const cudaError_t attr = set_smem<FMT, true>();
   if (attr != cudaSuccess) return attr;
-  const PassPlan pp = fit_plan(N, K);
+  const FitPlan pp = fit_plan(N, K);
   const PassPlan pprep = plan_pass(N, K);
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
-  double* errp = reinterpret_cast<double*>(reinterpret_cast<char*>(ws) + fit_ctl_bytes());
   uint8_t* cbytes = reinterpret_cast<uint8_t*>(ws) + fit_ws_bytes(N, K);
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
                                                    pprep.ncb, pprep.rows_per_chunk);
-  pack_setup<<<1, kFitThreads, 0, st>>>(ctl, T, ncodes(FMT), T_bf16);
+  pack_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), T_bf16);
   const float tau = choice_tau(S);
   const PackOut po{codes, scales_tagged, cbytes, err_final};
   fit_pass<FMT, true><<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
-      W, (int)N, (int)K, I, scales, g, S, flags, ctl, errp, pp.ncb, pp.rows_per_chunk, tau, po,
+      W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items, tau, po,
       RoundOut{nullptr, nullptr, nullptr, 0});
   int launches = 3;
   if (S != g) {

@@ -142,10 +142,11 @@ aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
  * for integration only.
  *   Arguments and results are those of aaac_fit_layer, without ws/ws_bytes.
  *   Scratch: a 256 KiB array inside the library (every GPU that loads the
- *   library holds it until the process exits).  Layers whose scratch need,
- *   aaac_workspace_size's fit share, exceeds it are rejected with
- *   AAAC_ERR_WORKSPACE before anything is launched (in practice only layers
- *   with K above about 8 million).
+ *   library holds it until the process exits).  The fit's scratch is its
+ *   control block (a few KB, the same for every layer), so every layer that
+ *   passes the shape checks (N*K < 2^31, rejected with AAAC_ERR_SHAPE before
+ *   anything is launched) fits; a scratch need above the array would be
+ *   rejected with AAAC_ERR_WORKSPACE, also before any launch.
  *   The first call on a device looks up the array's device address with that
  *   device current; make that first call before any stream capture.
  *   All calls share the one array and it keeps the previous call's contents

@@ -46,11 +46,13 @@ def test_fixed_scratch_matches_workspace_fit(fmt, g, S):
         assert bb.decode_stats(st) == ref_stats
 
 
-def test_fixed_scratch_rejects_oversized_layer():
+def test_fixed_scratch_rejects_layers_past_the_size_limit():
+    """Layers with N*K >= 2^31 are rejected before anything is launched (the
+    pointers below are never dereferenced: the shape check fails first)."""
     lib = bb.load()
     cfg = bb.Config(bb.INT4, 128, 128, 1).c()
-    fake = ctypes.c_void_p(1 << 20)  # never touched: the size check fails first
-    st = lib.aaac_fit_layer_fixed_scratch(fake, 1, 1 << 30, fake, fake, ctypes.byref(cfg), fake,
-                                          None, None, None)
-    assert st == 6  # AAAC_ERR_WORKSPACE
-    assert b"fixed scratch" in lib.aaac_last_error()
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.aaac_fit_layer_fixed_scratch(fake, 1 << 20, 4096, fake, fake, ctypes.byref(cfg),
+                                          fake, None, None, None)
+    assert st == 2  # AAAC_ERR_SHAPE
+    assert b"2^31" in lib.aaac_last_error()
