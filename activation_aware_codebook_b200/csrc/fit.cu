@@ -148,6 +148,19 @@ static size_t smem_bytes(bool pack) {
   return b;
 }
 
+// Claim counters for a pass of wt warps: warp g first takes chunk g / ncb of
+// strip g % ncb without a claim (so it can start before the previous round
+// has finished); the counters start past those chunks.
+__device__ void seed_claims(FitCtl* ctl, int wt, int cpc, int n_items) {
+  const int ncb = n_items / cpc;
+  for (int i = threadIdx.x; i < kMaxStrips; i += blockDim.x) {
+    unsigned v = 0u;
+    if (i < ncb && i < wt) v = (unsigned)min((wt - i + ncb - 1) / ncb, cpc);
+    ctl->strip_next[i] = v;
+  }
+  if (threadIdx.x == 0) ctl->next_item = (unsigned)min(wt, n_items);
+}
+
 // ---------------------------------------------------------------------------
 // buckets and tables
 // ---------------------------------------------------------------------------
@@ -417,8 +430,10 @@ __device__ float bucket_scale(const FitCtl* ctl) {
 
 // L = B - E(I_max) - E(S2_max) - max(0, E(U_max)), B = min(40, 61 - ceil(log2 M))
 __global__ void __launch_bounds__(kFitThreads)
-fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st) {
+fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st, int wt, int cpc,
+          int n_items) {
   __shared__ Tables tb;
+  seed_claims(ctl, wt, cpc, n_items);
   if (threadIdx.x == 0) {
     int c = 0;
     while (((int64_t)1 << c) < M) c++;
@@ -510,7 +525,8 @@ __device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsign
 // the integer sums (section 2, core mechanism 4), T = fp32(fp64(num) /
 // fp64(den)) when den > 0, else unchanged; then sorted books and new tables.
 // Everything is staged in shared memory and spread over the block's threads.
-__device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const RoundOut& ro) {
+__device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const RoundOut& ro,
+                               int cpc, int n_items) {
   __shared__ float sT[2][16];
   __shared__ long long sb[64];
   __shared__ int s_upd[2];
@@ -562,10 +578,9 @@ __device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const Ro
     }
     ctl->near_ties = 0;
     ctl->groups_t1 = 0;
-    ctl->next_item = 0;
     ctl->ticket = 0;
   }
-  for (int i = tid; i < kMaxStrips; i += blockDim.x) ctl->strip_next[i] = 0u;
+  seed_claims(ctl, (int)gridDim.x * kFitWarps, cpc, n_items);
 }
 
 // Chunk j (16 bytes) of a warp's 1 KB row segment sits at ring slot j ^ bit 3
@@ -657,47 +672,50 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   unsigned char* bins = ring + kFitWarps * kStages * kRingRowBytes;
   __shared__ int s_last;
 
-  {
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(&ctl->tb);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(&tb);
-    for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
-    if (!PACK) {
-      double2* b = reinterpret_cast<double2*>(bins);
-      for (int i = threadIdx.x; i < kFitWarps * kWarpBinBytes / 16; i += blockDim.x)
-        b[i] = make_double2(kNumBias, kDenBias);
-    }
+  // ---- up to the dependency wait nothing is read that the previous round
+  // writes (W, I and the scales do not change between rounds), so this part
+  // can run while the previous round's last block is still finishing.
+  if (!PACK) {
+    double2* b = reinterpret_cast<double2*>(bins);
+    for (int i = threadIdx.x; i < kFitWarps * kWarpBinBytes / 16; i += blockDim.x)
+      b[i] = make_double2(kNumBias, kDenBias);
   }
-  const double twoL = ctl->twoL;
-  const double twoLe = ctl->twoLe;
-  __syncthreads();
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned full = 0xffffffffu;
   const int G = K / g, KS = K / S;
   const int lanes_s = S >> 4;               // lanes per choice group when S >= 16
   const int leader_lane = S >= 16 ? (lane & ~(lanes_s - 1)) : lane;
   const bool single = (flags & AAAC_SINGLE_CODEBOOK) != 0;
-  const float la = tb.la;
   unsigned char* wring = ring + warp * kStages * kRingRowBytes;
   const int wr0 = ring_slot(lane) * 16, wr1 = ring_slot(32 + lane) * 16;
   const int rd0 = ring_slot(2 * lane) * 16, rd1 = ring_slot(2 * lane + 1) * 16;
   unsigned char* mybins = bins + warp * kWarpBinBytes + lane * 16;
 
   // ---- the warp's rows: work items (kItemRows rows of one 512-column strip)
-  // claimed from a global counter, one claim in flight ahead of its use, in a
-  // small FIFO that the W prefetch fills and the row loop drains.
+  // in a small FIFO that the W prefetch fills and the row loop drains.  The
+  // first item is fixed (chunk gw / ncb of strip gw % ncb, gw the warp's index
+  // in the grid); the rest are claimed from counters, one claim in flight
+  // ahead of its use.  Strips: a warp stays on its home strip and moves to the
+  // next one when it runs dry (per-strip counters keep the importance
+  // registers unchanged); with more than kMaxStrips strips a single counter
+  // hands out items in order.
   __shared__ int s_fifo[kFitWarps][8];
   int* fifo = s_fifo[warp];
-  // Strips: each warp starts on its home strip and moves to the next strip
-  // when one runs dry (per-strip counters keep a warp on one strip, so its
-  // importance registers rarely change); with more than kMaxStrips strips a
-  // single counter hands out items in order.
   const int ncb = n_items / cpc;
   const bool per_strip = ncb <= kMaxStrips;
-  int cur_strip = (int)((blockIdx.x * kFitWarps + warp) % (unsigned)ncb), tried = 0;
+  const int gw = (int)blockIdx.x * kFitWarps + warp;
+  int cur_strip = gw % ncb, tried = 0;
+  int first = -1;
+  if (per_strip) {
+    if (gw / ncb < cpc) first = cur_strip * cpc + gw / ncb;
+  } else if (gw < n_items) {
+    first = gw;
+  }
   unsigned pend = 0u;
-  bool pend_ok = false, no_more = false;
-  int claimed = 0, tail = 0;
+  bool pend_ok = false, no_more = first < 0;  // no fixed item: nothing is left
+  int claimed = first >= 0 ? 1 : 0, tail = 1;
+  if (lane == 0) fifo[0] = first;
+  __syncwarp();
   auto claim = [&]() {  // warp-uniform: start one claim
     pend_ok = !no_more && claimed < max_items;
     if (pend_ok) {
@@ -729,8 +747,6 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     __syncwarp();
     claim();
   };
-  claim();
-  land_push();
 
   // prefetch cursor: FIFO position pq, next row pr and end pe of that item,
   // and the item's strip values (set when the cursor enters the item)
@@ -749,16 +765,17 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     pact = pcol0 < K;
     pgi = pact ? pcol0 / g : 0;
   };
-  enter(fifo[0]);
-  float sq0 = 0.0f, sq1 = 0.0f, sq2 = 0.0f;  // scales of the rows in flight
-  // issue the row at the prefetch cursor into ring slot ps; returns its scale
+  // the row at the prefetch cursor into ring slot ps; returns its scale
+  auto issue = [&](int ps) -> float {
+    const uint16_t* src = psrc + (int64_t)pr * K;
+    if (pc0) cp_async16(wring + ps * kRingRowBytes + wr0, src);
+    if (pc1) cp_async16(wring + ps * kRingRowBytes + wr1, src + 256);
+    return pact ? load_scale<FMT>(scales, (int64_t)pr * G + pgi) : 0.0f;
+  };
   auto prefetch = [&](int ps) -> float {
     float sc = 0.0f;
     if (fifo[pq & 7] >= 0) {
-      const uint16_t* src = psrc + (int64_t)pr * K;
-      if (pc0) cp_async16(wring + ps * kRingRowBytes + wr0, src);
-      if (pc1) cp_async16(wring + ps * kRingRowBytes + wr1, src + 256);
-      if (pact) sc = load_scale<FMT>(scales, (int64_t)pr * G + pgi);
+      sc = issue(ps);
       if (++pr >= pe) {
         pq++;
         if (pq == tail) land_push();
@@ -768,12 +785,23 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     cp_async_commit();
     return sc;
   };
-  sq0 = prefetch(0);
-  sq1 = prefetch(1);
-  sq2 = prefetch(2);
+  enter(first);
+  // ring prologue, first part: rows of the fixed item that do not end it
+  float sqv[kStages];
+  int npre = 0;
+#pragma unroll
+  for (int k = 0; k < kStages; k++) {
+    sqv[k] = 0.0f;
+    if (first >= 0 && npre == k && pr + 1 < pe) {
+      sqv[k] = issue(k);
+      pr++;
+      cp_async_commit();
+      npre++;
+    }
+  }
 
   // consumer cursor: FIFO position cq, row cr, item end ce, strip ccb; and
-  // the strip whose importance is loaded
+  // the strip whose importance is loaded (the fixed item's, before the wait)
   int cq = 0, cr = 0, ce = 0, ccb = 0;
   auto centre = [&](int it) {
     if (it < 0) return;
@@ -781,15 +809,46 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     cr = (it % cpc) * kItemRows;
     ce = min(N, cr + kItemRows);
   };
-  centre(fifo[0]);
+  centre(first);
   int cur_cb = -1, col0 = 0;
   bool active = false;
   unsigned long long I2[8];
   double Id[16];
+  auto load_importance = [&](int cb) {  // fp32 pairs (choice) and fp64 (refine)
+    cur_cb = cb;
+    col0 = cb * kWarpCols + lane * kLaneCols;
+    active = col0 < K;
+    float Iv[16];
 #pragma unroll
-  for (int p = 0; p < 8; p++) I2[p] = 0ull;
+    for (int q = 0; q < 4; q++) {
+      const float4 a = active ? __ldg(reinterpret_cast<const float4*>(I + col0) + q)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      Iv[4 * q] = a.x; Iv[4 * q + 1] = a.y; Iv[4 * q + 2] = a.z; Iv[4 * q + 3] = a.w;
+    }
 #pragma unroll
-  for (int i = 0; i < 16; i++) Id[i] = 0.0;
+    for (int p = 0; p < 8; p++) I2[p] = f2pack(Iv[2 * p], Iv[2 * p + 1]);
+#pragma unroll
+    for (int i = 0; i < 16; i++) Id[i] = (double)Iv[i];
+  };
+  if (first >= 0) load_importance(ccb);
+
+  // ---- the previous round's results: tables, fixed-point scales, counters
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  {
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(&ctl->tb);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(&tb);
+    for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
+  }
+  const double twoL = ctl->twoL;
+  const double twoLe = ctl->twoLe;
+  __syncthreads();
+  const float la = tb.la;
+  claim();
+  // ring prologue, second part: the remaining positions (may claim)
+#pragma unroll
+  for (int k = 0; k < kStages; k++)
+    if (k >= npre) sqv[k] = prefetch(k);
+  float sq0 = sqv[0], sq1 = sqv[1], sq2 = sqv[2];
 
   GroupStats gs{0u, 0u, 0u, 0ull};
   int slot = 0;
@@ -799,22 +858,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     if (fifo[cq & 7] < 0) break;
     const int r = cr;
     const int cb = ccb;
-    if (cb != cur_cb) {  // importance of the lane's columns: fp32 pairs and fp64
-      cur_cb = cb;
-      col0 = cb * kWarpCols + lane * kLaneCols;
-      active = col0 < K;
-      float Iv[16];
-#pragma unroll
-      for (int q = 0; q < 4; q++) {
-        const float4 a = active ? __ldg(reinterpret_cast<const float4*>(I + col0) + q)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-        Iv[4 * q] = a.x; Iv[4 * q + 1] = a.y; Iv[4 * q + 2] = a.z; Iv[4 * q + 3] = a.w;
-      }
-#pragma unroll
-      for (int p = 0; p < 8; p++) I2[p] = f2pack(Iv[2 * p], Iv[2 * p + 1]);
-#pragma unroll
-      for (int i = 0; i < 16; i++) Id[i] = (double)Iv[i];
-    }
+    if (cb != cur_cb) load_importance(cb);
     if (++cr >= ce) {
       cq++;
       centre(fifo[cq & 7]);  // already pushed: the prefetch runs ahead
@@ -995,6 +1039,9 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     }
   }
   cp_async_wait<0>();
+  // the next round may start its blocks (they wait for this grid to finish
+  // before reading anything it writes)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   for (int o = 16; o > 0; o >>= 1) {
     gs.near += __shfl_xor_sync(0xffffffffu, gs.near, o);
@@ -1033,16 +1080,15 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   if (!s_last) return;
   __threadfence();
   if (!PACK) {
-    round_finalize(ctl, tb, flags, ro);
+    round_finalize(ctl, tb, flags, ro, cpc, n_items);
   } else {
     if (threadIdx.x == 0) {
       const long long acc = (long long)__ldcg(&ctl->err_acc);
       if (po.err_final) *po.err_final = (double)acc / ctl->twoLe;
       ctl->err_acc = 0ull;
-      ctl->next_item = 0;
       ctl->ticket = 0;
     }
-    for (int i = threadIdx.x; i < kMaxStrips; i += blockDim.x) ctl->strip_next[i] = 0u;
+    seed_claims(ctl, (int)gridDim.x * kFitWarps, cpc, n_items);
   }
 }
 
@@ -1072,12 +1118,28 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
                                                    pprep.ncb, pprep.rows_per_chunk);
-  fit_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), stats);
+  fit_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), stats, pp.blocks * kFitWarps,
+                                       pp.cpc, pp.items);
   const float tau = choice_tau(S);
+  // rounds launched with programmatic stream serialization: a round's blocks
+  // may start (and prefetch) while the previous launch finishes; they wait
+  // with griddepcontrol.wait before reading what it writes
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)pp.blocks);
+  lc.blockDim = dim3(kFitThreads);
+  lc.dynamicSmemBytes = smem_bytes(false);
+  lc.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
   for (int it = 0; it < iters; it++) {
-    fit_pass<FMT, false><<<pp.blocks, kFitThreads, smem_bytes(false), st>>>(
-        W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items, tau,
-        PackOut{nullptr, nullptr, nullptr, nullptr}, RoundOut{err_hist, T, stats, it});
+    const cudaError_t e = cudaLaunchKernelEx(
+        &lc, fit_pass<FMT, false>, W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items,
+        pp.max_items, tau, PackOut{nullptr, nullptr, nullptr, nullptr},
+        RoundOut{err_hist, T, stats, it});
+    if (e != cudaSuccess) return e;
   }
   count_launches(2 + iters);
   return cudaSuccess;
@@ -1132,9 +1194,11 @@ cudaError_t fixed_scratch_ptr(void** out) {
 // pack
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kFitThreads)
-pack_setup(FitCtl* ctl, const float* T_user, int64_t M, int n, uint16_t* T_bf16) {
+pack_setup(FitCtl* ctl, const float* T_user, int64_t M, int n, uint16_t* T_bf16, int wt,
+           int cpc, int n_items) {
   __shared__ Tables tb;
   __shared__ float sT[2][16];
+  seed_claims(ctl, wt, cpc, n_items);
   if (threadIdx.x == 0) {
     ctl->n = n;
     ctl->twoLe = objective_scale(ctl, M);
@@ -1184,7 +1248,8 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
                                                    pprep.ncb, pprep.rows_per_chunk);
-  pack_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), T_bf16);
+  pack_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), T_bf16,
+                                        pp.blocks * kFitWarps, pp.cpc, pp.items);
   const float tau = choice_tau(S);
   const PackOut po{codes, scales_tagged, cbytes, err_final};
   fit_pass<FMT, true><<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
