@@ -683,6 +683,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned full = 0xffffffffu;
   const int G = K / g, KS = K / S;
+  const int lg = __ffs(g) - 1;              // g is a power of two
   const int lanes_s = S >> 4;               // lanes per choice group when S >= 16
   const int leader_lane = S >= 16 ? (lane & ~(lanes_s - 1)) : lane;
   const bool single = (flags & AAAC_SINGLE_CODEBOOK) != 0;
@@ -699,22 +700,31 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   // next one when it runs dry (per-strip counters keep the importance
   // registers unchanged); with more than kMaxStrips strips a single counter
   // hands out items in order.
-  __shared__ int s_fifo[kFitWarps][8];
+  __shared__ int s_fifo[kFitWarps][8];   // item strip, -1 = no more items
+  __shared__ int s_fifoc[kFitWarps][8];  // item chunk within its strip
   int* fifo = s_fifo[warp];
+  int* fifoc = s_fifoc[warp];
   const int ncb = n_items / cpc;
   const bool per_strip = ncb <= kMaxStrips;
   const int gw = (int)blockIdx.x * kFitWarps + warp;
   int cur_strip = gw % ncb, tried = 0;
-  int first = -1;
+  int first = -1, first_c = 0;  // strip and chunk of the fixed item
   if (per_strip) {
-    if (gw / ncb < cpc) first = cur_strip * cpc + gw / ncb;
+    if (gw / ncb < cpc) {
+      first = cur_strip;
+      first_c = gw / ncb;
+    }
   } else if (gw < n_items) {
-    first = gw;
+    first = gw / cpc;
+    first_c = gw - first * cpc;
   }
   unsigned pend = 0u;
   bool pend_ok = false, no_more = first < 0;  // no fixed item: nothing is left
   int claimed = first >= 0 ? 1 : 0, tail = 1;
-  if (lane == 0) fifo[0] = first;
+  if (lane == 0) {
+    fifo[0] = first;
+    fifoc[0] = first_c;
+  }
   __syncwarp();
   auto claim = [&]() {  // warp-uniform: start one claim
     pend_ok = !no_more && claimed < max_items;
@@ -725,15 +735,19 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     }
   };
   auto land_push = [&]() {  // the pending claim's item (or -1) into the FIFO, next claim
-    int it = -1;
+    int it = -1, itc = 0;
     while (pend_ok) {
       const int v = __shfl_sync(full, (int)pend, 0);
       if (!per_strip) {
-        if (v < n_items) it = v;
+        if (v < n_items) {
+          it = v / cpc;
+          itc = v - it * cpc;
+        }
         break;
       }
       if (v < cpc) {
-        it = cur_strip * cpc + v;
+        it = cur_strip;
+        itc = v;
         break;
       }
       claimed--;  // this strip has run dry: try the next one
@@ -742,7 +756,10 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
       claim();
     }
     if (it < 0) no_more = true;
-    if (lane == 0) fifo[tail & 7] = it;
+    if (lane == 0) {
+      fifo[tail & 7] = it;
+      fifoc[tail & 7] = itc;
+    }
     tail++;
     __syncwarp();
     claim();
@@ -753,17 +770,17 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   int pq = 0, pr = 0, pe = 0, pgi = 0;
   const uint16_t* psrc = W;
   bool pc0 = false, pc1 = false, pact = false;
-  auto enter = [&](int it) {
+  auto enter = [&](int it, int itc) {
     if (it < 0) return;
-    const int pseg = (it / cpc) * kWarpCols;
-    pr = (it % cpc) * kItemRows;
+    const int pseg = it * kWarpCols;
+    pr = itc * kItemRows;
     pe = min(N, pr + kItemRows);
     psrc = W + pseg + lane * 8;
     pc0 = pseg + lane * 8 < K;
     pc1 = pseg + 256 + lane * 8 < K;
     const int pcol0 = pseg + lane * kLaneCols;
     pact = pcol0 < K;
-    pgi = pact ? pcol0 / g : 0;
+    pgi = pact ? (pcol0 >> lg) : 0;
   };
   // the row at the prefetch cursor into ring slot ps; returns its scale
   auto issue = [&](int ps) -> float {
@@ -779,13 +796,13 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
       if (++pr >= pe) {
         pq++;
         if (pq == tail) land_push();
-        enter(fifo[pq & 7]);
+        enter(fifo[pq & 7], fifoc[pq & 7]);
       }
     }
     cp_async_commit();
     return sc;
   };
-  enter(first);
+  enter(first, first_c);
   // ring prologue, first part: rows of the fixed item that do not end it
   float sqv[kStages];
   int npre = 0;
@@ -803,13 +820,13 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   // consumer cursor: FIFO position cq, row cr, item end ce, strip ccb; and
   // the strip whose importance is loaded (the fixed item's, before the wait)
   int cq = 0, cr = 0, ce = 0, ccb = 0;
-  auto centre = [&](int it) {
+  auto centre = [&](int it, int itc) {
     if (it < 0) return;
-    ccb = it / cpc;
-    cr = (it % cpc) * kItemRows;
+    ccb = it;
+    cr = itc * kItemRows;
     ce = min(N, cr + kItemRows);
   };
-  centre(first);
+  centre(first, first_c);
   int cur_cb = -1, col0 = 0;
   bool active = false;
   unsigned long long I2[8];
@@ -861,7 +878,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     if (cb != cur_cb) load_importance(cb);
     if (++cr >= ce) {
       cq++;
-      centre(fifo[cq & 7]);  // already pushed: the prefetch runs ahead
+      centre(fifo[cq & 7], fifoc[cq & 7]);  // already pushed: the prefetch runs ahead
     }
     cp_async_wait<kStages - 1>();
     __syncwarp();  // the row's chunks were copied by other lanes
@@ -1017,7 +1034,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
       gs.err += (unsigned long long)__double2ll_rn(err_w * twoLe);
       *reinterpret_cast<unsigned long long*>(po.codes + ((int64_t)r * K + col0) / 2) = packed;
       if ((lane & ((g >> 4) - 1)) == 0) {
-        const int64_t gi = (int64_t)r * G + col0 / g;
+        const int64_t gi = (int64_t)r * G + (col0 >> lg);
         const uint32_t tag = (S == g) ? (uint32_t)ch[0] : 0u;
         if (FMT == kInt4) {
           const uint32_t hs = reinterpret_cast<const unsigned short*>(scales)[gi];
@@ -1033,7 +1050,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
           po.choice_bytes[(int64_t)r * KS + col0 / 8] = (uint8_t)ch[0];
           po.choice_bytes[(int64_t)r * KS + col0 / 8 + 1] = (uint8_t)ch[1];
         } else if (lane == leader_lane) {
-          po.choice_bytes[(int64_t)r * KS + col0 / S] = (uint8_t)ch[0];
+          po.choice_bytes[(int64_t)r * KS + (col0 >> (__ffs(S) - 1))] = (uint8_t)ch[0];
         }
       }
     }
