@@ -41,6 +41,17 @@ paper/2605.08692) and what pins it (tests/test_oracle_*.py):
                     special case against numpy's textbook INT4 dequantisation.
   linear            Y = X W_hat^T in fp64.  Pinned by one-hot rows of X
                     (Y is a column of W_hat exactly) and by numpy's matmul.
+  awq_prescale      section 4 (AAAC combined with AWQ's weight scaling before
+                    quantisation; reading R16 for the scaling itself).  Pinned
+                    by: alpha = 0 is the identity, equal importance gives unit
+                    scales, a two-level importance gives 2^(+-j/4) in closed
+                    form, numpy's pow within one fp32 ulp, the importance of
+                    the rescaled activations recomputed from X, and the
+                    scaled layer computing the same map within bf16 rounding.
+  awq_search        plain grid search over alpha = j/16, keeping the first
+                    candidate with the lowest err_final.  Pinned by: alpha = 0
+                    reproduces the plain fit, and each candidate equals the
+                    plain fit of its rescaled layer.
   Final fitted values of a whole run: parity unpinned by the pages (they print
   no worked example); held only by the pins above.
 """
@@ -115,6 +126,10 @@ def lib():
         L.orc_linear.argtypes = [P, i64, i64, P, i64, i64, P]
         L.orc_unpack.restype = None
         L.orc_unpack.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, P]
+        L.orc_awq_scales.restype = None
+        L.orc_awq_scales.argtypes = [P, i64, i64, i32, P, P]
+        L.orc_awq_scale_weights.restype = None
+        L.orc_awq_scale_weights.argtypes = [P, i64, i64, P, P]
         _lib = L
     return _lib
 
@@ -321,3 +336,35 @@ def run_layer(W_u16, X_u16, fmt, g, S, iters, flags=0):
     out = pack(W_u16, I, scl, T, fmt, g, S, flags)
     out.update(I=I, scales=scl, T_init=T0, T=T, err_hist=err, stats=st)
     return out
+
+
+def awq_prescale(W_u16, I, tokens, j):
+    """(c, I', W') of reading R16 for alpha = j/16: per-channel scales, the
+    importance of the rescaled activations, and the rescaled bf16 weights."""
+    W = _u16(W_u16)
+    N, K = W.shape
+    I = np.ascontiguousarray(I, dtype=np.float32)
+    c = np.empty(K, dtype=np.float32)
+    Is = np.empty(K, dtype=np.float32)
+    lib().orc_awq_scales(_p(I), K, int(tokens), int(j), _p(c), _p(Is))
+    Ws = np.empty_like(W)
+    lib().orc_awq_scale_weights(_p(W), N, K, _p(c), _p(Ws))
+    return c, Is, Ws
+
+
+def awq_search(W_u16, I, tokens, fmt, g, S, iters, js, flags=0):
+    """Grid search over alpha = j/16 (j in js, ascending): fit and pack each
+    rescaled layer and keep the first candidate with the lowest err_final."""
+    js = [int(j) for j in js]
+    errs = []
+    best = None
+    for idx, j in enumerate(js):
+        c, Is, Ws = awq_prescale(W_u16, I, tokens, j)
+        scl, T0 = init_codebooks(Ws, fmt, g)
+        T, err, st = fit(Ws, Is, scl, T0, fmt, g, S, iters, flags)
+        out = pack(Ws, Is, scl, T, fmt, g, S, flags)
+        errs.append(out["err_final"])
+        if best is None or out["err_final"] < errs[best[0]]:
+            out.update(c=c, I=Is, W=Ws, scales=scl, T=T, err_hist=err, stats=st)
+            best = (idx, out)
+    return dict(best=best[0], err_alpha=np.array(errs, dtype=np.float64), **best[1])

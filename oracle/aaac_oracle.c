@@ -818,3 +818,67 @@ void orc_linear(const uint16_t* X, int64_t M, int64_t ldx, const uint16_t* w_hat
             Y[m * N + n] = acc;
         }
 }
+
+/* ------------------------------------------------------------------------ */
+/* AWQ-style pre-scaling ("Technical summary: AAAC", section 4: AAAC          */
+/* combined with AWQ, which scales the weights before quantisation).  The    */
+/* page gives no formula for the scaling; reading R16:                       */
+/*   v_k  = I_k / tokens                      (fp64; the channel's mean x^2) */
+/*   p_k  = v_k^(j/32), alpha = j/16 in [0, 1]: the product, in ascending i, */
+/*          of v^(2^(i-5)) over the set bits i of j, each power taken by     */
+/*          repeated fp64 square roots (v^(1/2), v^(1/4), ..., v^(1/32)), so */
+/*          every step is a correctly rounded IEEE operation;                */
+/*   z    = sqrt(max_k p_k * min_k p_k) over the live channels (I_k > 0);    */
+/*   c_k  = fp32_RN(p_k / z) for live channels, 1 for dead ones;             */
+/*   I'_k = fp32_RN(I_k / (c_k * c_k))        (fp64, c_k^2 exact);           */
+/*   W'   = bf16_RN(fp32_RN(w * c_k)).                                       */
+/* c scales the weights' input channels up where activations are large; the  */
+/* activations of the scaled layer are x / c, whose energy is I'.            */
+/* ------------------------------------------------------------------------ */
+static double awq_power(double v, int j)
+{
+    double q[5];
+    q[4] = sqrt(v);
+    for (int i = 3; i >= 0; i--) q[i] = sqrt(q[i + 1]);
+    double p = 1.0;
+    for (int i = 0; i < 5; i++)
+        if ((j >> i) & 1) p = p * q[i];
+    return p;
+}
+
+void orc_awq_scales(const float* I, int64_t K, int64_t tokens, int j, float* c, float* I_out)
+{
+    double pmax = 0.0, pmin = 0.0;
+    int any = 0;
+    for (int64_t k = 0; k < K; k++) {
+        if (!(I[k] > 0.0f)) continue;
+        double p = awq_power((double)I[k] / (double)tokens, j);
+        if (!any || p > pmax) pmax = p;
+        if (!any || p < pmin) pmin = p;
+        any = 1;
+    }
+    double z = any ? sqrt(pmax * pmin) : 1.0;
+    for (int64_t k = 0; k < K; k++) {
+        if (!(I[k] > 0.0f)) {
+            c[k] = 1.0f;
+            I_out[k] = I[k];
+            continue;
+        }
+        double p = awq_power((double)I[k] / (double)tokens, j);
+        c[k] = (float)(p / z);
+        double cc = (double)c[k] * (double)c[k];
+        I_out[k] = (float)((double)I[k] / cc);
+    }
+}
+
+void orc_awq_scale_weights(const uint16_t* W, int64_t N, int64_t K, const float* c,
+                           uint16_t* W_out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) {
+            float w = orc_bf16_to_f32(W[n * K + k]);
+            float p = w * c[k];
+            W_out[n * K + k] = orc_f32_to_bf16_rn(p);
+        }
+}

@@ -36,7 +36,7 @@ def packed_layer(N, K, fmt, g, S, seed, iters=3, dist="normal"):
 
 
 CASES = [(oracle.INT4, 128, 16), (oracle.INT4, 128, 128), (oracle.INT4, 64, 8),
-         (oracle.NVFP4, 16, 16)]
+         (oracle.NVFP4, 16, 16), (oracle.NVFP4, 16, 8)]
 
 
 @pytest.mark.parametrize("fmt,g,S", CASES)
@@ -110,7 +110,8 @@ def test_dequant_and_linear_full_size_gate():
 
 
 GEMM_CASES = [(oracle.INT4, 128, 16, 200, 640), (oracle.INT4, 128, 128, 130, 384),
-              (oracle.NVFP4, 16, 16, 70, 208), (oracle.INT4, 32, 8, 256, 96)]
+              (oracle.NVFP4, 16, 16, 70, 208), (oracle.INT4, 32, 8, 256, 96),
+              (oracle.NVFP4, 16, 8, 130, 176)]
 
 
 @pytest.mark.parametrize("fmt,g,S,N,K", GEMM_CASES)

@@ -73,7 +73,7 @@ def test_importance_accumulate_strided_and_boundary():
 # scales, init, fit, pack
 # --------------------------------------------------------------------------
 CASES = [(bb.INT4, 128, 128, 256, 512), (bb.INT4, 128, 16, 37, 640), (bb.NVFP4, 16, 16, 64, 512),
-         (bb.INT4, 32, 8, 48, 256), (bb.NVFP4, 16, 16, 33, 1040)]
+         (bb.INT4, 32, 8, 48, 256), (bb.NVFP4, 16, 16, 33, 1040), (bb.NVFP4, 16, 8, 40, 528)]
 
 
 @pytest.mark.parametrize("fmt,g,S,N,K", CASES)

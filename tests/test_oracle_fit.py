@@ -163,7 +163,8 @@ def test_one_refine_is_weighted_mean():
 
 @pytest.mark.parametrize("fmt,g,S,dist", [(oracle.INT4, 128, 128, "normal"),
                                           (oracle.INT4, 128, 16, "normal"),
-                                          (oracle.NVFP4, 16, 16, "student_t4")])
+                                          (oracle.NVFP4, 16, 16, "student_t4"),
+                                          (oracle.NVFP4, 16, 8, "student_t4")])
 def test_objective_monotone_and_books_sorted(fmt, g, S, dist):
     N, K = 48, 512
     Wb, Xb = _layer(N, K, seed=71 + S, dist=dist)
@@ -198,7 +199,7 @@ def _golden():
 
 
 @pytest.mark.parametrize("fmt,g,S", [(oracle.INT4, 128, 128), (oracle.INT4, 128, 16),
-                                     (oracle.NVFP4, 16, 16)])
+                                     (oracle.NVFP4, 16, 16), (oracle.NVFP4, 16, 8)])
 def test_pack_storage_arithmetic_and_round_trip(fmt, g, S):
     gold = _golden()
     N, K = 32, 512
