@@ -30,7 +30,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaaac.so"
 EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaac_fit_layer",
            "aaac_pack", "aaac_last_error", "aaac_version", "aaac_kernel_launches",
            "aaac_fit_layer_fixed_scratch", "aaac_dequant", "aaac_linear",
-           "aaac_device_timeouts")
+           "aaac_device_timeouts", "aaac_awq_prescale", "aaac_awq_workspace_size",
+           "aaac_awq_fit")
 
 
 class AaacError(RuntimeError):
@@ -107,6 +108,13 @@ def load(path: str = LIB_PATH):
     L.aaac_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     L.aaac_kernel_launches.restype = ctypes.c_uint64
     L.aaac_kernel_launches.argtypes = []
+    L.aaac_awq_prescale.restype = ctypes.c_int
+    L.aaac_awq_prescale.argtypes = [P, i64, i64, P, i64, ctypes.c_int, P, P, P, P]
+    L.aaac_awq_workspace_size.restype = sz
+    L.aaac_awq_workspace_size.argtypes = [P, i64, i64]
+    L.aaac_awq_fit.restype = ctypes.c_int
+    L.aaac_awq_fit.argtypes = [P, i64, i64, P, i64, P, P, ctypes.c_int, P, P, P, P, P, P, P, P,
+                               P, sz, P]
     _lib = L
     return L
 
@@ -320,4 +328,56 @@ def run_layer(W: torch.Tensor, X: torch.Tensor, cfg: Config, ws: Optional[torch.
     out = pack(W, I, scales, T, cfg, ws=ws, stream=stream)
     out.update(I=I, scales=scales, T_init=T_init, T=T, err_hist=err_hist[:cfg.iters],
                stats=stats)
+    return out
+
+
+def awq_prescale(W: torch.Tensor, I: torch.Tensor, tokens: int, alpha16: int, stream=None):
+    """AWQ-style pre-scaling for alpha = alpha16 / 16: (c, I', W') -- the
+    per-input-channel scales, the importance of the activations x / c, and
+    the rescaled bf16 weights (int16 bits)."""
+    _need_cuda()
+    W = _bits16(W)
+    N, K = W.shape
+    dev = W.device
+    c = torch.empty(K, dtype=torch.float32, device=dev)
+    Is = torch.empty(K, dtype=torch.float32, device=dev)
+    Ws = torch.empty(N, K, dtype=torch.int16, device=dev)
+    _check(load().aaac_awq_prescale(_ptr(W), N, K, _ptr(I), int(tokens), int(alpha16), _ptr(c),
+                                    _ptr(Is), _ptr(Ws), _stream(stream)))
+    return c, Is, Ws
+
+
+def awq_fit(W: torch.Tensor, I: torch.Tensor, tokens: int, cfg: Config, alphas16,
+            ws: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Grid search over alpha = j/16 for j in alphas16: pre-scale, fit and
+    pack each candidate on the device and keep the first with the lowest
+    err_final.  Returns the kept packed layer, c, err_final, the err_final of
+    every candidate (err_alpha) and the kept position (best), on the device."""
+    _need_cuda()
+    W = _bits16(W)
+    N, K = W.shape
+    dev = W.device
+    js = (ctypes.c_int32 * len(alphas16))(*[int(j) for j in alphas16])
+    c_cfg = cfg.c()
+    if ws is None:
+        need = load().aaac_awq_workspace_size(ctypes.byref(c_cfg), N, K)
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    G = K // cfg.g
+    sdt = torch.int16 if cfg.fmt == INT4 else torch.uint8
+    nb = (K // cfg.S + 7) // 8
+    out = dict(c=torch.empty(K, dtype=torch.float32, device=dev),
+               T_bf16=torch.zeros(2, 16, dtype=torch.int16, device=dev),
+               codes=torch.empty(N, K // 2, dtype=torch.uint8, device=dev),
+               scales_tagged=torch.empty(N, G, dtype=sdt, device=dev),
+               choice_bits=(torch.empty(N, nb, dtype=torch.uint8, device=dev)
+                            if cfg.S != cfg.g else None),
+               err_final=torch.zeros(1, dtype=torch.float64, device=dev),
+               err_alpha=torch.zeros(len(alphas16), dtype=torch.float64, device=dev),
+               best=torch.full((1,), -1, dtype=torch.int32, device=dev))
+    _check(load().aaac_awq_fit(_ptr(W), N, K, _ptr(I), int(tokens), ctypes.byref(c_cfg), js,
+                               len(alphas16), _ptr(out["c"]), _ptr(out["T_bf16"]),
+                               _ptr(out["codes"]), _ptr(out["scales_tagged"]),
+                               _ptr(out["choice_bits"]), _ptr(out["err_final"]),
+                               _ptr(out["err_alpha"]), _ptr(out["best"]), _ptr(ws), ws.numel(),
+                               _stream(stream)))
     return out

@@ -93,6 +93,38 @@ size_t weight_side_bytes(const aaac_config* cfg, int64_t N, int64_t K) {
   return m > init ? m : init;
 }
 
+// Workspace of aaac_awq_fit: the rescaled layer, one candidate's fit state
+// and packed output, and the fit's own workspace (shared by init, fit, pack).
+struct AwqLayout {
+  size_t Ws, Is, c, scales, T, Tb, codes, tagged, bits, hist, stats, fit, total;
+};
+AwqLayout awq_layout(const aaac_config* cfg, int64_t N, int64_t K) {
+  AwqLayout L{};
+  const int64_t G = K / cfg->g;
+  const size_t es = cfg->fmt == AAAC_INT4 ? 2 : 1;
+  const size_t nb = cfg->S != cfg->g ? (size_t)((K / cfg->S + 7) / 8) : 0;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += aaac::align256(bytes);
+    return at;
+  };
+  L.Ws = take((size_t)(N * K) * 2);
+  L.Is = take((size_t)K * 4);
+  L.c = take((size_t)K * 4);
+  L.scales = take((size_t)(N * G) * es);
+  L.T = take(2 * 16 * 4);
+  L.Tb = take(2 * 16 * 2);
+  L.codes = take((size_t)(N * K / 2));
+  L.tagged = take((size_t)(N * G) * es);
+  L.bits = take((size_t)N * nb);
+  L.hist = take((size_t)(cfg->iters > 0 ? cfg->iters : 1) * 8);
+  L.stats = take(sizeof(aaac_stats));
+  L.fit = take(weight_side_bytes(cfg, N, K));
+  L.total = o;
+  return L;
+}
+
 #define CHECK(x)                         \
   do {                                   \
     aaac_status _s = (x);                \
@@ -254,6 +286,99 @@ aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* co
                                        scales_tagged, choice_bits, T_bf16, N, K, cfg->fmt,
                                        cfg->g, cfg->S, Y, (cudaStream_t)stream),
                    "aaac_linear");
+}
+
+aaac_status aaac_awq_prescale(const void* W, int64_t N, int64_t K, const float* I,
+                              int64_t tokens, int alpha16, float* c, float* I_scaled,
+                              void* W_scaled, void* stream) {
+  if (N <= 0 || K <= 0) return fail(AAAC_ERR_SHAPE, "N and K must be positive");
+  if (K % 8) return fail(AAAC_ERR_ALIGN, "K=%lld is not a multiple of 8", (long long)K);
+  if (N > INT32_MAX || K > INT32_MAX || N * K >= ((int64_t)1 << 31))
+    return fail(AAAC_ERR_SHAPE, "N*K must be < 2^31 (N=%lld K=%lld)", (long long)N,
+                (long long)K);
+  if (tokens <= 0) return fail(AAAC_ERR_SHAPE, "tokens must be positive (%lld)", (long long)tokens);
+  if (alpha16 < 0 || alpha16 > 16)
+    return fail(AAAC_ERR_INVALID_ARG, "alpha16=%d is not in [0, 16]", alpha16);
+  CHECK(check_ptr(W, "W"));
+  CHECK(check_ptr(I, "I"));
+  CHECK(check_ptr(c, "c"));
+  CHECK(check_ptr(I_scaled, "I_scaled"));
+  CHECK(check_ptr(W_scaled, "W_scaled"));
+  return from_cuda(aaac::launch_awq_prescale(reinterpret_cast<const uint16_t*>(W), N, K, I,
+                                             tokens, alpha16, c, I_scaled,
+                                             reinterpret_cast<uint16_t*>(W_scaled),
+                                             (cudaStream_t)stream),
+                   "aaac_awq_prescale");
+}
+
+size_t aaac_awq_workspace_size(const aaac_config* cfg, int64_t N, int64_t K) {
+  if (!cfg || N <= 0 || K <= 0 || cfg->g <= 0 || cfg->S <= 0 || K % cfg->g) return 0;
+  return awq_layout(cfg, N, K).total;
+}
+
+aaac_status aaac_awq_fit(const void* W, int64_t N, int64_t K, const float* I, int64_t tokens,
+                         const aaac_config* cfg, const int32_t* alpha16, int n_alpha, float* c,
+                         uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
+                         uint8_t* choice_bits, double* err_final, double* err_alpha,
+                         int32_t* best, void* ws, size_t ws_bytes, void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  if (tokens <= 0) return fail(AAAC_ERR_SHAPE, "tokens must be positive (%lld)", (long long)tokens);
+  if (!alpha16) return fail(AAAC_ERR_INVALID_ARG, "alpha16 is NULL");
+  if (n_alpha < 1 || n_alpha > 17)
+    return fail(AAAC_ERR_INVALID_ARG, "n_alpha=%d is not in [1, 17]", n_alpha);
+  for (int i = 0; i < n_alpha; i++)
+    if (alpha16[i] < 0 || alpha16[i] > 16)
+      return fail(AAAC_ERR_INVALID_ARG, "alpha16[%d]=%d is not in [0, 16]", i, alpha16[i]);
+  CHECK(check_ptr(W, "W"));
+  CHECK(check_ptr(I, "I"));
+  CHECK(check_ptr(c, "c"));
+  CHECK(check_ptr(T_bf16, "T_bf16"));
+  CHECK(check_ptr(codes, "codes"));
+  CHECK(check_ptr(scales_tagged, "scales_tagged"));
+  CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
+  CHECK(check_ptr(err_final, "err_final", false));
+  CHECK(check_ptr(err_alpha, "err_alpha"));
+  CHECK(check_ptr(best, "best", false));
+  const AwqLayout L = awq_layout(cfg, N, K);
+  CHECK(check_ws(ws, ws_bytes, L.total));
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  uint16_t* Ws = reinterpret_cast<uint16_t*>(base + L.Ws);
+  float* Is = reinterpret_cast<float*>(base + L.Is);
+  float* cc = reinterpret_cast<float*>(base + L.c);
+  void* scl = base + L.scales;
+  float* T = reinterpret_cast<float*>(base + L.T);
+  uint16_t* Tb = reinterpret_cast<uint16_t*>(base + L.Tb);
+  uint8_t* cod = base + L.codes;
+  void* tag = base + L.tagged;
+  uint8_t* bits = cfg->S != cfg->g ? base + L.bits : nullptr;
+  double* hist = reinterpret_cast<double*>(base + L.hist);
+  aaac_stats* stats = reinterpret_cast<aaac_stats*>(base + L.stats);
+  void* fws = base + L.fit;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t G = K / cfg->g;
+  const size_t es = cfg->fmt == AAAC_INT4 ? 2 : 1;
+  const void* src[5] = {cod, tag, Tb, cc, bits};
+  void* dst[5] = {codes, scales_tagged, T_bf16, c, choice_bits};
+  const size_t bytes[5] = {(size_t)(N * K / 2), (size_t)(N * G) * es, 2 * 16 * 2,
+                           (size_t)K * 4, bits ? (size_t)N * ((K / cfg->S + 7) / 8) : 0};
+  const int segs = bits ? 5 : 4;
+  for (int i = 0; i < n_alpha; i++) {
+    cudaError_t e = aaac::launch_awq_prescale(reinterpret_cast<const uint16_t*>(W), N, K, I,
+                                              tokens, alpha16[i], cc, Is, Ws, st);
+    if (e == cudaSuccess)
+      e = aaac::launch_init(Ws, N, K, cfg->fmt, cfg->g, scl, T, fws, st);
+    if (e == cudaSuccess)
+      e = aaac::launch_fit(Ws, N, K, Is, scl, cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T,
+                           hist, stats, fws, st);
+    if (e == cudaSuccess)
+      e = aaac::launch_pack(Ws, N, K, Is, scl, cfg->fmt, cfg->g, cfg->S, cfg->flags, T, Tb, cod,
+                            tag, bits, err_alpha + i, fws, st);
+    if (e == cudaSuccess)
+      e = aaac::launch_awq_keep(i, err_alpha, src, dst, bytes, segs, err_final, best, st);
+    if (e != cudaSuccess) return from_cuda(e, "aaac_awq_fit");
+  }
+  return ok();
 }
 
 aaac_status aaac_device_timeouts(uint32_t* flag) {

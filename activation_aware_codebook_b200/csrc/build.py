@@ -15,7 +15,7 @@ PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libaaac.so")
-SOURCES = ["api.cu", "importance.cu", "init.cu", "fit.cu", "linear.cu", "gemm.cu"]
+SOURCES = ["api.cu", "importance.cu", "init.cu", "fit.cu", "linear.cu", "gemm.cu", "awq.cu"]
 BUILD_DIR = os.path.join(ROOT, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

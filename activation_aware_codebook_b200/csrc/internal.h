@@ -68,4 +68,11 @@ cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
                         int64_t K, int fmt, int lg, int ls, float* Y, cudaStream_t st);
 cudaError_t gemm_timeout_flag(unsigned int* out);
 
+cudaError_t launch_awq_prescale(const uint16_t* W, int64_t N, int64_t K, const float* I,
+                                int64_t tokens, int j, float* c, float* Is, uint16_t* Wout,
+                                cudaStream_t st);
+cudaError_t launch_awq_keep(int j, const double* err_alpha, const void* const* src,
+                            void* const* dst, const size_t* bytes, int segs, double* err_final,
+                            int32_t* best, cudaStream_t st);
+
 }  // namespace aaac

@@ -206,6 +206,56 @@ aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* co
                         const uint16_t* T_bf16, int64_t N, int64_t K, const aaac_config* cfg,
                         float* Y, void* stream);
 
+/* AWQ-style pre-scaling before the fit (section 4: AAAC combined with AWQ,
+ * which scales the weights before quantisation).  For alpha = alpha16 / 16:
+ *   v_k  = I_k / tokens;  p_k = v_k^(alpha16/32), the product in ascending i
+ *          of v^(2^(i-5)) over the set bits i of alpha16, each power by
+ *          repeated fp64 square roots;
+ *   z    = sqrt(max p * min p) over channels with I_k > 0;
+ *   c_k  = fp32_RN(p_k / z)  (1 where I_k is not > 0);
+ *   I'_k = fp32_RN(I_k / (c_k * c_k))  (fp64);
+ *   W'   = bf16_RN(fp32_RN(w * c_k)).
+ * The rescaled layer (W', activations x / c) computes the same map as the
+ * original up to the bf16 rounding of W', and I' is its importance vector.
+ *   W         device bf16 [N][K], K a multiple of 8, N*K < 2^31
+ *   I         device fp32 [K] (aaac_importance over `tokens` rows of X)
+ *   tokens    > 0
+ *   alpha16   in [0, 16]; 0 gives c = 1, I' = I, W' = W
+ *   c, I_scaled  device fp32 [K];  W_scaled  device bf16 [N][K]
+ * All pointers 16-byte aligned; outputs must not overlap the inputs.
+ * Two kernels, no workspace. */
+aaac_status aaac_awq_prescale(const void* W, int64_t N, int64_t K, const float* I,
+                              int64_t tokens, int alpha16, float* c, float* I_scaled,
+                              void* W_scaled, void* stream);
+
+/* Bytes of workspace aaac_awq_fit needs for this config and shape (0 when
+ * the config or shape is invalid): the rescaled layer (2 B per weight), one
+ * candidate's packed output, and the fit's own workspace. */
+size_t aaac_awq_workspace_size(const aaac_config* cfg, int64_t N, int64_t K);
+
+/* Grid search over the pre-scaling exponent.  For each i < n_alpha, in
+ * order: aaac_awq_prescale with alpha16[i], then aaac_init_codebooks,
+ * aaac_fit_layer (cfg->iters rounds) and aaac_pack on the rescaled layer
+ * (W', I'); err_alpha[i] receives that candidate's err_final (the
+ * activation-weighted error of the rescaled layer, which equals the error
+ * of W_hat'/c against W'/c in the original input space).  The first
+ * candidate with the lowest err_final is kept (strict improvement over all
+ * earlier ones): its c, T_bf16, codes, scales_tagged and choice_bits go to
+ * the outputs, its err_final to *err_final and its position i to *best.
+ * Everything runs on `stream` with no host synchronisation.
+ *   alpha16     HOST int32 [n_alpha], each in [0, 16]; n_alpha in [1, 17]
+ *   c           device fp32 [K] (deploy with activations x / c)
+ *   T_bf16, codes, scales_tagged, choice_bits: as aaac_pack
+ *   err_final   device fp64 [1] (may be NULL); err_alpha device fp64 [n_alpha]
+ *   best        device int32 [1] (may be NULL)
+ *   ws          aaac_awq_workspace_size(cfg, N, K) bytes
+ * A CUDA error part way leaves the outputs of earlier candidates in place. */
+aaac_status aaac_awq_fit(const void* W, int64_t N, int64_t K, const float* I, int64_t tokens,
+                         const aaac_config* cfg, const int32_t* alpha16, int n_alpha, float* c,
+                         uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
+                         uint8_t* choice_bits, double* err_final, double* err_alpha,
+                         int32_t* best, void* ws, size_t ws_bytes, void* stream);
+
 /* Device-side wait status of the current device: *flag = 1 when a bounded
  * wait inside one of the library's kernels (the tensor-core aaac_linear path)
  * has run out since the library was loaded, else 0.  A kernel whose wait ran

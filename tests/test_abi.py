@@ -102,3 +102,31 @@ def test_binding_refuses_without_cuda(lib):
         pytest.skip("a GPU is present")
     with pytest.raises(RuntimeError):
         binding.importance(torch.zeros(8, 8, dtype=torch.bfloat16))
+
+
+def test_awq_entry_points_validate_before_anything(lib):
+    """Every call below has NULL device pointers, so no path can reach a
+    launch; the status shows which check refused it."""
+    assert lib.aaac_awq_prescale(None, 4, 60, None, 10, 3, None, None, None, None) == 3  # K % 8
+    assert lib.aaac_awq_prescale(None, 4, 64, None, 0, 3, None, None, None, None) == 2   # tokens
+    assert lib.aaac_awq_prescale(None, 4, 64, None, 10, 17, None, None, None, None) == 1  # alpha
+    assert lib.aaac_awq_prescale(None, 4, 64, None, 10, 3, None, None, None, None) == 1   # W NULL
+    c = _cfg()
+    js = (ctypes.c_int32 * 2)(0, 20)
+    assert lib.aaac_awq_fit(None, 64, 256, None, 10, ctypes.byref(c), js, 2, None, None, None,
+                            None, None, None, None, None, None, 0, None) == 1  # alpha16[1]
+    assert lib.aaac_awq_fit(None, 64, 256, None, 10, ctypes.byref(c), None, 1, None, None, None,
+                            None, None, None, None, None, None, 0, None) == 1  # alpha16 NULL
+    assert lib.aaac_awq_fit(None, 64, 200, None, 10, ctypes.byref(c), js, 1, None, None, None,
+                            None, None, None, None, None, None, 0, None) == 2  # K % g
+
+
+def test_awq_workspace_size(lib):
+    c = _cfg()
+    small = lib.aaac_awq_workspace_size(ctypes.byref(c), 64, 256)
+    big = lib.aaac_awq_workspace_size(ctypes.byref(c), 128, 512)
+    assert 0 < small < big
+    # at least the rescaled weights, the codes and the fit's own workspace
+    assert small >= 64 * 256 * 2 + 64 * 128 + lib.aaac_workspace_size(ctypes.byref(c), 64, 256, 0)
+    assert lib.aaac_awq_workspace_size(ctypes.byref(c), 64, 200) == 0
+    assert lib.aaac_awq_workspace_size(None, 64, 256) == 0
