@@ -15,9 +15,10 @@
 // Every step is one correctly rounded IEEE operation (sqrt, mul, div, one
 // narrowing), so the results do not depend on a math library's pow.
 //
-//   awq_scales_kernel   one block: the K channel scales and the rescaled
-//                       importance (two sweeps over K; the max / min
-//                       reduction between them is exact in any order).
+//   awq_scales_kernel   one cluster of 8 blocks: the K channel scales and the
+//                       rescaled importance (two sweeps over K; the max /
+//                       min between them is exact in any order and is
+//                       combined over distributed shared memory).
 //   awq_weights_kernel  streams W once: 16 bytes in, 16 bytes out per 8
 //                       weights, c read through the read-only path.
 //   awq_keep_kernel     after candidate j is packed: when its err_final beats
@@ -25,8 +26,12 @@
 //                       wins), copy its packed layer and scales to the
 //                       outputs.  Every block takes the same decision from
 //                       values no block writes, so there is no race.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace aaac {
 
@@ -44,25 +49,11 @@ __device__ __forceinline__ double awq_power(double v, int j) {
   return p;
 }
 
-constexpr int kScaleThreads = 1024;
+constexpr int kScaleThreads = 512;
+constexpr int kScaleCluster = 8;  // blocks of one cluster share the max / min over DSMEM
 
-__global__ void __launch_bounds__(kScaleThreads)
-awq_scales_kernel(const float* __restrict__ I, int K, double tokens, int j, float* __restrict__ c,
-                  float* __restrict__ Is) {
-  __shared__ double s_max[kScaleThreads / 32], s_min[kScaleThreads / 32];
-  __shared__ int s_any[kScaleThreads / 32];
-  __shared__ double s_z;
-  double pmax = 0.0, pmin = 0.0;
-  int any = 0;
-  for (int k = threadIdx.x; k < K; k += kScaleThreads) {
-    const float ik = I[k];
-    if (!(ik > 0.0f)) continue;
-    const double p = awq_power(__ddiv_rn((double)ik, tokens), j);
-    if (!any || p > pmax) pmax = p;
-    if (!any || p < pmin) pmin = p;
-    any = 1;
-  }
-  // warp, then block reduction; a lane without live channels contributes none
+// Reduce (max, min, any) of the live channels' p over a warp.
+__device__ __forceinline__ void reduce_live(double& pmax, double& pmin, int& any) {
   for (int o = 16; o; o >>= 1) {
     const double omax = __shfl_xor_sync(0xffffffffu, pmax, o);
     const double omin = __shfl_xor_sync(0xffffffffu, pmin, o);
@@ -73,6 +64,33 @@ awq_scales_kernel(const float* __restrict__ I, int K, double tokens, int j, floa
       any = 1;
     }
   }
+}
+
+// One cluster of kScaleCluster blocks: each block takes every
+// (kScaleCluster * kScaleThreads)-th channel from its offset, reduces its
+// live max / min in shared memory, and every block then reads all blocks'
+// partials over distributed shared memory in rank order, so all of them
+// form the same z.
+__global__ void __cluster_dims__(kScaleCluster, 1, 1) __launch_bounds__(kScaleThreads)
+awq_scales_kernel(const float* __restrict__ I, int K, double tokens, int j, float* __restrict__ c,
+                  float* __restrict__ Is) {
+  __shared__ double s_max[kScaleThreads / 32], s_min[kScaleThreads / 32];
+  __shared__ int s_any[kScaleThreads / 32];
+  __shared__ double s_z;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int first = (int)cluster.block_rank() * kScaleThreads + threadIdx.x;
+  const int step = kScaleCluster * kScaleThreads;
+  double pmax = 0.0, pmin = 0.0;
+  int any = 0;
+  for (int k = first; k < K; k += step) {
+    const float ik = I[k];
+    if (!(ik > 0.0f)) continue;
+    const double p = awq_power(__ddiv_rn((double)ik, tokens), j);
+    if (!any || p > pmax) pmax = p;
+    if (!any || p < pmin) pmin = p;
+    any = 1;
+  }
+  reduce_live(pmax, pmin, any);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) {
     s_max[warp] = pmax;
@@ -80,20 +98,36 @@ awq_scales_kernel(const float* __restrict__ I, int K, double tokens, int j, floa
     s_any[warp] = any;
   }
   __syncthreads();
+  if (warp == 0) {  // the block's partial, left in slot 0
+    pmax = lane < kScaleThreads / 32 ? s_max[lane] : 0.0;
+    pmin = lane < kScaleThreads / 32 ? s_min[lane] : 0.0;
+    any = lane < kScaleThreads / 32 ? s_any[lane] : 0;
+    reduce_live(pmax, pmin, any);
+    __syncwarp();
+    if (lane == 0) {
+      s_max[0] = pmax;
+      s_min[0] = pmin;
+      s_any[0] = any;
+    }
+  }
+  cluster.sync();  // every block's partial is in its shared memory
   if (threadIdx.x == 0) {
     double mx = 0.0, mn = 0.0;
     int a = 0;
-    for (int w = 0; w < kScaleThreads / 32; w++) {
-      if (!s_any[w]) continue;
-      mx = a ? fmax(mx, s_max[w]) : s_max[w];
-      mn = a ? fmin(mn, s_min[w]) : s_min[w];
+    for (int r = 0; r < kScaleCluster; r++) {
+      const int ra = *cluster.map_shared_rank(&s_any[0], r);
+      if (!ra) continue;
+      const double rmax = *cluster.map_shared_rank(&s_max[0], r);
+      const double rmin = *cluster.map_shared_rank(&s_min[0], r);
+      mx = a ? fmax(mx, rmax) : rmax;
+      mn = a ? fmin(mn, rmin) : rmin;
       a = 1;
     }
     s_z = a ? __dsqrt_rn(__dmul_rn(mx, mn)) : 1.0;
   }
-  __syncthreads();
+  cluster.sync();  // no block leaves while another still reads its partial
   const double z = s_z;
-  for (int k = threadIdx.x; k < K; k += kScaleThreads) {
+  for (int k = first; k < K; k += step) {
     const float ik = I[k];
     if (!(ik > 0.0f)) {
       c[k] = 1.0f;
@@ -168,7 +202,7 @@ __global__ void __launch_bounds__(kThreads) awq_keep_kernel(KeepArgs a) {
 cudaError_t launch_awq_prescale(const uint16_t* W, int64_t N, int64_t K, const float* I,
                                 int64_t tokens, int j, float* c, float* Is, uint16_t* Wout,
                                 cudaStream_t st) {
-  awq_scales_kernel<<<1, kScaleThreads, 0, st>>>(I, (int)K, (double)tokens, j, c, Is);
+  awq_scales_kernel<<<kScaleCluster, kScaleThreads, 0, st>>>(I, (int)K, (double)tokens, j, c, Is);
   const uint32_t n_vec = (uint32_t)(N * K / 8), k_vec = (uint32_t)(K / 8);
   int blocks = (int)((n_vec + kThreads - 1) / kThreads);
   if (blocks > 148 * 8) blocks = 148 * 8;
