@@ -64,6 +64,7 @@ from . import build as _build
 
 INT4 = 0
 NVFP4 = 1
+NVFP4_GS = 2  # NVFP4 with a per-tensor fp32 scale (reading R17)
 FREEZE_T0 = 1
 FREEZE_T1 = 2
 SINGLE_CODEBOOK = 4
@@ -98,15 +99,17 @@ def lib():
         L.orc_importance.restype = None
         L.orc_importance.argtypes = [P, i64, i64, i64, P, P]
         L.orc_scales.restype = None
-        L.orc_scales.argtypes = [P, i64, i64, i32, i32, P]
+        L.orc_scales.argtypes = [P, i64, i64, i32, i32, P, ctypes.c_float]
         L.orc_u.restype = None
-        L.orc_u.argtypes = [P, i64, i64, i32, i32, P, P]
+        L.orc_u.argtypes = [P, i64, i64, i32, i32, P, P, ctypes.c_float]
         L.orc_rank_t0.restype = i64
         L.orc_rank_t0.argtypes = [i64, i32, i32]
         L.orc_rank_t1.restype = i64
         L.orc_rank_t1.argtypes = [i64, i32, i32]
         L.orc_init_codebooks.restype = i32
-        L.orc_init_codebooks.argtypes = [P, i64, i64, i32, i32, P, P]
+        L.orc_init_codebooks.argtypes = [P, i64, i64, i32, i32, P, P, P]
+        L.orc_global_scale.restype = ctypes.c_float
+        L.orc_global_scale.argtypes = [P, i64, i64]
         L.orc_assign.restype = None
         L.orc_assign.argtypes = [P, i32, P, i64, P]
         L.orc_group_error.restype = ctypes.c_double
@@ -116,16 +119,17 @@ def lib():
         L.orc_fixed_point_L.restype = i32
         L.orc_fixed_point_L.argtypes = [i64, ctypes.c_double, ctypes.c_double, ctypes.c_double]
         L.orc_fit.restype = i32
-        L.orc_fit.argtypes = [P, i64, i64, P, P, i32, i32, i32, i32, ctypes.c_uint, P, P, P]
+        L.orc_fit.argtypes = [P, i64, i64, P, P, i32, i32, i32, i32, ctypes.c_uint, P, P, P,
+                              ctypes.c_float]
         L.orc_pack.restype = i32
         L.orc_pack.argtypes = [P, i64, i64, P, P, i32, i32, i32, ctypes.c_uint, P, P, P, P, P,
-                               P, P]
+                               P, P, ctypes.c_float]
         L.orc_dequant_bf16.restype = None
-        L.orc_dequant_bf16.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P]
+        L.orc_dequant_bf16.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, ctypes.c_float]
         L.orc_linear.restype = None
         L.orc_linear.argtypes = [P, i64, i64, P, i64, i64, P]
         L.orc_unpack.restype = None
-        L.orc_unpack.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, P]
+        L.orc_unpack.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, P, ctypes.c_float]
         L.orc_awq_scales.restype = None
         L.orc_awq_scales.argtypes = [P, i64, i64, i32, P, P]
         L.orc_awq_scale_weights.restype = None
@@ -199,20 +203,27 @@ def importance(X_u16, I_in=None, ldx=None):
     return out
 
 
-def scales(W_u16, fmt, g):
+def global_scale(W_u16):
+    """Tensor scale of reading R17: fp32_RN(max |w| / 448), 0 for a zero tensor."""
+    W = _u16(W_u16)
+    N, K = W.shape
+    return float(np.float32(lib().orc_global_scale(_p(W), N, K)))
+
+
+def scales(W_u16, fmt, g, gs=0.0):
     W = _u16(W_u16)
     N, K = W.shape
     out = np.empty((N, K // g), dtype=scale_dtype(fmt))
-    lib().orc_scales(_p(W), N, K, fmt, g, _p(out))
+    lib().orc_scales(_p(W), N, K, fmt, g, _p(out), float(gs))
     return out
 
 
-def u_values(W_u16, scl, fmt, g):
+def u_values(W_u16, scl, fmt, g, gs=0.0):
     W = _u16(W_u16)
     N, K = W.shape
     scl = np.ascontiguousarray(scl, dtype=scale_dtype(fmt))
     out = np.empty((N, K), dtype=np.float32)
-    lib().orc_u(_p(W), N, K, fmt, g, _p(scl), _p(out))
+    lib().orc_u(_p(W), N, K, fmt, g, _p(scl), _p(out), float(gs))
     return out
 
 
@@ -224,14 +235,16 @@ def rank_t1(M, n, j):
     return lib().orc_rank_t1(M, n, j)
 
 
-def init_codebooks(W_u16, fmt, g):
+def init_codebooks(W_u16, fmt, g, with_gs=False):
+    """(scales, T), or (scales, T, gs) with with_gs (gs = 0 unless NVFP4_GS)."""
     W = _u16(W_u16)
     N, K = W.shape
     scl = np.empty((N, K // g), dtype=scale_dtype(fmt))
     T = np.zeros((2, 16), dtype=np.float32)
-    rc = lib().orc_init_codebooks(_p(W), N, K, fmt, g, _p(scl), _p(T))
+    gs = np.zeros(1, dtype=np.float32)
+    rc = lib().orc_init_codebooks(_p(W), N, K, fmt, g, _p(scl), _p(T), _p(gs))
     assert rc == 0
-    return scl, T
+    return (scl, T, float(gs[0])) if with_gs else (scl, T)
 
 
 def assign(T, n, u):
@@ -259,7 +272,7 @@ def fixed_point_L(M, I_max, S2_max, U_max):
     return lib().orc_fixed_point_L(M, I_max, S2_max, U_max)
 
 
-def fit(W_u16, I, scl, T_init, fmt, g, S, iters, flags=0):
+def fit(W_u16, I, scl, T_init, fmt, g, S, iters, flags=0, gs=0.0):
     W = _u16(W_u16)
     N, K = W.shape
     I = np.ascontiguousarray(I, dtype=np.float32)
@@ -268,12 +281,12 @@ def fit(W_u16, I, scl, T_init, fmt, g, S, iters, flags=0):
     err = np.zeros(max(iters, 1), dtype=np.float64)
     st = Stats()
     rc = lib().orc_fit(_p(W), N, K, _p(I), _p(scl), fmt, g, S, iters, flags, _p(T), _p(err),
-                       ctypes.cast(ctypes.pointer(st), ctypes.c_void_p))
+                       ctypes.cast(ctypes.pointer(st), ctypes.c_void_p), float(gs))
     assert rc == 0
     return T, err[:iters], st
 
 
-def pack(W_u16, I, scl, T, fmt, g, S, flags=0):
+def pack(W_u16, I, scl, T, fmt, g, S, flags=0, gs=0.0):
     W = _u16(W_u16)
     N, K = W.shape
     I = np.ascontiguousarray(I, dtype=np.float32)
@@ -287,33 +300,35 @@ def pack(W_u16, I, scl, T, fmt, g, S, flags=0):
     err = np.zeros(1, dtype=np.float64)
     ties = np.zeros(1, dtype=np.int64)
     rc = lib().orc_pack(_p(W), N, K, _p(I), _p(scl), fmt, g, S, flags, _p(T), _p(T_bf16),
-                        _p(codes), _p(tagged), _p(bits), _p(err), _p(ties))
+                        _p(codes), _p(tagged), _p(bits), _p(err), _p(ties), float(gs))
     assert rc == 0
     return dict(T_bf16=T_bf16, codes=codes, scales_tagged=tagged, choice_bits=bits,
                 err_final=float(err[0]), near_ties=int(ties[0]))
 
 
-def unpack(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S):
+def unpack(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S, gs=0.0):
+    """Exact dequantised values s * T_bf16[c][code] (fp64) and the choices."""
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     tagged = np.ascontiguousarray(scales_tagged, dtype=scale_dtype(fmt))
     bits = None if choice_bits is None else np.ascontiguousarray(choice_bits, dtype=np.uint8)
     T_bf16 = np.ascontiguousarray(T_bf16, dtype=np.uint16)
-    w_hat = np.empty((N, K), dtype=np.float32)
+    w_hat = np.empty((N, K), dtype=np.float64)
     ch = np.empty((N, K // S), dtype=np.uint8)
     lib().orc_unpack(_p(codes), _p(tagged), _p(bits), _p(T_bf16), N, K, fmt, g, S, _p(w_hat),
-                     _p(ch))
+                     _p(ch), float(gs))
     return w_hat, ch
 
 
-def dequant_bf16(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S):
-    """bf16 bits of bf16_RN(s * T_bf16[c][code]) per weight, [N, K] uint16."""
+def dequant_bf16(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S, gs=0.0):
+    """bf16 bits of bf16_RN(s * T_bf16[c][code]) per weight, [N, K] uint16
+    (with a tensor scale: bf16_RN(fp32_RN(fp32_RN(gs * s8) * T)))."""
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     tagged = np.ascontiguousarray(scales_tagged, dtype=scale_dtype(fmt))
     bits = None if choice_bits is None else np.ascontiguousarray(choice_bits, dtype=np.uint8)
     T_bf16 = np.ascontiguousarray(T_bf16, dtype=np.uint16)
     w_hat = np.empty((N, K), dtype=np.uint16)
     lib().orc_dequant_bf16(_p(codes), _p(tagged), _p(bits), _p(T_bf16), N, K, fmt, g, S,
-                           _p(w_hat))
+                           _p(w_hat), float(gs))
     return w_hat
 
 
@@ -331,10 +346,10 @@ def linear(X_u16, w_hat_u16):
 def run_layer(W_u16, X_u16, fmt, g, S, iters, flags=0):
     """importance -> init -> fit -> pack, all on the CPU."""
     I = importance(X_u16)
-    scl, T0 = init_codebooks(W_u16, fmt, g)
-    T, err, st = fit(W_u16, I, scl, T0, fmt, g, S, iters, flags)
-    out = pack(W_u16, I, scl, T, fmt, g, S, flags)
-    out.update(I=I, scales=scl, T_init=T0, T=T, err_hist=err, stats=st)
+    scl, T0, gs = init_codebooks(W_u16, fmt, g, with_gs=True)
+    T, err, st = fit(W_u16, I, scl, T0, fmt, g, S, iters, flags, gs)
+    out = pack(W_u16, I, scl, T, fmt, g, S, flags, gs)
+    out.update(I=I, scales=scl, T_init=T0, T=T, err_hist=err, stats=st, gs=gs)
     return out
 
 
@@ -360,11 +375,11 @@ def awq_search(W_u16, I, tokens, fmt, g, S, iters, js, flags=0):
     best = None
     for idx, j in enumerate(js):
         c, Is, Ws = awq_prescale(W_u16, I, tokens, j)
-        scl, T0 = init_codebooks(Ws, fmt, g)
-        T, err, st = fit(Ws, Is, scl, T0, fmt, g, S, iters, flags)
-        out = pack(Ws, Is, scl, T, fmt, g, S, flags)
+        scl, T0, gs = init_codebooks(Ws, fmt, g, with_gs=True)
+        T, err, st = fit(Ws, Is, scl, T0, fmt, g, S, iters, flags, gs)
+        out = pack(Ws, Is, scl, T, fmt, g, S, flags, gs)
         errs.append(out["err_final"])
         if best is None or out["err_final"] < errs[best[0]]:
-            out.update(c=c, I=Is, W=Ws, scales=scl, T=T, err_hist=err, stats=st)
+            out.update(c=c, I=Is, W=Ws, scales=scl, T=T, err_hist=err, stats=st, gs=gs)
             best = (idx, out)
     return dict(best=best[0], err_alpha=np.array(errs, dtype=np.float64), **best[1])

@@ -43,6 +43,7 @@ typedef __int128 i128;
 
 #define ORC_INT4 0
 #define ORC_NVFP4 1
+#define ORC_NVFP4_GS 2   /* NVFP4 with a per-tensor fp32 scale (reading R17) */
 #define ORC_FREEZE_T0 1u
 #define ORC_FREEZE_T1 2u
 #define ORC_SINGLE_CODEBOOK 4u
@@ -256,9 +257,25 @@ void orc_importance(const uint16_t* X, int64_t T, int64_t K, int64_t ldx,
 /* ------------------------------------------------------------------------ */
 /* R1: per-group absmax scale.  INT4: s = bf16_RN(fp32_RN(a / 7)).           */
 /*     NVFP4: s = e4m3_RN_satfinite(a).  a = max |w| over the g weights.     */
+/* R17: NVFP4 with a per-tensor fp32 scale gs = fp32_RN(amax / 448), amax    */
+/*     the largest |w| of the tensor (gs = 0 when amax = 0); the stored     */
+/*     group scale is s8 = e4m3_RN_satfinite(fp32_RN(a / gs)) (0 when       */
+/*     gs = 0) and the group's effective scale is fp32_RN(gs * s8).  The    */
+/*     largest group maps to the top of E4M3's range, so small weights keep */
+/*     normal (4-significant-bit) scales instead of E4M3 subnormals.        */
 /* ------------------------------------------------------------------------ */
 
-void orc_scales(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* scales)
+float orc_global_scale(const uint16_t* W, int64_t N, int64_t K)
+{
+    float a = 0.0f;
+    for (int64_t i = 0; i < N * K; i++) {
+        float w = fabsf(orc_bf16_to_f32(W[i]));
+        if (w > a) a = w;
+    }
+    return a > 0.0f ? a / 448.0f : 0.0f;
+}
+
+void orc_scales(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* scales, float gs)
 {
     int64_t G = K / g;
 #pragma omp parallel for schedule(static)
@@ -272,19 +289,28 @@ void orc_scales(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* s
             if (fmt == ORC_INT4) {
                 float d = a / 7.0f;
                 ((uint16_t*)scales)[r * G + j] = orc_f32_to_bf16_rn(d);
-            } else {
+            } else if (fmt == ORC_NVFP4) {
                 ((uint8_t*)scales)[r * G + j] = orc_f32_to_e4m3_rn_sat(a);
+            } else {
+                ((uint8_t*)scales)[r * G + j] = gs > 0.0f ? orc_f32_to_e4m3_rn_sat(a / gs) : 0;
             }
         }
     }
 }
 
 /* Decoded magnitude of a stored scale; the sign bit (a choice tag) is
- * ignored. */
+ * ignored.  For NVFP4 with a tensor scale this is the E4M3 factor s8. */
 static float scale_value(const void* scales, int fmt, int64_t idx)
 {
     if (fmt == ORC_INT4) return orc_bf16_to_f32(((const uint16_t*)scales)[idx] & 0x7fffu);
     return orc_e4m3_to_f32(((const uint8_t*)scales)[idx] & 0x7fu);
+}
+
+/* The scale that multiplies the codebook value: s itself, or fp32_RN(gs * s8)
+ * with a tensor scale (R17). */
+static float eff_scale(float s, int fmt, float gs)
+{
+    return fmt == ORC_NVFP4_GS ? gs * s : s;
 }
 
 /* R2: r = fp32_RN(1/s); u = fp32_RN(w * r).  A group is "live" when s > 0
@@ -300,14 +326,15 @@ static int group_live(float s, float* r_out)
 }
 
 void orc_u(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, const void* scales,
-           float* u)
+           float* u, float gs)
 {
     int64_t G = K / g;
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < N; r++) {
         for (int64_t k = 0; k < K; k++) {
             float s = scale_value(scales, fmt, r * G + k / g), rc;
-            if (group_live(s, &rc)) u[r * K + k] = orc_bf16_to_f32(W[r * K + k]) * rc;
+            if (group_live(eff_scale(s, fmt, gs), &rc))
+                u[r * K + k] = orc_bf16_to_f32(W[r * K + k]) * rc;
             else u[r * K + k] = 0.0f;
         }
     }
@@ -344,15 +371,17 @@ int64_t orc_rank_t1(int64_t M, int n, int j)
 }
 
 int orc_init_codebooks(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* scales,
-                       float* T /* [2][16] */)
+                       float* T /* [2][16] */, float* gs_out /* NVFP4_GS: the tensor scale */)
 {
     int64_t M = N * K;
     int n = (fmt == ORC_INT4) ? 16 : 15;
-    orc_scales(W, N, K, fmt, g, scales);
+    float gs = fmt == ORC_NVFP4_GS ? orc_global_scale(W, N, K) : 0.0f;
+    if (gs_out) *gs_out = gs;
+    orc_scales(W, N, K, fmt, g, scales, gs);
     float* u = (float*)malloc(sizeof(float) * (size_t)M);
     uint32_t* key = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)M);
     if (!u || !key) { free(u); free(key); return 1; }
-    orc_u(W, N, K, fmt, g, scales, u);
+    orc_u(W, N, K, fmt, g, scales, u, gs);
     for (int64_t i = 0; i < M; i++) key[i] = total_order_key(u[i]);
     qsort(key, (size_t)M, sizeof(uint32_t), cmp_u32);
     for (int j = 0; j < 16; j++) {
@@ -537,6 +566,7 @@ typedef struct {
     const void* scales;
     int fmt, g, S, n;
     unsigned flags;
+    float gs;  /* tensor scale (NVFP4_GS only) */
 } layer_t;
 
 /* One assign pass with codebooks T ([2][16]).  Fills per-group choice and
@@ -566,7 +596,7 @@ static void assign_pass(const layer_t* Ly, const float* T, int L, uint8_t* choic
             for (int64_t j = 0; j < NS; j++) {
                 int64_t k0 = j * S;
                 float s = scale_value(Ly->scales, Ly->fmt, r * G + k0 / Ly->g), rc;
-                int live = group_live(s, &rc);
+                int live = group_live(eff_scale(s, Ly->fmt, Ly->gs), &rc);
                 for (int i = 0; i < S; i++) {
                     u[i] = live ? orc_bf16_to_f32(Ly->W[r * K + k0 + i]) * rc : 0.0f;
                     Ik[i] = Ly->I[k0 + i];
@@ -625,7 +655,7 @@ static void layer_maxima(const layer_t* Ly, double* I_max, double* S2_max, doubl
     for (int64_t r = 0; r < N; r++) {
         for (int64_t j = 0; j < G; j++) {
             float s = scale_value(Ly->scales, Ly->fmt, r * G + j), rc;
-            if (!group_live(s, &rc)) { nd++; continue; }
+            if (!group_live(eff_scale(s, Ly->fmt, Ly->gs), &rc)) { nd++; continue; }
             double s2 = (double)s * (double)s;
             if (s2 > sm) sm = s2;
             for (int i = 0; i < Ly->g; i++) {
@@ -640,9 +670,9 @@ static void layer_maxima(const layer_t* Ly, double* I_max, double* S2_max, doubl
 
 int orc_fit(const uint16_t* W, int64_t N, int64_t K, const float* I, const void* scales,
             int fmt, int g, int S, int iters, unsigned flags, float* T /* [2][16] inout */,
-            double* err_hist, orc_stats* st)
+            double* err_hist, orc_stats* st, float gs)
 {
-    layer_t Ly = { W, N, K, I, scales, fmt, g, S, (fmt == ORC_INT4) ? 16 : 15, flags };
+    layer_t Ly = { W, N, K, I, scales, fmt, g, S, (fmt == ORC_INT4) ? 16 : 15, flags, gs };
     int64_t NS = N * (K / S);
     uint8_t* choice = (uint8_t*)malloc((size_t)NS);
     double* D = (double*)malloc(sizeof(double) * (size_t)NS);
@@ -668,7 +698,9 @@ int orc_fit(const uint16_t* W, int64_t N, int64_t K, const float* I, const void*
             err = err + s2[i] * D[i];
             nt1 += choice[i];
         }
-        err_hist[it] = err;
+        /* R17: the centroid weights and this sum use s8; the tensor scale is
+         * common to every group and enters the objective as one factor. */
+        err_hist[it] = fmt == ORC_NVFP4_GS ? err * ((double)gs * (double)gs) : err;
         local.near_ties = ties;
         local.groups_t1 = nt1;
         local.empty_cells = 0;
@@ -698,9 +730,9 @@ int orc_pack(const uint16_t* W, int64_t N, int64_t K, const float* I, const void
              int fmt, int g, int S, unsigned flags, const float* T_in /* [2][16] */,
              uint16_t* T_bf16 /* [2][16] */, uint8_t* codes /* [N][K/2] */,
              void* scales_tagged /* like scales */, uint8_t* choice_bits /* [N][K/S/8] */,
-             double* err_final, int64_t* near_ties)
+             double* err_final, int64_t* near_ties, float gs)
 {
-    layer_t Ly = { W, N, K, I, scales, fmt, g, S, (fmt == ORC_INT4) ? 16 : 15, flags };
+    layer_t Ly = { W, N, K, I, scales, fmt, g, S, (fmt == ORC_INT4) ? 16 : 15, flags, gs };
     int64_t G = K / g, NS = K / S;
     float T[32], Tq[32];
     memcpy(T, T_in, sizeof(T));
@@ -743,7 +775,7 @@ int orc_pack(const uint16_t* W, int64_t N, int64_t K, const float* I, const void
     double err = 0.0;
     for (int64_t r = 0; r < N; r++)
         for (int64_t k = 0; k < K; k++) {
-            float s = scale_value(scales, fmt, r * G + k / g);
+            float s = eff_scale(scale_value(scales, fmt, r * G + k / g), fmt, gs);
             int c = choice[r * NS + k / S];
             double wh = (double)s * (double)Tq[c * 16 + q[r * K + k]];
             double d = (double)orc_bf16_to_f32(W[r * K + k]) - wh;
@@ -757,7 +789,7 @@ int orc_pack(const uint16_t* W, int64_t N, int64_t K, const float* I, const void
 /* Per-weight dequantisation from the packed format (round-trip checks). */
 void orc_unpack(const uint8_t* codes, const void* scales_tagged, const uint8_t* choice_bits,
                 const uint16_t* T_bf16, int64_t N, int64_t K, int fmt, int g, int S,
-                float* w_hat, uint8_t* choice_per_group /* [N][K/S] */)
+                double* w_hat, uint8_t* choice_per_group /* [N][K/S] */, float gs)
 {
     int64_t G = K / g, NS = K / S, nb = (NS + 7) / 8;
     for (int64_t r = 0; r < N; r++)
@@ -772,14 +804,14 @@ void orc_unpack(const uint8_t* codes, const void* scales_tagged, const uint8_t* 
             } else {
                 uint8_t v = ((const uint8_t*)scales_tagged)[gi];
                 tag = v >> 7;
-                s = orc_e4m3_to_f32(v & 0x7fu);
+                s = eff_scale(orc_e4m3_to_f32(v & 0x7fu), fmt, gs);
             }
             int64_t j = k / S;
             c = (S == g) ? tag : ((choice_bits[r * nb + j / 8] >> (j % 8)) & 1);
             if (k % S == 0) choice_per_group[r * NS + j] = (uint8_t)c;
             uint8_t byte = codes[r * (K / 2) + k / 2];
             int qv = (k & 1) ? (byte >> 4) : (byte & 15);
-            w_hat[r * K + k] = (float)((double)s * (double)orc_bf16_to_f32(T_bf16[c * 16 + qv]));
+            w_hat[r * K + k] = (double)s * (double)orc_bf16_to_f32(T_bf16[c * 16 + qv]);
         }
 }
 
@@ -789,17 +821,19 @@ void orc_unpack(const uint8_t* codes, const void* scales_tagged, const uint8_t* 
 /*      BF16 tables, choice in the scale's sign bit or in a bitmask).        */
 /*      w_hat[n][k] = bf16_RN(s[n][k/g] * T_bf16[c][code[n][k]]): the exact  */
 /*      product (at most 16 significant bits, exact in fp32) rounded once   */
-/*      to the 16-bit activation type.                                       */
+/*      to the 16-bit activation type.  With a tensor scale (R17) s is the  */
+/*      effective fp32 scale and the product is rounded to fp32 first:      */
+/*      w_hat = bf16_RN(fp32_RN(fp32_RN(gs * s8) * T)).                      */
 /* ------------------------------------------------------------------------ */
 void orc_dequant_bf16(const uint8_t* codes, const void* scales_tagged, const uint8_t* choice_bits,
                       const uint16_t* T_bf16, int64_t N, int64_t K, int fmt, int g, int S,
-                      uint16_t* w_hat)
+                      uint16_t* w_hat, float gs)
 {
-    float* wf = (float*)malloc(sizeof(float) * (size_t)(N * K));
+    double* wd = (double*)malloc(sizeof(double) * (size_t)(N * K));
     uint8_t* ch = (uint8_t*)malloc((size_t)(N * (K / S)));
-    orc_unpack(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S, wf, ch);
-    for (int64_t i = 0; i < N * K; i++) w_hat[i] = orc_f32_to_bf16_rn(wf[i]);
-    free(wf);
+    orc_unpack(codes, scales_tagged, choice_bits, T_bf16, N, K, fmt, g, S, wd, ch, gs);
+    for (int64_t i = 0; i < N * K; i++) w_hat[i] = orc_f32_to_bf16_rn((float)wd[i]);
+    free(wd);
     free(ch);
 }
 
