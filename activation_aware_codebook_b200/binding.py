@@ -15,6 +15,7 @@ import torch
 
 INT4 = 0
 NVFP4 = 1
+NVFP4_GS = 2  # NVFP4 with a per-tensor fp32 scale
 FREEZE_T0 = 1
 FREEZE_T1 = 2
 SINGLE_CODEBOOK = 4
@@ -42,7 +43,8 @@ class AaacError(RuntimeError):
 
 class CConfig(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("g", ctypes.c_int32), ("S", ctypes.c_int32),
-                ("iters", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+                ("iters", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("global_scale", ctypes.c_void_p)]
 
 
 class CStats(ctypes.Structure):
@@ -62,9 +64,17 @@ class Config:
     S: int = 128
     iters: int = 20
     flags: int = 0
+    # NVFP4_GS: device fp32 [1] holding the per-tensor scale (init_codebooks
+    # allocates it on the weights' device when it is None)
+    global_scale: Optional[torch.Tensor] = None
 
     def c(self) -> CConfig:
-        return CConfig(self.fmt, self.g, self.S, self.iters, self.flags)
+        gs = self.global_scale.data_ptr() if self.global_scale is not None else None
+        return CConfig(self.fmt, self.g, self.S, self.iters, self.flags, gs)
+
+    def ensure_global_scale(self, device) -> None:
+        if self.fmt == NVFP4_GS and self.global_scale is None:
+            self.global_scale = torch.zeros(1, dtype=torch.float32, device=device)
 
     @property
     def n(self) -> int:
@@ -197,6 +207,7 @@ def init_codebooks(W: torch.Tensor, cfg: Config, ws: Optional[torch.Tensor] = No
         T = torch.empty(2, 16, dtype=torch.float32, device=W.device)
     if ws is None:
         ws = workspace(cfg, N, K, 0, W.device)
+    cfg.ensure_global_scale(W.device)
     c = cfg.c()
     _check(load().aaac_init_codebooks(_ptr(W), N, K, ctypes.byref(c), _ptr(scales), _ptr(T),
                                       _ptr(ws), ws.numel(), _stream(stream)))
@@ -326,6 +337,7 @@ def run_layer(W: torch.Tensor, X: torch.Tensor, cfg: Config, ws: Optional[torch.
     T_init = T.clone()
     T, err_hist, stats = fit_layer(W, I, scales, T, cfg, ws=ws, stream=stream)
     out = pack(W, I, scales, T, cfg, ws=ws, stream=stream)
+    out.update(global_scale=cfg.global_scale)
     out.update(I=I, scales=scales, T_init=T_init, T=T, err_hist=err_hist[:cfg.iters],
                stats=stats)
     return out
@@ -358,6 +370,7 @@ def awq_fit(W: torch.Tensor, I: torch.Tensor, tokens: int, cfg: Config, alphas16
     N, K = W.shape
     dev = W.device
     js = (ctypes.c_int32 * len(alphas16))(*[int(j) for j in alphas16])
+    cfg.ensure_global_scale(dev)
     c_cfg = cfg.c()
     if ws is None:
         need = load().aaac_awq_workspace_size(ctypes.byref(c_cfg), N, K)

@@ -41,10 +41,17 @@ bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 aaac_status check_cfg(const aaac_config* cfg) {
   if (!cfg) return fail(AAAC_ERR_INVALID_ARG, "cfg is NULL");
-  if (cfg->fmt != AAAC_INT4 && cfg->fmt != AAAC_NVFP4)
-    return fail(AAAC_ERR_UNSUPPORTED, "fmt %d is not AAAC_INT4 or AAAC_NVFP4", cfg->fmt);
-  if (cfg->fmt == AAAC_NVFP4 && cfg->g != 16)
+  if (cfg->fmt != AAAC_INT4 && cfg->fmt != AAAC_NVFP4 && cfg->fmt != AAAC_NVFP4_GS)
+    return fail(AAAC_ERR_UNSUPPORTED, "fmt %d is not AAAC_INT4, AAAC_NVFP4 or AAAC_NVFP4_GS",
+                cfg->fmt);
+  if (cfg->fmt != AAAC_INT4 && cfg->g != 16)
     return fail(AAAC_ERR_UNSUPPORTED, "NVFP4 needs g == 16 (got %d)", cfg->g);
+  if (cfg->fmt == AAAC_NVFP4_GS) {
+    if (!cfg->global_scale)
+      return fail(AAAC_ERR_INVALID_ARG, "AAAC_NVFP4_GS needs cfg->global_scale");
+    if (reinterpret_cast<uintptr_t>(cfg->global_scale) & 3u)
+      return fail(AAAC_ERR_ALIGN, "cfg->global_scale is not 4-byte aligned");
+  }
   if (!pow2(cfg->g) || cfg->g < 16 || cfg->g > 256)
     return fail(AAAC_ERR_UNSUPPORTED, "g must be a power of two in [16, 256] (got %d)", cfg->g);
   if (!pow2(cfg->S) || cfg->S < 8 || cfg->S > cfg->g)
@@ -96,7 +103,7 @@ size_t weight_side_bytes(const aaac_config* cfg, int64_t N, int64_t K) {
 // Workspace of aaac_awq_fit: the rescaled layer, one candidate's fit state
 // and packed output, and the fit's own workspace (shared by init, fit, pack).
 struct AwqLayout {
-  size_t Ws, Is, c, scales, T, Tb, codes, tagged, bits, hist, stats, fit, total;
+  size_t Ws, Is, c, scales, T, Tb, codes, tagged, bits, hist, stats, gs, fit, total;
 };
 AwqLayout awq_layout(const aaac_config* cfg, int64_t N, int64_t K) {
   AwqLayout L{};
@@ -120,6 +127,7 @@ AwqLayout awq_layout(const aaac_config* cfg, int64_t N, int64_t K) {
   L.bits = take((size_t)N * nb);
   L.hist = take((size_t)(cfg->iters > 0 ? cfg->iters : 1) * 8);
   L.stats = take(sizeof(aaac_stats));
+  L.gs = take(sizeof(float));
   L.fit = take(weight_side_bytes(cfg, N, K));
   L.total = o;
   return L;
@@ -176,7 +184,7 @@ aaac_status aaac_init_codebooks(const void* W, int64_t N, int64_t K, const aaac_
   CHECK(check_ptr(T, "T"));
   CHECK(check_ws(ws, ws_bytes, aaac::init_ctl_bytes()));
   return from_cuda(aaac::launch_init(reinterpret_cast<const uint16_t*>(W), N, K, cfg->fmt, cfg->g,
-                                     scales, T, ws, (cudaStream_t)stream),
+                                     scales, T, ws, cfg->global_scale, (cudaStream_t)stream),
                    "aaac_init_codebooks");
 }
 
@@ -195,7 +203,7 @@ aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
   CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K)));
   return from_cuda(aaac::launch_fit(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
                                     cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T, err_hist,
-                                    stats, ws, (cudaStream_t)stream),
+                                    stats, ws, cfg->global_scale, (cudaStream_t)stream),
                    "aaac_fit_layer");
 }
 
@@ -221,7 +229,7 @@ aaac_status aaac_fit_layer_fixed_scratch(const void* W, int64_t N, int64_t K, co
   if (e != cudaSuccess) return from_cuda(e, "aaac_fit_layer_fixed_scratch: scratch address");
   return from_cuda(aaac::launch_fit(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
                                     cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T, err_hist,
-                                    stats, ws, (cudaStream_t)stream),
+                                    stats, ws, cfg->global_scale, (cudaStream_t)stream),
                    "aaac_fit_layer_fixed_scratch");
 }
 
@@ -243,7 +251,7 @@ aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const
   CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K) + aaac::pack_extra_bytes(N, K, cfg->S)));
   return from_cuda(aaac::launch_pack(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
                                      cfg->fmt, cfg->g, cfg->S, cfg->flags, T, T_bf16, codes,
-                                     scales_tagged, choice_bits, err_final, ws,
+                                     scales_tagged, choice_bits, err_final, ws, cfg->global_scale,
                                      (cudaStream_t)stream),
                    "aaac_pack");
 }
@@ -259,7 +267,8 @@ aaac_status aaac_dequant(const uint8_t* codes, const void* scales_tagged,
   CHECK(check_ptr(T_bf16, "T_bf16"));
   CHECK(check_ptr(W_hat, "W_hat"));
   return from_cuda(aaac::launch_dequant(codes, scales_tagged, choice_bits, T_bf16, N, K, cfg->fmt,
-                                        cfg->g, cfg->S, W_hat, (cudaStream_t)stream),
+                                        cfg->g, cfg->S, W_hat, cfg->global_scale,
+                                        (cudaStream_t)stream),
                    "aaac_dequant");
 }
 
@@ -284,7 +293,7 @@ aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* co
   CHECK(check_ptr(Y, "Y"));
   return from_cuda(aaac::launch_linear(reinterpret_cast<const uint16_t*>(X), M, ldx, codes,
                                        scales_tagged, choice_bits, T_bf16, N, K, cfg->fmt,
-                                       cfg->g, cfg->S, Y, (cudaStream_t)stream),
+                                       cfg->g, cfg->S, Y, cfg->global_scale, (cudaStream_t)stream),
                    "aaac_linear");
 }
 
@@ -355,27 +364,29 @@ aaac_status aaac_awq_fit(const void* W, int64_t N, int64_t K, const float* I, in
   double* hist = reinterpret_cast<double*>(base + L.hist);
   aaac_stats* stats = reinterpret_cast<aaac_stats*>(base + L.stats);
   void* fws = base + L.fit;
+  // candidates keep their tensor scale (NVFP4_GS) in the workspace; the kept
+  // one is copied to cfg->global_scale with the rest of its output
+  float* gs = cfg->fmt == AAAC_NVFP4_GS ? reinterpret_cast<float*>(base + L.gs) : nullptr;
   cudaStream_t st = (cudaStream_t)stream;
   const int64_t G = K / cfg->g;
   const size_t es = cfg->fmt == AAAC_INT4 ? 2 : 1;
-  const void* src[5] = {cod, tag, Tb, cc, bits};
-  void* dst[5] = {codes, scales_tagged, T_bf16, c, choice_bits};
-  const size_t bytes[5] = {(size_t)(N * K / 2), (size_t)(N * G) * es, 2 * 16 * 2,
-                           (size_t)K * 4, bits ? (size_t)N * ((K / cfg->S + 7) / 8) : 0};
-  const int segs = bits ? 5 : 4;
+  const void* src[6] = {cod, tag, Tb, cc, bits, gs};
+  void* dst[6] = {codes, scales_tagged, T_bf16, c, choice_bits, cfg->global_scale};
+  const size_t bytes[6] = {(size_t)(N * K / 2), (size_t)(N * G) * es, 2 * 16 * 2, (size_t)K * 4,
+                           bits ? (size_t)N * ((K / cfg->S + 7) / 8) : 0, gs ? sizeof(float) : 0};
   for (int i = 0; i < n_alpha; i++) {
     cudaError_t e = aaac::launch_awq_prescale(reinterpret_cast<const uint16_t*>(W), N, K, I,
                                               tokens, alpha16[i], cc, Is, Ws, st);
     if (e == cudaSuccess)
-      e = aaac::launch_init(Ws, N, K, cfg->fmt, cfg->g, scl, T, fws, st);
+      e = aaac::launch_init(Ws, N, K, cfg->fmt, cfg->g, scl, T, fws, gs, st);
     if (e == cudaSuccess)
       e = aaac::launch_fit(Ws, N, K, Is, scl, cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T,
-                           hist, stats, fws, st);
+                           hist, stats, fws, gs, st);
     if (e == cudaSuccess)
       e = aaac::launch_pack(Ws, N, K, Is, scl, cfg->fmt, cfg->g, cfg->S, cfg->flags, T, Tb, cod,
-                            tag, bits, err_alpha + i, fws, st);
+                            tag, bits, err_alpha + i, fws, gs, st);
     if (e == cudaSuccess)
-      e = aaac::launch_awq_keep(i, err_alpha, src, dst, bytes, segs, err_final, best, st);
+      e = aaac::launch_awq_keep(i, err_alpha, src, dst, bytes, 6, err_final, best, st);
     if (e != cudaSuccess) return from_cuda(e, "aaac_awq_fit");
   }
   return ok();

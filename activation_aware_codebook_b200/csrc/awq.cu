@@ -164,10 +164,12 @@ awq_weights_kernel(const uint4* __restrict__ W, uint32_t n_vec, uint32_t k_vec,
   }
 }
 
+constexpr int kKeepSegs = 6;
+
 struct KeepArgs {
-  const unsigned char* src[5];
-  unsigned char* dst[5];
-  size_t bytes[5];
+  const unsigned char* src[kKeepSegs];
+  unsigned char* dst[kKeepSegs];
+  size_t bytes[kKeepSegs];
   int segs;
   int j;
   const double* err_alpha;
@@ -218,7 +220,8 @@ cudaError_t launch_awq_keep(int j, const double* err_alpha, const void* const* s
                             int32_t* best, cudaStream_t st) {
   KeepArgs a{};
   size_t total = 0;
-  for (int s = 0; s < segs && s < 5; s++) {
+  for (int s = 0; s < segs && s < kKeepSegs; s++) {
+    if (bytes[s] == 0) continue;  // absent output (no choice bits, no tensor scale)
     a.src[a.segs] = static_cast<const unsigned char*>(src[s]);
     a.dst[a.segs] = static_cast<unsigned char*>(dst[s]);
     a.bytes[a.segs] = bytes[s];

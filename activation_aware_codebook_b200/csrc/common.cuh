@@ -17,6 +17,7 @@ namespace aaac {
 
 constexpr int kInt4 = 0;
 constexpr int kNvfp4 = 1;
+constexpr int kNvfp4G = 2;            // NVFP4 with a per-tensor fp32 scale
 constexpr int kWarps = 8;             // warps per block of the streaming kernels
 constexpr int kThreads = kWarps * 32;
 constexpr int kSegCols = 256;         // columns a warp covers per row (32 lanes x 8)
@@ -45,6 +46,13 @@ __device__ __forceinline__ float load_scale(const void* scales, int64_t idx) {
     uint32_t v = __ldg(reinterpret_cast<const unsigned char*>(scales) + idx);
     return e4m3_mag(v & 0x7fu);
   }
+}
+
+// The scale that multiplies a codebook value: the stored scale itself, or,
+// with a per-tensor scale gs, fp32_RN(gs * s8) for the stored E4M3 factor s8.
+template <int FMT>
+__device__ __forceinline__ float eff_scale(float s, float gs) {
+  return FMT == kNvfp4G ? __fmul_rn(gs, s) : s;
 }
 
 // r = fp32_RN(1/s); a group is live when s > 0 and r is finite.

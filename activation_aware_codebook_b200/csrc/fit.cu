@@ -343,8 +343,10 @@ __device__ void store_tables(FitCtl* ctl, const Tables& tb) {
 template <int FMT>
 __global__ void __launch_bounds__(kThreads)
 fit_prep(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
-         const void* __restrict__ scales, int g, FitCtl* ctl, int ncb, int rows_per_chunk) {
+         const void* __restrict__ scales, int g, FitCtl* ctl, int ncb, int rows_per_chunk,
+         const float* __restrict__ gsc) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float gsv = FMT == kNvfp4G ? __ldg(gsc) : 1.0f;
   uint32_t im = 0;
   for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < K; k += gridDim.x * blockDim.x)
     im = max(im, __float_as_uint(I[k]));
@@ -361,7 +363,7 @@ fit_prep(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     for (int r = r0 + warp; r < r1; r += kWarps) {
       const float s = load_scale<FMT>(scales, (int64_t)r * G + col0 / g);
       float rcp;
-      if (!scale_live(s, &rcp)) {
+      if (!scale_live(eff_scale<FMT>(s, gsv), &rcp)) {
         if ((lane & (lanes_g - 1)) == 0) dead++;
         continue;
       }
@@ -397,14 +399,16 @@ __device__ inline int frexp_exponent(double x) {
 
 // 2^Le for the objective sums: every contribution is a group's s^2 D (or a
 // row's weight-space error), rounded to an integer after scaling by 2^Le.
-// Both are below M * I_max * S2_max * (2 U_max)^2 in total (|u - T| <= 2 U_max,
-// |w - s T| <= 2 sqrt(S2_max) U_max), and Le keeps that bound below 2^61, so
-// the int64 sums cannot overflow and do not depend on the order of addition.
-__device__ double objective_scale(const FitCtl* ctl, int64_t M) {
+// Both are below M * I_max * S2_max * g2 * (2 U_max)^2 in total (|u - T| <=
+// 2 U_max, |w - s T| <= 2 sqrt(S2_max g2) U_max, g2 the square of a per-tensor
+// scale for the weight-space error, else 1), and Le keeps that bound below
+// 2^61, so the int64 sums cannot overflow and do not depend on the order of
+// addition.
+__device__ double objective_scale(const FitCtl* ctl, int64_t M, double g2 = 1.0) {
   const double Imax = (double)__uint_as_float(ctl->Imax_bits);
   const double S2max = __longlong_as_double((long long)ctl->S2max_bits);
   const double Umax = (double)__uint_as_float(ctl->Umax_bits);
-  const double bound = (double)M * Imax * S2max * 4.0 * Umax * Umax;
+  const double bound = (double)M * Imax * S2max * g2 * 4.0 * Umax * Umax;
   if (!(bound > 0.0)) return 1.0;
   int Le = 61 - frexp_exponent(bound);
   if (Le > 1000) Le = 1000;
@@ -526,7 +530,7 @@ __device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsign
 // fp64(den)) when den > 0, else unchanged; then sorted books and new tables.
 // Everything is staged in shared memory and spread over the block's threads.
 __device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const RoundOut& ro,
-                               int cpc, int n_items) {
+                               int cpc, int n_items, double g2) {
   __shared__ float sT[2][16];
   __shared__ long long sb[64];
   __shared__ int s_upd[2];
@@ -536,7 +540,9 @@ __device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const Ro
   if (tid < 2) s_upd[tid] = 0;
   if (tid == 0) {
     const long long acc = (long long)__ldcg(&ctl->err_acc);
-    if (ro.err_hist) ro.err_hist[ro.it] = (double)acc / ctl->twoLe;
+    // the rounds sum s^2 D with the stored scale factor; a per-tensor scale
+    // enters the objective once, as g2 = gs^2
+    if (ro.err_hist) ro.err_hist[ro.it] = __dmul_rn((double)acc / ctl->twoLe, g2);
     ctl->err_acc = 0ull;
   }
   __syncthreads();
@@ -665,7 +671,7 @@ __global__ void __launch_bounds__(kFitThreads, kFitBlocksPerSM)
 fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
          const void* __restrict__ scales, int g, int S, uint32_t flags, FitCtl* ctl,
          int cpc, int n_items, int max_items, float tau, PackOut po,
-         RoundOut ro) {
+         RoundOut ro, const float* __restrict__ gsc) {
   extern __shared__ __align__(128) unsigned char smem[];
   Tables& tb = *reinterpret_cast<Tables*>(smem);
   unsigned char* ring = smem + kTablesBytes;
@@ -687,6 +693,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   const int lanes_s = S >> 4;               // lanes per choice group when S >= 16
   const int leader_lane = S >= 16 ? (lane & ~(lanes_s - 1)) : lane;
   const bool single = (flags & AAAC_SINGLE_CODEBOOK) != 0;
+  const float gsv = FMT == kNvfp4G ? __ldg(gsc) : 1.0f;  // written before the fit starts
   unsigned char* wring = ring + warp * kStages * kRingRowBytes;
   const int wr0 = ring_slot(lane) * 16, wr1 = ring_slot(32 + lane) * 16;
   const int rd0 = ring_slot(2 * lane) * 16, rd1 = ring_slot(2 * lane + 1) * 16;
@@ -893,7 +900,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     slot = (slot + 1 == kStages) ? 0 : slot + 1;
 
     float rcp;
-    const bool live = active && scale_live(s, &rcp);  // dead: rcp = 0, u = +-0
+    const bool live = active && scale_live(eff_scale<FMT>(s, gsv), &rcp);  // dead: u = +-0
     const uint32_t wv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
     const unsigned long long rr2 = f2pack(rcp, rcp);
     unsigned long long u2[8];
@@ -1027,7 +1034,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
         const Book& bc = tb.bk[ch[h]];
         packed |= (unsigned long long)bc.idx[q] << (4 * i);
         const float wf = (i & 1) ? bf16_hi(wv[i >> 1]) : bf16_lo(wv[i >> 1]);
-        const double wh = (double)s * (double)bc.val[q];
+        const double wh = (double)eff_scale<FMT>(s, gsv) * (double)bc.val[q];
         const double d = __dsub_rn((double)wf, wh);
         err_w = __fma_rn(Id[i], __dmul_rn(d, d), err_w);
       }
@@ -1097,7 +1104,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   if (!s_last) return;
   __threadfence();
   if (!PACK) {
-    round_finalize(ctl, tb, flags, ro, cpc, n_items);
+    round_finalize(ctl, tb, flags, ro, cpc, n_items, __dmul_rn((double)gsv, (double)gsv));
   } else {
     if (threadIdx.x == 0) {
       const long long acc = (long long)__ldcg(&ctl->err_acc);
@@ -1125,7 +1132,7 @@ template <int FMT>
 static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const float* I,
                                 const void* scales, int g, int S, int iters, uint32_t flags,
                                 float* T, double* err_hist, aaac_stats* stats, void* ws,
-                                cudaStream_t st) {
+                                const float* gsc, cudaStream_t st) {
   // per call: the attribute belongs to the current device's copy of the kernel
   const cudaError_t attr = set_smem<FMT, false>();
   if (attr != cudaSuccess) return attr;
@@ -1134,7 +1141,7 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
-                                                   pprep.ncb, pprep.rows_per_chunk);
+                                                   pprep.ncb, pprep.rows_per_chunk, gsc);
   fit_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), stats, pp.blocks * kFitWarps,
                                        pp.cpc, pp.items);
   const float tau = choice_tau(S);
@@ -1155,7 +1162,7 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
     const cudaError_t e = cudaLaunchKernelEx(
         &lc, fit_pass<FMT, false>, W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items,
         pp.max_items, tau, PackOut{nullptr, nullptr, nullptr, nullptr},
-        RoundOut{err_hist, T, stats, it});
+        RoundOut{err_hist, T, stats, it}, gsc);
     if (e != cudaSuccess) return e;
   }
   count_launches(2 + iters);
@@ -1164,12 +1171,15 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
 
 cudaError_t launch_fit(const uint16_t* W, int64_t N, int64_t K, const float* I,
                        const void* scales, int fmt, int g, int S, int iters, uint32_t flags,
-                       float* T, double* err_hist, aaac_stats* stats, void* ws, cudaStream_t st) {
-  cudaError_t e = (fmt == kInt4)
-                      ? launch_fit_t<kInt4>(W, N, K, I, scales, g, S, iters, flags, T, err_hist,
-                                            stats, ws, st)
-                      : launch_fit_t<kNvfp4>(W, N, K, I, scales, g, S, iters, flags, T, err_hist,
-                                             stats, ws, st);
+                       float* T, double* err_hist, aaac_stats* stats, void* ws, const float* gsc,
+                       cudaStream_t st) {
+  cudaError_t e =
+      (fmt == kInt4) ? launch_fit_t<kInt4>(W, N, K, I, scales, g, S, iters, flags, T, err_hist,
+                                           stats, ws, gsc, st)
+      : (fmt == kNvfp4) ? launch_fit_t<kNvfp4>(W, N, K, I, scales, g, S, iters, flags, T, err_hist,
+                                               stats, ws, gsc, st)
+                        : launch_fit_t<kNvfp4G>(W, N, K, I, scales, g, S, iters, flags, T,
+                                                err_hist, stats, ws, gsc, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1212,13 +1222,14 @@ cudaError_t fixed_scratch_ptr(void** out) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kFitThreads)
 pack_setup(FitCtl* ctl, const float* T_user, int64_t M, int n, uint16_t* T_bf16, int wt,
-           int cpc, int n_items) {
+           int cpc, int n_items, const float* gsc) {
   __shared__ Tables tb;
   __shared__ float sT[2][16];
   seed_claims(ctl, wt, cpc, n_items);
   if (threadIdx.x == 0) {
     ctl->n = n;
-    ctl->twoLe = objective_scale(ctl, M);
+    const double gs = gsc ? (double)*gsc : 1.0;  // the pack's error is in weight space
+    ctl->twoLe = objective_scale(ctl, M, gs * gs);
     ctl->err_acc = 0ull;
     tb.la = bucket_scale(ctl);
   }
@@ -1255,7 +1266,7 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
                                  const void* scales, int g, int S, uint32_t flags, const float* T,
                                  uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
                                  uint8_t* choice_bits, double* err_final, void* ws,
-                                 cudaStream_t st) {
+                                 const float* gsc, cudaStream_t st) {
   const cudaError_t attr = set_smem<FMT, true>();
   if (attr != cudaSuccess) return attr;
   const FitPlan pp = fit_plan(N, K);
@@ -1264,14 +1275,15 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
   uint8_t* cbytes = reinterpret_cast<uint8_t*>(ws) + fit_ws_bytes(N, K);
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
-                                                   pprep.ncb, pprep.rows_per_chunk);
+                                                   pprep.ncb, pprep.rows_per_chunk, gsc);
   pack_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), T_bf16,
-                                        pp.blocks * kFitWarps, pp.cpc, pp.items);
+                                        pp.blocks * kFitWarps, pp.cpc, pp.items,
+                                        FMT == kNvfp4G ? gsc : nullptr);
   const float tau = choice_tau(S);
   const PackOut po{codes, scales_tagged, cbytes, err_final};
   fit_pass<FMT, true><<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
       W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items, tau, po,
-      RoundOut{nullptr, nullptr, nullptr, 0});
+      RoundOut{nullptr, nullptr, nullptr, 0}, gsc);
   int launches = 3;
   if (S != g) {
     const int KS = (int)(K / S);
@@ -1286,12 +1298,16 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
 cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const float* I,
                         const void* scales, int fmt, int g, int S, uint32_t flags, const float* T,
                         uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
-                        uint8_t* choice_bits, double* err_final, void* ws, cudaStream_t st) {
-  cudaError_t e = (fmt == kInt4)
-                      ? launch_pack_t<kInt4>(W, N, K, I, scales, g, S, flags, T, T_bf16, codes,
-                                             scales_tagged, choice_bits, err_final, ws, st)
-                      : launch_pack_t<kNvfp4>(W, N, K, I, scales, g, S, flags, T, T_bf16, codes,
-                                              scales_tagged, choice_bits, err_final, ws, st);
+                        uint8_t* choice_bits, double* err_final, void* ws, const float* gsc,
+                        cudaStream_t st) {
+  cudaError_t e =
+      (fmt == kInt4) ? launch_pack_t<kInt4>(W, N, K, I, scales, g, S, flags, T, T_bf16, codes,
+                                            scales_tagged, choice_bits, err_final, ws, gsc, st)
+      : (fmt == kNvfp4) ? launch_pack_t<kNvfp4>(W, N, K, I, scales, g, S, flags, T, T_bf16, codes,
+                                                scales_tagged, choice_bits, err_final, ws, gsc, st)
+                        : launch_pack_t<kNvfp4G>(W, N, K, I, scales, g, S, flags, T, T_bf16,
+                                                 codes, scales_tagged, choice_bits, err_final, ws,
+                                                 gsc, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

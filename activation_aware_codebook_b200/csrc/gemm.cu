@@ -198,6 +198,26 @@ __device__ __forceinline__ uint4 expand8(uint32_t cw, uint32_t sbf, uint32_t c,
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// expand8 with an fp32 scale (NVFP4 with a per-tensor scale):
+// bf16_RN(fp32_RN(se * T)) per weight.
+__device__ __forceinline__ uint4 expand8g(uint32_t cw, float se, uint32_t c,
+                                          const unsigned short* sT) {
+  const uint32_t cb = c ? 0x20202020u : 0u;
+  const uint32_t ev = ((cw << 1) & 0x1e1e1e1eu) | cb;
+  const uint32_t od = ((cw >> 3) & 0x1e1e1e1eu) | cb;
+  const unsigned char* tb = reinterpret_cast<const unsigned char*>(sT);
+  uint32_t o[4];
+#pragma unroll
+  for (int p = 0; p < 4; p++) {
+    const uint32_t lo = *reinterpret_cast<const unsigned short*>(tb + __byte_perm(ev, 0u, 0x4440u + p));
+    const uint32_t hi = *reinterpret_cast<const unsigned short*>(tb + __byte_perm(od, 0u, 0x4440u + p));
+    const __nv_bfloat162 r = __floats2bfloat162_rn(__fmul_rn(se, __uint_as_float(lo << 16)),
+                                                   __fmul_rn(se, __uint_as_float(hi << 16)));
+    o[p] = *reinterpret_cast<const uint32_t*>(&r);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 struct GemmArgs {
   const uint8_t* codes;
   const void* tagged;
@@ -206,6 +226,7 @@ struct GemmArgs {
   float* Y;
   int M, N, K, lg, ls;
   int split;  // 1: one CTA per tile; 2: two K halves added into a zeroed Y
+  const float* gsc;  // per-tensor scale (NVFP4 with a tensor scale only)
 };
 
 template <int FMT, int BT>
@@ -290,6 +311,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
     const int h = p & 1;
     const int G = a.K >> a.lg, nb = ((a.K >> a.ls) + 7) >> 3;
     const bool sign_choice = a.lg == a.ls;
+    const float gsv = FMT == kNvfp4G ? __ldg(a.gsc) : 1.0f;
     const int rowi = p >> 1;
     const int nrow_p = n0 + rowi;
     const bool rok = nrow_p < a.N;
@@ -354,9 +376,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
           uint4 v = make_uint4(0u, 0u, 0u, 0u);
           if (rok && k < a.K) {
             uint32_t tag;
-            const uint32_t sbf = scale_bits<FMT>(R.sv[u][j >> 1], &tag);
-            const uint32_t ch = sign_choice ? tag : (R.cb[u] >> ((k >> a.ls) & 7)) & 1u;
-            v = expand8(words[j], sbf, ch, sT);
+            if (FMT == kNvfp4G) {
+              const uint32_t sv = R.sv[u][j >> 1];
+              tag = sv >> 7;
+              const uint32_t ch = sign_choice ? tag : (R.cb[u] >> ((k >> a.ls) & 7)) & 1u;
+              v = expand8g(words[j], __fmul_rn(gsv, e4m3_mag(sv & 0x7fu)), ch, sT);
+            } else {
+              const uint32_t sbf = scale_bits<FMT>(R.sv[u][j >> 1], &tag);
+              const uint32_t ch = sign_choice ? tag : (R.cb[u] >> ((k >> a.ls) & 7)) & 1u;
+              v = expand8(words[j], sbf, ch, sT);
+            }
           }
           const uint32_t c = (uint32_t)(h * 4 + j);
           *reinterpret_cast<uint4*>(dst + ((c ^ rsw) << 4)) = v;
@@ -471,22 +500,25 @@ cudaError_t launch_gemm_t(const uint16_t* X, int64_t M, int64_t ldx, const GemmA
 
 cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                         const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
-                        int64_t K, int fmt, int lg, int ls, float* Y, cudaStream_t st) {
-  GemmArgs ga{codes, tagged, cbits, Tb, Y, (int)M, (int)N, (int)K, lg, ls, 1};
-  cudaError_t e;
+                        int64_t K, int fmt, int lg, int ls, float* Y, const float* gsc,
+                        cudaStream_t st) {
+  GemmArgs ga{codes, tagged, cbits, Tb, Y, (int)M, (int)N, (int)K, lg, ls, 1, gsc};
   // token tile: 64 up to 64 tokens, then 128 (two CTAs fit on an SM), and 256
   // once there are at least two such tiles (less re-expansion of W per token)
-  if (M <= 64) {
-    e = fmt == kInt4 ? launch_gemm_t<kInt4, 64>(X, M, ldx, ga, st)
-                     : launch_gemm_t<kNvfp4, 64>(X, M, ldx, ga, st);
-  } else if (M < 512) {
-    e = fmt == kInt4 ? launch_gemm_t<kInt4, 128>(X, M, ldx, ga, st)
-                     : launch_gemm_t<kNvfp4, 128>(X, M, ldx, ga, st);
-  } else {
-    e = fmt == kInt4 ? launch_gemm_t<kInt4, 256>(X, M, ldx, ga, st)
+  const int bt = M <= 64 ? 64 : (M < 512 ? 128 : 256);
+  if (fmt == kInt4) {
+    return bt == 64 ? launch_gemm_t<kInt4, 64>(X, M, ldx, ga, st)
+         : bt == 128 ? launch_gemm_t<kInt4, 128>(X, M, ldx, ga, st)
+                     : launch_gemm_t<kInt4, 256>(X, M, ldx, ga, st);
+  }
+  if (fmt == kNvfp4) {
+    return bt == 64 ? launch_gemm_t<kNvfp4, 64>(X, M, ldx, ga, st)
+         : bt == 128 ? launch_gemm_t<kNvfp4, 128>(X, M, ldx, ga, st)
                      : launch_gemm_t<kNvfp4, 256>(X, M, ldx, ga, st);
   }
-  return e;
+  return bt == 64 ? launch_gemm_t<kNvfp4G, 64>(X, M, ldx, ga, st)
+       : bt == 128 ? launch_gemm_t<kNvfp4G, 128>(X, M, ldx, ga, st)
+                   : launch_gemm_t<kNvfp4G, 256>(X, M, ldx, ga, st);
 }
 
 cudaError_t gemm_timeout_flag(unsigned int* out) {

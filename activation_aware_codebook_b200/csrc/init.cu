@@ -16,6 +16,10 @@
 //                   match one of the (at most 32) prefixes still being
 //                   resolved, found with one probe of a two-entry-bucket hash
 //                   table in shared memory.
+//   tensor_amax     (NVFP4 with a per-tensor scale only) the largest |w| of
+//                   the tensor, as the max of the bf16 magnitude bits; every
+//                   radix pass then forms gs = fp32_RN(amax / 448) from it and
+//                   the first radix_select stores gs for the caller.
 //   radix_select    one thread per target rank walks its prefix's histogram
 //                   and fixes the next digit (4 passes of 8 bits resolve the
 //                   32-bit key exactly, ties included); it also builds the
@@ -34,6 +38,7 @@ struct InitCtl {
   int32_t nranks;
   int32_t n;
   uint32_t hmult;           // multiplier of the prefix hash (0: binary search)
+  uint32_t amax_bits;       // bf16 magnitude bits of the tensor's largest |w|
   uint4 htab[256];          // bucket: {prefix, slot, prefix, slot}, empty = ~0
   uint32_t hist[32][256];
 };
@@ -54,17 +59,43 @@ PassPlan plan_pass(int64_t N, int64_t K, int target, int seg_cols) {
 
 // Scale of one group from the max of its bf16 magnitude bits; *stored gets
 // the stored bits (bf16 for INT4, E4M3 for NVFP4), the result its value.
+// With a per-tensor scale gs the stored E4M3 factor is that of a / gs (0 when
+// gs is 0: the whole tensor is zero).
 template <int FMT>
-__device__ __forceinline__ float group_scale(uint32_t mx, uint32_t* stored) {
+__device__ __forceinline__ float group_scale(uint32_t mx, uint32_t* stored, float gs) {
   const float a = __uint_as_float(mx << 16);
   if (FMT == kInt4) {
     const __nv_bfloat16 s = __float2bfloat16_rn(__fdiv_rn(a, 7.0f));
     *stored = __bfloat16_as_ushort(s);
     return __uint_as_float(*stored << 16);
-  } else {
+  } else if (FMT == kNvfp4) {
     *stored = (uint32_t)__nv_cvt_float_to_fp8(a, __NV_SATFINITE, __NV_E4M3);
     return e4m3_mag(*stored & 0x7fu);
+  } else {
+    *stored = gs > 0.0f ? (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(a, gs), __NV_SATFINITE,
+                                                          __NV_E4M3)
+                        : 0u;
+    return e4m3_mag(*stored & 0x7fu);
   }
+}
+
+// gs = fp32_RN(amax / 448), 0 for a zero tensor.
+__device__ __forceinline__ float tensor_scale(uint32_t amax_bits) {
+  const float a = __uint_as_float(amax_bits << 16);
+  return a > 0.0f ? __fdiv_rn(a, 448.0f) : 0.0f;
+}
+
+__global__ void __launch_bounds__(kThreads)
+tensor_amax(const uint4* __restrict__ W, uint32_t n_vec, InitCtl* c) {
+  uint32_t mx = 0;
+  for (uint32_t i = blockIdx.x * kThreads + threadIdx.x; i < n_vec; i += gridDim.x * kThreads) {
+    const uint4 v = __ldg(W + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; k++) mx = max(mx, max(w[k] & 0x7fffu, (w[k] >> 16) & 0x7fffu));
+  }
+  for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0 && mx) atomicMax(&c->amax_bits, mx);
 }
 
 constexpr int kRadixRows = 4;  // rows per lane loaded ahead in a radix pass
@@ -87,6 +118,7 @@ __global__ void init_setup(InitCtl* c, RankInit ri, int nranks, int n) {
     c->nranks = nranks;
     c->n = n;
     c->hmult = 0u;
+    c->amax_bits = 0u;
   }
 }
 
@@ -101,7 +133,8 @@ struct RadixArgs {
 // passes with the prefix hash; 2: later passes with the binary search.
 template <int FMT, int MODE>
 __device__ __forceinline__ void radix_rows(const RadixArgs& a, uint32_t (*sh)[256], const uint4* tab,
-                                           uint32_t mult, const uint32_t* sp, int nslots) {
+                                           uint32_t mult, const uint32_t* sp, int nslots,
+                                           float gs) {
   const int shift = 24 - 8 * a.pass;
   const int K = a.K, g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -139,7 +172,7 @@ __device__ __forceinline__ void radix_rows(const RadixArgs& a, uint32_t (*sh)[25
         }
         for (int o = 1; o < lanes_g; o <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         uint32_t stored;
-        s = group_scale<FMT>(mx, &stored);
+        s = group_scale<FMT>(mx, &stored, gs);
         if (active && (lane & (lanes_g - 1)) == 0) {
           const int64_t gi = (int64_t)r * G + col0 / g;
           if (FMT == kInt4) reinterpret_cast<unsigned short*>(a.scales)[gi] = (unsigned short)stored;
@@ -147,7 +180,7 @@ __device__ __forceinline__ void radix_rows(const RadixArgs& a, uint32_t (*sh)[25
         }
       }
       float rcp;
-      const bool live = scale_live(s, &rcp);
+      const bool live = scale_live(eff_scale<FMT>(s, gs), &rcp);
 #pragma unroll
       for (int i = 0; i < 8; i++) {
         const float wf = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
@@ -198,9 +231,10 @@ radix_pass(RadixArgs a, InitCtl* c) {
   }
   __syncthreads();
   const int nslots = FIRST ? 1 : ns;
-  if (FIRST) radix_rows<FMT, 0>(a, sh, tab, 0u, sp, 1);
-  else if (smult) radix_rows<FMT, 1>(a, sh, tab, smult, sp, nslots);
-  else radix_rows<FMT, 2>(a, sh, tab, 0u, sp, nslots);
+  const float gs = FMT == kNvfp4G ? tensor_scale(c->amax_bits) : 1.0f;
+  if (FIRST) radix_rows<FMT, 0>(a, sh, tab, 0u, sp, 1, gs);
+  else if (smult) radix_rows<FMT, 1>(a, sh, tab, smult, sp, nslots, gs);
+  else radix_rows<FMT, 2>(a, sh, tab, 0u, sp, nslots, gs);
   __syncthreads();
   if (FIRST) {
     for (int d = threadIdx.x; d < 256; d += blockDim.x) {
@@ -221,7 +255,8 @@ radix_pass(RadixArgs a, InitCtl* c) {
 // the digit.  Warp 0 then sorts and deduplicates the new prefixes and builds
 // the next pass's prefix hash table (bucket (p * mult) >> 24 of 256, two
 // entries each; multipliers are tried until no bucket receives three).
-__global__ void __launch_bounds__(256) radix_select(InitCtl* c, int pass, float* T) {
+__global__ void __launch_bounds__(256) radix_select(InitCtl* c, int pass, float* T,
+                                                    float* gs_out) {
   __shared__ uint32_t hist[32][256];
   __shared__ uint32_t sp[32];
   __shared__ uint32_t newp[32];
@@ -363,6 +398,7 @@ __global__ void __launch_bounds__(256) radix_select(InitCtl* c, int pass, float*
     c->htab[tid] = stab[tid];
     if (tid == 0) c->hmult = mult;
   }
+  if (pass == 0 && gs_out && tid == 0) *gs_out = tensor_scale(c->amax_bits);
   if (pass == 3 && tid < 32) {
     const int n = c->n;
     const int j = tid & 15, b = tid >> 4;
@@ -370,8 +406,15 @@ __global__ void __launch_bounds__(256) radix_select(InitCtl* c, int pass, float*
   }
 }
 
+template <int FMT>
+static void radix_pass_launch(int pass, int blocks, const RadixArgs& a, InitCtl* c,
+                              cudaStream_t st) {
+  if (pass == 0) radix_pass<FMT, true><<<blocks, kThreads, 0, st>>>(a, c);
+  else radix_pass<FMT, false><<<blocks, kThreads, 0, st>>>(a, c);
+}
+
 cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* scales,
-                        float* T, void* ws, cudaStream_t st) {
+                        float* T, void* ws, float* gs_out, cudaStream_t st) {
   const PassPlan pp = plan_pass(N, K);
   InitCtl* c = reinterpret_cast<InitCtl*>(ws);
   const int n = ncodes(fmt);
@@ -384,18 +427,22 @@ cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g,
   }
   for (int j = 2 * n; j < 32; j++) ri.rank[j] = 0;
   init_setup<<<1, 256, 0, st>>>(c, ri, 2 * n, n);
+  int launches = 9;
+  if (fmt == kNvfp4G) {
+    const uint32_t n_vec = (uint32_t)(M / 8);
+    int blocks = (int)((n_vec + kThreads - 1) / kThreads);
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    tensor_amax<<<blocks, kThreads, 0, st>>>(reinterpret_cast<const uint4*>(W), n_vec, c);
+    launches++;
+  }
   for (int pass = 0; pass < 4; pass++) {
     const RadixArgs a{W, (int)N, (int)K, g, scales, pass, pp.ncb, pp.rows_per_chunk};
-    if (fmt == kInt4) {
-      if (pass == 0) radix_pass<kInt4, true><<<pp.blocks, kThreads, 0, st>>>(a, c);
-      else radix_pass<kInt4, false><<<pp.blocks, kThreads, 0, st>>>(a, c);
-    } else {
-      if (pass == 0) radix_pass<kNvfp4, true><<<pp.blocks, kThreads, 0, st>>>(a, c);
-      else radix_pass<kNvfp4, false><<<pp.blocks, kThreads, 0, st>>>(a, c);
-    }
-    radix_select<<<1, 256, 0, st>>>(c, pass, T);
+    if (fmt == kInt4) radix_pass_launch<kInt4>(pass, pp.blocks, a, c, st);
+    else if (fmt == kNvfp4) radix_pass_launch<kNvfp4>(pass, pp.blocks, a, c, st);
+    else radix_pass_launch<kNvfp4G>(pass, pp.blocks, a, c, st);
+    radix_select<<<1, 256, 0, st>>>(c, pass, T, fmt == kNvfp4G ? gs_out : nullptr);
   }
-  count_launches(9);
+  count_launches(launches);
   return cudaGetLastError();
 }
 

@@ -46,26 +46,32 @@ void count_launches(int n);
 // ---- launchers (return cudaGetLastError() of their launches) --------------
 cudaError_t launch_importance(const uint16_t* X, int64_t T, int64_t K, int64_t ldx, uint32_t flags,
                               float* I, void* ws, cudaStream_t st);
+// gs_out / gsc: the per-tensor scale of AAAC_NVFP4_GS (device fp32 [1]);
+// ignored for the other formats.
 cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* scales,
-                        float* T, void* ws, cudaStream_t st);
+                        float* T, void* ws, float* gs_out, cudaStream_t st);
 cudaError_t launch_fit(const uint16_t* W, int64_t N, int64_t K, const float* I,
                        const void* scales, int fmt, int g, int S, int iters, uint32_t flags,
-                       float* T, double* err_hist, aaac_stats* stats, void* ws, cudaStream_t st);
+                       float* T, double* err_hist, aaac_stats* stats, void* ws, const float* gsc,
+                       cudaStream_t st);
 cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const float* I,
                         const void* scales, int fmt, int g, int S, uint32_t flags, const float* T,
                         uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
-                        uint8_t* choice_bits, double* err_final, void* ws, cudaStream_t st);
+                        uint8_t* choice_bits, double* err_final, void* ws, const float* gsc,
+                        cudaStream_t st);
 
 cudaError_t launch_dequant(const uint8_t* codes, const void* tagged, const uint8_t* cbits,
                            const uint16_t* Tb, int64_t N, int64_t K, int fmt, int g, int S,
-                           uint16_t* W_hat, cudaStream_t st);
+                           uint16_t* W_hat, const float* gsc, cudaStream_t st);
 cudaError_t launch_linear(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                           const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
-                          int64_t K, int fmt, int g, int S, float* Y, cudaStream_t st);
+                          int64_t K, int fmt, int g, int S, float* Y, const float* gsc,
+                          cudaStream_t st);
 
 cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                         const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
-                        int64_t K, int fmt, int lg, int ls, float* Y, cudaStream_t st);
+                        int64_t K, int fmt, int lg, int ls, float* Y, const float* gsc,
+                        cudaStream_t st);
 cudaError_t gemm_timeout_flag(unsigned int* out);
 
 cudaError_t launch_awq_prescale(const uint16_t* W, int64_t N, int64_t K, const float* I,

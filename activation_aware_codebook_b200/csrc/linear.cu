@@ -8,7 +8,9 @@
 //   W_hat[n][k] = bf16_RN(s[n][k/g] * T_bf16[c][code[n][k]])
 // The product of two bf16-representable values has at most 16 significant
 // bits; the bf16x2 multiply rounds the exact product once, which is that
-// definition.
+// definition.  With a per-tensor scale gs (NVFP4 variant) the scale is
+// fp32_RN(gs * s8) and the value bf16_RN(fp32_RN(scale * T)): an fp32
+// multiply, then the bf16x2 conversion.
 //
 //   dequant_kernel  one warp per row, 16 weights per lane per step: 8 bytes
 //                   of codes in, 32 bytes of bf16 out; the 32-entry table
@@ -80,14 +82,42 @@ __device__ __forceinline__ void expand8(uint32_t cw, uint32_t sbf, uint32_t c,
   }
 }
 
+// expand8 with an fp32 scale (NVFP4 with a per-tensor scale): each product
+// is rounded to fp32 and then to bf16, bf16_RN(fp32_RN(se * T)).
+__device__ __forceinline__ void expand8g(uint32_t cw, float se, uint32_t c,
+                                         const unsigned short* sT, uint32_t out[4]) {
+  const uint32_t cb = c ? 0x20202020u : 0u;
+  const uint32_t ev = ((cw << 1) & 0x1e1e1e1eu) | cb;
+  const uint32_t od = ((cw >> 3) & 0x1e1e1e1eu) | cb;
+  const unsigned char* tb = reinterpret_cast<const unsigned char*>(sT);
+#pragma unroll
+  for (int p = 0; p < 4; p++) {
+    const uint32_t lo = *reinterpret_cast<const unsigned short*>(tb + __byte_perm(ev, 0u, 0x4440u + p));
+    const uint32_t hi = *reinterpret_cast<const unsigned short*>(tb + __byte_perm(od, 0u, 0x4440u + p));
+    const __nv_bfloat162 r = __floats2bfloat162_rn(__fmul_rn(se, __uint_as_float(lo << 16)),
+                                                   __fmul_rn(se, __uint_as_float(hi << 16)));
+    out[p] = *reinterpret_cast<const uint32_t*>(&r);
+  }
+}
+
 // Sixteen weights of one lane and row: codes (8 bytes), the scale of the
 // group (g >= 16 holds all 16), the choice byte (S >= 8: both 8-column halves
-// fall in one byte), expanded to 8 bf16x2 pairs.
+// fall in one byte), expanded to 8 bf16x2 pairs.  gsv: the per-tensor scale
+// (NVFP4 with a tensor scale only).
 template <int FMT>
 __device__ __forceinline__ void expand16(uint2 cw, uint32_t sv, uint32_t cbyte, int k0, int ls,
-                                         bool sign_choice, const unsigned short* sT,
+                                         bool sign_choice, const unsigned short* sT, float gsv,
                                          uint32_t out[8]) {
   uint32_t tag;
+  if (FMT == kNvfp4G) {
+    tag = sv >> 7;
+    const float se = __fmul_rn(gsv, e4m3_mag(sv & 0x7fu));
+    const uint32_t c0 = sign_choice ? tag : ((cbyte >> ((k0 >> ls) & 7)) & 1u);
+    const uint32_t c1 = sign_choice ? tag : ((cbyte >> (((k0 + 8) >> ls) & 7)) & 1u);
+    expand8g(cw.x, se, c0, sT, out);
+    expand8g(cw.y, se, c1, sT, out + 4);
+    return;
+  }
   const uint32_t sbf = decode_scale<FMT>(sv, &tag);
   const uint32_t c0 = sign_choice ? tag : ((cbyte >> ((k0 >> ls) & 7)) & 1u);
   const uint32_t c1 = sign_choice ? tag : ((cbyte >> (((k0 + 8) >> ls) & 7)) & 1u);
@@ -103,8 +133,9 @@ template <int FMT>
 __global__ void __launch_bounds__(kLinWarps * 32)
 dequant_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ tagged,
                const uint8_t* __restrict__ cbits, const uint16_t* __restrict__ Tb, int N, int K,
-               int lg, int ls, uint16_t* __restrict__ W_hat) {
+               int lg, int ls, uint16_t* __restrict__ W_hat, const float* __restrict__ gsc) {
   __shared__ unsigned short sT[32];
+  const float gsv = FMT == kNvfp4G ? __ldg(gsc) : 1.0f;
   if (threadIdx.x < 32) sT[threadIdx.x] = Tb[threadIdx.x];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -122,7 +153,7 @@ dequant_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ tagge
           : (uint32_t)__ldg(reinterpret_cast<const unsigned char*>(tagged) + grow + (k0 >> lg));
       const uint32_t cbyte = sign_choice ? 0u : (uint32_t)__ldg(brow + (k0 >> (ls + 3)));
       uint32_t out[8];
-      expand16<FMT>(cw, sv, cbyte, k0, ls, sign_choice, sT, out);
+      expand16<FMT>(cw, sv, cbyte, k0, ls, sign_choice, sT, gsv, out);
       uint4* dst = reinterpret_cast<uint4*>(wrow + k0);
       dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
       dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
@@ -138,8 +169,10 @@ template <int FMT, int MT, int R>
 __global__ void __launch_bounds__(kLinWarps * 32)
 gemv_kernel(const uint16_t* __restrict__ X, int M, int ldx, const uint8_t* __restrict__ codes,
             const void* __restrict__ tagged, const uint8_t* __restrict__ cbits,
-            const uint16_t* __restrict__ Tb, int N, int K, int lg, int ls, float* __restrict__ Y) {
+            const uint16_t* __restrict__ Tb, int N, int K, int lg, int ls, float* __restrict__ Y,
+            const float* __restrict__ gsc) {
   __shared__ unsigned short sT[32];
+  const float gsv = FMT == kNvfp4G ? __ldg(gsc) : 1.0f;
   if (threadIdx.x < 32) sT[threadIdx.x] = Tb[threadIdx.x];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -184,7 +217,7 @@ gemv_kernel(const uint16_t* __restrict__ X, int M, int ldx, const uint8_t* __res
 #pragma unroll
     for (int r = 0; r < R; r++) {
       uint32_t w[8];
-      expand16<FMT>(cw[r], sv[r], cbyte[r], k0, ls, sign_choice, sT, w);
+      expand16<FMT>(cw[r], sv[r], cbyte[r], k0, ls, sign_choice, sT, gsv, w);
 #pragma unroll
       for (int p = 0; p < 8; p++) {
         const unsigned long long wf = f2pack(bf16_lo(w[p]), bf16_hi(w[p]));
@@ -207,21 +240,25 @@ gemv_kernel(const uint16_t* __restrict__ X, int M, int ldx, const uint8_t* __res
 template <int FMT, int MT, int R>
 void launch_gemv_t(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                    const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
-                   int64_t K, int lg, int ls, float* Y, cudaStream_t st) {
+                   int64_t K, int lg, int ls, float* Y, const float* gsc, cudaStream_t st) {
   // token tiles along x (consecutive blocks reuse the same codes from L2)
   const unsigned rows_per_block = kLinWarps * R;
   const dim3 grid((unsigned)((M + MT - 1) / MT), (unsigned)((N + rows_per_block - 1) / rows_per_block));
   gemv_kernel<FMT, MT, R><<<grid, kLinWarps * 32, 0, st>>>(X, (int)M, (int)ldx, codes, tagged,
-                                                           cbits, Tb, (int)N, (int)K, lg, ls, Y);
+                                                           cbits, Tb, (int)N, (int)K, lg, ls, Y,
+                                                           gsc);
 }
 
 template <int FMT>
 void launch_gemv(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                  const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
-                 int64_t K, int lg, int ls, float* Y, cudaStream_t st) {
-  if (M == 1) launch_gemv_t<FMT, 1, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
-  else if (M == 2) launch_gemv_t<FMT, 2, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
-  else launch_gemv_t<FMT, 4, 1>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
+                 int64_t K, int lg, int ls, float* Y, const float* gsc, cudaStream_t st) {
+  if (M == 1)
+    launch_gemv_t<FMT, 1, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
+  else if (M == 2)
+    launch_gemv_t<FMT, 2, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
+  else
+    launch_gemv_t<FMT, 4, 1>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
 }
 
 }  // namespace
@@ -236,31 +273,41 @@ static int log2_of(int v) {
 
 cudaError_t launch_dequant(const uint8_t* codes, const void* tagged, const uint8_t* cbits,
                            const uint16_t* Tb, int64_t N, int64_t K, int fmt, int g, int S,
-                           uint16_t* W_hat, cudaStream_t st) {
+                           uint16_t* W_hat, const float* gsc, cudaStream_t st) {
   const int lg = log2_of(g), ls = log2_of(S);
   const int64_t want = (N + kLinWarps - 1) / kLinWarps;
   const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
+  const unsigned th = kLinWarps * 32;
   if (fmt == kInt4)
-    dequant_kernel<kInt4><<<blocks, kLinWarps * 32, 0, st>>>(codes, tagged, cbits, Tb, (int)N, (int)K, lg, ls,
-                                                  W_hat);
+    dequant_kernel<kInt4><<<blocks, th, 0, st>>>(codes, tagged, cbits, Tb, (int)N, (int)K, lg, ls,
+                                                 W_hat, gsc);
+  else if (fmt == kNvfp4)
+    dequant_kernel<kNvfp4><<<blocks, th, 0, st>>>(codes, tagged, cbits, Tb, (int)N, (int)K, lg,
+                                                  ls, W_hat, gsc);
   else
-    dequant_kernel<kNvfp4><<<blocks, kLinWarps * 32, 0, st>>>(codes, tagged, cbits, Tb, (int)N, (int)K, lg,
-                                                   ls, W_hat);
+    dequant_kernel<kNvfp4G><<<blocks, th, 0, st>>>(codes, tagged, cbits, Tb, (int)N, (int)K, lg,
+                                                   ls, W_hat, gsc);
   count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_linear(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                           const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
-                          int64_t K, int fmt, int g, int S, float* Y, cudaStream_t st) {
+                          int64_t K, int fmt, int g, int S, float* Y, const float* gsc,
+                          cudaStream_t st) {
   const int lg = log2_of(g), ls = log2_of(S);
   if (M > kGemvMaxM) {  // tensor cores: dequantised tiles in shared memory
-    const cudaError_t e = launch_gemm(X, M, ldx, codes, tagged, cbits, Tb, N, K, fmt, lg, ls, Y, st);
+    const cudaError_t e =
+        launch_gemm(X, M, ldx, codes, tagged, cbits, Tb, N, K, fmt, lg, ls, Y, gsc, st);
     if (e == cudaSuccess) count_launches(1);
     return e;
   }
-  if (fmt == kInt4) launch_gemv<kInt4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
-  else launch_gemv<kNvfp4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, st);
+  if (fmt == kInt4)
+    launch_gemv<kInt4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
+  else if (fmt == kNvfp4)
+    launch_gemv<kNvfp4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
+  else
+    launch_gemv<kNvfp4G>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
   count_launches(1);
   return cudaGetLastError();
 }

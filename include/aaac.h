@@ -48,10 +48,18 @@ typedef enum {
 } aaac_status;
 
 /* Section 1 / 4: the two 4-bit layouts evaluated on the page.
- *   AAAC_INT4  : g = 128 (any multiple of 8 up to 256 accepted), codebooks of
- *                16 entries, scale stored as bf16.
- *   AAAC_NVFP4 : g = 16, codebooks of 15 entries, scale stored as FP8 E4M3. */
-typedef enum { AAAC_INT4 = 0, AAAC_NVFP4 = 1 } aaac_format;
+ *   AAAC_INT4     : g = 128 (any power of two in [16, 256] accepted),
+ *                   codebooks of 16 entries, scale stored as bf16.
+ *   AAAC_NVFP4    : g = 16, codebooks of 15 entries, scale stored as FP8 E4M3
+ *                   (s = e4m3_RN_satfinite(group absmax)).
+ *   AAAC_NVFP4_GS : NVFP4 with a per-tensor fp32 scale, the page leaving open
+ *                   whether one is used: gs = fp32_RN(max|w| / 448) in
+ *                   *cfg->global_scale, the stored E4M3 factor
+ *                   s8 = e4m3_RN_satfinite(fp32_RN(absmax / gs)), and the
+ *                   group's scale fp32_RN(gs * s8).  Refine weights and the
+ *                   round objective use s8 (gs^2 is common to every group and
+ *                   multiplies err_hist once). */
+typedef enum { AAAC_INT4 = 0, AAAC_NVFP4 = 1, AAAC_NVFP4_GS = 2 } aaac_format;
 
 /* flags of aaac_config */
 #define AAAC_FREEZE_T0 1u         /* never refine T0                            */
@@ -64,6 +72,9 @@ typedef struct {
     int32_t S;       /* selection group size: S % 8 == 0, g % S == 0           */
     int32_t iters;   /* assign+refine rounds of aaac_fit_layer, >= 0           */
     uint32_t flags;  /* AAAC_FREEZE_T0 | AAAC_FREEZE_T1 | AAAC_SINGLE_CODEBOOK */
+    float* global_scale; /* AAAC_NVFP4_GS only (else ignored): device fp32 [1],
+                          * 4-byte aligned; aaac_init_codebooks writes gs there,
+                          * every other call reads it */
 } aaac_config;
 
 /* flags of aaac_importance */
@@ -102,6 +113,9 @@ aaac_status aaac_importance(const void* X, int64_t T, int64_t K, int64_t ldx, ui
  * (initialisation: evenly spaced quantiles of the normalised weights, T1
  * shifted by half a step), with the scale of section 1 / 4 read as
  *   INT4 : s = bf16_RN(fp32_RN(max|w| / 7))      NVFP4 : s = e4m3_RN_sat(max|w|)
+ *   NVFP4_GS : gs = fp32_RN(max over W of |w| / 448) written to
+ *              *cfg->global_scale, stored s8 = e4m3_RN_sat(fp32_RN(max|w| / gs)),
+ *              s = fp32_RN(gs * s8)
  *   u = fp32_RN(w * fp32_RN(1/s)); groups with s == 0 or 1/s = inf have u = 0.
  *   T0[j] = u_(floor((2j+1)M / 2n)),  T1[j] = u_(min(M-1, floor((j+1)M/n)))
  * over the ascending IEEE total order of all M = N*K values, n = 16 (INT4) or
@@ -182,7 +196,9 @@ aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const
  *   W_hat[n][k] = bf16_RN(s[n][k/g] * T_bf16[c][code[n][k]])
  * where s is the magnitude of the stored scale and c is its sign bit (S == g)
  * or bit (k/S)%8 of choice_bits[n][(k/S)/8] (S < g).  The product has at most
- * 16 significant bits, so it is exact in fp32 and rounded once.
+ * 16 significant bits, so it is exact in fp32 and rounded once.  For
+ * AAAC_NVFP4_GS, s = fp32_RN(gs * s8) and
+ *   W_hat[n][k] = bf16_RN(fp32_RN(s * T_bf16[c][code[n][k]])).
  *   codes, scales_tagged, choice_bits, T_bf16: as aaac_pack writes them
  *                 (choice_bits may be NULL when S == g)
  *   cfg           fmt, g and S of the packed layer (iters and flags ignored)
@@ -241,7 +257,8 @@ size_t aaac_awq_workspace_size(const aaac_config* cfg, int64_t N, int64_t K);
  * of W_hat'/c against W'/c in the original input space).  The first
  * candidate with the lowest err_final is kept (strict improvement over all
  * earlier ones): its c, T_bf16, codes, scales_tagged and choice_bits go to
- * the outputs, its err_final to *err_final and its position i to *best.
+ * the outputs, its err_final to *err_final and its position i to *best
+ * (AAAC_NVFP4_GS: its tensor scale to *cfg->global_scale).
  * Everything runs on `stream` with no host synchronisation.
  *   alpha16     HOST int32 [n_alpha], each in [0, 16]; n_alpha in [1, 17]
  *   c           device fp32 [K] (deploy with activations x / c)

@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_struct_layouts_match_header():
-    assert ctypes.sizeof(binding.CConfig) == 20
+    assert ctypes.sizeof(binding.CConfig) == 32
     assert ctypes.sizeof(binding.CStats) == 48
 
 
@@ -56,7 +56,7 @@ def _cfg(**kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(fmt=2), 4), (dict(fmt=1, g=32), 4), (dict(g=48), 4), (dict(S=4), 2), (dict(S=256), 2),
+    (dict(fmt=3), 4), (dict(fmt=2, g=16, S=16), 1), (dict(fmt=2, g=32), 4), (dict(fmt=1, g=32), 4), (dict(g=48), 4), (dict(S=4), 2), (dict(S=256), 2),
     (dict(S=24), 2), (dict(iters=-1), 1), (dict(flags=8), 1)])
 def test_invalid_config_rejected_without_launch(lib, kw, status):
     c = _cfg(**kw)

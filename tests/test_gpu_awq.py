@@ -64,14 +64,14 @@ def test_prescale_extreme_importance_range():
 
 
 CASES = [(bb.INT4, 128, 16, 48, 512), (bb.INT4, 128, 128, 37, 384), (bb.NVFP4, 16, 16, 40, 256),
-         (bb.NVFP4, 16, 8, 24, 208)]
+         (bb.NVFP4, 16, 8, 24, 208), (bb.NVFP4_GS, 16, 16, 40, 256)]
 
 
 @pytest.mark.parametrize("fmt,g,S,N,K", CASES)
 def test_search_bit_exact(fmt, g, S, N, K):
     iters = 3
     js = [0, 4, 8, 12, 16]
-    W, Wb, Xb = _layer(N, K, seed=5 * N + K, dist="student_t4" if fmt == bb.NVFP4 else "normal")
+    W, Wb, Xb = _layer(N, K, seed=5 * N + K, dist="normal" if fmt == bb.INT4 else "student_t4")
     I = oracle.importance(Xb)
     cfg = bb.Config(fmt, g, S, iters)
     out = bb.awq_fit(W.cuda(), torch.from_numpy(I).cuda(), Xb.shape[0], cfg, js)
@@ -87,6 +87,8 @@ def test_search_bit_exact(fmt, g, S, N, K):
     if S != g:
         assert np.array_equal(out["choice_bits"].cpu().numpy(), ref["choice_bits"])
     np.testing.assert_allclose(float(out["err_final"][0]), ref["err_final"], rtol=RTOL)
+    if fmt == bb.NVFP4_GS:  # the kept candidate's tensor scale
+        assert np.float32(cfg.global_scale.item()) == np.float32(ref["gs"])
 
 
 def test_search_single_candidate_is_the_plain_fit():

@@ -24,7 +24,9 @@ def f32_of_bf16(h):
 
 
 def packed_layer(N, K, fmt, g, S, seed, iters=3, dist="normal"):
-    """A layer fitted and packed by the oracle; returns (host dict, device dict)."""
+    """A layer fitted and packed by the oracle; returns (host dict, device dict).
+    dev["cfg"] is the layer's config (with its tensor scale on the device for
+    NVFP4_GS)."""
     W, X = synth.small_layer(N, K, seed, T=64, heavy=True, dist=dist)
     host = oracle.run_layer(u16(W), u16(X), fmt, g, S, iters)
     dev = {}
@@ -32,22 +34,28 @@ def packed_layer(N, K, fmt, g, S, seed, iters=3, dist="normal"):
         a = host[key]
         dev[key] = None if a is None else torch.from_numpy(
             np.ascontiguousarray(a).view(np.int16 if a.dtype == np.uint16 else a.dtype)).cuda()
+    gs = (torch.tensor([host["gs"]], dtype=torch.float32).cuda() if fmt == oracle.NVFP4_GS
+          else None)
+    dev["cfg"] = bb.Config(fmt, g, S, 0, global_scale=gs)
     return host, dev
 
 
+def ref_dequant(host, N, K, fmt, g, S):
+    return oracle.dequant_bf16(host["codes"], host["scales_tagged"], host["choice_bits"],
+                               host["T_bf16"], N, K, fmt, g, S, host["gs"])
+
+
 CASES = [(oracle.INT4, 128, 16), (oracle.INT4, 128, 128), (oracle.INT4, 64, 8),
-         (oracle.NVFP4, 16, 16), (oracle.NVFP4, 16, 8)]
+         (oracle.NVFP4, 16, 16), (oracle.NVFP4, 16, 8), (oracle.NVFP4_GS, 16, 16),
+         (oracle.NVFP4_GS, 16, 8)]
 
 
 @pytest.mark.parametrize("fmt,g,S", CASES)
 @pytest.mark.parametrize("N,K", [(96, 512), (33, 384)])
 def test_dequant_bit_exact(fmt, g, S, N, K):
     host, dev = packed_layer(N, K, fmt, g, S, seed=N + K + S)
-    cfg = bb.Config(fmt, g, S, 0)
-    W_hat = bb.dequant(dev, cfg, N, K)
-    ref = oracle.dequant_bf16(host["codes"], host["scales_tagged"], host["choice_bits"],
-                              host["T_bf16"], N, K, fmt, g, S)
-    assert np.array_equal(u16(W_hat), ref)
+    W_hat = bb.dequant(dev, dev["cfg"], N, K)
+    assert np.array_equal(u16(W_hat), ref_dequant(host, N, K, fmt, g, S))
 
 
 def check_linear(Y, Xb, Wh):
@@ -64,12 +72,9 @@ def check_linear(Y, Xb, Wh):
 def test_linear_within_bound(fmt, g, S, M):
     N, K = 70, 640
     host, dev = packed_layer(N, K, fmt, g, S, seed=7 + M)
-    cfg = bb.Config(fmt, g, S, 0)
     X = synth.make_activations(M, K, seed=100 + M, heavy=True).cuda()
-    Y = bb.linear(X, dev, cfg, N, K)
-    Wh = oracle.dequant_bf16(host["codes"], host["scales_tagged"], host["choice_bits"],
-                             host["T_bf16"], N, K, fmt, g, S)
-    check_linear(Y, u16(X), Wh)
+    Y = bb.linear(X, dev, dev["cfg"], N, K)
+    check_linear(Y, u16(X), ref_dequant(host, N, K, fmt, g, S))
 
 
 def test_linear_strided_x_and_one_hot():
@@ -111,7 +116,7 @@ def test_dequant_and_linear_full_size_gate():
 
 GEMM_CASES = [(oracle.INT4, 128, 16, 200, 640), (oracle.INT4, 128, 128, 130, 384),
               (oracle.NVFP4, 16, 16, 70, 208), (oracle.INT4, 32, 8, 256, 96),
-              (oracle.NVFP4, 16, 8, 130, 176)]
+              (oracle.NVFP4, 16, 8, 130, 176), (oracle.NVFP4_GS, 16, 16, 150, 272)]
 
 
 @pytest.mark.parametrize("fmt,g,S,N,K", GEMM_CASES)
@@ -121,14 +126,11 @@ def test_linear_tensor_core_path(fmt, g, S, N, K, M):
     (N not a multiple of 128), partial token tiles, and a last K block that
     is only partly inside K (K = 208, 96)."""
     host, dev = packed_layer(N, K, fmt, g, S, seed=M + N)
-    cfg = bb.Config(fmt, g, S, 0)
     X = synth.make_activations(M, K, seed=200 + M, heavy=True).cuda()
-    Y = bb.linear(X, dev, cfg, N, K)
+    Y = bb.linear(X, dev, dev["cfg"], N, K)
     torch.cuda.synchronize()
     assert bb.device_timeouts() == 0
-    Wh = oracle.dequant_bf16(host["codes"], host["scales_tagged"], host["choice_bits"],
-                             host["T_bf16"], N, K, fmt, g, S)
-    check_linear(Y, u16(X), Wh)
+    check_linear(Y, u16(X), ref_dequant(host, N, K, fmt, g, S))
 
 
 def test_linear_tensor_core_many_tiles():

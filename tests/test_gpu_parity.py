@@ -73,7 +73,8 @@ def test_importance_accumulate_strided_and_boundary():
 # scales, init, fit, pack
 # --------------------------------------------------------------------------
 CASES = [(bb.INT4, 128, 128, 256, 512), (bb.INT4, 128, 16, 37, 640), (bb.NVFP4, 16, 16, 64, 512),
-         (bb.INT4, 32, 8, 48, 256), (bb.NVFP4, 16, 16, 33, 1040), (bb.NVFP4, 16, 8, 40, 528)]
+         (bb.INT4, 32, 8, 48, 256), (bb.NVFP4, 16, 16, 33, 1040), (bb.NVFP4, 16, 8, 40, 528),
+         (bb.NVFP4_GS, 16, 16, 64, 512), (bb.NVFP4_GS, 16, 8, 33, 1040)]
 
 
 @pytest.mark.parametrize("fmt,g,S,N,K", CASES)
@@ -81,15 +82,17 @@ def test_init_bit_exact(fmt, g, S, N, K):
     W, _ = layer(N, K, seed=N * K + g)
     cfg = cfg_of(fmt, g, S, 0)
     scl, T = bb.init_codebooks(W, cfg)
-    rscl, rT = oracle.init_codebooks(u16(W), fmt, g)
+    rscl, rT, rgs = oracle.init_codebooks(u16(W), fmt, g, with_gs=True)
     assert np.array_equal(scl.cpu().numpy().view(rscl.dtype), rscl)
     assert np.array_equal(npbits(T), rT.view(np.uint32))
+    if fmt == bb.NVFP4_GS:
+        assert np.float32(cfg.global_scale.item()) == np.float32(rgs)
 
 
 @pytest.mark.parametrize("fmt,g,S,N,K", CASES)
 @pytest.mark.parametrize("iters", [1, 6])
 def test_fit_and_pack_bit_exact(fmt, g, S, N, K, iters):
-    W, X = layer(N, K, seed=3 * N + K + iters, dist="student_t4" if fmt == bb.NVFP4 else "normal")
+    W, X = layer(N, K, seed=3 * N + K + iters, dist="normal" if fmt == bb.INT4 else "student_t4")
     cfg = cfg_of(fmt, g, S, iters)
     out = bb.run_layer(W, X, cfg)
     ref = oracle.run_layer(u16(W), u16(X), fmt, g, S, iters)
@@ -100,6 +103,8 @@ def check_against_oracle(out, ref, cfg, label=""):
     torch.cuda.synchronize()
     assert np.array_equal(npbits(out["I"]), ref["I"].view(np.uint32)), label
     assert np.array_equal(out["scales"].cpu().numpy().view(ref["scales"].dtype), ref["scales"])
+    if cfg.fmt == bb.NVFP4_GS:
+        assert np.float32(out["global_scale"].item()) == np.float32(ref["gs"]), label
     assert np.array_equal(npbits(out["T_init"]), ref["T_init"].view(np.uint32)), label
     T, rT = out["T"].cpu().numpy(), ref["T"]
     assert np.array_equal(T.view(np.uint32), rT.view(np.uint32)), (label, T, rT)
@@ -146,12 +151,29 @@ def test_dead_groups_constant_weights_and_duplicates():
     W[2:10] = 0.5                 # constant groups: heavy duplicate u values
     X = synth.make_activations(32, K, seed=91, heavy=True)
     X[:, 10:20] = 0               # columns with zero importance
-    for fmt, S in ((bb.NVFP4, 16), (bb.INT4, 16)):
+    for fmt, S in ((bb.NVFP4, 16), (bb.INT4, 16), (bb.NVFP4_GS, 16)):
         cfg = cfg_of(fmt, g, S, 5)
         out = bb.run_layer(W.cuda(), X.cuda(), cfg)
         ref = oracle.run_layer(u16(W), u16(X), fmt, g, S, 5)
         check_against_oracle(out, ref, cfg, label=f"fmt{fmt}")
         assert bb.decode_stats(out["stats"])["dead_groups"] > 0
+
+
+@pytest.mark.parametrize("sigma", [1e-3, 0.0])
+def test_tensor_scale_small_and_zero_weights(sigma):
+    """NVFP4 with a per-tensor scale on weights whose group maxima are E4M3
+    subnormals without it (about 2e-3), and on an all-zero tensor (gs = 0,
+    every group dead)."""
+    N, K = 48, 512
+    W = (synth.make_weight(N, K, seed=95).float() * (sigma / 0.02)).to(torch.bfloat16)
+    X = synth.make_activations(64, K, seed=96, heavy=True)
+    cfg = cfg_of(bb.NVFP4_GS, 16, 16, 4)
+    out = bb.run_layer(W.cuda(), X.cuda(), cfg)
+    ref = oracle.run_layer(u16(W), u16(X), bb.NVFP4_GS, 16, 16, 4)
+    check_against_oracle(out, ref, cfg)
+    if sigma == 0.0:
+        assert float(out["global_scale"][0]) == 0.0
+        assert bb.decode_stats(out["stats"])["dead_groups"] == N * K // 16
 
 
 def test_all_equal_weights():
