@@ -26,6 +26,7 @@ import torch
 
 INT4 = 0
 NVFP4 = 1
+NVFP4_GS = 2  # NVFP4 with a per-tensor fp32 scale
 
 
 @dataclasses.dataclass(frozen=True)
@@ -86,6 +87,12 @@ WORKLOADS = {
         (Linear("gate_27648x5120", 27648, 5120, "h"), Linear("up_27648x5120", 27648, 5120, "h"),
          Linear("down_5120x27648", 5120, 27648, "a")),
         131072, "student_t4", False, NVFP4, 16, 16, 30),
+    # the same layers with NVFP4's per-tensor fp32 scale
+    "qwen32b-nvfp4-gs": Workload(
+        "qwen32b-nvfp4-gs",
+        (Linear("gate_27648x5120", 27648, 5120, "h"), Linear("up_27648x5120", 27648, 5120, "h"),
+         Linear("down_5120x27648", 5120, 27648, "a")),
+        131072, "student_t4", False, NVFP4_GS, 16, 16, 30),
 }
 
 

@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -205,7 +206,11 @@ class Block:
                   for k, x in Xs.items()}
         sdt = torch.int16 if wl.fmt == bb.INT4 else torch.uint8
         self.scales, self.T, self.eh, self.st, self.out = {}, {}, {}, {}, {}
+        self.cfgs = {}  # per linear: its own tensor scale (NVFP4 with a tensor scale)
         for l in wl.linears:
+            gs = (torch.zeros(1, dtype=torch.float32, device=dev) if wl.fmt == bb.NVFP4_GS
+                  else None)
+            self.cfgs[l.name] = bb.Config(wl.fmt, wl.g, wl.S, wl.iters, global_scale=gs)
             self.scales[l.name] = torch.empty(l.N, l.K // wl.g, dtype=sdt, device=dev)
             self.T[l.name] = torch.zeros(2, 16, dtype=torch.float32, device=dev)
             self.eh[l.name] = torch.zeros(wl.iters, dtype=torch.float64, device=dev)
@@ -218,14 +223,17 @@ class Block:
                 choice_bits=(torch.empty(l.N, nb, dtype=torch.uint8, device=dev)
                              if wl.S != wl.g else None),
                 err_final=torch.zeros(1, dtype=torch.float64, device=dev))
+            if gs is not None:  # part of the packed layer
+                self.out[l.name]["global_scale"] = gs
         self.weight_iters = sum(l.N * l.K for l in wl.linears) * wl.iters
 
     def step(self, fit_events=None, probe=None):
-        bb, cfg = self.bb, self.cfg
+        bb = self.bb
         for k, X in self.Xs.items():
             bb.importance(X, I=self.I[k], ws=self.ws)
         for l in self.wl.linears:
             W = self.Ws[l.name]
+            cfg = self.cfgs[l.name]
             bb.init_codebooks(W, cfg, ws=self.ws, scales=self.scales[l.name], T=self.T[l.name])
             if fit_events is not None and l.name == probe:
                 fit_events[0].record()
@@ -249,7 +257,7 @@ def fit_setup_ms(blk, lin, reps=5):
     """Time of a fit call with zero rounds (prep + setup) on the probe layer."""
     import torch
     bb = blk.bb
-    cfg0 = bb.Config(blk.cfg.fmt, blk.cfg.g, blk.cfg.S, 0)
+    cfg0 = dataclasses.replace(blk.cfgs[lin.name], iters=0)
     W = blk.Ws[lin.name]
     T = blk.T[lin.name].clone()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -341,7 +349,8 @@ def run_ours(args, rank, local_rank, world):
             "config": {"workload": wl.name, "linears": [f"{l.name} {l.N}x{l.K}"
                                                         for l in wl.linears],
                        "weights_per_block": sum(l.N * l.K for l in wl.linears),
-                       "tokens": tokens, "format": "INT4" if wl.fmt == bb.INT4 else "NVFP4",
+                       "tokens": tokens,
+                       "format": {bb.INT4: "INT4", bb.NVFP4: "NVFP4"}.get(wl.fmt, "NVFP4+tensor scale"),
                        "g": wl.g, "S": wl.S, "iters": wl.iters,
                        "blocks": world, "parallelism": f"layer-parallel x{world} (no collective)",
                        "l2": "inputs larger than L2 (activations %.1f GiB per step)" % (
