@@ -100,6 +100,16 @@ tensor_amax(const uint4* __restrict__ W, uint32_t n_vec, InitCtl* c) {
 
 constexpr int kRadixRows = 4;  // rows per lane loaded ahead in a radix pass
 
+// *p += v in shared memory when cond holds: one predicated reduction, no
+// branch (lanes that do not count skip the access).
+__device__ __forceinline__ void shared_add_if(uint32_t* p, uint32_t v, bool cond) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q red.shared.add.u32 [%0], %1;\n\t}"
+      ::"r"(a), "r"(v), "r"((uint32_t)cond)
+      : "memory");
+}
+
 struct RankInit {
   int64_t rank[32];
 };
@@ -190,7 +200,8 @@ __device__ __forceinline__ void radix_rows(const RadixArgs& a, uint32_t (*sh)[25
           // lanes holding the same top digit add once (fewer same-address atomics)
           const uint32_t d = active ? (key >> 24) : 0x100u;
           const uint32_t peers = __match_any_sync(0xffffffffu, d);
-          if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&sh[warp][d], (uint32_t)__popc(peers));
+          shared_add_if(&sh[warp][d & 255u], (uint32_t)__popc(peers),
+                        d < 256u && lane == __ffs(peers) - 1);
         } else {
           const uint32_t pre = key >> (shift + 8);
           int slot;
@@ -205,7 +216,7 @@ __device__ __forceinline__ void radix_rows(const RadixArgs& a, uint32_t (*sh)[25
             }
             slot = (lo < nslots && sp[lo] == pre) ? lo : -1;
           }
-          if (slot >= 0) atomicAdd(&sh[slot][(key >> shift) & 255u], 1u);
+          shared_add_if(&sh[slot >= 0 ? slot : 0][(key >> shift) & 255u], 1u, slot >= 0);
         }
       }
     }
