@@ -24,7 +24,7 @@ IMPORTANCE_EXACT = 2
 
 STATUS = {0: "AAAC_OK", 1: "AAAC_ERR_INVALID_ARG", 2: "AAAC_ERR_SHAPE", 3: "AAAC_ERR_ALIGN",
           4: "AAAC_ERR_UNSUPPORTED", 5: "AAAC_ERR_CUDA", 6: "AAAC_ERR_WORKSPACE",
-          7: "AAAC_ERR_TIMEOUT"}
+          7: "AAAC_ERR_TIMEOUT", 8: "AAAC_ERR_COLLECTIVE"}
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaaac.so")
 
@@ -32,7 +32,14 @@ EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaa
            "aaac_pack", "aaac_last_error", "aaac_version", "aaac_kernel_launches",
            "aaac_fit_layer_fixed_scratch", "aaac_dequant", "aaac_linear",
            "aaac_device_timeouts", "aaac_awq_prescale", "aaac_awq_workspace_size",
-           "aaac_awq_fit")
+           "aaac_awq_fit", "aaac_init_codebooks_sharded", "aaac_fit_layer_sharded",
+           "aaac_pack_sharded")
+
+
+# reduction callback of the row-sharded calls: (user, buf, count, op, stream) -> 0 | error
+REDUCE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                             ctypes.c_int, ctypes.c_void_p)
+REDUCE_SUM_I64, REDUCE_MAX_I64, REDUCE_SUM_I32, REDUCE_MAX_I32 = 0, 1, 2, 3
 
 
 class AaacError(RuntimeError):
@@ -125,6 +132,13 @@ def load(path: str = LIB_PATH):
     L.aaac_awq_fit.restype = ctypes.c_int
     L.aaac_awq_fit.argtypes = [P, i64, i64, P, i64, P, P, ctypes.c_int, P, P, P, P, P, P, P, P,
                                P, sz, P]
+    R = REDUCE_FN
+    L.aaac_init_codebooks_sharded.restype = ctypes.c_int
+    L.aaac_init_codebooks_sharded.argtypes = [P, i64, i64, i64, P, P, P, R, P, P, sz, P]
+    L.aaac_fit_layer_sharded.restype = ctypes.c_int
+    L.aaac_fit_layer_sharded.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, R, P, P, sz, P]
+    L.aaac_pack_sharded.restype = ctypes.c_int
+    L.aaac_pack_sharded.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, P, P, P, R, P, P, sz, P]
     _lib = L
     return L
 
@@ -393,4 +407,118 @@ def awq_fit(W: torch.Tensor, I: torch.Tensor, tokens: int, cfg: Config, alphas16
                                _ptr(out["choice_bits"]), _ptr(out["err_final"]),
                                _ptr(out["err_alpha"]), _ptr(out["best"]), _ptr(ws), ws.numel(),
                                _stream(stream)))
+    return out
+
+
+# --------------------------------------------------------------------------
+# row-sharded calls (one layer's rows over several processes / GPUs)
+# --------------------------------------------------------------------------
+class ShardReducer:
+    """Adapts a Python all-reduce to the library's callback.  The library
+    hands a buffer inside the workspace `ws`; `allreduce(t, op)` receives a
+    torch view of it (int64 or int32) and op "sum" or "max", and must combine
+    it in place over all shards on the current stream (for example
+    torch.distributed.all_reduce with NCCL)."""
+
+    def __init__(self, ws: torch.Tensor, allreduce):
+        self.ws, self.allreduce, self.error = ws, allreduce, None
+
+        def cb(user, buf, count, op, stream):
+            try:
+                off = int(buf) - self.ws.data_ptr()
+                esz = 8 if op in (REDUCE_SUM_I64, REDUCE_MAX_I64) else 4
+                dt = torch.int64 if esz == 8 else torch.int32
+                assert 0 <= off and off + count * esz <= self.ws.numel()
+                t = self.ws[off:off + count * esz].view(dt)
+                self.allreduce(t, "sum" if op in (REDUCE_SUM_I64, REDUCE_SUM_I32) else "max")
+                return 0
+            except Exception as e:  # reported by the call as AAAC_ERR_COLLECTIVE
+                self.error = e
+                return 1
+
+        self.fn = REDUCE_FN(cb)  # kept alive with the reducer
+
+    def check(self, status: int):
+        if status == 8 and self.error is not None:
+            raise AaacError(status, f"reduce callback failed: {self.error!r}")
+        _check(status)
+
+
+def torch_allreduce(group=None):
+    """An allreduce for ShardReducer over torch.distributed (NCCL on GPUs)."""
+    import torch.distributed as dist
+
+    def run(t, op):
+        dist.all_reduce(t, op=dist.ReduceOp.SUM if op == "sum" else dist.ReduceOp.MAX,
+                        group=group)
+    return run
+
+
+def init_codebooks_sharded(W: torch.Tensor, N_total: int, cfg: Config, allreduce,
+                           ws: Optional[torch.Tensor] = None, stream=None):
+    """init_codebooks over a layer whose rows are split over shards; this
+    shard holds W [N, K].  Returns (scales [N, K/g], T [2, 16]); T is the
+    whole layer's quantile initialisation on every shard."""
+    _need_cuda()
+    W = _bits16(W)
+    N, K = W.shape
+    sdt = torch.int16 if cfg.fmt == INT4 else torch.uint8
+    scales = torch.empty(N, K // cfg.g, dtype=sdt, device=W.device)
+    T = torch.empty(2, 16, dtype=torch.float32, device=W.device)
+    if ws is None:
+        ws = workspace(cfg, N, K, 0, W.device)
+    cfg.ensure_global_scale(W.device)
+    red = ShardReducer(ws, allreduce)
+    c = cfg.c()
+    red.check(load().aaac_init_codebooks_sharded(_ptr(W), N, K, int(N_total), ctypes.byref(c),
+                                                 _ptr(scales), _ptr(T), red.fn, None, _ptr(ws),
+                                                 ws.numel(), _stream(stream)))
+    return scales, T
+
+
+def fit_layer_sharded(W: torch.Tensor, N_total: int, I: torch.Tensor, scales: torch.Tensor,
+                      T: torch.Tensor, cfg: Config, allreduce, ws: Optional[torch.Tensor] = None,
+                      stream=None):
+    """fit_layer over a row-sharded layer.  Returns (T, err_hist, stats); every
+    shard gets the whole layer's tables, history and counters."""
+    _need_cuda()
+    W = _bits16(W)
+    N, K = W.shape
+    err_hist = torch.zeros(max(cfg.iters, 1), dtype=torch.float64, device=W.device)
+    stats = torch.zeros(STATS_BYTES, dtype=torch.uint8, device=W.device)
+    if ws is None:
+        ws = workspace(cfg, N, K, 0, W.device)
+    red = ShardReducer(ws, allreduce)
+    c = cfg.c()
+    red.check(load().aaac_fit_layer_sharded(_ptr(W), N, K, int(N_total), _ptr(I), _ptr(scales),
+                                            ctypes.byref(c), _ptr(T), _ptr(err_hist),
+                                            _ptr(stats), red.fn, None, _ptr(ws), ws.numel(),
+                                            _stream(stream)))
+    return T, err_hist, stats
+
+
+def pack_sharded(W: torch.Tensor, N_total: int, I: torch.Tensor, scales: torch.Tensor,
+                 T: torch.Tensor, cfg: Config, allreduce, ws: Optional[torch.Tensor] = None,
+                 stream=None) -> dict:
+    """pack of this shard's rows; err_final is the whole layer's."""
+    _need_cuda()
+    W = _bits16(W)
+    N, K = W.shape
+    dev = W.device
+    nb = (K // cfg.S + 7) // 8
+    out = dict(T_bf16=torch.zeros(2, 16, dtype=torch.int16, device=dev),
+               codes=torch.empty(N, K // 2, dtype=torch.uint8, device=dev),
+               scales_tagged=torch.empty_like(scales),
+               choice_bits=(torch.empty(N, nb, dtype=torch.uint8, device=dev)
+                            if cfg.S != cfg.g else None),
+               err_final=torch.zeros(1, dtype=torch.float64, device=dev))
+    if ws is None:
+        ws = workspace(cfg, N, K, 0, dev)
+    red = ShardReducer(ws, allreduce)
+    c = cfg.c()
+    red.check(load().aaac_pack_sharded(_ptr(W), N, K, int(N_total), _ptr(I), _ptr(scales),
+                                       ctypes.byref(c), _ptr(T), _ptr(out["T_bf16"]),
+                                       _ptr(out["codes"]), _ptr(out["scales_tagged"]),
+                                       _ptr(out["choice_bits"]), _ptr(out["err_final"]),
+                                       red.fn, None, _ptr(ws), ws.numel(), _stream(stream)))
     return out

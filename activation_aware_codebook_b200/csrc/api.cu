@@ -392,6 +392,85 @@ aaac_status aaac_awq_fit(const void* W, int64_t N, int64_t K, const float* I, in
   return ok();
 }
 
+static aaac_status check_shards(int64_t N, int64_t K, int64_t N_total, const aaac_config* cfg,
+                                aaac_reduce_fn reduce) {
+  if (!reduce) return fail(AAAC_ERR_INVALID_ARG, "reduce is NULL");
+  if (N_total < N)
+    return fail(AAAC_ERR_SHAPE, "N_total=%lld < N=%lld", (long long)N_total, (long long)N);
+  return check_layer(N_total, K, cfg);  // the whole layer obeys the unsharded limits
+}
+
+aaac_status aaac_init_codebooks_sharded(const void* W, int64_t N, int64_t K, int64_t N_total,
+                                        const aaac_config* cfg, void* scales, float* T,
+                                        aaac_reduce_fn reduce, void* user, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  CHECK(check_shards(N, K, N_total, cfg, reduce));
+  CHECK(check_ptr(W, "W"));
+  CHECK(check_ptr(scales, "scales"));
+  CHECK(check_ptr(T, "T"));
+  CHECK(check_ws(ws, ws_bytes, aaac::init_ctl_bytes()));
+  aaac::Reducer red{reduce, user, false};
+  const cudaError_t e = aaac::launch_init_sharded(reinterpret_cast<const uint16_t*>(W), N, K,
+                                                  N_total * K, cfg->fmt, cfg->g, scales, T, ws,
+                                                  cfg->global_scale, red, (cudaStream_t)stream);
+  if (red.failed) return fail(AAAC_ERR_COLLECTIVE, "aaac_init_codebooks_sharded: reduce failed");
+  return from_cuda(e, "aaac_init_codebooks_sharded");
+}
+
+aaac_status aaac_fit_layer_sharded(const void* W, int64_t N, int64_t K, int64_t N_total,
+                                   const float* I, const void* scales, const aaac_config* cfg,
+                                   float* T, double* err_hist, aaac_stats* stats,
+                                   aaac_reduce_fn reduce, void* user, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  CHECK(check_shards(N, K, N_total, cfg, reduce));
+  CHECK(check_ptr(W, "W"));
+  CHECK(check_ptr(I, "I"));
+  CHECK(check_ptr(scales, "scales"));
+  CHECK(check_ptr(T, "T"));
+  CHECK(check_ptr(err_hist, "err_hist", false));
+  CHECK(check_ptr(stats, "stats", false));
+  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K)));
+  aaac::Reducer red{reduce, user, false};
+  const cudaError_t e = aaac::launch_fit_sharded(
+      reinterpret_cast<const uint16_t*>(W), N, K, N_total * K, I, scales, cfg->fmt, cfg->g,
+      cfg->S, cfg->iters, cfg->flags, T, err_hist, stats, ws, cfg->global_scale, red,
+      (cudaStream_t)stream);
+  if (red.failed) return fail(AAAC_ERR_COLLECTIVE, "aaac_fit_layer_sharded: reduce failed");
+  return from_cuda(e, "aaac_fit_layer_sharded");
+}
+
+aaac_status aaac_pack_sharded(const void* W, int64_t N, int64_t K, int64_t N_total,
+                              const float* I, const void* scales, const aaac_config* cfg,
+                              const float* T, uint16_t* T_bf16, uint8_t* codes,
+                              void* scales_tagged, uint8_t* choice_bits, double* err_final,
+                              aaac_reduce_fn reduce, void* user, void* ws, size_t ws_bytes,
+                              void* stream) {
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  CHECK(check_shards(N, K, N_total, cfg, reduce));
+  CHECK(check_ptr(W, "W"));
+  CHECK(check_ptr(I, "I"));
+  CHECK(check_ptr(scales, "scales"));
+  CHECK(check_ptr(T, "T"));
+  CHECK(check_ptr(T_bf16, "T_bf16"));
+  CHECK(check_ptr(codes, "codes"));
+  CHECK(check_ptr(scales_tagged, "scales_tagged"));
+  CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
+  CHECK(check_ptr(err_final, "err_final", false));
+  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K) + aaac::pack_extra_bytes(N, K, cfg->S)));
+  aaac::Reducer red{reduce, user, false};
+  const cudaError_t e = aaac::launch_pack_sharded(
+      reinterpret_cast<const uint16_t*>(W), N, K, N_total * K, I, scales, cfg->fmt, cfg->g,
+      cfg->S, cfg->flags, T, T_bf16, codes, scales_tagged, choice_bits, err_final, ws,
+      cfg->global_scale, red, (cudaStream_t)stream);
+  if (red.failed) return fail(AAAC_ERR_COLLECTIVE, "aaac_pack_sharded: reduce failed");
+  return from_cuda(e, "aaac_pack_sharded");
+}
+
 aaac_status aaac_device_timeouts(uint32_t* flag) {
   if (!flag) return fail(AAAC_ERR_INVALID_ARG, "flag is NULL");
   unsigned int v = 0;

@@ -39,6 +39,7 @@
 //   launch plan bounds the rows per lane to keep it there.  Bins are laid out
 //   [book*16 + entry][lane] in 16-byte cells: a warp's read-modify-write of
 //   its bins touches 32 distinct bank quads, with no conflicts.
+#include <cstddef>
 #include <mutex>
 
 #include "common.cuh"
@@ -90,17 +91,24 @@ struct FitCtl {
   uint32_t Umax_bits;
   unsigned long long S2max_bits;
   unsigned long long dead_groups;
+  // A round's integer sums, contiguous: a row-sharded fit adds them over the
+  // shards with one int64 sum-reduction of kShardSums values.
   long long bins[2][16][2];
+  unsigned long long err_acc;  // sum of rint(s^2 D 2^Le) of the running pass
   unsigned long long near_ties;
   unsigned long long groups_t1;
   unsigned long long exact_groups;
   unsigned long long empty_cells;
+  unsigned long long exact_total;   // row-sharded fit: exact decisions of earlier rounds
+  unsigned long long shard_max[3];  // row-sharded fit: Imax, Umax, S2max bits (max-reduced)
   unsigned int ticket;
   unsigned int next_item;  // work-item counter of the running pass (many strips)
   unsigned int strip_next[kMaxStrips];  // per-strip item counters of the running pass
   double twoLe;            // fixed-point scale of the objective sums
-  unsigned long long err_acc;  // sum of rint(s^2 D 2^Le) of the running pass
 };
+constexpr int kShardSums = 64 + 4;  // bins, err_acc, near_ties, groups_t1, exact_groups
+static_assert(offsetof(FitCtl, exact_groups) == offsetof(FitCtl, bins) + (kShardSums - 1) * 8,
+              "the round sums must be contiguous");
 
 size_t fit_ctl_bytes() { return align256(sizeof(FitCtl)); }
 
@@ -112,13 +120,14 @@ struct FitPlan {
   int ncb, cpc, items, max_items, blocks;
 };
 
-static FitPlan fit_plan(int64_t N, int64_t K) {
+// M: the weights of the whole layer (of every row shard), which fixes B.
+static FitPlan fit_plan(int64_t N, int64_t K, int64_t M) {
   FitPlan p;
   p.ncb = (int)((K + kWarpCols - 1) / kWarpCols);
   p.cpc = (int)((N + kItemRows - 1) / kItemRows);
   p.items = p.ncb * p.cpc;
   int c = 0;
-  while (((int64_t)1 << c) < N * K) c++;
+  while (((int64_t)1 << c) < M) c++;
   const int Bmax = (61 - c) < 40 ? (61 - c) : 40;
   const int64_t cap_rows = ((int64_t)1 << (50 - Bmax)) / kLaneCols;  // >= 64
   p.max_items = (int)(cap_rows / kItemRows);
@@ -530,7 +539,7 @@ __device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsign
 // fp64(den)) when den > 0, else unchanged; then sorted books and new tables.
 // Everything is staged in shared memory and spread over the block's threads.
 __device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const RoundOut& ro,
-                               int cpc, int n_items, double g2) {
+                               int wt, int cpc, int n_items, double g2) {
   __shared__ float sT[2][16];
   __shared__ long long sb[64];
   __shared__ int s_upd[2];
@@ -586,7 +595,7 @@ __device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const Ro
     ctl->groups_t1 = 0;
     ctl->ticket = 0;
   }
-  seed_claims(ctl, (int)gridDim.x * kFitWarps, cpc, n_items);
+  seed_claims(ctl, wt, cpc, n_items);
 }
 
 // Chunk j (16 bytes) of a warp's 1 KB row segment sits at ring slot j ^ bit 3
@@ -671,7 +680,7 @@ __global__ void __launch_bounds__(kFitThreads, kFitBlocksPerSM)
 fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
          const void* __restrict__ scales, int g, int S, uint32_t flags, FitCtl* ctl,
          int cpc, int n_items, int max_items, float tau, PackOut po,
-         RoundOut ro, const float* __restrict__ gsc) {
+         RoundOut ro, const float* __restrict__ gsc, int finalize) {
   extern __shared__ __align__(128) unsigned char smem[];
   Tables& tb = *reinterpret_cast<Tables*>(smem);
   unsigned char* ring = smem + kTablesBytes;
@@ -1103,8 +1112,14 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  if (!PACK) {
-    round_finalize(ctl, tb, flags, ro, cpc, n_items, __dmul_rn((double)gsv, (double)gsv));
+  const int wt = (int)gridDim.x * kFitWarps;
+  if (!finalize) {
+    // row-sharded: the sums are reduced over the shards before the round
+    // ends (shard_round_end / shard_pack_end); only the claims are reset
+    if (threadIdx.x == 0) ctl->ticket = 0;
+    seed_claims(ctl, wt, cpc, n_items);
+  } else if (!PACK) {
+    round_finalize(ctl, tb, flags, ro, wt, cpc, n_items, __dmul_rn((double)gsv, (double)gsv));
   } else {
     if (threadIdx.x == 0) {
       const long long acc = (long long)__ldcg(&ctl->err_acc);
@@ -1112,8 +1127,55 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
       ctl->err_acc = 0ull;
       ctl->ticket = 0;
     }
-    seed_claims(ctl, (int)gridDim.x * kFitWarps, cpc, n_items);
+    seed_claims(ctl, wt, cpc, n_items);
   }
+}
+
+// ---------------------------------------------------------------------------
+// row-sharded fit: the pieces between the reductions
+// ---------------------------------------------------------------------------
+// dir 0: the maxima into shard_max (for a max-reduction); dir 1: back.
+__global__ void shard_maxima(FitCtl* ctl, int dir) {
+  if (threadIdx.x != 0) return;
+  if (dir == 0) {
+    ctl->shard_max[0] = ctl->Imax_bits;
+    ctl->shard_max[1] = ctl->Umax_bits;
+    ctl->shard_max[2] = ctl->S2max_bits;
+  } else {
+    ctl->Imax_bits = (uint32_t)ctl->shard_max[0];
+    ctl->Umax_bits = (uint32_t)ctl->shard_max[1];
+    ctl->S2max_bits = ctl->shard_max[2];
+  }
+}
+
+// The end of a round once its sums hold every shard's: the refine of
+// round_finalize on the round's tables, with the exact-decision count kept
+// as a running total of the reduced per-round counts.
+__global__ void __launch_bounds__(kFitThreads)
+shard_round_end(FitCtl* ctl, uint32_t flags, RoundOut ro, int wt, int cpc, int n_items,
+                const float* __restrict__ gsc, int fmt) {
+  __shared__ Tables tb;
+  {
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(&ctl->tb);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(&tb);
+    for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
+  }
+  if (threadIdx.x == 0) {
+    ctl->exact_total += ctl->exact_groups;
+    ctl->exact_groups = ctl->exact_total;
+  }
+  __syncthreads();
+  const double gs = fmt == kNvfp4G ? (double)__ldg(gsc) : 1.0;
+  round_finalize(ctl, tb, flags, ro, wt, cpc, n_items, __dmul_rn(gs, gs));
+  __syncthreads();
+  if (threadIdx.x == 0) ctl->exact_groups = 0ull;  // the next round counts its own
+}
+
+__global__ void shard_pack_end(FitCtl* ctl, double* err_final) {
+  if (threadIdx.x != 0) return;
+  const long long acc = (long long)ctl->err_acc;
+  if (err_final) *err_final = (double)acc / ctl->twoLe;
+  ctl->err_acc = 0ull;
 }
 
 static float choice_tau(int S) {
@@ -1136,7 +1198,7 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
   // per call: the attribute belongs to the current device's copy of the kernel
   const cudaError_t attr = set_smem<FMT, false>();
   if (attr != cudaSuccess) return attr;
-  const FitPlan pp = fit_plan(N, K);
+  const FitPlan pp = fit_plan(N, K, N * K);
   const PassPlan pprep = plan_pass(N, K);
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
@@ -1162,7 +1224,7 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
     const cudaError_t e = cudaLaunchKernelEx(
         &lc, fit_pass<FMT, false>, W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items,
         pp.max_items, tau, PackOut{nullptr, nullptr, nullptr, nullptr},
-        RoundOut{err_hist, T, stats, it}, gsc);
+        RoundOut{err_hist, T, stats, it}, gsc, 1);
     if (e != cudaSuccess) return e;
   }
   count_launches(2 + iters);
@@ -1182,6 +1244,64 @@ cudaError_t launch_fit(const uint16_t* W, int64_t N, int64_t K, const float* I,
                                                 err_hist, stats, ws, gsc, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// Row-sharded fit: this process fits rows [its N] of a layer of M_total
+// weights.  The maxima that fix L, Le and the bucket scale are max-reduced
+// over the shards before the first round; each round's integer sums (bins,
+// objective, counters) are sum-reduced before its refine, which every shard
+// then runs on identical sums -- so every shard holds the same tables, and
+// they equal the unsharded fit's bit for bit (the sums are exact integers).
+template <int FMT>
+static cudaError_t launch_fit_sharded_t(const uint16_t* W, int64_t N, int64_t K, int64_t M_total,
+                                        const float* I, const void* scales, int g, int S,
+                                        int iters, uint32_t flags, float* T, double* err_hist,
+                                        aaac_stats* stats, void* ws, const float* gsc,
+                                        Reducer& red, cudaStream_t st) {
+  const cudaError_t attr = set_smem<FMT, false>();
+  if (attr != cudaSuccess) return attr;
+  const FitPlan pp = fit_plan(N, K, M_total);
+  const PassPlan pprep = plan_pass(N, K);
+  FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
+  cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
+  fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
+                                                   pprep.ncb, pprep.rows_per_chunk, gsc);
+  shard_maxima<<<1, 32, 0, st>>>(ctl, 0);
+  int launches = 3;
+  if (!red.run(ctl->shard_max, 3, AAAC_REDUCE_MAX_I64, st)) return cudaGetLastError();
+  if (!red.run(&ctl->dead_groups, 1, AAAC_REDUCE_SUM_I64, st)) return cudaGetLastError();
+  shard_maxima<<<1, 32, 0, st>>>(ctl, 1);
+  fit_setup<<<1, kFitThreads, 0, st>>>(ctl, T, M_total, ncodes(FMT), stats,
+                                       pp.blocks * kFitWarps, pp.cpc, pp.items);
+  launches += 2;
+  const float tau = choice_tau(S);
+  for (int it = 0; it < iters; it++) {
+    fit_pass<FMT, false><<<pp.blocks, kFitThreads, smem_bytes(false), st>>>(
+        W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items, tau,
+        PackOut{nullptr, nullptr, nullptr, nullptr}, RoundOut{nullptr, nullptr, nullptr, it}, gsc,
+        0);
+    if (!red.run(&ctl->bins[0][0][0], kShardSums, AAAC_REDUCE_SUM_I64, st)) break;
+    shard_round_end<<<1, kFitThreads, 0, st>>>(ctl, flags, RoundOut{err_hist, T, stats, it},
+                                               pp.blocks * kFitWarps, pp.cpc, pp.items, gsc, FMT);
+    launches += 2;
+  }
+  count_launches(launches);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fit_sharded(const uint16_t* W, int64_t N, int64_t K, int64_t M_total,
+                               const float* I, const void* scales, int fmt, int g, int S,
+                               int iters, uint32_t flags, float* T, double* err_hist,
+                               aaac_stats* stats, void* ws, const float* gsc, Reducer& red,
+                               cudaStream_t st) {
+  if (fmt == kInt4)
+    return launch_fit_sharded_t<kInt4>(W, N, K, M_total, I, scales, g, S, iters, flags, T,
+                                       err_hist, stats, ws, gsc, red, st);
+  if (fmt == kNvfp4)
+    return launch_fit_sharded_t<kNvfp4>(W, N, K, M_total, I, scales, g, S, iters, flags, T,
+                                        err_hist, stats, ws, gsc, red, st);
+  return launch_fit_sharded_t<kNvfp4G>(W, N, K, M_total, I, scales, g, S, iters, flags, T,
+                                       err_hist, stats, ws, gsc, red, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -1269,7 +1389,7 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
                                  const float* gsc, cudaStream_t st) {
   const cudaError_t attr = set_smem<FMT, true>();
   if (attr != cudaSuccess) return attr;
-  const FitPlan pp = fit_plan(N, K);
+  const FitPlan pp = fit_plan(N, K, N * K);
   const PassPlan pprep = plan_pass(N, K);
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
   uint8_t* cbytes = reinterpret_cast<uint8_t*>(ws) + fit_ws_bytes(N, K);
@@ -1283,7 +1403,7 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
   const PackOut po{codes, scales_tagged, cbytes, err_final};
   fit_pass<FMT, true><<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
       W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items, tau, po,
-      RoundOut{nullptr, nullptr, nullptr, 0}, gsc);
+      RoundOut{nullptr, nullptr, nullptr, 0}, gsc, 1);
   int launches = 3;
   if (S != g) {
     const int KS = (int)(K / S);
@@ -1293,6 +1413,70 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
   }
   count_launches(launches);
   return cudaSuccess;
+}
+
+// Row-sharded pack: every shard packs its rows with the final tables; the
+// fixed-point scale of the error comes from the max-reduced maxima and the
+// error is the sum-reduced integer total, as in the unsharded pack.
+template <int FMT>
+static cudaError_t launch_pack_sharded_t(const uint16_t* W, int64_t N, int64_t K,
+                                         int64_t M_total, const float* I, const void* scales,
+                                         int g, int S, uint32_t flags, const float* T,
+                                         uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
+                                         uint8_t* choice_bits, double* err_final, void* ws,
+                                         const float* gsc, Reducer& red, cudaStream_t st) {
+  const cudaError_t attr = set_smem<FMT, true>();
+  if (attr != cudaSuccess) return attr;
+  const FitPlan pp = fit_plan(N, K, M_total);
+  const PassPlan pprep = plan_pass(N, K);
+  FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
+  uint8_t* cbytes = reinterpret_cast<uint8_t*>(ws) + fit_ws_bytes(N, K);
+  cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
+  fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
+                                                   pprep.ncb, pprep.rows_per_chunk, gsc);
+  shard_maxima<<<1, 32, 0, st>>>(ctl, 0);
+  int launches = 2;
+  if (red.run(ctl->shard_max, 3, AAAC_REDUCE_MAX_I64, st)) {
+    shard_maxima<<<1, 32, 0, st>>>(ctl, 1);
+    pack_setup<<<1, kFitThreads, 0, st>>>(ctl, T, M_total, ncodes(FMT), T_bf16,
+                                          pp.blocks * kFitWarps, pp.cpc, pp.items,
+                                          FMT == kNvfp4G ? gsc : nullptr);
+    const PackOut po{codes, scales_tagged, cbytes, err_final};
+    fit_pass<FMT, true><<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
+        W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items,
+        choice_tau(S), po, RoundOut{nullptr, nullptr, nullptr, 0}, gsc, 0);
+    launches += 3;
+    if (S != g) {
+      const int KS = (int)(K / S);
+      const int64_t total = N * ((KS + 7) / 8);
+      pack_bits<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(cbytes, N, KS, choice_bits);
+      launches++;
+    }
+    if (red.run(&ctl->err_acc, 1, AAAC_REDUCE_SUM_I64, st)) {
+      shard_pack_end<<<1, 32, 0, st>>>(ctl, err_final);
+      launches++;
+    }
+  }
+  count_launches(launches);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_sharded(const uint16_t* W, int64_t N, int64_t K, int64_t M_total,
+                                const float* I, const void* scales, int fmt, int g, int S,
+                                uint32_t flags, const float* T, uint16_t* T_bf16, uint8_t* codes,
+                                void* scales_tagged, uint8_t* choice_bits, double* err_final,
+                                void* ws, const float* gsc, Reducer& red, cudaStream_t st) {
+  if (fmt == kInt4)
+    return launch_pack_sharded_t<kInt4>(W, N, K, M_total, I, scales, g, S, flags, T, T_bf16,
+                                        codes, scales_tagged, choice_bits, err_final, ws, gsc,
+                                        red, st);
+  if (fmt == kNvfp4)
+    return launch_pack_sharded_t<kNvfp4>(W, N, K, M_total, I, scales, g, S, flags, T, T_bf16,
+                                         codes, scales_tagged, choice_bits, err_final, ws, gsc,
+                                         red, st);
+  return launch_pack_sharded_t<kNvfp4G>(W, N, K, M_total, I, scales, g, S, flags, T, T_bf16,
+                                        codes, scales_tagged, choice_bits, err_final, ws, gsc,
+                                        red, st);
 }
 
 cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const float* I,

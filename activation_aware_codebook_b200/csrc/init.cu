@@ -457,4 +457,50 @@ cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g,
   return cudaGetLastError();
 }
 
+// Row-sharded init: this process holds N rows of a layer of M_total weights.
+// The target ranks come from M_total; the tensor maximum (NVFP4 with a
+// tensor scale) is max-reduced and each pass's histograms are sum-reduced
+// over the shards before the select, so every shard selects the same keys:
+// the order statistics of the whole layer.
+cudaError_t launch_init_sharded(const uint16_t* W, int64_t N, int64_t K, int64_t M_total, int fmt,
+                                int g, void* scales, float* T, void* ws, float* gs_out,
+                                Reducer& red, cudaStream_t st) {
+  const PassPlan pp = plan_pass(N, K);
+  InitCtl* c = reinterpret_cast<InitCtl*>(ws);
+  const int n = ncodes(fmt);
+  const int64_t M = M_total;
+  RankInit ri;
+  for (int j = 0; j < n; j++) {
+    ri.rank[j] = (int64_t)(((__int128)(2 * j + 1) * M) / (2 * n));
+    int64_t r1 = (int64_t)(((__int128)(j + 1) * M) / n);
+    ri.rank[n + j] = r1 > M - 1 ? M - 1 : r1;
+  }
+  for (int j = 2 * n; j < 32; j++) ri.rank[j] = 0;
+  init_setup<<<1, 256, 0, st>>>(c, ri, 2 * n, n);
+  int launches = 1;
+  if (fmt == kNvfp4G) {
+    const uint32_t n_vec = (uint32_t)(N * K / 8);
+    int blocks = (int)((n_vec + kThreads - 1) / kThreads);
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    tensor_amax<<<blocks, kThreads, 0, st>>>(reinterpret_cast<const uint4*>(W), n_vec, c);
+    launches++;
+    if (!red.run(&c->amax_bits, 1, AAAC_REDUCE_MAX_I32, st)) {
+      count_launches(launches);
+      return cudaGetLastError();
+    }
+  }
+  for (int pass = 0; pass < 4; pass++) {
+    const RadixArgs a{W, (int)N, (int)K, g, scales, pass, pp.ncb, pp.rows_per_chunk};
+    if (fmt == kInt4) radix_pass_launch<kInt4>(pass, pp.blocks, a, c, st);
+    else if (fmt == kNvfp4) radix_pass_launch<kNvfp4>(pass, pp.blocks, a, c, st);
+    else radix_pass_launch<kNvfp4G>(pass, pp.blocks, a, c, st);
+    launches++;
+    if (!red.run(&c->hist[0][0], 32 * 256, AAAC_REDUCE_SUM_I32, st)) break;
+    radix_select<<<1, 256, 0, st>>>(c, pass, T, fmt == kNvfp4G ? gs_out : nullptr);
+    launches++;
+  }
+  count_launches(launches);
+  return cudaGetLastError();
+}
+
 }  // namespace aaac

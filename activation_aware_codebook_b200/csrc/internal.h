@@ -60,6 +60,34 @@ cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const float* I,
                         uint8_t* choice_bits, double* err_final, void* ws, const float* gsc,
                         cudaStream_t st);
 
+// ---- row-sharded fit: the caller's reduction over the shards ----------------
+// fn enqueues an in-place reduction of `count` elements at the device address
+// buf on `stream` (op: AAAC_REDUCE_SUM_I64, AAAC_REDUCE_MAX_I64,
+// AAAC_REDUCE_SUM_I32, AAAC_REDUCE_MAX_I32) and returns 0 on success.
+struct Reducer {
+  aaac_reduce_fn fn;
+  void* user;
+  bool failed;
+  bool run(void* buf, int64_t count, int op, cudaStream_t st) {
+    if (failed) return false;
+    if (fn(user, buf, count, op, (void*)st) != 0) failed = true;
+    return !failed;
+  }
+};
+cudaError_t launch_init_sharded(const uint16_t* W, int64_t N, int64_t K, int64_t M_total, int fmt,
+                                int g, void* scales, float* T, void* ws, float* gs_out,
+                                Reducer& red, cudaStream_t st);
+cudaError_t launch_fit_sharded(const uint16_t* W, int64_t N, int64_t K, int64_t M_total,
+                               const float* I, const void* scales, int fmt, int g, int S,
+                               int iters, uint32_t flags, float* T, double* err_hist,
+                               aaac_stats* stats, void* ws, const float* gsc, Reducer& red,
+                               cudaStream_t st);
+cudaError_t launch_pack_sharded(const uint16_t* W, int64_t N, int64_t K, int64_t M_total,
+                                const float* I, const void* scales, int fmt, int g, int S,
+                                uint32_t flags, const float* T, uint16_t* T_bf16, uint8_t* codes,
+                                void* scales_tagged, uint8_t* choice_bits, double* err_final,
+                                void* ws, const float* gsc, Reducer& red, cudaStream_t st);
+
 cudaError_t launch_dequant(const uint8_t* codes, const void* tagged, const uint8_t* cbits,
                            const uint16_t* Tb, int64_t N, int64_t K, int fmt, int g, int S,
                            uint16_t* W_hat, const float* gsc, cudaStream_t st);

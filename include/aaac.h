@@ -44,7 +44,8 @@ typedef enum {
     AAAC_ERR_UNSUPPORTED = 4, /* format / group size this build does not do  */
     AAAC_ERR_CUDA = 5,        /* a CUDA runtime error (see aaac_last_error)    */
     AAAC_ERR_WORKSPACE = 6,   /* ws is NULL or smaller than required           */
-    AAAC_ERR_TIMEOUT = 7      /* reserved: a bounded device wait ran out       */
+    AAAC_ERR_TIMEOUT = 7,     /* reserved: a bounded device wait ran out       */
+    AAAC_ERR_COLLECTIVE = 8   /* a sharded call's reduction callback failed    */
 } aaac_status;
 
 /* Section 1 / 4: the two 4-bit layouts evaluated on the page.
@@ -272,6 +273,44 @@ aaac_status aaac_awq_fit(const void* W, int64_t N, int64_t K, const float* I, in
                          uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
                          uint8_t* choice_bits, double* err_final, double* err_alpha,
                          int32_t* best, void* ws, size_t ws_bytes, void* stream);
+
+/* Row-sharded calls: one layer's rows split over several processes (one per
+ * GPU), each holding N of the layer's N_total rows (its W, scales, codes
+ * rows; I is the whole K columns).  Where the unsharded call reduces over all
+ * rows -- the quantile histograms, the maxima that fix the fixed-point
+ * exponents, each round's refine sums and objective -- the sharded call
+ * hands a buffer in its workspace to the caller's reduction, which must
+ * combine it over all shards in place (an all-reduce, e.g. NCCL over
+ * NVLink), enqueued on `stream`.  Every reduced quantity is an integer, so
+ * the result does not depend on the reduction's order: every shard ends
+ * with the tables of the unsharded call on the whole layer, bit for bit,
+ * and packs its own rows exactly as the unsharded pack would.  Per fit round
+ * the exchange is 68 int64 values (544 bytes).
+ *   op AAAC_REDUCE_SUM_I64 / MAX_I64: int64 elements; SUM_I32 / MAX_I32: int32.
+ *   The callback returns 0 on success; any other value stops the call, which
+ *   returns AAAC_ERR_COLLECTIVE (work already enqueued stays enqueued).
+ * Every shard must make the same calls with the same cfg, K and N_total. */
+#define AAAC_REDUCE_SUM_I64 0
+#define AAAC_REDUCE_MAX_I64 1
+#define AAAC_REDUCE_SUM_I32 2
+#define AAAC_REDUCE_MAX_I32 3
+typedef int (*aaac_reduce_fn)(void* user, void* buf, int64_t count, int op, void* stream);
+
+aaac_status aaac_init_codebooks_sharded(const void* W, int64_t N, int64_t K, int64_t N_total,
+                                        const aaac_config* cfg, void* scales, float* T,
+                                        aaac_reduce_fn reduce, void* user, void* ws,
+                                        size_t ws_bytes, void* stream);
+aaac_status aaac_fit_layer_sharded(const void* W, int64_t N, int64_t K, int64_t N_total,
+                                   const float* I, const void* scales, const aaac_config* cfg,
+                                   float* T, double* err_hist, aaac_stats* stats,
+                                   aaac_reduce_fn reduce, void* user, void* ws, size_t ws_bytes,
+                                   void* stream);
+aaac_status aaac_pack_sharded(const void* W, int64_t N, int64_t K, int64_t N_total,
+                              const float* I, const void* scales, const aaac_config* cfg,
+                              const float* T, uint16_t* T_bf16, uint8_t* codes,
+                              void* scales_tagged, uint8_t* choice_bits, double* err_final,
+                              aaac_reduce_fn reduce, void* user, void* ws, size_t ws_bytes,
+                              void* stream);
 
 /* Device-side wait status of the current device: *flag = 1 when a bounded
  * wait inside one of the library's kernels (the tensor-core aaac_linear path)
