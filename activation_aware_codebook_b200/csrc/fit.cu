@@ -11,10 +11,12 @@
 //
 // One fit round is ONE launch of fit_pass<false>: a streaming pass over W whose
 // last block to finish (atomic ticket, no waiting) does the refine, sorts the
-// books, rebuilds the tables and records the error.  Per block: 2 warps; a warp
+// books, rebuilds the tables and records the error.  Per block: 3 warps; a warp
 // covers 512 columns of a row, 16 per lane (32 bytes), and walks the rows of
-// its chunk with a 3-deep cp.async ring.  The grid is one wave (5 blocks per
-// SM, bounded by the refine bins' shared memory).
+// its work items with a 2-deep cp.async ring.  The grid is one wave (4 blocks,
+// 12 warps, per SM, bounded by the refine bins' shared memory: 16 KB a warp;
+// the last block's table rebuild borrows the idle ring for its scratch, so
+// the pass holds almost no static shared memory).
 //
 // Nearest entry in both books at once (exact):
 //   the midpoint thresholds of both books, merged and deduplicated (at most
@@ -48,10 +50,10 @@
 namespace aaac {
 
 constexpr int kNB = 128;                  // bucket LUT entries
-constexpr int kFitWarps = 2;
+constexpr int kFitWarps = 3;
 constexpr int kFitThreads = kFitWarps * 32;
-constexpr int kStages = 3;                // rows per warp in flight
-constexpr int kFitBlocksPerSM = 5;
+constexpr int kStages = 2;                // rows per warp in flight
+constexpr int kFitBlocksPerSM = 4;
 constexpr int kLaneCols = 16;             // columns per lane
 constexpr int kItemRows = 4;              // rows of one work item
 constexpr int kMaxStrips = 256;           // per-strip work counters (more strips: one counter)
@@ -199,12 +201,28 @@ __device__ inline int bucket_raw(float x, float la) {
 //      bucket b counts the thresholds below it or opening it, and is crowded
 //      when two or more fall strictly inside.
 // When sort_first, sT is left sorted (the callers write it back as T).
-__device__ void build_tables(Tables& tb, float (*sT)[16], int n, bool sort_first) {
-  __shared__ float s_sorted[2][16];
-  __shared__ float s_slot[32];
-  __shared__ int s_src[32];
-  __shared__ int s_cc[2][kMerged];
-  __shared__ int s_A[kNB + 2], s_F[kNB + 2];
+// Shared-memory scratch of the table rebuild and the refine.  The fit pass's
+// last block places it in its (by then idle) row ring, so the pass holds no
+// static shared memory for work that only one block does.
+struct FinalizeScratch {
+  float s_sorted[2][16];
+  float s_slot[32];
+  int s_src[32];
+  int s_cc[2][kMerged];
+  int s_A[kNB + 2], s_F[kNB + 2];
+  float sT[2][16];
+  long long sb[64];
+  int s_upd[2];
+};
+
+__device__ void build_tables(Tables& tb, float (*sT)[16], int n, bool sort_first,
+                             FinalizeScratch& sc) {
+  float (*s_sorted)[16] = sc.s_sorted;
+  float* s_slot = sc.s_slot;
+  int* s_src = sc.s_src;
+  int (*s_cc)[kMerged] = sc.s_cc;
+  int* s_A = sc.s_A;
+  int* s_F = sc.s_F;
   const int tid = threadIdx.x, lane = tid & 31;
   const unsigned full = 0xffffffffu;
   for (int i = tid; i < kNB + 2; i += blockDim.x) {
@@ -441,11 +459,16 @@ __device__ float bucket_scale(const FitCtl* ctl) {
   return Umax > 0.0f ? __fdiv_rn(62.5f, Umax) : 0.0f;  // |u| * la < 63: buckets 1..127
 }
 
+static_assert(sizeof(FinalizeScratch) <= (size_t)kFitWarps * kStages * kRingRowBytes,
+              "the last block's finalize scratch lives in the row ring");
+static_assert(kFitThreads >= 64, "the bin flush takes one thread per (cell, num | den)");
+
 // L = B - E(I_max) - E(S2_max) - max(0, E(U_max)), B = min(40, 61 - ceil(log2 M))
 __global__ void __launch_bounds__(kFitThreads)
 fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st, int wt, int cpc,
           int n_items) {
   __shared__ Tables tb;
+  __shared__ FinalizeScratch sc;
   seed_claims(ctl, wt, cpc, n_items);
   if (threadIdx.x == 0) {
     int c = 0;
@@ -468,10 +491,10 @@ fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st, int wt, 
     ctl->n = n;
     tb.la = bucket_scale(ctl);
   }
-  __shared__ float sT[2][16];
+  float (*sT)[16] = sc.sT;
   if (threadIdx.x < 32) sT[threadIdx.x >> 4][threadIdx.x & 15] = T_user[threadIdx.x];
   __syncthreads();
-  build_tables(tb, sT, n, true);
+  build_tables(tb, sT, n, true, sc);
   store_tables(ctl, tb);
   if (threadIdx.x < 32) {
     const float t = sT[threadIdx.x >> 4][threadIdx.x & 15];
@@ -539,10 +562,10 @@ __device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsign
 // fp64(den)) when den > 0, else unchanged; then sorted books and new tables.
 // Everything is staged in shared memory and spread over the block's threads.
 __device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const RoundOut& ro,
-                               int wt, int cpc, int n_items, double g2) {
-  __shared__ float sT[2][16];
-  __shared__ long long sb[64];
-  __shared__ int s_upd[2];
+                               int wt, int cpc, int n_items, double g2, FinalizeScratch& sc) {
+  float (*sT)[16] = sc.sT;
+  long long* sb = sc.sb;
+  int* s_upd = sc.s_upd;
   const int tid = threadIdx.x;
   if (tid < 64) sb[tid] = __ldcg(&ctl->bins[0][0][0] + tid);
   if (tid < 32) sT[tid >> 4][tid & 15] = ctl->T[tid >> 4][tid & 15];
@@ -571,7 +594,7 @@ __device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const Ro
   __syncthreads();
   const bool f0 = (flags & AAAC_FREEZE_T0) != 0, f1 = (flags & AAAC_FREEZE_T1) != 0;
   const int empty = (f0 ? 0 : n - s_upd[0]) + (f1 ? 0 : n - s_upd[1]);
-  build_tables(tb, sT, n, true);
+  build_tables(tb, sT, n, true, sc);
   store_tables(ctl, tb);
   if (tid < 32) {
     const float t = sT[tid >> 4][tid & 15];
@@ -881,7 +904,6 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
 #pragma unroll
   for (int k = 0; k < kStages; k++)
     if (k >= npre) sqv[k] = prefetch(k);
-  float sq0 = sqv[0], sq1 = sqv[1], sq2 = sqv[2];
 
   GroupStats gs{0u, 0u, 0u, 0ull};
   int slot = 0;
@@ -902,10 +924,10 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     const uint4 va = *reinterpret_cast<const uint4*>(srow + rd0);
     const uint4 vb = *reinterpret_cast<const uint4*>(srow + rd1);
     __syncwarp();  // every lane has read the slot before it is refilled
-    const float s = sq0;
-    sq0 = sq1;
-    sq1 = sq2;
-    sq2 = prefetch(slot);  // the row kStages positions ahead into this slot
+    const float s = sqv[0];
+#pragma unroll
+    for (int k = 0; k + 1 < kStages; k++) sqv[k] = sqv[k + 1];
+    sqv[kStages - 1] = prefetch(slot);  // the row kStages positions ahead into this slot
     slot = (slot + 1 == kStages) ? 0 : slot + 1;
 
     float rcp;
@@ -1090,7 +1112,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   for (int o = 16; o > 0; o >>= 1) gs.err += __shfl_xor_sync(0xffffffffu, gs.err, o);
   if (lane == 0 && gs.err) atomicAdd(&ctl->err_acc, gs.err);
   __syncthreads();  // every lane's bins are complete
-  if (!PACK) {
+  if (!PACK && threadIdx.x < 64) {
     // lane bins -> exact integer partials (bias removed exactly), one
     // (book, entry, num | den) per thread, summed over the block's lanes
     const int bc = threadIdx.x >> 1, which = threadIdx.x & 1;
@@ -1119,7 +1141,8 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     if (threadIdx.x == 0) ctl->ticket = 0;
     seed_claims(ctl, wt, cpc, n_items);
   } else if (!PACK) {
-    round_finalize(ctl, tb, flags, ro, wt, cpc, n_items, __dmul_rn((double)gsv, (double)gsv));
+    round_finalize(ctl, tb, flags, ro, wt, cpc, n_items, __dmul_rn((double)gsv, (double)gsv),
+                   *reinterpret_cast<FinalizeScratch*>(ring));  // the ring is idle now
   } else {
     if (threadIdx.x == 0) {
       const long long acc = (long long)__ldcg(&ctl->err_acc);
@@ -1155,6 +1178,7 @@ __global__ void __launch_bounds__(kFitThreads)
 shard_round_end(FitCtl* ctl, uint32_t flags, RoundOut ro, int wt, int cpc, int n_items,
                 const float* __restrict__ gsc, int fmt) {
   __shared__ Tables tb;
+  __shared__ FinalizeScratch sc;
   {
     const uint32_t* src = reinterpret_cast<const uint32_t*>(&ctl->tb);
     uint32_t* dst = reinterpret_cast<uint32_t*>(&tb);
@@ -1166,7 +1190,7 @@ shard_round_end(FitCtl* ctl, uint32_t flags, RoundOut ro, int wt, int cpc, int n
   }
   __syncthreads();
   const double gs = fmt == kNvfp4G ? (double)__ldg(gsc) : 1.0;
-  round_finalize(ctl, tb, flags, ro, wt, cpc, n_items, __dmul_rn(gs, gs));
+  round_finalize(ctl, tb, flags, ro, wt, cpc, n_items, __dmul_rn(gs, gs), sc);
   __syncthreads();
   if (threadIdx.x == 0) ctl->exact_groups = 0ull;  // the next round counts its own
 }
@@ -1344,7 +1368,8 @@ __global__ void __launch_bounds__(kFitThreads)
 pack_setup(FitCtl* ctl, const float* T_user, int64_t M, int n, uint16_t* T_bf16, int wt,
            int cpc, int n_items, const float* gsc) {
   __shared__ Tables tb;
-  __shared__ float sT[2][16];
+  __shared__ FinalizeScratch sc;
+  float (*sT)[16] = sc.sT;
   seed_claims(ctl, wt, cpc, n_items);
   if (threadIdx.x == 0) {
     ctl->n = n;
@@ -1364,7 +1389,7 @@ pack_setup(FitCtl* ctl, const float* T_user, int64_t M, int n, uint16_t* T_bf16,
     sT[b][j] = __uint_as_float((uint32_t)h << 16);
   }
   __syncthreads();
-  build_tables(tb, sT, n, false);
+  build_tables(tb, sT, n, false, sc);
   store_tables(ctl, tb);
   if (threadIdx.x < 32) ctl->T[threadIdx.x >> 4][threadIdx.x & 15] = sT[threadIdx.x >> 4][threadIdx.x & 15];
 }
