@@ -54,6 +54,7 @@ constexpr int kFitWarps = 3;
 constexpr int kFitThreads = kFitWarps * 32;
 constexpr int kStages = 2;                // rows per warp in flight
 constexpr int kFitBlocksPerSM = 4;
+constexpr int kPrepRows = 4;  // rows per lane loaded ahead by fit_prep
 constexpr int kLaneCols = 16;             // columns per lane
 constexpr int kItemRows = 4;              // rows of one work item
 constexpr int kMaxStrips = 256;           // per-strip work counters (more strips: one counter)
@@ -387,20 +388,34 @@ fit_prep(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   unsigned long long dead = 0;
   const int r0 = rc * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
   if (active) {
-    for (int r = r0 + warp; r < r1; r += kWarps) {
-      const float s = load_scale<FMT>(scales, (int64_t)r * G + col0 / g);
-      float rcp;
-      if (!scale_live(eff_scale<FMT>(s, gsv), &rcp)) {
-        if ((lane & (lanes_g - 1)) == 0) dead++;
-        continue;
-      }
-      s2m = fmax(s2m, (double)s * (double)s);
-      uint4 v = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)r * K + col0));
-      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    // kPrepRows rows per lane are loaded before any is used (loads in flight)
+    for (int rb = r0 + warp; rb < r1; rb += kWarps * kPrepRows) {
+      float sv[kPrepRows];
+      uint4 wv[kPrepRows];
 #pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const float wf = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
-        um = max(um, __float_as_uint(fabsf(__fmul_rn(wf, rcp))));
+      for (int k = 0; k < kPrepRows; k++) {
+        const int r = rb + k * kWarps;
+        const bool in = r < r1;
+        sv[k] = in ? load_scale<FMT>(scales, (int64_t)r * G + col0 / g) : 0.0f;
+        wv[k] = in ? __ldg(reinterpret_cast<const uint4*>(W + (int64_t)r * K + col0))
+                   : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < kPrepRows; k++) {
+        if (rb + k * kWarps >= r1) break;  // warp-uniform
+        const float s = sv[k];
+        float rcp;
+        if (!scale_live(eff_scale<FMT>(s, gsv), &rcp)) {
+          if ((lane & (lanes_g - 1)) == 0) dead++;
+          continue;
+        }
+        s2m = fmax(s2m, (double)s * (double)s);
+        const uint32_t w[4] = {wv[k].x, wv[k].y, wv[k].z, wv[k].w};
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+          const float wf = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+          um = max(um, __float_as_uint(fabsf(__fmul_rn(wf, rcp))));
+        }
       }
     }
   }
@@ -410,7 +425,24 @@ fit_prep(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     s2m = fmax(s2m, __shfl_xor_sync(0xffffffffu, s2m, o));
     dead += __shfl_xor_sync(0xffffffffu, dead, o);
   }
+  // one atomic per block and quantity (same-address atomics serialise)
+  __shared__ uint32_t s_im[kWarps], s_um[kWarps];
+  __shared__ double s_s2[kWarps];
+  __shared__ unsigned long long s_dead[kWarps];
   if (lane == 0) {
+    s_im[warp] = im;
+    s_um[warp] = um;
+    s_s2[warp] = s2m;
+    s_dead[warp] = dead;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kWarps; w++) {
+      im = max(im, s_im[w]);
+      um = max(um, s_um[w]);
+      s2m = fmax(s2m, s_s2[w]);
+      dead += s_dead[w];
+    }
     if (im) atomicMax(&ctl->Imax_bits, im);
     if (um) atomicMax(&ctl->Umax_bits, um);
     if (s2m > 0.0) atomicMax(&ctl->S2max_bits, (unsigned long long)__double_as_longlong(s2m));
