@@ -486,7 +486,8 @@ def run_sharded(args, rank, local_rank, world):
 
 def run_e2e(blk, steps, dev):
     """Same step through the public API with host-resident inputs: pinned H2D
-    of every activation and weight, the four calls, D2H of every output."""
+    of every activation and weight, the four calls, D2H of every output, with
+    the copies overlapping the compute (three streams)."""
     import torch
     hostX = {k: torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for k, x in blk.Xs.items()}
     hostW = {k: torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for k, w in blk.Ws.items()}
@@ -500,24 +501,70 @@ def run_e2e(blk, steps, dev):
     h2d = sum(v.numel() * v.element_size() for v in list(hostX.values()) + list(hostW.values()))
     d2h = blk.output_bytes()
 
+    # Copies overlap the compute: the inputs go host -> device on one stream
+    # in the order the step uses them, the compute stream waits for each
+    # input just before its first use, and each linear's outputs go device ->
+    # host on a third stream as soon as its pack is done.  Events guard the
+    # reuse of every buffer across steps.
+    bb = blk.bb
+    comp = torch.cuda.current_stream()
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    x_free = {k: None for k in hostX}
+    w_free = {l.name: None for l in blk.wl.linears}
+    out_free = {l.name: None for l in blk.wl.linears}
+
     def one():
-        for k in hostX:
-            blk.Xs[k].copy_(hostX[k], non_blocking=True)
-        for k in hostW:
-            blk.Ws[k].copy_(hostW[k], non_blocking=True)
-        blk.step()
+        x_ready, w_ready = {}, {}
+        with torch.cuda.stream(h2d_s):
+            for k in hostX:
+                if x_free[k] is not None:
+                    h2d_s.wait_event(x_free[k])
+                blk.Xs[k].copy_(hostX[k], non_blocking=True)
+                x_ready[k] = ev()
+                x_ready[k].record(h2d_s)
+            for l in blk.wl.linears:
+                if w_free[l.name] is not None:
+                    h2d_s.wait_event(w_free[l.name])
+                blk.Ws[l.name].copy_(hostW[l.name], non_blocking=True)
+                w_ready[l.name] = ev()
+                w_ready[l.name].record(h2d_s)
+        for k, X in blk.Xs.items():
+            comp.wait_event(x_ready[k])
+            bb.importance(X, I=blk.I[k], ws=blk.ws)
+            x_free[k] = ev()
+            x_free[k].record(comp)
         for l in blk.wl.linears:
-            for k, v in blk.out[l.name].items():
-                if v is not None:
-                    hostOut[l.name][k].copy_(v, non_blocking=True)
+            W, cfg = blk.Ws[l.name], blk.cfgs[l.name]
+            comp.wait_event(w_ready[l.name])
+            if out_free[l.name] is not None:
+                comp.wait_event(out_free[l.name])
+            bb.init_codebooks(W, cfg, ws=blk.ws, scales=blk.scales[l.name], T=blk.T[l.name])
+            bb.fit_layer(W, blk.I[l.x_key], blk.scales[l.name], blk.T[l.name], cfg, ws=blk.ws,
+                         err_hist=blk.eh[l.name], stats=blk.st[l.name])
+            bb.pack(W, blk.I[l.x_key], blk.scales[l.name], blk.T[l.name], cfg, ws=blk.ws,
+                    out=blk.out[l.name])
+            done = ev()
+            done.record(comp)
+            w_free[l.name] = done
+            d2h_s.wait_event(done)
+            with torch.cuda.stream(d2h_s):
+                for k, v in blk.out[l.name].items():
+                    if v is not None:
+                        hostOut[l.name][k].copy_(v, non_blocking=True)
+                out_free[l.name] = ev()
+                out_free[l.name].record(d2h_s)
 
     one()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(comp)
+    h2d_s.wait_event(e0)
     for _ in range(steps):
         one()
-    e1.record()
+    comp.wait_stream(d2h_s)
+    comp.wait_stream(h2d_s)
+    e1.record(comp)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     return {"value": blk.weight_iters / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
