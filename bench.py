@@ -194,7 +194,11 @@ def build_block(wl, block, tokens, dev):
 
 
 class Block:
-    """Device buffers and the step of one block of linears."""
+    """Device buffers and the step of one block of linears.  The linears are
+    independent once the importance vectors exist, so each runs its init,
+    fit and pack on its own stream with its own workspace (biggest first):
+    one layer's short phases (the refine tail of a round, the radix selects,
+    small layers' rounds) overlap another's streaming passes."""
 
     def __init__(self, wl, Xs, Ws, dev):
         import torch
@@ -229,23 +233,47 @@ class Block:
             if gs is not None:  # part of the packed layer
                 self.out[l.name]["global_scale"] = gs
         self.weight_iters = sum(l.N * l.K for l in wl.linears) * wl.iters
+        self.order = sorted(wl.linears, key=lambda l: -l.N * l.K)
+        self.streams = {l.name: torch.cuda.Stream(device=dev) for l in wl.linears}
+        self.wss = {l.name: torch.empty(bb.workspace_size(self.cfgs[l.name], l.N, l.K, 0),
+                                        dtype=torch.uint8, device=dev) for l in wl.linears}
 
-    def step(self, fit_events=None, probe=None):
+    def step(self, fit_events=None, probe=None, waits=None):
+        """importance on the current stream, then every linear on its own
+        stream; the current stream waits for all of them before returning.
+        waits: optional {linear name: [events]} a linear's stream waits for
+        (e2e: its weight copy, the previous copy-out of its outputs).
+        Returns (event after the importance, {linear name: event after its
+        pack})."""
+        import torch
         bb = self.bb
+        comp = torch.cuda.current_stream()
         for k, X in self.Xs.items():
             bb.importance(X, I=self.I[k], ws=self.ws)
-        for l in self.wl.linears:
-            W = self.Ws[l.name]
-            cfg = self.cfgs[l.name]
-            bb.init_codebooks(W, cfg, ws=self.ws, scales=self.scales[l.name], T=self.T[l.name])
-            if fit_events is not None and l.name == probe:
-                fit_events[0].record()
-            bb.fit_layer(W, self.I[l.x_key], self.scales[l.name], self.T[l.name], cfg,
-                         ws=self.ws, err_hist=self.eh[l.name], stats=self.st[l.name])
-            if fit_events is not None and l.name == probe:
-                fit_events[1].record()
-            bb.pack(W, self.I[l.x_key], self.scales[l.name], self.T[l.name], cfg, ws=self.ws,
-                    out=self.out[l.name])
+        imp = torch.cuda.Event()
+        imp.record(comp)
+        done = {}
+        for l in self.order:
+            s = self.streams[l.name]
+            s.wait_event(imp)
+            for e in (waits or {}).get(l.name, ()):
+                s.wait_event(e)
+            with torch.cuda.stream(s):
+                W, cfg, ws = self.Ws[l.name], self.cfgs[l.name], self.wss[l.name]
+                bb.init_codebooks(W, cfg, ws=ws, scales=self.scales[l.name], T=self.T[l.name])
+                if fit_events is not None and l.name == probe:
+                    fit_events[0].record(s)
+                bb.fit_layer(W, self.I[l.x_key], self.scales[l.name], self.T[l.name], cfg,
+                             ws=ws, err_hist=self.eh[l.name], stats=self.st[l.name])
+                if fit_events is not None and l.name == probe:
+                    fit_events[1].record(s)
+                bb.pack(W, self.I[l.x_key], self.scales[l.name], self.T[l.name], cfg, ws=ws,
+                        out=self.out[l.name])
+                done[l.name] = torch.cuda.Event()
+                done[l.name].record(s)
+        for l in self.order:
+            comp.wait_event(done[l.name])
+        return imp, done
 
     def output_bytes(self):
         tot = 0
@@ -268,6 +296,27 @@ def fit_setup_ms(blk, lin, reps=5):
     for _ in range(reps + 1):
         e0.record()
         bb.fit_layer(W, blk.I[lin.x_key], blk.scales[lin.name], T, cfg0, ws=blk.ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times[1:])
+
+
+def fit_alone_ms(blk, lin, reps=5):
+    """Time of the probe layer's whole fit (prep, setup, every round) with
+    nothing else on the GPU: the roofline of the fit pass is taken from it,
+    while the timed step runs the linears concurrently."""
+    import torch
+    bb = blk.bb
+    W = blk.Ws[lin.name]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    for _ in range(reps + 1):
+        T = blk.T[lin.name].clone()
+        torch.cuda.synchronize()
+        e0.record()
+        bb.fit_layer(W, blk.I[lin.x_key], blk.scales[lin.name], T, blk.cfgs[lin.name],
+                     ws=blk.ws, err_hist=blk.eh[lin.name], stats=blk.st[lin.name])
         e1.record()
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
@@ -323,8 +372,11 @@ def run_ours(args, rank, local_rank, world):
     fit_ms = statistics.median(a.elapsed_time(b) for a, b in fit_ev)
     ms_max = max_over_ranks(ms, world, dev)
 
-    # roofline of one fit round (one fit_pass launch) on the probe layer
-    iter_ms = (fit_ms - setup_ms) / wl.iters
+    # roofline of one fit round (one fit_pass launch) on the probe layer: the
+    # probe's fit timed alone (the step overlaps it with the other linears)
+    alone_ms = fit_alone_ms(blk, probe)
+    iter_ms = (alone_ms - setup_ms) / wl.iters
+    iter_in_step_ms = (fit_ms - setup_ms) / wl.iters
     scale_bytes = 2 if wl.fmt == bb.INT4 else 1
     bytes_per_iter = (probe.N * probe.K * 2 + probe.N * (probe.K // wl.g) * scale_bytes
                       + probe.K * 4)
@@ -355,7 +407,8 @@ def run_ours(args, rank, local_rank, world):
                        "tokens": tokens,
                        "format": {bb.INT4: "INT4", bb.NVFP4: "NVFP4"}.get(wl.fmt, "NVFP4+tensor scale"),
                        "g": wl.g, "S": wl.S, "iters": wl.iters,
-                       "blocks": world, "parallelism": f"layer-parallel x{world} (no collective)",
+                       "blocks": world, "parallelism": f"layer-parallel x{world} (no collective); "
+                                                      "the linears of a block on concurrent streams",
                        "l2": "inputs larger than L2 (activations %.1f GiB per step)" % (
                            sum(x.numel() * 2 for x in Xs.values()) / 2 ** 30)},
             "roofline": {"kernel": "fit_pass (one fit round; refine fused in its last block)",
@@ -363,7 +416,8 @@ def run_ours(args, rank, local_rank, world):
                          "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "bytes_per_launch": bytes_per_iter,
-                         "round_ms": iter_ms},
+                         "round_ms": iter_ms, "timing": "the probe's fit alone, CUDA events",
+                         "round_ms_in_step": iter_in_step_ms},
             "gpu_launches": int(launches),
             "clocks": clocks,
         }
@@ -502,11 +556,10 @@ def run_e2e(blk, steps, dev):
     d2h = blk.output_bytes()
 
     # Copies overlap the compute: the inputs go host -> device on one stream
-    # in the order the step uses them, the compute stream waits for each
-    # input just before its first use, and each linear's outputs go device ->
-    # host on a third stream as soon as its pack is done.  Events guard the
-    # reuse of every buffer across steps.
-    bb = blk.bb
+    # in the order the step uses them, the importance waits for the
+    # activations and each linear's stream for its weights, and each linear's
+    # outputs go device -> host on a third stream as soon as its pack is done.
+    # Events guard the reuse of every buffer across steps.
     comp = torch.cuda.current_stream()
     h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()  # noqa: E731
@@ -523,31 +576,22 @@ def run_e2e(blk, steps, dev):
                 blk.Xs[k].copy_(hostX[k], non_blocking=True)
                 x_ready[k] = ev()
                 x_ready[k].record(h2d_s)
-            for l in blk.wl.linears:
+            for l in blk.order:
                 if w_free[l.name] is not None:
                     h2d_s.wait_event(w_free[l.name])
                 blk.Ws[l.name].copy_(hostW[l.name], non_blocking=True)
                 w_ready[l.name] = ev()
                 w_ready[l.name].record(h2d_s)
-        for k, X in blk.Xs.items():
+        for k in hostX:
             comp.wait_event(x_ready[k])
-            bb.importance(X, I=blk.I[k], ws=blk.ws)
-            x_free[k] = ev()
-            x_free[k].record(comp)
-        for l in blk.wl.linears:
-            W, cfg = blk.Ws[l.name], blk.cfgs[l.name]
-            comp.wait_event(w_ready[l.name])
-            if out_free[l.name] is not None:
-                comp.wait_event(out_free[l.name])
-            bb.init_codebooks(W, cfg, ws=blk.ws, scales=blk.scales[l.name], T=blk.T[l.name])
-            bb.fit_layer(W, blk.I[l.x_key], blk.scales[l.name], blk.T[l.name], cfg, ws=blk.ws,
-                         err_hist=blk.eh[l.name], stats=blk.st[l.name])
-            bb.pack(W, blk.I[l.x_key], blk.scales[l.name], blk.T[l.name], cfg, ws=blk.ws,
-                    out=blk.out[l.name])
-            done = ev()
-            done.record(comp)
-            w_free[l.name] = done
-            d2h_s.wait_event(done)
+        waits = {l.name: [w_ready[l.name]] + ([out_free[l.name]] if out_free[l.name] else [])
+                 for l in blk.order}
+        imp, done = blk.step(waits=waits)
+        for k in hostX:
+            x_free[k] = imp
+        for l in blk.order:
+            w_free[l.name] = done[l.name]
+            d2h_s.wait_event(done[l.name])
             with torch.cuda.stream(d2h_s):
                 for k, v in blk.out[l.name].items():
                     if v is not None:
