@@ -237,25 +237,45 @@ class Block:
         self.streams = {l.name: torch.cuda.Stream(device=dev) for l in wl.linears}
         self.wss = {l.name: torch.empty(bb.workspace_size(self.cfgs[l.name], l.N, l.K, 0),
                                         dtype=torch.uint8, device=dev) for l in wl.linears}
+        # importance of each activation set on its own stream and workspace, in
+        # the order the linears (biggest first) need them
+        self.keys = []
+        for l in self.order:
+            if l.x_key not in self.keys:
+                self.keys.append(l.x_key)
+        self.kstreams = {k: torch.cuda.Stream(device=dev) for k in self.keys}
+        self.kws = {k: torch.empty(bb.workspace_size(None, 0, Xs[k].shape[1], tokens),
+                                   dtype=torch.uint8, device=dev) for k in self.keys}
 
-    def step(self, fit_events=None, probe=None, waits=None):
-        """importance on the current stream, then every linear on its own
-        stream; the current stream waits for all of them before returning.
+    def step(self, fit_events=None, probe=None, waits=None, key_waits=None):
+        """The importance of each activation set on its own stream, then
+        every linear on its own stream once its importance is done; the
+        current stream waits for all of them before returning.
         waits: optional {linear name: [events]} a linear's stream waits for
-        (e2e: its weight copy, the previous copy-out of its outputs).
-        Returns (event after the importance, {linear name: event after its
-        pack})."""
+        (e2e: its weight copy, the previous copy-out of its outputs);
+        key_waits: optional {key: [events]} an importance waits for (e2e:
+        the activations' copy).  Returns ({key: event after its importance},
+        {linear name: event after its pack})."""
         import torch
         bb = self.bb
         comp = torch.cuda.current_stream()
-        for k, X in self.Xs.items():
-            bb.importance(X, I=self.I[k], ws=self.ws)
-        imp = torch.cuda.Event()
-        imp.record(comp)
+        start = torch.cuda.Event()
+        start.record(comp)
+        imp = {}
+        for k in self.keys:
+            ks = self.kstreams[k]
+            ks.wait_event(start)
+            for e in (key_waits or {}).get(k, ()):
+                ks.wait_event(e)
+            with torch.cuda.stream(ks):
+                bb.importance(self.Xs[k], I=self.I[k], ws=self.kws[k])
+                imp[k] = torch.cuda.Event()
+                imp[k].record(ks)
         done = {}
         for l in self.order:
             s = self.streams[l.name]
-            s.wait_event(imp)
+            s.wait_event(start)
+            s.wait_event(imp[l.x_key])
             for e in (waits or {}).get(l.name, ()):
                 s.wait_event(e)
             with torch.cuda.stream(s):
@@ -273,6 +293,8 @@ class Block:
                 done[l.name].record(s)
         for l in self.order:
             comp.wait_event(done[l.name])
+        for k in self.keys:
+            comp.wait_event(imp[k])
         return imp, done
 
     def output_bytes(self):
@@ -570,25 +592,25 @@ def run_e2e(blk, steps, dev):
     def one():
         x_ready, w_ready = {}, {}
         with torch.cuda.stream(h2d_s):
-            for k in hostX:
-                if x_free[k] is not None:
-                    h2d_s.wait_event(x_free[k])
-                blk.Xs[k].copy_(hostX[k], non_blocking=True)
-                x_ready[k] = ev()
-                x_ready[k].record(h2d_s)
+            # in the order of use: each linear's activations (once), then its weights
             for l in blk.order:
+                k = l.x_key
+                if k not in x_ready:
+                    if x_free[k] is not None:
+                        h2d_s.wait_event(x_free[k])
+                    blk.Xs[k].copy_(hostX[k], non_blocking=True)
+                    x_ready[k] = ev()
+                    x_ready[k].record(h2d_s)
                 if w_free[l.name] is not None:
                     h2d_s.wait_event(w_free[l.name])
                 blk.Ws[l.name].copy_(hostW[l.name], non_blocking=True)
                 w_ready[l.name] = ev()
                 w_ready[l.name].record(h2d_s)
-        for k in hostX:
-            comp.wait_event(x_ready[k])
         waits = {l.name: [w_ready[l.name]] + ([out_free[l.name]] if out_free[l.name] else [])
                  for l in blk.order}
-        imp, done = blk.step(waits=waits)
+        imp, done = blk.step(waits=waits, key_waits={k: [x_ready[k]] for k in hostX})
         for k in hostX:
-            x_free[k] = imp
+            x_free[k] = imp[k]
         for l in blk.order:
             w_free[l.name] = done[l.name]
             d2h_s.wait_event(done[l.name])
