@@ -35,6 +35,7 @@ import hashlib
 import json
 import os
 import time
+from concurrent.futures import ThreadPoolExecutor
 from typing import Callable, Dict, Iterable, List, Optional
 
 import numpy as np
@@ -129,34 +130,52 @@ Runner = Callable[[Unit], Dict[str, np.ndarray]]
 
 def run_rank(out_dir: str, units: List[Unit], rank: int, world: int, runner: Runner,
              log: Optional[Callable[[str], None]] = None) -> dict:
-    """Fit and store this rank's share of `units`, skipping done ones."""
+    """Fit and store this rank's share of `units`, skipping done ones.  A
+    unit's result is written by a background writer while the next unit
+    runs on the GPU; the writer is the only thread that touches the files and
+    the manifest, so the manifest keeps the units' order."""
     os.makedirs(out_dir, exist_ok=True)
     manifest = os.path.join(out_dir, f"manifest_r{rank}.jsonl")
     done = load_done(out_dir)
     mine = partition(units, world)[rank]
-    ran = skipped = failed = 0
+    skipped = 0
     t_all = time.time()
-    for u in mine:
-        if u.uid in done:
-            skipped += 1
-            continue
-        t0 = time.time()
+    writes = []
+
+    def write_ok(u: Unit, arrays: Dict[str, np.ndarray], seconds: float) -> bool:
         try:
-            arrays = runner(u)
             rel = _save(out_dir, u.uid, arrays)
-            rec = {"unit": u.uid, "status": "ok", "file": rel,
-                   "sha256": _sha256(os.path.join(out_dir, rel)), "rank": rank,
-                   "seconds": time.time() - t0, "N": u.linear.N, "K": u.linear.K}
-            _append(manifest, rec)
-            ran += 1
+            _append(manifest, {"unit": u.uid, "status": "ok", "file": rel,
+                               "sha256": _sha256(os.path.join(out_dir, rel)), "rank": rank,
+                               "seconds": seconds, "N": u.linear.N, "K": u.linear.K})
+            return True
         except Exception as e:  # recorded, retried by the next run
-            _append(manifest, {"unit": u.uid, "status": "failed", "rank": rank,
-                               "error": f"{type(e).__name__}: {e}"})
-            failed += 1
-            if log:
-                log(f"rank {rank}: {u.uid} failed: {e}")
+            write_failed(u, e)
+            return False
+
+    def write_failed(u: Unit, e: Exception) -> bool:
+        _append(manifest, {"unit": u.uid, "status": "failed", "rank": rank,
+                           "error": f"{type(e).__name__}: {e}"})
+        if log:
+            log(f"rank {rank}: {u.uid} failed: {e}")
+        return False
+
+    with ThreadPoolExecutor(max_workers=1) as writer:
+        for u in mine:
+            if u.uid in done:
+                skipped += 1
+                continue
+            t0 = time.time()
+            try:
+                arrays = runner(u)
+            except Exception as e:
+                writes.append(writer.submit(write_failed, u, e))
+                continue
+            writes.append(writer.submit(write_ok, u, arrays, time.time() - t0))
+        ok = [f.result() for f in writes]
+    ran = sum(ok)
     return {"rank": rank, "world": world, "assigned": len(mine), "ran": ran,
-            "skipped": skipped, "failed": failed, "seconds": time.time() - t_all,
+            "skipped": skipped, "failed": len(ok) - ran, "seconds": time.time() - t_all,
             "weights": int(sum(u.weights for u in mine))}
 
 
