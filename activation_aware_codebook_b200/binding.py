@@ -33,7 +33,7 @@ EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaa
            "aaac_fit_layer_fixed_scratch", "aaac_dequant", "aaac_linear",
            "aaac_device_timeouts", "aaac_awq_prescale", "aaac_awq_workspace_size",
            "aaac_awq_fit", "aaac_init_codebooks_sharded", "aaac_fit_layer_sharded",
-           "aaac_pack_sharded")
+           "aaac_pack_sharded", "aaac_linear_workspace_size", "aaac_linear_ws")
 
 
 # reduction callback of the row-sharded calls: (user, buf, count, op, stream) -> 0 | error
@@ -132,6 +132,10 @@ def load(path: str = LIB_PATH):
     L.aaac_awq_fit.restype = ctypes.c_int
     L.aaac_awq_fit.argtypes = [P, i64, i64, P, i64, P, P, ctypes.c_int, P, P, P, P, P, P, P, P,
                                P, sz, P]
+    L.aaac_linear_workspace_size.restype = sz
+    L.aaac_linear_workspace_size.argtypes = [P, i64, i64, i64]
+    L.aaac_linear_ws.restype = ctypes.c_int
+    L.aaac_linear_ws.argtypes = [P, i64, i64, P, P, P, P, i64, i64, P, P, P, sz, P]
     R = REDUCE_FN
     L.aaac_init_codebooks_sharded.restype = ctypes.c_int
     L.aaac_init_codebooks_sharded.argtypes = [P, i64, i64, i64, P, P, P, R, P, P, sz, P]
@@ -322,9 +326,19 @@ def dequant(packed: dict, cfg: Config, N: int, K: int, out: Optional[torch.Tenso
     return out
 
 
+def linear_workspace_size(cfg: Config, M: int, N: int, K: int) -> int:
+    """Bytes of the workspace that lets linear() dequantise once (0 when the
+    fused kernels are used for this token count)."""
+    c = cfg.c()
+    return int(load().aaac_linear_workspace_size(ctypes.byref(c), M, N, K))
+
+
 def linear(X: torch.Tensor, packed: dict, cfg: Config, N: int, K: int,
-           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """W4A16 linear on a packed layer: Y[M, N] = X[M, K] @ W_hat^T, fp32."""
+           out: Optional[torch.Tensor] = None, stream=None,
+           ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """W4A16 linear on a packed layer: Y[M, N] = X[M, K] @ W_hat^T, fp32.
+    With a workspace (linear_workspace_size bytes) large token counts
+    dequantise W once and use the TMA-fed tensor-core GEMM."""
     _need_cuda()
     assert X.dtype in (torch.bfloat16, torch.int16, torch.uint16), X.dtype
     if X.stride(1) != 1 or X.stride(0) % 8:
@@ -333,6 +347,13 @@ def linear(X: torch.Tensor, packed: dict, cfg: Config, N: int, K: int,
     if out is None:
         out = torch.empty(M, N, dtype=torch.float32, device=X.device)
     c = cfg.c()
+    if ws is not None:
+        _check(load().aaac_linear_ws(_ptr(X), M, ldx, _ptr(packed["codes"]),
+                                     _ptr(packed["scales_tagged"]),
+                                     _ptr(packed.get("choice_bits")), _ptr(packed["T_bf16"]), N,
+                                     K, ctypes.byref(c), _ptr(out), _ptr(ws), ws.numel(),
+                                     _stream(stream)))
+        return out
     _check(load().aaac_linear(_ptr(X), M, ldx, _ptr(packed["codes"]),
                               _ptr(packed["scales_tagged"]), _ptr(packed.get("choice_bits")),
                               _ptr(packed["T_bf16"]), N, K, ctypes.byref(c), _ptr(out),

@@ -471,6 +471,48 @@ aaac_status aaac_pack_sharded(const void* W, int64_t N, int64_t K, int64_t N_tot
   return from_cuda(e, "aaac_pack_sharded");
 }
 
+// Token counts from which aaac_linear_ws dequantises W once into its
+// workspace and runs the TMA-fed GEMM (below it the fused kernels are faster).
+static const int64_t kDequantMinM = 512;
+
+size_t aaac_linear_workspace_size(const aaac_config* cfg, int64_t M, int64_t N, int64_t K) {
+  if (!cfg || M < kDequantMinM || N <= 0 || K <= 0) return 0;
+  return aaac::align256((size_t)N * (size_t)K * 2);
+}
+
+aaac_status aaac_linear_ws(const void* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                           const void* scales_tagged, const uint8_t* choice_bits,
+                           const uint16_t* T_bf16, int64_t N, int64_t K, const aaac_config* cfg,
+                           float* Y, void* ws, size_t ws_bytes, void* stream) {
+  const size_t need = aaac_linear_workspace_size(cfg, M, N, K);
+  if (need == 0 || !ws || ws_bytes < need || !aligned16(ws))
+    return aaac_linear(X, M, ldx, codes, scales_tagged, choice_bits, T_bf16, N, K, cfg, Y, stream);
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  if (M > ((int64_t)1 << 20))
+    return fail(AAAC_ERR_SHAPE, "M=%lld must be in [1, 2^20]", (long long)M);
+  if (ldx < K) return fail(AAAC_ERR_SHAPE, "ldx=%lld < K=%lld", (long long)ldx, (long long)K);
+  if (ldx % 8) return fail(AAAC_ERR_ALIGN, "ldx=%lld is not a multiple of 8", (long long)ldx);
+  if (M * ldx >= ((int64_t)1 << 40))
+    return fail(AAAC_ERR_SHAPE, "M*ldx is too large (M=%lld ldx=%lld)", (long long)M,
+                (long long)ldx);
+  CHECK(check_ptr(X, "X"));
+  CHECK(check_ptr(codes, "codes"));
+  CHECK(check_ptr(scales_tagged, "scales_tagged"));
+  CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
+  CHECK(check_ptr(T_bf16, "T_bf16"));
+  CHECK(check_ptr(Y, "Y"));
+  uint16_t* Wh = static_cast<uint16_t*>(ws);
+  cudaError_t e = aaac::launch_dequant(codes, scales_tagged, choice_bits, T_bf16, N, K, cfg->fmt,
+                                       cfg->g, cfg->S, Wh, cfg->global_scale,
+                                       (cudaStream_t)stream);
+  if (e == cudaSuccess)
+    e = aaac::launch_gemm_dequantised(reinterpret_cast<const uint16_t*>(X), M, ldx, Wh, N, K, Y,
+                                      (cudaStream_t)stream);
+  if (e == cudaSuccess) aaac::count_launches(1);
+  return from_cuda(e, "aaac_linear_ws");
+}
+
 aaac_status aaac_device_timeouts(uint32_t* flag) {
   if (!flag) return fail(AAAC_ERR_INVALID_ARG, "flag is NULL");
   unsigned int v = 0;

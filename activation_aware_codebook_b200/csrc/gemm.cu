@@ -436,6 +436,122 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Large token counts: W_hat dequantised once into the caller's workspace
+// (aaac_dequant's kernel), then a plain bf16 x bf16 tcgen05 GEMM with both
+// operands brought in by TMA.  The fused kernel above expands W again for
+// every token tile; here the expansion is paid once, and the producer warps
+// are free for the epilogue.
+//   warp 0      one lane issues the TMA loads of the W_hat tile (128 rows x 64)
+//               and the X tile (BT x 64) of each stage, no multicast;
+//   warp 1      TMEM allocation and MMA issue, as in gemm_kernel;
+//   warps 2..9  epilogue, as in gemm_kernel.
+// ---------------------------------------------------------------------------
+constexpr int kStagesT = 4;
+
+template <int BT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
+                GemmArgs a) {
+  extern __shared__ __align__(1024) unsigned char gsm[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(gsm) + 1023) & ~(uintptr_t)1023);
+  unsigned char* sA = base;                                   // kStagesT x 16 KB
+  unsigned char* sB = base + kStagesT * kATileBytes;          // kStagesT x BT*128
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStagesT * BT * 128);
+  uint64_t* empty = full + kStagesT;
+  uint64_t* accum = empty + kStagesT;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  __shared__ int s_fail;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBN, t0 = blockIdx.y * BT;
+  const int nkb_all = (a.K + kBK - 1) / kBK;
+  const int kb_lo = a.split == 2 ? (blockIdx.z ? (nkb_all + 1) / 2 : 0) : 0;
+  const int nkb = a.split == 2 ? (blockIdx.z ? nkb_all - kb_lo : (nkb_all + 1) / 2) : nkb_all;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStagesT; s++) {
+      mbar_init(&full[s], 1);   // the TMA thread's expect_tx
+      mbar_init(&empty[s], 1);  // MMA commit
+    }
+    mbar_init(accum, 1);
+    s_fail = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(BT));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {  // W_hat and X tiles by TMA
+      int issued = 0;
+      for (int kb = 0; kb < nkb; kb++) {
+        const int s = kb % kStagesT;
+        const uint32_t wrap = kb / kStagesT;
+        if (kb >= kStagesT && !mbar_wait(&empty[s], (wrap - 1) & 1)) { s_fail = 1; break; }
+        mbar_arrive_expect_tx(&full[s], kATileBytes + BT * 128);
+        const int k = (kb_lo + kb) * kBK;
+        tma_load_2d(sA + s * kATileBytes, &wmap, &full[s], k, n0);
+        tma_load_2d(sB + s * BT * 128, &xmap, &full[s], k, t0);
+        issued = kb + 1;
+      }
+      for (int kb = issued > kStagesT ? issued - kStagesT : 0; kb < issued; kb++)
+        if (!mbar_wait(&full[kb % kStagesT], (kb / kStagesT) & 1)) { s_fail = 1; break; }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issue
+      const uint32_t idesc = mma_idesc(kBN, BT);
+      for (int kb = 0; kb < nkb; kb++) {
+        const int s = kb % kStagesT;
+        if (!mbar_wait(&full[s], (kb / kStagesT) & 1)) { s_fail = 1; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * kATileBytes), b0 = smem_u32(sB + s * BT * 128);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; k++)
+          mma_bf16(tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
+                   (kb > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accum);
+    }
+  } else {
+    const bool got = __all_sync(0xffffffffu, mbar_wait(accum, 0));
+    tc_fence_after();
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int nrow = n0 + q * 32 + lane;
+    const bool fail = !got || s_fail;
+    for (int j0 = half * (BT / 2); j0 < (half + 1) * (BT / 2); j0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)j0, r);
+#pragma unroll
+      for (int j = 0; j < 32; j++) {
+        const int t = t0 + j0 + j;
+        if (nrow < a.N && t < a.M) {
+          float* y = a.Y + (int64_t)t * a.N + nrow;
+          const float v = fail ? __int_as_float(0x7fc00000) : __uint_as_float(r[j]);
+          if (a.split == 2) atomicAdd(y, v);
+          else *y = v;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BT));
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host: tensor map for X through the driver entry point (no link to libcuda)
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -496,6 +612,53 @@ cudaError_t launch_gemm_t(const uint16_t* X, int64_t M, int64_t ldx, const GemmA
   return cudaGetLastError();
 }
 
+template <int BT>
+size_t gemm_tma_smem() {
+  return 1024 + (size_t)kStagesT * (kATileBytes + BT * 128) + (2 * kStagesT + 1) * 8 + 16;
+}
+
+template <int BT>
+cudaError_t launch_gemm_tma_t(const uint16_t* X, int64_t M, int64_t ldx, const uint16_t* Wh,
+                              const GemmArgs& ga, cudaStream_t st) {
+  EncodeTiledFn enc;
+  cudaError_t e = encode_fn(&enc);
+  if (e != cudaSuccess) return e;
+  CUtensorMap xmap, wmap;
+  const cuuint32_t estr[2] = {1, 1};
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)ga.K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BT};
+    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)ga.K, (cuuint64_t)ga.N};
+    const cuuint64_t strides[1] = {(cuuint64_t)ga.K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBN};
+    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(Wh), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const size_t smem = gemm_tma_smem<BT>();
+  e = cudaFuncSetAttribute(gemm_tma_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned nblk = (unsigned)((ga.N + kBN - 1) / kBN), tblk = (unsigned)((M + BT - 1) / BT);
+  GemmArgs g2 = ga;
+  g2.split = ((int64_t)nblk * tblk < 148 && ga.K > kBK) ? 2 : 1;
+  if (g2.split == 2) {
+    e = cudaMemsetAsync(ga.Y, 0, (size_t)M * (size_t)ga.N * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+  }
+  const dim3 grid(nblk, tblk, (unsigned)g2.split);
+  gemm_tma_kernel<BT><<<grid, kGemmThreads, smem, st>>>(xmap, wmap, g2);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
@@ -519,6 +682,16 @@ cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
   return bt == 64 ? launch_gemm_t<kNvfp4G, 64>(X, M, ldx, ga, st)
        : bt == 128 ? launch_gemm_t<kNvfp4G, 128>(X, M, ldx, ga, st)
                    : launch_gemm_t<kNvfp4G, 256>(X, M, ldx, ga, st);
+}
+
+cudaError_t launch_gemm_dequantised(const uint16_t* X, int64_t M, int64_t ldx,
+                                    const uint16_t* Wh, int64_t N, int64_t K, float* Y,
+                                    cudaStream_t st) {
+  GemmArgs ga{nullptr, nullptr, nullptr, nullptr, Y, (int)M, (int)N, (int)K, 0, 0, 1, nullptr};
+  const int bt = M <= 64 ? 64 : (M < 512 ? 128 : 256);
+  return bt == 64 ? launch_gemm_tma_t<64>(X, M, ldx, Wh, ga, st)
+       : bt == 128 ? launch_gemm_tma_t<128>(X, M, ldx, Wh, ga, st)
+                   : launch_gemm_tma_t<256>(X, M, ldx, Wh, ga, st);
 }
 
 cudaError_t gemm_timeout_flag(unsigned int* out) {

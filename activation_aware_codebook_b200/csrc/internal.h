@@ -100,6 +100,10 @@ cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
                         const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
                         int64_t K, int fmt, int lg, int ls, float* Y, const float* gsc,
                         cudaStream_t st);
+// Y = X W_hat^T from an already dequantised bf16 W_hat [N][K] (both operands by TMA)
+cudaError_t launch_gemm_dequantised(const uint16_t* X, int64_t M, int64_t ldx,
+                                    const uint16_t* Wh, int64_t N, int64_t K, float* Y,
+                                    cudaStream_t st);
 cudaError_t gemm_timeout_flag(unsigned int* out);
 
 cudaError_t launch_awq_prescale(const uint16_t* W, int64_t N, int64_t K, const float* I,

@@ -739,14 +739,16 @@ def run_linear(args):
         x = synth.make_activations(M, K, 93 + M, True, device=dev)
         Y = torch.empty(M, N, dtype=torch.float32, device=dev)
         st = torch.cuda.current_stream()
+        need = bb.linear_workspace_size(cfg, M, N, K)
+        lws = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
         for _ in range(args.warmup):
-            bb.linear(x, packed, cfg, N, K, out=Y)
+            bb.linear(x, packed, cfg, N, K, out=Y, ws=lws)
         times = []
         for _ in range(args.steps):
             flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(st)
-            bb.linear(x, packed, cfg, N, K, out=Y)
+            bb.linear(x, packed, cfg, N, K, out=Y, ws=lws)
             e1.record(st)
             torch.cuda.synchronize()
             times.append(e0.elapsed_time(e1))
@@ -761,7 +763,8 @@ def run_linear(args):
                     "peak_kind": tf_kind, "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
         points.append({"tokens": M, "us": ms * 1e3, "tokens_per_s": M / (ms * 1e-3),
-                       "path": "gemv" if M <= 4 else "tcgen05", "roofline": roof})
+                       "path": ("gemv" if M <= 4 else "tcgen05 fused expansion" if not need
+                                else "dequant + TMA-fed tcgen05"), "roofline": roof})
     clocks = sampler.stop()
     launches = bb.kernel_launches() - launches0
     head = points[0]

@@ -312,6 +312,19 @@ aaac_status aaac_pack_sharded(const void* W, int64_t N, int64_t K, int64_t N_tot
                               aaac_reduce_fn reduce, void* user, void* ws, size_t ws_bytes,
                               void* stream);
 
+/* aaac_linear with a workspace.  From a token count the library chooses
+ * (aaac_linear_workspace_size returns 0 below it), the layer is dequantised
+ * once into the workspace (as aaac_dequant) and Y = X W_hat^T runs as a bf16
+ * tcgen05 GEMM with both operands fed by TMA; the fused kernels instead
+ * expand W again for every token tile.  Same contract and accuracy bound as
+ * aaac_linear; with a NULL or too small workspace it is aaac_linear.
+ *   ws   device, aaac_linear_workspace_size(cfg, M, N, K) bytes (N*K bf16) */
+size_t aaac_linear_workspace_size(const aaac_config* cfg, int64_t M, int64_t N, int64_t K);
+aaac_status aaac_linear_ws(const void* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                           const void* scales_tagged, const uint8_t* choice_bits,
+                           const uint16_t* T_bf16, int64_t N, int64_t K, const aaac_config* cfg,
+                           float* Y, void* ws, size_t ws_bytes, void* stream);
+
 /* Device-side wait status of the current device: *flag = 1 when a bounded
  * wait inside one of the library's kernels (the tensor-core aaac_linear path)
  * has run out since the library was loaded, else 0.  A kernel whose wait ran

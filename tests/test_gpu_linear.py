@@ -146,3 +146,31 @@ def test_linear_tensor_core_many_tiles():
     Wh = oracle.dequant_bf16(host["codes"], host["scales_tagged"], host["choice_bits"],
                              host["T_bf16"], N, K, oracle.INT4, 128, 16)
     check_linear(Y, u16(X), Wh)
+
+
+@pytest.mark.parametrize("fmt,g,S,N,K", GEMM_CASES)
+@pytest.mark.parametrize("M", [512, 700])
+def test_linear_dequantised_path(fmt, g, S, N, K, M):
+    """From 512 tokens, aaac_linear_ws dequantises W once into its workspace
+    and runs the TMA-fed tcgen05 GEMM: partial weight-row and token tiles and
+    a K tail inside the last 64-wide block (K = 208, 96) come from the tensor
+    maps' zero fill.  Within the same bound as the fused kernels."""
+    host, dev = packed_layer(N, K, fmt, g, S, seed=M + N + 1)
+    cfg = dev["cfg"]
+    need = bb.linear_workspace_size(cfg, M, N, K)
+    assert need >= N * K * 2
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    X = synth.make_activations(M, K, seed=300 + M, heavy=True).cuda()
+    Y = bb.linear(X, dev, cfg, N, K, ws=ws)
+    torch.cuda.synchronize()
+    assert bb.device_timeouts() == 0
+    check_linear(Y, u16(X), ref_dequant(host, N, K, fmt, g, S))
+    # the workspace holds the dequantised weights, bit-exact
+    assert np.array_equal(u16(ws[:N * K * 2].view(torch.int16).view(N, K)),
+                          ref_dequant(host, N, K, fmt, g, S))
+
+
+def test_linear_workspace_size_threshold():
+    cfg = bb.Config(bb.INT4, 128, 16, 0)
+    assert bb.linear_workspace_size(cfg, 511, 256, 512) == 0
+    assert bb.linear_workspace_size(cfg, 512, 256, 512) >= 256 * 512 * 2
