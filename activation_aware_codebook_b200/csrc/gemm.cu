@@ -437,51 +437,57 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
 
 // ---------------------------------------------------------------------------
 // Large token counts: W_hat dequantised once into the caller's workspace
-// (aaac_dequant's kernel), then a plain bf16 x bf16 tcgen05 GEMM with both
-// operands brought in by TMA.  The fused kernel above expands W again for
-// every token tile; here the expansion is paid once, and the producer warps
-// are free for the epilogue.
+// (aaac_dequant's kernel), then a persistent bf16 x bf16 tcgen05 GEMM with
+// both operands brought in by TMA.  The fused kernel above expands W again
+// for every token tile; here the expansion is paid once.
+//   one CTA per SM walks the 128 x 256 output tiles t = blockIdx.x, +grid, ...
+//   (weight-row tile major, so the CTAs in flight share their W rows in L2);
 //   warp 0      one lane issues the TMA loads of the W_hat tile (128 rows x 64)
-//               and the X tile (BT x 64) of each stage, no multicast;
-//   warp 1      TMEM allocation and MMA issue, as in gemm_kernel;
-//   warps 2..9  epilogue, as in gemm_kernel.
+//               and the X tile (256 x 64) of every stage, no multicast;
+//   warp 1      allocates all 512 TMEM columns: two 256-column accumulators,
+//               tiles alternating between them; one lane issues the MMAs and
+//               commits each tile's accumulator to acc_full[b];
+//   warps 2..9  epilogue of tile i from accumulator i & 1 while the MMAs of
+//               tile i + 1 run in the other one; acc_empty[b] hands it back.
+// Waits are bounded as in gemm_kernel.
 // ---------------------------------------------------------------------------
 constexpr int kStagesT = 4;
+constexpr int kBTT = 256;  // tokens per tile
 
-template <int BT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
-                GemmArgs a) {
+                GemmArgs a, int tiles_t, int tiles) {
   extern __shared__ __align__(1024) unsigned char gsm[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(gsm) + 1023) & ~(uintptr_t)1023);
   unsigned char* sA = base;                                   // kStagesT x 16 KB
-  unsigned char* sB = base + kStagesT * kATileBytes;          // kStagesT x BT*128
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStagesT * BT * 128);
+  unsigned char* sB = base + kStagesT * kATileBytes;          // kStagesT x 32 KB
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStagesT * kBTT * 128);
   uint64_t* empty = full + kStagesT;
-  uint64_t* accum = empty + kStagesT;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  uint64_t* acc_full = empty + kStagesT;   // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   __shared__ int s_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kBN, t0 = blockIdx.y * BT;
-  const int nkb_all = (a.K + kBK - 1) / kBK;
-  const int kb_lo = a.split == 2 ? (blockIdx.z ? (nkb_all + 1) / 2 : 0) : 0;
-  const int nkb = a.split == 2 ? (blockIdx.z ? nkb_all - kb_lo : (nkb_all + 1) / 2) : nkb_all;
+  const int nkb = (a.K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesT; s++) {
       mbar_init(&full[s], 1);   // the TMA thread's expect_tx
       mbar_init(&empty[s], 1);  // MMA commit
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < 2; b++) {
+      mbar_init(&acc_full[b], 1);           // MMA commit of a tile
+      mbar_init(&acc_empty[b], kProdWarps);  // one arrive per epilogue warp
+    }
     s_fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(BT));
+                 "r"(2 * kBTT));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -490,64 +496,84 @@ gemm_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {  // W_hat and X tiles by TMA
-      int issued = 0;
-      for (int kb = 0; kb < nkb; kb++) {
-        const int s = kb % kStagesT;
-        const uint32_t wrap = kb / kStagesT;
-        if (kb >= kStagesT && !mbar_wait(&empty[s], (wrap - 1) & 1)) { s_fail = 1; break; }
-        mbar_arrive_expect_tx(&full[s], kATileBytes + BT * 128);
-        const int k = (kb_lo + kb) * kBK;
-        tma_load_2d(sA + s * kATileBytes, &wmap, &full[s], k, n0);
-        tma_load_2d(sB + s * BT * 128, &xmap, &full[s], k, t0);
-        issued = kb + 1;
+    if (lane == 0) {  // W_hat and X tiles by TMA, stage after stage across the tiles
+      int it = 0;     // stage uses so far
+      for (int tile = blockIdx.x; tile < tiles && !s_fail; tile += gridDim.x) {
+        const int n0 = (tile / tiles_t) * kBN, t0 = (tile % tiles_t) * kBTT;
+        for (int kb = 0; kb < nkb; kb++, it++) {
+          const int s = it % kStagesT;
+          if (it >= kStagesT && !mbar_wait(&empty[s], ((it / kStagesT) - 1) & 1)) {
+            s_fail = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kATileBytes + kBTT * 128);
+          tma_load_2d(sA + s * kATileBytes, &wmap, &full[s], kb * kBK, n0);
+          tma_load_2d(sB + s * kBTT * 128, &xmap, &full[s], kb * kBK, t0);
+        }
       }
-      for (int kb = issued > kStagesT ? issued - kStagesT : 0; kb < issued; kb++)
-        if (!mbar_wait(&full[kb % kStagesT], (kb / kStagesT) & 1)) { s_fail = 1; break; }
+      // the last copies have landed before the CTA can exit (bounded)
+      for (int j = it > kStagesT ? it - kStagesT : 0; j < it; j++)
+        if (!mbar_wait(&full[j % kStagesT], (j / kStagesT) & 1)) { s_fail = 1; break; }
     }
   } else if (warp == 1) {
     if (lane == 0) {  // MMA issue
-      const uint32_t idesc = mma_idesc(kBN, BT);
-      for (int kb = 0; kb < nkb; kb++) {
-        const int s = kb % kStagesT;
-        if (!mbar_wait(&full[s], (kb / kStagesT) & 1)) { s_fail = 1; break; }
+      const uint32_t idesc = mma_idesc(kBN, kBTT);
+      int it = 0, i = 0;
+      for (int tile = blockIdx.x; tile < tiles && !s_fail; tile += gridDim.x, i++) {
+        const int b = i & 1;
+        // the accumulator's previous tile (i - 2) has been read out
+        if (i >= 2 && !mbar_wait(&acc_empty[b], ((i >> 1) - 1) & 1)) { s_fail = 1; break; }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * kATileBytes), b0 = smem_u32(sB + s * BT * 128);
+        const uint32_t d = tmem + (uint32_t)(b * kBTT);
+        bool ok = true;
+        for (int kb = 0; kb < nkb; kb++, it++) {
+          const int s = it % kStagesT;
+          if (!mbar_wait(&full[s], (it / kStagesT) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kATileBytes), b0 = smem_u32(sB + s * kBTT * 128);
 #pragma unroll
-        for (int k = 0; k < kBK / 16; k++)
-          mma_bf16(tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
-                   (kb > 0 || k > 0) ? 1u : 0u);
-        mma_commit(&empty[s]);
+          for (int k = 0; k < kBK / 16; k++)
+            mma_bf16(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
+                     (kb > 0 || k > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);
+        }
+        if (!ok) { s_fail = 1; break; }
+        mma_commit(&acc_full[b]);
       }
-      mma_commit(accum);
     }
   } else {
-    const bool got = __all_sync(0xffffffffu, mbar_wait(accum, 0));
-    tc_fence_after();
-    const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int nrow = n0 + q * 32 + lane;
-    const bool fail = !got || s_fail;
-    for (int j0 = half * (BT / 2); j0 < (half + 1) * (BT / 2); j0 += 32) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)j0, r);
+    const int q = warp & 3;               // TMEM lane quadrant this warp may read
+    const int half = (warp - 2) >> 2;     // which half of the token columns
+    int i = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, i++) {
+      const int b = i & 1;
+      const int n0 = (tile / tiles_t) * kBN, t0 = (tile % tiles_t) * kBTT;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], (i >> 1) & 1));
+      tc_fence_after();
+      const bool fail = !got || s_fail;
+      const int nrow = n0 + q * 32 + lane;
+      for (int j0 = half * (kBTT / 2); j0 < (half + 1) * (kBTT / 2); j0 += 32) {
+        uint32_t r[32];
+        if (!fail) tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kBTT + j0), r);
 #pragma unroll
-      for (int j = 0; j < 32; j++) {
-        const int t = t0 + j0 + j;
-        if (nrow < a.N && t < a.M) {
-          float* y = a.Y + (int64_t)t * a.N + nrow;
-          const float v = fail ? __int_as_float(0x7fc00000) : __uint_as_float(r[j]);
-          if (a.split == 2) atomicAdd(y, v);
-          else *y = v;
+        for (int j = 0; j < 32; j++) {
+          const int t = t0 + j0 + j;
+          if (nrow < a.N && t < a.M)
+            a.Y[(int64_t)t * a.N + nrow] = fail ? __int_as_float(0x7fc00000) : __uint_as_float(r[j]);
         }
       }
+      if (fail) break;  // the MMA warp stopped; nothing more to read
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BT));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(2 * kBTT));
   }
 }
 
@@ -612,14 +638,12 @@ cudaError_t launch_gemm_t(const uint16_t* X, int64_t M, int64_t ldx, const GemmA
   return cudaGetLastError();
 }
 
-template <int BT>
 size_t gemm_tma_smem() {
-  return 1024 + (size_t)kStagesT * (kATileBytes + BT * 128) + (2 * kStagesT + 1) * 8 + 16;
+  return 1024 + (size_t)kStagesT * (kATileBytes + kBTT * 128) + (2 * kStagesT + 4) * 8 + 16;
 }
 
-template <int BT>
-cudaError_t launch_gemm_tma_t(const uint16_t* X, int64_t M, int64_t ldx, const uint16_t* Wh,
-                              const GemmArgs& ga, cudaStream_t st) {
+cudaError_t launch_gemm_tma(const uint16_t* X, int64_t M, int64_t ldx, const uint16_t* Wh,
+                            const GemmArgs& ga, cudaStream_t st) {
   EncodeTiledFn enc;
   cudaError_t e = encode_fn(&enc);
   if (e != cudaSuccess) return e;
@@ -628,7 +652,7 @@ cudaError_t launch_gemm_tma_t(const uint16_t* X, int64_t M, int64_t ldx, const u
   {
     const cuuint64_t dims[2] = {(cuuint64_t)ga.K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BT};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBTT};
     if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -643,19 +667,13 @@ cudaError_t launch_gemm_tma_t(const uint16_t* X, int64_t M, int64_t ldx, const u
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const size_t smem = gemm_tma_smem<BT>();
-  e = cudaFuncSetAttribute(gemm_tma_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
+  const size_t smem = gemm_tma_smem();
+  e = cudaFuncSetAttribute(gemm_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const unsigned nblk = (unsigned)((ga.N + kBN - 1) / kBN), tblk = (unsigned)((M + BT - 1) / BT);
-  GemmArgs g2 = ga;
-  g2.split = ((int64_t)nblk * tblk < 148 && ga.K > kBK) ? 2 : 1;
-  if (g2.split == 2) {
-    e = cudaMemsetAsync(ga.Y, 0, (size_t)M * (size_t)ga.N * sizeof(float), st);
-    if (e != cudaSuccess) return e;
-  }
-  const dim3 grid(nblk, tblk, (unsigned)g2.split);
-  gemm_tma_kernel<BT><<<grid, kGemmThreads, smem, st>>>(xmap, wmap, g2);
+  const int tiles_n = (int)((ga.N + kBN - 1) / kBN), tiles_t = (int)((M + kBTT - 1) / kBTT);
+  const int tiles = tiles_n * tiles_t;
+  const int grid = tiles < 148 ? tiles : 148;
+  gemm_tma_kernel<<<grid, kGemmThreads, smem, st>>>(xmap, wmap, ga, tiles_t, tiles);
   return cudaGetLastError();
 }
 
@@ -687,11 +705,9 @@ cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
 cudaError_t launch_gemm_dequantised(const uint16_t* X, int64_t M, int64_t ldx,
                                     const uint16_t* Wh, int64_t N, int64_t K, float* Y,
                                     cudaStream_t st) {
-  GemmArgs ga{nullptr, nullptr, nullptr, nullptr, Y, (int)M, (int)N, (int)K, 0, 0, 1, nullptr};
-  const int bt = M <= 64 ? 64 : (M < 512 ? 128 : 256);
-  return bt == 64 ? launch_gemm_tma_t<64>(X, M, ldx, Wh, ga, st)
-       : bt == 128 ? launch_gemm_tma_t<128>(X, M, ldx, Wh, ga, st)
-                   : launch_gemm_tma_t<256>(X, M, ldx, Wh, ga, st);
+  const GemmArgs ga{nullptr, nullptr, nullptr, nullptr, Y, (int)M, (int)N, (int)K, 0, 0, 1,
+                     nullptr};
+  return launch_gemm_tma(X, M, ldx, Wh, ga, st);
 }
 
 cudaError_t gemm_timeout_flag(unsigned int* out) {
