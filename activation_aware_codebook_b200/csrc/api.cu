@@ -473,7 +473,7 @@ aaac_status aaac_pack_sharded(const void* W, int64_t N, int64_t K, int64_t N_tot
 
 // Token counts from which aaac_linear_ws dequantises W once into its
 // workspace and runs the TMA-fed GEMM (below it the fused kernels are faster).
-static const int64_t kDequantMinM = 512;
+static const int64_t kDequantMinM = 192;
 
 size_t aaac_linear_workspace_size(const aaac_config* cfg, int64_t M, int64_t N, int64_t K) {
   if (!cfg || M < kDequantMinM || N <= 0 || K <= 0) return 0;

@@ -149,9 +149,9 @@ def test_linear_tensor_core_many_tiles():
 
 
 @pytest.mark.parametrize("fmt,g,S,N,K", GEMM_CASES)
-@pytest.mark.parametrize("M", [512, 700])
+@pytest.mark.parametrize("M", [192, 700])
 def test_linear_dequantised_path(fmt, g, S, N, K, M):
-    """From 512 tokens, aaac_linear_ws dequantises W once into its workspace
+    """From 192 tokens, aaac_linear_ws dequantises W once into its workspace
     and runs the TMA-fed tcgen05 GEMM: partial weight-row and token tiles and
     a K tail inside the last 64-wide block (K = 208, 96) come from the tensor
     maps' zero fill.  Within the same bound as the fused kernels."""
@@ -172,5 +172,5 @@ def test_linear_dequantised_path(fmt, g, S, N, K, M):
 
 def test_linear_workspace_size_threshold():
     cfg = bb.Config(bb.INT4, 128, 16, 0)
-    assert bb.linear_workspace_size(cfg, 511, 256, 512) == 0
-    assert bb.linear_workspace_size(cfg, 512, 256, 512) >= 256 * 512 * 2
+    assert bb.linear_workspace_size(cfg, 191, 256, 512) == 0
+    assert bb.linear_workspace_size(cfg, 192, 256, 512) >= 256 * 512 * 2
