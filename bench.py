@@ -405,9 +405,21 @@ def run_ours(args, rank, local_rank, world):
     achieved = bytes_per_iter / (iter_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     traffic = None
+    issue = None
     tr = committed_traffic(source_hash("fit.cu", "common.cuh"))
     if tr is not None and tr.get("N") and tr.get("K"):
-        traffic = tr["dram_bytes_per_launch"] * (probe.N * probe.K) / (tr["N"] * tr["K"])
+        scale = (probe.N * probe.K) / (tr["N"] * tr["K"])
+        traffic = tr["dram_bytes_per_launch"] * scale
+        if tr.get("warp_instructions_per_launch"):
+            # what actually bounds the pass: instruction issue, against one
+            # warp instruction per scheduler per cycle (148 SMs x 4 at the
+            # sampled SM clock)
+            inst = tr["warp_instructions_per_launch"] * scale
+            peak_issue = 148 * 4 * (clocks.get("sm_mhz") or 1965.0) * 1e6
+            issue = {"warp_instructions_per_launch": inst,
+                     "achieved_per_s": inst / (iter_ms * 1e-3), "peak_per_s": peak_issue,
+                     "frac": inst / (iter_ms * 1e-3) / peak_issue,
+                     "source": "warp instructions from the committed ncu capture"}
 
     # end to end through the C ABI with host buffers (pinned), copies timed
     e2e = None
@@ -439,7 +451,7 @@ def run_ours(args, rank, local_rank, world):
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "bytes_per_launch": bytes_per_iter,
                          "round_ms": iter_ms, "timing": "the probe's fit alone, CUDA events",
-                         "round_ms_in_step": iter_in_step_ms},
+                         "round_ms_in_step": iter_in_step_ms, "issue": issue},
             "gpu_launches": int(launches),
             "clocks": clocks,
         }
