@@ -730,12 +730,15 @@ __device__ __forceinline__ void count_group(GroupStats& gs, bool exact, double E
   gs.t1 += ch;
 }
 
-template <int FMT, bool PACK>
+// SC: the selection group size when it is 8 or 16 (the common layouts,
+// compiled with S known), or 0 for S >= 32 taken from S_rt.
+template <int FMT, bool PACK, int SC>
 __global__ void __launch_bounds__(kFitThreads, kFitBlocksPerSM)
 fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
-         const void* __restrict__ scales, int g, int S, uint32_t flags, FitCtl* ctl,
+         const void* __restrict__ scales, int g, int S_rt, uint32_t flags, FitCtl* ctl,
          int cpc, int n_items, int max_items, float tau, PackOut po,
          RoundOut ro, const float* __restrict__ gsc, int finalize) {
+  const int S = SC ? SC : S_rt;
   extern __shared__ __align__(128) unsigned char smem[];
   Tables& tb = *reinterpret_cast<Tables*>(smem);
   unsigned char* ring = smem + kTablesBytes;
@@ -1240,9 +1243,18 @@ static float choice_tau(int S) {
   return (float)((12 + lg) * ldexp(1.0, -22));
 }
 
+// The fit pass compiled for this selection group size, with its shared
+// memory attribute set (per call: the attribute belongs to the current
+// device's copy of the kernel).
+using FitPassFn = void (*)(const uint16_t*, int, int, const float*, const void*, int, int,
+                           uint32_t, FitCtl*, int, int, int, float, PackOut, RoundOut,
+                           const float*, int);
 template <int FMT, bool PACK>
-static cudaError_t set_smem() {
-  return cudaFuncSetAttribute(fit_pass<FMT, PACK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+static cudaError_t fit_kernel(int S, FitPassFn* out) {
+  const FitPassFn k = S == 8 ? fit_pass<FMT, PACK, 8>
+                    : S == 16 ? fit_pass<FMT, PACK, 16> : fit_pass<FMT, PACK, 0>;
+  *out = k;
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)smem_bytes(PACK));
 }
 
@@ -1252,7 +1264,8 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
                                 float* T, double* err_hist, aaac_stats* stats, void* ws,
                                 const float* gsc, cudaStream_t st) {
   // per call: the attribute belongs to the current device's copy of the kernel
-  const cudaError_t attr = set_smem<FMT, false>();
+  FitPassFn kern;
+  const cudaError_t attr = fit_kernel<FMT, false>(S, &kern);
   if (attr != cudaSuccess) return attr;
   const FitPlan pp = fit_plan(N, K, N * K);
   const PassPlan pprep = plan_pass(N, K);
@@ -1278,7 +1291,7 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
   lc.numAttrs = 1;
   for (int it = 0; it < iters; it++) {
     const cudaError_t e = cudaLaunchKernelEx(
-        &lc, fit_pass<FMT, false>, W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items,
+        &lc, kern, W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items,
         pp.max_items, tau, PackOut{nullptr, nullptr, nullptr, nullptr},
         RoundOut{err_hist, T, stats, it}, gsc, 1);
     if (e != cudaSuccess) return e;
@@ -1314,7 +1327,8 @@ static cudaError_t launch_fit_sharded_t(const uint16_t* W, int64_t N, int64_t K,
                                         int iters, uint32_t flags, float* T, double* err_hist,
                                         aaac_stats* stats, void* ws, const float* gsc,
                                         Reducer& red, cudaStream_t st) {
-  const cudaError_t attr = set_smem<FMT, false>();
+  FitPassFn kern;
+  const cudaError_t attr = fit_kernel<FMT, false>(S, &kern);
   if (attr != cudaSuccess) return attr;
   const FitPlan pp = fit_plan(N, K, M_total);
   const PassPlan pprep = plan_pass(N, K);
@@ -1332,7 +1346,7 @@ static cudaError_t launch_fit_sharded_t(const uint16_t* W, int64_t N, int64_t K,
   launches += 2;
   const float tau = choice_tau(S);
   for (int it = 0; it < iters; it++) {
-    fit_pass<FMT, false><<<pp.blocks, kFitThreads, smem_bytes(false), st>>>(
+    kern<<<pp.blocks, kFitThreads, smem_bytes(false), st>>>(
         W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items, tau,
         PackOut{nullptr, nullptr, nullptr, nullptr}, RoundOut{nullptr, nullptr, nullptr, it}, gsc,
         0);
@@ -1444,7 +1458,8 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
                                  uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
                                  uint8_t* choice_bits, double* err_final, void* ws,
                                  const float* gsc, cudaStream_t st) {
-  const cudaError_t attr = set_smem<FMT, true>();
+  FitPassFn kern;
+  const cudaError_t attr = fit_kernel<FMT, true>(S, &kern);
   if (attr != cudaSuccess) return attr;
   const FitPlan pp = fit_plan(N, K, N * K);
   const PassPlan pprep = plan_pass(N, K);
@@ -1458,7 +1473,7 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
                                         FMT == kNvfp4G ? gsc : nullptr);
   const float tau = choice_tau(S);
   const PackOut po{codes, scales_tagged, cbytes, err_final};
-  fit_pass<FMT, true><<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
+  kern<<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
       W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items, tau, po,
       RoundOut{nullptr, nullptr, nullptr, 0}, gsc, 1);
   int launches = 3;
@@ -1482,7 +1497,8 @@ static cudaError_t launch_pack_sharded_t(const uint16_t* W, int64_t N, int64_t K
                                          uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
                                          uint8_t* choice_bits, double* err_final, void* ws,
                                          const float* gsc, Reducer& red, cudaStream_t st) {
-  const cudaError_t attr = set_smem<FMT, true>();
+  FitPassFn kern;
+  const cudaError_t attr = fit_kernel<FMT, true>(S, &kern);
   if (attr != cudaSuccess) return attr;
   const FitPlan pp = fit_plan(N, K, M_total);
   const PassPlan pprep = plan_pass(N, K);
@@ -1499,7 +1515,7 @@ static cudaError_t launch_pack_sharded_t(const uint16_t* W, int64_t N, int64_t K
                                           pp.blocks * kFitWarps, pp.cpc, pp.items,
                                           FMT == kNvfp4G ? gsc : nullptr);
     const PackOut po{codes, scales_tagged, cbytes, err_final};
-    fit_pass<FMT, true><<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
+    kern<<<pp.blocks, kFitThreads, smem_bytes(true), st>>>(
         W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items,
         choice_tau(S), po, RoundOut{nullptr, nullptr, nullptr, 0}, gsc, 0);
     launches += 3;
