@@ -105,7 +105,8 @@ def check_against_oracle(out, ref, cfg, label=""):
     assert np.array_equal(out["scales"].cpu().numpy().view(ref["scales"].dtype), ref["scales"])
     if cfg.fmt == bb.NVFP4_GS:
         assert np.float32(out["global_scale"].item()) == np.float32(ref["gs"]), label
-    assert np.array_equal(npbits(out["T_init"]), ref["T_init"].view(np.uint32)), label
+    if "T_init" in out:  # the bench's block keeps no copy of the initial tables
+        assert np.array_equal(npbits(out["T_init"]), ref["T_init"].view(np.uint32)), label
     T, rT = out["T"].cpu().numpy(), ref["T"]
     assert np.array_equal(T.view(np.uint32), rT.view(np.uint32)), (label, T, rT)
     st = bb.decode_stats(out["stats"])
@@ -291,3 +292,28 @@ def test_qwen32b_nvfp4_full_layer_few_rounds():
     out = bb.run_layer(W, X, cfg)
     ref = oracle.run_layer(u16(W), u16(X), wl.fmt, wl.g, wl.S, 2)
     check_against_oracle(out, ref, cfg, label="qwen32b gate")
+
+
+
+def test_bench_launch_configuration_full_size():
+    """The bench step as bench.py launches it: the Llama-3-8B-shaped block,
+    every linear on its own stream with its own workspace (biggest first) and
+    each activation set's importance on its own stream, all in flight at once.
+    Layer sizes are the bench's; the calibration set is cut to 4096 tokens so
+    that the oracle can redo the whole 20-round fit of gate_proj (58.7M
+    weights) and of k_proj on the CPU."""
+    import bench
+    wl = synth.WORKLOADS["llama8b-int4-s16"]
+    dev = torch.device("cuda", 0)
+    Xs, Ws = bench.build_block(wl, 0, 4096, dev)
+    blk = bench.Block(wl, Xs, Ws, dev)
+    blk.step()
+    torch.cuda.synchronize()
+    cfg = cfg_of(wl.fmt, wl.g, wl.S, wl.iters)
+    for name in ("gate_proj", "k_proj"):
+        lin = next(l for l in wl.linears if l.name == name)
+        ref = oracle.run_layer(u16(Ws[name]), u16(Xs[lin.x_key]), wl.fmt, wl.g, wl.S, wl.iters)
+        out = dict(blk.out[name], I=blk.I[lin.x_key], scales=blk.scales[name], T=blk.T[name],
+                   stats=blk.st[name], err_hist=blk.eh[name])
+        check_against_oracle(out, ref, cfg, label=name)
+    assert bb.device_timeouts() == 0
