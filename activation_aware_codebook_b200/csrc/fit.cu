@@ -56,7 +56,7 @@ constexpr int kStages = 2;                // rows per warp in flight
 constexpr int kFitBlocksPerSM = 4;
 constexpr int kPrepRows = 4;  // rows per lane loaded ahead by fit_prep
 constexpr int kLaneCols = 16;             // columns per lane
-constexpr int kItemRows = 4;              // rows of one work item
+constexpr int kItemRows = 6;              // rows of one work item
 constexpr int kMaxStrips = 256;           // per-strip work counters (more strips: one counter)
 constexpr int kWarpCols = 32 * kLaneCols; // columns per warp (one row segment)
 constexpr int kRingRowBytes = kWarpCols * 2;
