@@ -110,6 +110,15 @@ __device__ __forceinline__ void shared_add_if(uint32_t* p, uint32_t v, bool cond
       : "memory");
 }
 
+// The same at a 32-bit shared address base + 4 idx (idx need not be valid
+// where cond is false: the access is then not made).
+__device__ __forceinline__ void shared_add_at(uint32_t base, uint32_t idx, uint32_t v, bool cond) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q red.shared.add.u32 [%0], %1;\n\t}"
+      ::"r"(base + 4u * idx), "r"(v), "r"((uint32_t)cond)
+      : "memory");
+}
+
 struct RankInit {
   int64_t rank[32];
 };
@@ -155,17 +164,20 @@ __device__ __forceinline__ void radix_rows(const RadixArgs& a, uint32_t (*sh)[25
   const int G = K / g;
   const int r0 = rc * a.rows_per_chunk, r1 = min(a.N, r0 + a.rows_per_chunk);
   if (MODE != 0 && !active) return;  // no warp collectives in later passes
+  const uint32_t sh_base = (uint32_t)__cvta_generic_to_shared(&sh[0][0]);
+  const int cl = active ? col0 : K - 8;  // the column a lane loads from
   // kRadixRows rows per lane are loaded before any is processed (loads in flight)
   for (int rb = r0 + warp; rb < r1; rb += kWarps * kRadixRows) {  // warp-uniform
     uint4 vr[kRadixRows];
     float sr[kRadixRows];
 #pragma unroll
     for (int k = 0; k < kRadixRows; k++) {
+      // unconditional loads: a row past the chunk reads the chunk's last row
+      // and a lane past K the last 8 columns; neither value is counted
       const int r = rb + k * kWarps;
-      const bool ok = active && r < r1;
-      vr[k] = ok ? __ldg(reinterpret_cast<const uint4*>(a.W + (int64_t)r * K + col0))
-                 : make_uint4(0u, 0u, 0u, 0u);
-      sr[k] = (MODE != 0 && ok) ? load_scale<FMT>(a.scales, (int64_t)r * G + col0 / g) : 0.0f;
+      const int rr = r < r1 ? r : r1 - 1;
+      vr[k] = __ldg(reinterpret_cast<const uint4*>(a.W + (int64_t)rr * K + cl));
+      sr[k] = MODE != 0 ? load_scale<FMT>(a.scales, (int64_t)rr * G + cl / g) : 0.0f;
     }
 #pragma unroll
     for (int k = 0; k < kRadixRows; k++) {
@@ -204,19 +216,23 @@ __device__ __forceinline__ void radix_rows(const RadixArgs& a, uint32_t (*sh)[25
                         d < 256u && lane == __ffs(peers) - 1);
         } else {
           const uint32_t pre = key >> (shift + 8);
-          int slot;
-          if (MODE == 1) {
+          uint32_t slot;
+          bool hit;
+          if (MODE == 1) {  // selects, no branches: slot is only used on a hit
             const uint4 e = tab[(pre * mult) >> 24];
-            slot = e.x == pre ? (int)e.y : (e.z == pre ? (int)e.w : -1);
+            const bool hx = e.x == pre;
+            hit = hx || e.z == pre;
+            slot = hx ? e.y : e.w;
           } else {
             int lo = 0, hi = nslots;  // sorted distinct prefixes
             while (lo < hi) {
               const int mid = (lo + hi) >> 1;
               if (sp[mid] < pre) lo = mid + 1; else hi = mid;
             }
-            slot = (lo < nslots && sp[lo] == pre) ? lo : -1;
+            hit = lo < nslots && sp[lo] == pre;
+            slot = (uint32_t)lo;
           }
-          shared_add_if(&sh[slot >= 0 ? slot : 0][(key >> shift) & 255u], 1u, slot >= 0);
+          shared_add_at(sh_base, slot * 256u + ((key >> shift) & 255u), 1u, hit);
         }
       }
     }
