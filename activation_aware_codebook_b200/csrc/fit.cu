@@ -394,28 +394,29 @@ fit_prep(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
       uint4 wv[kPrepRows];
 #pragma unroll
       for (int k = 0; k < kPrepRows; k++) {
+        // unconditional loads: a row past the chunk reads the chunk's last
+        // row, which is not used
         const int r = rb + k * kWarps;
-        const bool in = r < r1;
-        sv[k] = in ? load_scale<FMT>(scales, (int64_t)r * G + col0 / g) : 0.0f;
-        wv[k] = in ? __ldg(reinterpret_cast<const uint4*>(W + (int64_t)r * K + col0))
-                   : make_uint4(0u, 0u, 0u, 0u);
+        const int rr = r < r1 ? r : r1 - 1;
+        sv[k] = load_scale<FMT>(scales, (int64_t)rr * G + col0 / g);
+        wv[k] = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)rr * K + col0));
       }
 #pragma unroll
       for (int k = 0; k < kPrepRows; k++) {
         if (rb + k * kWarps >= r1) break;  // warp-uniform
         const float s = sv[k];
         float rcp;
-        if (!scale_live(eff_scale<FMT>(s, gsv), &rcp)) {
-          if ((lane & (lanes_g - 1)) == 0) dead++;
-          continue;
-        }
-        s2m = fmax(s2m, (double)s * (double)s);
+        const bool live = scale_live(eff_scale<FMT>(s, gsv), &rcp);
+        dead += (!live && (lane & (lanes_g - 1)) == 0) ? 1ull : 0ull;
+        if (live) s2m = fmax(s2m, (double)s * (double)s);
         const uint32_t w[4] = {wv[k].x, wv[k].y, wv[k].z, wv[k].w};
+        uint32_t rm = 0;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
           const float wf = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
-          um = max(um, __float_as_uint(fabsf(__fmul_rn(wf, rcp))));
+          rm = max(rm, __float_as_uint(fabsf(__fmul_rn(wf, rcp))));
         }
+        um = max(um, live ? rm : 0u);  // a dead group's weights are not counted
       }
     }
   }
