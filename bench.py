@@ -345,6 +345,24 @@ def fit_alone_ms(blk, lin, reps=5):
     return statistics.median(times[1:])
 
 
+def per_linear_fit(blk, wl, peak):
+    """Every linear's fit timed alone (prep and setup subtracted): per round,
+    weights/s and algorithmic GB/s against the HBM peak.  W of every linear
+    here is below the 126 MB L2, so rounds after the first can hit in L2."""
+    bb = blk.bb
+    scale_bytes = 2 if wl.fmt == bb.INT4 else 1
+    rows = {}
+    for l in wl.linears:
+        it_ms = (fit_alone_ms(blk, l) - fit_setup_ms(blk, l)) / wl.iters
+        b = l.N * l.K * 2 + l.N * (l.K // wl.g) * scale_bytes + l.K * 4
+        rows[l.name] = {"shape": f"{l.N}x{l.K}", "round_us": it_ms * 1e3,
+                        "weights_per_s": l.N * l.K / (it_ms * 1e-3),
+                        "GB_per_s": b / (it_ms * 1e-3) / 1e9,
+                        "frac": b / (it_ms * 1e-3) / 1e9 / peak,
+                        "W_in_l2": l.N * l.K * 2 < 126 * 2 ** 20}
+    return rows
+
+
 def run_ours(args, rank, local_rank, world):
     import torch
     import torch.distributed as dist
@@ -421,6 +439,8 @@ def run_ours(args, rank, local_rank, world):
                      "frac": inst / (iter_ms * 1e-3) / peak_issue,
                      "source": "warp instructions from the committed ncu capture"}
 
+    per_linear = per_linear_fit(blk, wl, peak)
+
     # end to end through the C ABI with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
@@ -452,6 +472,7 @@ def run_ours(args, rank, local_rank, world):
                          "traffic": traffic, "bytes_per_launch": bytes_per_iter,
                          "round_ms": iter_ms, "timing": "the probe's fit alone, CUDA events",
                          "round_ms_in_step": iter_in_step_ms, "issue": issue},
+            "per_linear_fit": per_linear,
             "gpu_launches": int(launches),
             "clocks": clocks,
         }

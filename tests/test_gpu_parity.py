@@ -126,6 +126,18 @@ def check_against_oracle(out, ref, cfg, label=""):
     np.testing.assert_allclose(float(out["err_final"][0]), ref["err_final"], rtol=RTOL)
 
 
+def test_many_strips_single_counter():
+    """K = 131584 (257 strips of 512 columns): past the per-strip counters the
+    pass hands out fixed-size items from one counter; with 48 rows there are
+    more items than warps in a full wave, so some are claimed."""
+    N, K, iters = 48, 257 * 512, 3
+    W, X = layer(N, K, seed=257, T=32)
+    cfg = cfg_of(bb.INT4, 128, 16, iters)
+    out = bb.run_layer(W, X, cfg)
+    ref = oracle.run_layer(u16(W), u16(X), bb.INT4, 128, 16, iters)
+    check_against_oracle(out, ref, cfg, label="257 strips")
+
+
 def test_single_256x512_int4_workload():
     """The 256x512 INT4 g=128 S=128 layer, X[128, 512], 10 iterations, seed 0."""
     wl = synth.WORKLOADS["single-256x512-int4"]
