@@ -19,6 +19,7 @@ NVFP4_GS = 2  # NVFP4 with a per-tensor fp32 scale
 FREEZE_T0 = 1
 FREEZE_T1 = 2
 SINGLE_CODEBOOK = 4
+CONCURRENT = 8  # grids sized by the layer's weights, for layers fitted side by side
 IMPORTANCE_ACCUMULATE = 1
 IMPORTANCE_EXACT = 2
 

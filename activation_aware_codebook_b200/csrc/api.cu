@@ -58,7 +58,7 @@ aaac_status check_cfg(const aaac_config* cfg) {
     return fail(AAAC_ERR_SHAPE, "S must be a power of two with 8 <= S <= g (S=%d, g=%d)",
                 cfg->S, cfg->g);
   if (cfg->iters < 0) return fail(AAAC_ERR_INVALID_ARG, "iters < 0 (%d)", cfg->iters);
-  if (cfg->flags & ~7u) return fail(AAAC_ERR_INVALID_ARG, "unknown flags 0x%x", cfg->flags);
+  if (cfg->flags & ~15u) return fail(AAAC_ERR_INVALID_ARG, "unknown flags 0x%x", cfg->flags);
   return AAAC_OK;
 }
 

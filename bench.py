@@ -217,7 +217,9 @@ class Block:
         for l in wl.linears:
             gs = (torch.zeros(1, dtype=torch.float32, device=dev) if wl.fmt == bb.NVFP4_GS
                   else None)
-            self.cfgs[l.name] = bb.Config(wl.fmt, wl.g, wl.S, wl.iters, global_scale=gs)
+            # the linears run side by side: grids sized by each one's weights
+            self.cfgs[l.name] = bb.Config(wl.fmt, wl.g, wl.S, wl.iters, flags=bb.CONCURRENT,
+                                          global_scale=gs)
             self.scales[l.name] = torch.empty(l.N, l.K // wl.g, dtype=sdt, device=dev)
             self.T[l.name] = torch.zeros(2, 16, dtype=torch.float32, device=dev)
             self.eh[l.name] = torch.zeros(wl.iters, dtype=torch.float64, device=dev)
@@ -310,7 +312,7 @@ def fit_setup_ms(blk, lin, reps=5):
     """Time of a fit call with zero rounds (prep + setup) on the probe layer."""
     import torch
     bb = blk.bb
-    cfg0 = dataclasses.replace(blk.cfgs[lin.name], iters=0)
+    cfg0 = dataclasses.replace(blk.cfgs[lin.name], iters=0, flags=0)  # alone: full grid
     W = blk.Ws[lin.name]
     T = blk.T[lin.name].clone()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -337,7 +339,8 @@ def fit_alone_ms(blk, lin, reps=5):
         T = blk.T[lin.name].clone()
         torch.cuda.synchronize()
         e0.record()
-        bb.fit_layer(W, blk.I[lin.x_key], blk.scales[lin.name], T, blk.cfgs[lin.name],
+        bb.fit_layer(W, blk.I[lin.x_key], blk.scales[lin.name], T,
+                     dataclasses.replace(blk.cfgs[lin.name], flags=0),  # alone: full grid
                      ws=blk.ws, err_hist=blk.eh[lin.name], stats=blk.st[lin.name])
         e1.record()
         torch.cuda.synchronize()

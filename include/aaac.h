@@ -66,13 +66,20 @@ typedef enum { AAAC_INT4 = 0, AAAC_NVFP4 = 1, AAAC_NVFP4_GS = 2 } aaac_format;
 #define AAAC_FREEZE_T0 1u         /* never refine T0                            */
 #define AAAC_FREEZE_T1 2u         /* never refine T1                            */
 #define AAAC_SINGLE_CODEBOOK 4u   /* every group takes T0                       */
+/* The fit and pack passes of this layer share the GPU with other layers' on
+ * concurrent streams: their grids take one block per 196608 weights (at
+ * least 16, never more than fill the GPU) instead of always filling it, so
+ * a small layer's latency-bound rounds hold few of the SMs' block slots.
+ * Results are identical with and without it. */
+#define AAAC_CONCURRENT 8u
 
 typedef struct {
     int32_t fmt;     /* aaac_format                                            */
     int32_t g;       /* scale group size along K                               */
     int32_t S;       /* selection group size: S % 8 == 0, g % S == 0           */
     int32_t iters;   /* assign+refine rounds of aaac_fit_layer, >= 0           */
-    uint32_t flags;  /* AAAC_FREEZE_T0 | AAAC_FREEZE_T1 | AAAC_SINGLE_CODEBOOK */
+    uint32_t flags;  /* AAAC_FREEZE_T0 | AAAC_FREEZE_T1 | AAAC_SINGLE_CODEBOOK
+                      * | AAAC_CONCURRENT                                      */
     float* global_scale; /* AAAC_NVFP4_GS only (else ignored): device fp32 [1],
                           * 4-byte aligned; aaac_init_codebooks writes gs there,
                           * every other call reads it */

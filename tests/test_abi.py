@@ -57,7 +57,7 @@ def _cfg(**kw):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(fmt=3), 4), (dict(fmt=2, g=16, S=16), 1), (dict(fmt=2, g=32), 4), (dict(fmt=1, g=32), 4), (dict(g=48), 4), (dict(S=4), 2), (dict(S=256), 2),
-    (dict(S=24), 2), (dict(iters=-1), 1), (dict(flags=8), 1)])
+    (dict(S=24), 2), (dict(iters=-1), 1), (dict(flags=16), 1)])
 def test_invalid_config_rejected_without_launch(lib, kw, status):
     c = _cfg(**kw)
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first

@@ -126,6 +126,21 @@ def check_against_oracle(out, ref, cfg, label=""):
     np.testing.assert_allclose(float(out["err_final"][0]), ref["err_final"], rtol=RTOL)
 
 
+@pytest.mark.parametrize("fmt,g,S,N,K", [(bb.INT4, 128, 16, 1024, 4096),
+                                         (bb.NVFP4_GS, 16, 16, 2048, 2048),
+                                         (bb.INT4, 128, 128, 14336, 4096)])
+def test_concurrent_grid_same_results(fmt, g, S, N, K):
+    """AAAC_CONCURRENT only resizes the fit and pack grids: every output is
+    the full-grid call's, bit for bit."""
+    W, X = layer(N, K, seed=N + K, T=256, dist="normal" if fmt == bb.INT4 else "student_t4")
+    ref = bb.run_layer(W, X, cfg_of(fmt, g, S, 4))
+    out = bb.run_layer(W, X, cfg_of(fmt, g, S, 4, flags=bb.CONCURRENT))
+    torch.cuda.synchronize()
+    for k in ("I", "scales", "T_init", "T", "err_hist", "stats", "T_bf16", "codes",
+              "scales_tagged", "err_final") + (("choice_bits",) if S != g else ()):
+        assert torch.equal(out[k], ref[k]), k
+
+
 def test_many_strips_single_counter():
     """K = 131584 (257 strips of 512 columns): past the per-strip counters the
     pass hands out fixed-size items from one counter; with 48 rows there are
