@@ -250,9 +250,10 @@ class Block:
                                    dtype=torch.uint8, device=dev) for k in self.keys}
 
     def step(self, fit_events=None, probe=None, waits=None, key_waits=None):
-        """The importance of each activation set on its own stream, then
-        every linear on its own stream once its importance is done; the
-        current stream waits for all of them before returning.
+        """The importance of each activation set on its own stream, and
+        every linear on its own stream: its init at once (it needs only W),
+        its fit and pack once its importance is done; the current stream
+        waits for all of them before returning.
         waits: optional {linear name: [events]} a linear's stream waits for
         (e2e: its weight copy, the previous copy-out of its outputs);
         key_waits: optional {key: [events]} an importance waits for (e2e:
@@ -277,12 +278,14 @@ class Block:
         for l in self.order:
             s = self.streams[l.name]
             s.wait_event(start)
-            s.wait_event(imp[l.x_key])
             for e in (waits or {}).get(l.name, ()):
                 s.wait_event(e)
             with torch.cuda.stream(s):
                 W, cfg, ws = self.Ws[l.name], self.cfgs[l.name], self.wss[l.name]
+                # the init reads only W: it overlaps the importance passes,
+                # and the fit waits for its importance vector
                 bb.init_codebooks(W, cfg, ws=ws, scales=self.scales[l.name], T=self.T[l.name])
+                s.wait_event(imp[l.x_key])
                 if fit_events is not None and l.name == probe:
                     fit_events[0].record(s)
                 bb.fit_layer(W, self.I[l.x_key], self.scales[l.name], self.T[l.name], cfg,
