@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--tokens", type=int, default=0, help="override calibration tokens")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-per-linear", action="store_true",
+                   help="skip the per-linear fit timings (e.g. for an ncu launch list of the step)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--linear", action="store_true",
                    help="time the W4A16 linear on a packed 14336x4096 layer instead of the fit")
@@ -445,7 +447,7 @@ def run_ours(args, rank, local_rank, world):
                      "frac": inst / (iter_ms * 1e-3) / peak_issue,
                      "source": "warp instructions from the committed ncu capture"}
 
-    per_linear = per_linear_fit(blk, wl, peak)
+    per_linear = None if args.no_per_linear else per_linear_fit(blk, wl, peak)
 
     # end to end through the C ABI with host buffers (pinned), copies timed
     e2e = None
@@ -478,7 +480,7 @@ def run_ours(args, rank, local_rank, world):
                          "traffic": traffic, "bytes_per_launch": bytes_per_iter,
                          "round_ms": iter_ms, "timing": "the probe's fit alone, CUDA events",
                          "round_ms_in_step": iter_in_step_ms, "issue": issue},
-            "per_linear_fit": per_linear,
+            **({"per_linear_fit": per_linear} if per_linear is not None else {}),
             "gpu_launches": int(launches),
             "clocks": clocks,
         }
