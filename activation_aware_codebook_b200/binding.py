@@ -34,7 +34,8 @@ EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaa
            "aaac_fit_layer_fixed_scratch", "aaac_dequant", "aaac_linear",
            "aaac_device_timeouts", "aaac_awq_prescale", "aaac_awq_workspace_size",
            "aaac_awq_fit", "aaac_init_codebooks_sharded", "aaac_fit_layer_sharded",
-           "aaac_pack_sharded", "aaac_linear_workspace_size", "aaac_linear_ws")
+           "aaac_pack_sharded", "aaac_linear_workspace_size", "aaac_linear_ws",
+           "aaac_fit_launch_plan")
 
 
 # reduction callback of the row-sharded calls: (user, buf, count, op, stream) -> 0 | error
@@ -126,6 +127,8 @@ def load(path: str = LIB_PATH):
     L.aaac_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     L.aaac_kernel_launches.restype = ctypes.c_uint64
     L.aaac_kernel_launches.argtypes = []
+    L.aaac_fit_launch_plan.restype = ctypes.c_int
+    L.aaac_fit_launch_plan.argtypes = [P, i64, i64, i64, ctypes.POINTER(ctypes.c_int32)]
     L.aaac_awq_prescale.restype = ctypes.c_int
     L.aaac_awq_prescale.argtypes = [P, i64, i64, P, i64, ctypes.c_int, P, P, P, P]
     L.aaac_awq_workspace_size.restype = sz
@@ -180,6 +183,15 @@ def _need_cuda():
 def workspace_size(cfg: Optional[Config], N: int = 0, K: int = 0, T: int = 0) -> int:
     c = cfg.c() if cfg is not None else None
     return int(load().aaac_workspace_size(ctypes.byref(c) if c is not None else None, N, K, T))
+
+
+def fit_launch_plan(cfg: Config, N: int, K: int, N_total: Optional[int] = None) -> dict:
+    """The fit/pack passes' launch plan for these sizes (host-only query)."""
+    out = (ctypes.c_int32 * 5)()
+    _check(load().aaac_fit_launch_plan(ctypes.byref(cfg.c()), N, K,
+                                       N if N_total is None else N_total, out))
+    return dict(blocks=out[0], strips=out[1], items_per_strip=out[2], item_rows=out[3],
+                max_items=out[4])
 
 
 def workspace(cfg: Optional[Config], N: int = 0, K: int = 0, T: int = 0,

@@ -149,6 +149,18 @@ const char* aaac_version(void) { return "libaaac 0.1 (sm_100a)"; }
 
 uint64_t aaac_kernel_launches(void) { return aaac::g_launches.load(std::memory_order_relaxed); }
 
+aaac_status aaac_fit_launch_plan(const aaac_config* cfg, int64_t N, int64_t K, int64_t N_total,
+                                 int32_t* out) {
+  if (!out) return fail(AAAC_ERR_INVALID_ARG, "out is NULL");
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  if (N_total < N)
+    return fail(AAAC_ERR_SHAPE, "N_total=%lld < N=%lld", (long long)N_total, (long long)N);
+  CHECK(check_layer(N_total, K, cfg));
+  aaac::fit_launch_plan(N, K, N_total * K, cfg->flags, out);
+  return ok();
+}
+
 size_t aaac_workspace_size(const aaac_config* cfg, int64_t N, int64_t K, int64_t T) {
   size_t need = weight_side_bytes(cfg, N, K);
   if (T > 0 && K > 0) {

@@ -155,6 +155,15 @@ static FitPlan fit_plan(int64_t N, int64_t K, int64_t M, bool concurrent) {
   return p;
 }
 
+void fit_launch_plan(int64_t N, int64_t K, int64_t M_total, uint32_t flags, int32_t out[5]) {
+  const FitPlan p = fit_plan(N, K, M_total, (flags & AAAC_CONCURRENT) != 0);
+  out[0] = p.blocks;
+  out[1] = p.ncb;
+  out[2] = p.cpc;
+  out[3] = kItemRows;
+  out[4] = p.max_items;
+}
+
 size_t fit_ws_bytes(int64_t N, int64_t K) {
   (void)N;
   (void)K;

@@ -35,6 +35,9 @@ size_t fit_ctl_bytes();
 size_t init_ctl_bytes();
 size_t pack_extra_bytes(int64_t N, int64_t K, int S);
 size_t fit_ws_bytes(int64_t N, int64_t K);
+// the fit/pack launch plan: blocks, strips, items per strip, rows per item,
+// items per warp
+void fit_launch_plan(int64_t N, int64_t K, int64_t M_total, uint32_t flags, int32_t out[5]);
 
 // ---- the fit's library-owned scratch (fit.cu) -----------------------------
 size_t fixed_scratch_bytes();

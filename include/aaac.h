@@ -346,6 +346,22 @@ const char* aaac_last_error(void);
 /* Library version string. */
 const char* aaac_version(void);
 
+/* Launch plan of the fit and pack passes (aaac_fit_layer, aaac_pack and their
+ * row-sharded forms) for N rows x K columns of a layer of N_total rows (N_total
+ * = N when it is not sharded), as those calls compute it from cfg.  A host-only
+ * query: no GPU work, no device memory.  out (host int32[5]):
+ *   out[0]  blocks of the pass (3 warps each)
+ *   out[1]  strips of 512 columns
+ *   out[2]  work items per strip (runs of out[3] rows)
+ *   out[3]  rows per work item
+ *   out[4]  work items one warp may take: the bound that keeps its lanes'
+ *           fixed-point refine partials exact
+ * Errors as the calls': AAAC_ERR_INVALID_ARG (NULL cfg or out, bad flags or
+ * iters), AAAC_ERR_UNSUPPORTED / AAAC_ERR_SHAPE (format, g, S, sizes,
+ * N_total < N). */
+aaac_status aaac_fit_launch_plan(const aaac_config* cfg, int64_t N, int64_t K, int64_t N_total,
+                                 int32_t* out);
+
 /* Number of CUDA kernels this library has launched in the process so far
  * (all threads, all devices).  A measurement aid: the difference across a
  * region counts the library's kernel launches in it. */
