@@ -153,6 +153,21 @@ def test_many_strips_single_counter():
     check_against_oracle(out, ref, cfg, label="257 strips")
 
 
+@pytest.mark.parametrize("fmt,g,S,N,K", [(bb.INT4, 128, 128, 1, 128), (bb.NVFP4, 16, 16, 1, 16),
+                                         (bb.NVFP4, 16, 8, 3, 16), (bb.INT4, 16, 8, 5, 48),
+                                         (bb.NVFP4_GS, 16, 16, 2, 32)])
+@pytest.mark.parametrize("iters", [0, 3])
+def test_tiny_layers(fmt, g, S, N, K, iters):
+    """One row, one scale group, a 16-weight layer, and zero rounds (the pack
+    straight after the init): every output bit-exact against the oracle."""
+    W, X = layer(N, K, seed=7 * N + K + iters, T=32,
+                 dist="normal" if fmt == bb.INT4 else "student_t4")
+    cfg = cfg_of(fmt, g, S, iters)
+    out = bb.run_layer(W, X, cfg)
+    ref = oracle.run_layer(u16(W), u16(X), fmt, g, S, iters)
+    check_against_oracle(out, ref, cfg, label=f"{N}x{K}")
+
+
 def test_single_256x512_int4_workload():
     """The 256x512 INT4 g=128 S=128 layer, X[128, 512], 10 iterations, seed 0."""
     wl = synth.WORKLOADS["single-256x512-int4"]
