@@ -41,6 +41,8 @@
 //   launch plan bounds the rows per lane to keep it there.  Bins are laid out
 //   [book*16 + entry][lane] in 16-byte cells: a warp's read-modify-write of
 //   its bins touches 32 distinct bank quads, with no conflicts.
+#include <cuda.h>
+
 #include <cstddef>
 #include <mutex>
 
@@ -736,15 +738,15 @@ struct GroupStats {
 // Counters of one live group: near ties, exact decisions, T1 groups, and
 // its objective s^2 D in fixed point (scale twoLe).
 __device__ __forceinline__ void count_group(GroupStats& gs, bool exact, double E0, double E1,
-                                            float d0, float d1, int ch, bool single, float s,
-                                            double twoLe) {
+                                            float d0, float d1, int ch, float s, double twoLe) {
   double e;
   if (exact) {
     gs.exact++;
     if (fabs(E1 - E0) < 1e-6 * fmax(E0, E1)) gs.near++;
     e = (double)(s * s) * (ch ? E1 : E0);  // s*s exact in fp32
   } else {
-    if (!single && fabsf(d1 - d0) < 1e-6f * fmaxf(d0, d1)) gs.near++;
+    // never true for a decided group: its gap exceeds tau (d0 + d1) > 1e-6 max
+    if (fabsf(d1 - d0) < 1e-6f * fmaxf(d0, d1)) gs.near++;
     e = (double)(s * s) * (double)(ch ? d1 : d0);
   }
   gs.err += (unsigned long long)__double2ll_rn(e * twoLe);
@@ -1043,10 +1045,16 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     int ch[2] = {0, 0};
     bool ex[2] = {false, false};
     float g0[2] = {D0[0], D0[1]}, g1[2] = {D1[0], D1[1]};
+    // SINGLE_CODEBOOK forces T0, but an undecided group still takes the exact
+    // rule below, so that its near-tie count is that of the sequential fp64
+    // errors, as for the other variants.
     if (S == 8) {
 #pragma unroll
       for (int h = 0; h < 2; h++)
-        if (live && !single) ch[h] = fast_choice(D0[h], D1[h], tau, &ex[h]);
+        if (live) {
+          ch[h] = fast_choice(D0[h], D1[h], tau, &ex[h]);
+          if (single) ch[h] = 0;
+        }
     } else {
       float d0 = __fadd_rn(D0[0], D0[1]), d1 = __fadd_rn(D1[0], D1[1]);
       for (int o = 1; o < lanes_s; o <<= 1) {
@@ -1055,7 +1063,10 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
       }
       g0[0] = g0[1] = d0;
       g1[0] = g1[1] = d1;
-      if (live && !single) ch[0] = fast_choice(d0, d1, tau, &ex[0]);
+      if (live) {
+        ch[0] = fast_choice(d0, d1, tau, &ex[0]);
+        if (single) ch[0] = 0;
+      }
       ch[1] = ch[0];
       ex[1] = ex[0];
     }
@@ -1067,12 +1078,12 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
         for (int h = 0; h < 2; h++)
           if (ex[h]) {
             exact_group_errors(wrow + 8 * h, I + col0 + 8 * h, 8, rcp, tb, &E0[h], &E1[h]);
-            ch[h] = (E1[h] < E0[h]) ? 1 : 0;
+            ch[h] = (!single && E1[h] < E0[h]) ? 1 : 0;
           }
       } else {
         if (ex[0] && lane == leader_lane) {
           exact_group_errors(wrow, I + col0, S, rcp, tb, &E0[0], &E1[0]);
-          ch[0] = (E1[0] < E0[0]) ? 1 : 0;
+          ch[0] = (!single && E1[0] < E0[0]) ? 1 : 0;
         }
         ch[0] = __shfl_sync(0xffffffffu, ch[0], leader_lane);
         ch[1] = ch[0];
@@ -1080,10 +1091,10 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     }
     if (live) {
       if (S == 8) {
-        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], single, s, PACK ? 0.0 : twoLe);
-        count_group(gs, ex[1], E0[1], E1[1], g0[1], g1[1], ch[1], single, s, PACK ? 0.0 : twoLe);
+        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], s, PACK ? 0.0 : twoLe);
+        count_group(gs, ex[1], E0[1], E1[1], g0[1], g1[1], ch[1], s, PACK ? 0.0 : twoLe);
       } else if (lane == leader_lane) {
-        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], single, s, PACK ? 0.0 : twoLe);
+        count_group(gs, ex[0], E0[0], E1[0], g0[0], g1[0], ch[0], s, PACK ? 0.0 : twoLe);
       }
     }
     const uint32_t sel0 = ch[0] ? 0x4432u : 0x4410u;  // book-1 or book-0 half of moff
@@ -1398,33 +1409,64 @@ cudaError_t launch_fit_sharded(const uint16_t* W, int64_t N, int64_t K, int64_t 
 // ---------------------------------------------------------------------------
 // library-owned scratch for aaac_fit_layer_fixed_scratch
 // ---------------------------------------------------------------------------
-// The fit's scratch (control block + one fp64 per block) in a file-scope device
-// array: every GPU that loads the library holds it until the process exits.
-// All calls share it, so calls whose work overlaps on the GPU would race.
+// The fit's scratch (its control block) in a file-scope device array: every
+// GPU that loads the library holds it until the process exits.  All calls
+// share it, so calls whose work overlaps on the GPU would race.
 constexpr size_t kFixedScratchBytes = 256 * 1024;
 static __device__ __align__(256) unsigned char g_fit_scratch[kFixedScratchBytes];
+static_assert(sizeof(FitCtl) + 255 <= kFixedScratchBytes,
+              "the fit's control block must fit the library-owned scratch");
 
 size_t fixed_scratch_bytes() { return kFixedScratchBytes; }
 
 // In host code g_fit_scratch names a host-side stand-in, not device memory:
-// the device address is looked up with cudaGetSymbolAddress, once per device,
-// with that device current, and cached.
+// the device address is looked up with cudaGetSymbolAddress with the device
+// current.  The address belongs to the copy of the module loaded in the
+// current context, so it is cached per device together with that context's
+// unique id, and looked up again when the current context is another one
+// (for example the primary context made anew after cudaDeviceReset).
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+static CtxGetIdFn ctx_get_id_fn() {
+  static CtxGetIdFn fn = []() -> CtxGetIdFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<CtxGetIdFn>(p);
+  }();
+  return fn;
+}
+
 cudaError_t fixed_scratch_ptr(void** out) {
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
+  static unsigned long long ctx_id[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const CtxGetIdFn get_id = ctx_get_id_fn();
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_fit_scratch);
-    if (e != cudaSuccess) return e;
-    addr[dev] = p;
+  unsigned long long id = 0;
+  // a NULL context means "the current one"; no id (no context yet, or no
+  // driver entry point) means no cached address is trusted
+  const bool have_id = get_id && get_id(nullptr, &id) == CUDA_SUCCESS && id != 0;
+  if (addr[dev] != nullptr && have_id && ctx_id[dev] == id) {
+    *out = addr[dev];
+    return cudaSuccess;
   }
-  *out = addr[dev];
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_fit_scratch);  // makes the device's context current
+  if (e != cudaSuccess) return e;
+  if (get_id && get_id(nullptr, &id) == CUDA_SUCCESS && id != 0) {
+    addr[dev] = p;
+    ctx_id[dev] = id;
+  } else {
+    addr[dev] = nullptr;
+  }
+  *out = p;
   return cudaSuccess;
 }
 

@@ -11,7 +11,8 @@
  *  - All tensors are caller-allocated DEVICE memory on the current CUDA device,
  *    except the aaac_config struct, which is host memory read during the call.
  *    The library allocates nothing: scratch memory is the caller's workspace
- *    (ws, ws_bytes), sized by aaac_workspace_size().
+ *    (ws, ws_bytes), sized by aaac_workspace_size().  The one exception is
+ *    aaac_fit_layer_fixed_scratch, which uses an array inside the library.
  *  - W is the weight, row-major [N][K] bf16 (N output rows, K input columns);
  *    groups of g (scale) and S (codebook choice) weights run along K.
  *    X is the calibration activation, row-major [T][ldx] bf16 (T tokens).
@@ -170,7 +171,9 @@ aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
  *   anything is launched) fits; a scratch need above the array would be
  *   rejected with AAAC_ERR_WORKSPACE, also before any launch.
  *   The first call on a device looks up the array's device address with that
- *   device current; make that first call before any stream capture.
+ *   device current; make that first call before any stream capture.  The
+ *   address is cached with the id of the context it was taken in and looked
+ *   up again when another context is current (after cudaDeviceReset, say).
  *   All calls share the one array and it keeps the previous call's contents
  *   (the call clears what must start at zero).  Calls whose work overlaps on
  *   the GPU -- concurrent streams, or concurrent host threads -- race on it:

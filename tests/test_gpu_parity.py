@@ -115,6 +115,10 @@ def check_against_oracle(out, ref, cfg, label=""):
         assert st["groups_t1"] == ref["stats"].groups_t1
         assert st["empty_cells"] == ref["stats"].empty_cells
         assert st["dead_groups"] == ref["stats"].dead_groups
+        # near ties (reading R13) of the last round; each was decided by the
+        # exact fp64 rule, which the exact-decision count (all rounds) includes
+        assert st["near_ties"] == ref["stats"].near_ties, label
+        assert st["exact_groups"] >= st["near_ties"], label
         eh = out["err_hist"].cpu().numpy()
         np.testing.assert_allclose(eh, ref["err_hist"], rtol=RTOL, atol=0)
     assert np.array_equal(out["T_bf16"].cpu().numpy().view(np.uint16), ref["T_bf16"])
