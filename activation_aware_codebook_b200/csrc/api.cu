@@ -93,8 +93,8 @@ aaac_status from_cuda(cudaError_t e, const char* where) {
 
 size_t weight_side_bytes(const aaac_config* cfg, int64_t N, int64_t K) {
   if (!cfg || N <= 0 || K <= 0 || cfg->S <= 0) return 0;
-  size_t fit = aaac::fit_ws_bytes(N, K);
-  size_t pack = fit + aaac::pack_extra_bytes(N, K, cfg->S);
+  size_t fit = aaac::fit_ws_bytes(N, K, cfg->g);
+  size_t pack = aaac::fit_ctl_bytes() + aaac::pack_extra_bytes(N, K, cfg->S);
   size_t init = aaac::init_ctl_bytes();
   size_t m = fit > pack ? fit : pack;
   return m > init ? m : init;
@@ -212,10 +212,11 @@ aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
   CHECK(check_ptr(T, "T"));
   CHECK(check_ptr(err_hist, "err_hist", false));
   CHECK(check_ptr(stats, "stats", false));
-  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K)));
+  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K, cfg->g)));
+  float2* rsc = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(ws) + aaac::fit_ctl_bytes());
   return from_cuda(aaac::launch_fit(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
                                     cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T, err_hist,
-                                    stats, ws, cfg->global_scale, (cudaStream_t)stream),
+                                    stats, ws, rsc, cfg->global_scale, (cudaStream_t)stream),
                    "aaac_fit_layer");
 }
 
@@ -230,7 +231,9 @@ aaac_status aaac_fit_layer_fixed_scratch(const void* W, int64_t N, int64_t K, co
   CHECK(check_ptr(T, "T"));
   CHECK(check_ptr(err_hist, "err_hist", false));
   CHECK(check_ptr(stats, "stats", false));
-  const size_t need = aaac::fit_ws_bytes(N, K);
+  // with no room for per-layer tables the rounds run fit_pass, whose only
+  // scratch is the control block
+  const size_t need = aaac::fit_ctl_bytes();
   if (need > aaac::fixed_scratch_bytes())
     return fail(AAAC_ERR_WORKSPACE,
                 "this layer (N=%lld K=%lld) needs %zu bytes of scratch but the library's fixed "
@@ -241,7 +244,7 @@ aaac_status aaac_fit_layer_fixed_scratch(const void* W, int64_t N, int64_t K, co
   if (e != cudaSuccess) return from_cuda(e, "aaac_fit_layer_fixed_scratch: scratch address");
   return from_cuda(aaac::launch_fit(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
                                     cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T, err_hist,
-                                    stats, ws, cfg->global_scale, (cudaStream_t)stream),
+                                    stats, ws, nullptr, cfg->global_scale, (cudaStream_t)stream),
                    "aaac_fit_layer_fixed_scratch");
 }
 
@@ -260,7 +263,7 @@ aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const
   CHECK(check_ptr(scales_tagged, "scales_tagged"));
   CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
   CHECK(check_ptr(err_final, "err_final", false));
-  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K) + aaac::pack_extra_bytes(N, K, cfg->S)));
+  CHECK(check_ws(ws, ws_bytes, aaac::fit_ctl_bytes() + aaac::pack_extra_bytes(N, K, cfg->S)));
   return from_cuda(aaac::launch_pack(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
                                      cfg->fmt, cfg->g, cfg->S, cfg->flags, T, T_bf16, codes,
                                      scales_tagged, choice_bits, err_final, ws, cfg->global_scale,
@@ -393,7 +396,10 @@ aaac_status aaac_awq_fit(const void* W, int64_t N, int64_t K, const float* I, in
       e = aaac::launch_init(Ws, N, K, cfg->fmt, cfg->g, scl, T, fws, gs, st);
     if (e == cudaSuccess)
       e = aaac::launch_fit(Ws, N, K, Is, scl, cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T,
-                           hist, stats, fws, gs, st);
+                           hist, stats, fws,
+                           reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(fws) +
+                                                     aaac::fit_ctl_bytes()),
+                           gs, st);
     if (e == cudaSuccess)
       e = aaac::launch_pack(Ws, N, K, Is, scl, cfg->fmt, cfg->g, cfg->S, cfg->flags, T, Tb, cod,
                             tag, bits, err_alpha + i, fws, gs, st);
@@ -445,7 +451,7 @@ aaac_status aaac_fit_layer_sharded(const void* W, int64_t N, int64_t K, int64_t 
   CHECK(check_ptr(T, "T"));
   CHECK(check_ptr(err_hist, "err_hist", false));
   CHECK(check_ptr(stats, "stats", false));
-  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K)));
+  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K, cfg->g)));
   aaac::Reducer red{reduce, user, false};
   const cudaError_t e = aaac::launch_fit_sharded(
       reinterpret_cast<const uint16_t*>(W), N, K, N_total * K, I, scales, cfg->fmt, cfg->g,
@@ -473,7 +479,7 @@ aaac_status aaac_pack_sharded(const void* W, int64_t N, int64_t K, int64_t N_tot
   CHECK(check_ptr(scales_tagged, "scales_tagged"));
   CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
   CHECK(check_ptr(err_final, "err_final", false));
-  CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K) + aaac::pack_extra_bytes(N, K, cfg->S)));
+  CHECK(check_ws(ws, ws_bytes, aaac::fit_ctl_bytes() + aaac::pack_extra_bytes(N, K, cfg->S)));
   aaac::Reducer red{reduce, user, false};
   const cudaError_t e = aaac::launch_pack_sharded(
       reinterpret_cast<const uint16_t*>(W), N, K, N_total * K, I, scales, cfg->fmt, cfg->g,

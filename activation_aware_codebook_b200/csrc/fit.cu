@@ -79,6 +79,7 @@ struct Tables {
   float mv1[kMerged];      // book-1 value of merged cell m (NaN at kCrowded)
   uint32_t moff[kMerged];  // bin offsets of cell m: book 0 low 16 bits, book 1 high
   uint8_t mlut[kNB];       // bucket -> merged base count, kCrowded = crowded bucket
+  uint8_t mlut4[kNB];      // 4 * mlut: the base count as a byte offset into the 4-byte arrays
   Book bk[2];
   float la;
   int32_t nm;              // number of merged thresholds
@@ -100,6 +101,7 @@ struct FitCtl {
   // shards with one int64 sum-reduction of kShardSums values.
   long long bins[2][16][2];
   unsigned long long err_acc;  // sum of rint(s^2 D 2^Le) of the running pass
+  unsigned long long err_fine;  // the same at 2^30 times the scale (see objective_value)
   unsigned long long near_ties;
   unsigned long long groups_t1;
   unsigned long long exact_groups;
@@ -111,11 +113,14 @@ struct FitCtl {
   unsigned int strip_next[kMaxStrips];  // per-strip item counters of the running pass
   double twoLe;            // fixed-point scale of the objective sums
 };
-constexpr int kShardSums = 64 + 4;  // bins, err_acc, near_ties, groups_t1, exact_groups
+constexpr int kShardSums = 64 + 5;  // bins, err_acc, err_fine, near_ties, groups_t1, exact_groups
 static_assert(offsetof(FitCtl, exact_groups) == offsetof(FitCtl, bins) + (kShardSums - 1) * 8,
               "the round sums must be contiguous");
 
 size_t fit_ctl_bytes() { return align256(sizeof(FitCtl)); }
+
+// Scale pairs per row of the pair table: the group count rounded up to even.
+__host__ __device__ inline int pair_stride(int G) { return G + (G & 1); }
 
 // Work items: kItemRows rows of one 512-column strip; warps claim them from
 // a global counter.  A lane's refine partial over its rows (16 terms a row,
@@ -132,7 +137,9 @@ struct FitPlan {
 // linears on concurrent streams: 14.12 ms per step with full grids, 13.1 ms).
 constexpr int64_t kConcurrentWeights = 196608;
 constexpr int64_t kConcurrentMinBlocks = 16;
-static FitPlan fit_plan(int64_t N, int64_t K, int64_t M, bool concurrent) {
+// bps: blocks per SM of one full wave.
+static FitPlan fit_plan(int64_t N, int64_t K, int64_t M, bool concurrent,
+                        int bps = kFitBlocksPerSM) {
   FitPlan p;
   p.ncb = (int)((K + kWarpCols - 1) / kWarpCols);
   p.cpc = (int)((N + kItemRows - 1) / kItemRows);
@@ -145,7 +152,7 @@ static FitPlan fit_plan(int64_t N, int64_t K, int64_t M, bool concurrent) {
   const int64_t per_block = (int64_t)kFitWarps * p.max_items;
   const int64_t need = (p.items + per_block - 1) / per_block;
   const int64_t useful = (p.items + kFitWarps - 1) / kFitWarps;
-  int64_t blocks = 148 * kFitBlocksPerSM;
+  int64_t blocks = 148 * (int64_t)bps;
   if (concurrent) {
     int64_t share = (N * K + kConcurrentWeights - 1) / kConcurrentWeights;
     if (share < kConcurrentMinBlocks) share = kConcurrentMinBlocks;
@@ -166,10 +173,10 @@ void fit_launch_plan(int64_t N, int64_t K, int64_t M_total, uint32_t flags, int3
   out[4] = p.max_items;
 }
 
-size_t fit_ws_bytes(int64_t N, int64_t K) {
-  (void)N;
-  (void)K;
-  return fit_ctl_bytes();  // the control block: work counter, sums, tables
+// The fit's workspace: the control block (work counters, sums, tables), then
+// the (s, 1/s_eff) pair of every scale group.
+size_t fit_ws_bytes(int64_t N, int64_t K, int g) {
+  return fit_ctl_bytes() + align256((size_t)N * (size_t)pair_stride(K / g) * sizeof(float2));
 }
 
 size_t pack_extra_bytes(int64_t N, int64_t K, int S) {
@@ -373,6 +380,7 @@ __device__ void build_tables(Tables& tb, float (*sT)[16], int n, bool sort_first
         const int base = run + s_F[k];
         const int inner = v[i] - s_F[k];
         tb.mlut[k - 1] = (uint8_t)(inner > 1 ? kCrowded : base);
+        tb.mlut4[k - 1] = (uint8_t)(4 * (inner > 1 ? kCrowded : base));
       }
       run += v[i];
     }
@@ -390,11 +398,15 @@ __device__ void store_tables(FitCtl* ctl, const Tables& tb) {
 // prep: the exact maxima that fix the refine's fixed-point exponent and the
 // bucket scale
 // ---------------------------------------------------------------------------
+// rsc (optional): per (row, scale group) the stored scale's magnitude s and
+// r = fp32_RN(1/s_eff) of the effective scale, or (s, 0) for a dead group --
+// what every fit round needs of the scales, computed once per fit.  Rows are
+// pair_stride(K/g) pairs apart (an even count: 16-byte aligned rows).
 template <int FMT>
 __global__ void __launch_bounds__(kThreads)
 fit_prep(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
          const void* __restrict__ scales, int g, FitCtl* ctl, int ncb, int rows_per_chunk,
-         const float* __restrict__ gsc) {
+         const float* __restrict__ gsc, float2* __restrict__ rsc) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float gsv = FMT == kNvfp4G ? __ldg(gsc) : 1.0f;
   uint32_t im = 0;
@@ -430,6 +442,8 @@ fit_prep(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
         float rcp;
         const bool live = scale_live(eff_scale<FMT>(s, gsv), &rcp);
         dead += (!live && (lane & (lanes_g - 1)) == 0) ? 1ull : 0ull;
+        if (rsc && (lane & (lanes_g - 1)) == 0)
+          rsc[(int64_t)(rb + k * kWarps) * pair_stride(G) + col0 / g] = make_float2(s, rcp);
         if (live) s2m = fmax(s2m, (double)s * (double)s);
         const uint32_t w[4] = {wv[k].x, wv[k].y, wv[k].z, wv[k].w};
         uint32_t rm = 0;
@@ -498,6 +512,21 @@ __device__ double objective_scale(const FitCtl* ctl, int64_t M, double g2 = 1.0)
   return ldexp(1.0, Le);
 }
 
+// The objective is summed in fixed point so that its value does not depend on
+// the order of the additions.  2^Le comes from a bound on the whole sum that
+// is rigorous but loose (every weight at the largest importance, scale and
+// error), so one unit can be a sizeable part of a group's contribution: with
+// many groups below a unit the rounding biases the total.  A second sum at
+// 2^30 times the scale keeps that rounding far below the result; it is the
+// one used unless the coarse total shows it may have overflowed (2^31 coarse
+// units or more, where the coarse sum is itself fine enough).
+constexpr double kFineScale = 1073741824.0;  // 2^30
+__device__ __forceinline__ double objective_value(unsigned long long coarse,
+                                                  unsigned long long fine, double twoLe) {
+  return coarse < (1ull << 31) ? (double)(long long)fine / (twoLe * kFineScale)
+                               : (double)(long long)coarse / twoLe;
+}
+
 __device__ void write_stats(const FitCtl* ctl, aaac_stats* st) {
   if (!st) return;
   st->near_ties = (int64_t)ctl->near_ties;
@@ -543,6 +572,7 @@ fit_setup(FitCtl* ctl, float* T_user, int64_t M, int n, aaac_stats* st, int wt, 
     ctl->twoL = ldexp(1.0, L);
     ctl->twoLe = objective_scale(ctl, M);
     ctl->err_acc = 0ull;
+    ctl->err_fine = 0ull;
     ctl->n = n;
     tb.la = bucket_scale(ctl);
   }
@@ -626,11 +656,12 @@ __device__ void round_finalize(FitCtl* ctl, Tables& tb, uint32_t flags, const Ro
   if (tid < 32) sT[tid >> 4][tid & 15] = ctl->T[tid >> 4][tid & 15];
   if (tid < 2) s_upd[tid] = 0;
   if (tid == 0) {
-    const long long acc = (long long)__ldcg(&ctl->err_acc);
+    const double acc = objective_value(__ldcg(&ctl->err_acc), __ldcg(&ctl->err_fine), ctl->twoLe);
     // the rounds sum s^2 D with the stored scale factor; a per-tensor scale
     // enters the objective once, as g2 = gs^2
-    if (ro.err_hist) ro.err_hist[ro.it] = __dmul_rn((double)acc / ctl->twoLe, g2);
+    if (ro.err_hist) ro.err_hist[ro.it] = __dmul_rn(acc, g2);
     ctl->err_acc = 0ull;
+    ctl->err_fine = 0ull;
   }
   __syncthreads();
   const int n = ctl->n;
@@ -732,8 +763,14 @@ __device__ __forceinline__ int fast_choice(float d0, float d1, float tau, bool* 
 
 struct GroupStats {
   unsigned int near, exact, t1;
-  unsigned long long err;  // sum of rint(contribution * 2^Le), modulo 2^64
+  unsigned long long err;   // sum of rint(contribution * 2^Le), modulo 2^64
+  unsigned long long errf;  // sum of rint(contribution * 2^Le * 2^30)
 };
+
+__device__ __forceinline__ void add_objective(GroupStats& gs, double e, double twoLe) {
+  gs.err += (unsigned long long)__double2ll_rn(e * twoLe);
+  gs.errf += (unsigned long long)__double2ll_rn(e * (twoLe * kFineScale));
+}
 
 // Counters of one live group: near ties, exact decisions, T1 groups, and
 // its objective s^2 D in fixed point (scale twoLe).
@@ -749,7 +786,7 @@ __device__ __forceinline__ void count_group(GroupStats& gs, bool exact, double E
     if (fabsf(d1 - d0) < 1e-6f * fmaxf(d0, d1)) gs.near++;
     e = (double)(s * s) * (double)(ch ? d1 : d0);
   }
-  gs.err += (unsigned long long)__double2ll_rn(e * twoLe);
+  add_objective(gs, e, twoLe);
   gs.t1 += ch;
 }
 
@@ -963,7 +1000,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
   for (int k = 0; k < kStages; k++)
     if (k >= npre) sqv[k] = prefetch(k);
 
-  GroupStats gs{0u, 0u, 0u, 0ull};
+  GroupStats gs{0u, 0u, 0u, 0ull, 0ull};
   int slot = 0;
   const unsigned long long la2 = f2pack(la, la);
   const unsigned long long cc2 = f2pack(kBucketMagic + (float)(kNB / 2), kBucketMagic + (float)(kNB / 2));
@@ -1136,7 +1173,7 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
         const double d = __dsub_rn((double)wf, wh);
         err_w = __fma_rn(Id[i], __dmul_rn(d, d), err_w);
       }
-      gs.err += (unsigned long long)__double2ll_rn(err_w * twoLe);
+      add_objective(gs, err_w, twoLe);
       *reinterpret_cast<unsigned long long*>(po.codes + ((int64_t)r * K + col0) / 2) = packed;
       if ((lane & ((g >> 4) - 1)) == 0) {
         const int64_t gi = (int64_t)r * G + (col0 >> lg);
@@ -1176,8 +1213,12 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
     if (gs.t1) atomicAdd(&ctl->groups_t1, (unsigned long long)gs.t1);
   }
   // objective: integer sums, the same whatever the order
-  for (int o = 16; o > 0; o >>= 1) gs.err += __shfl_xor_sync(0xffffffffu, gs.err, o);
+  for (int o = 16; o > 0; o >>= 1) {
+    gs.err += __shfl_xor_sync(0xffffffffu, gs.err, o);
+    gs.errf += __shfl_xor_sync(0xffffffffu, gs.errf, o);
+  }
   if (lane == 0 && gs.err) atomicAdd(&ctl->err_acc, gs.err);
+  if (lane == 0 && gs.errf) atomicAdd(&ctl->err_fine, gs.errf);
   __syncthreads();  // every lane's bins are complete
   if (!PACK && threadIdx.x < 64) {
     // lane bins -> exact integer partials (bias removed exactly), one
@@ -1212,12 +1253,548 @@ fit_pass(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__
                    *reinterpret_cast<FinalizeScratch*>(ring));  // the ring is idle now
   } else {
     if (threadIdx.x == 0) {
-      const long long acc = (long long)__ldcg(&ctl->err_acc);
-      if (po.err_final) *po.err_final = (double)acc / ctl->twoLe;
+      if (po.err_final)
+        *po.err_final = objective_value(__ldcg(&ctl->err_acc), __ldcg(&ctl->err_fine), ctl->twoLe);
       ctl->err_acc = 0ull;
+      ctl->err_fine = 0ull;
       ctl->ticket = 0;
     }
     seed_claims(ctl, wt, cpc, n_items);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the fit round
+// ---------------------------------------------------------------------------
+// fit_round is fit_pass<fit> rebuilt around the same arithmetic with less work
+// per weight and per row:
+//   - W arrives by cp.async.bulk: one lane issues a 1 KB row segment into a
+//     2-slot ring on an mbarrier (the other lanes compute no addresses);
+//   - the scales arrive as (s, 1/s_eff) pairs that fit_prep computes once
+//     per fit, instead of a correctly rounded reciprocal per row;
+//   - every per-lane decision (live group, choice, objective, refine) is a
+//     select: the refine of a dead or inactive lane adds exact zeros, so the
+//     row has no divergent branch outside the rare crowded-bucket and exact
+//     choice paths;
+//   - the bucket table holds byte offsets (4 c), so a cell's address needs no
+//     multiply.
+// The refine sums, the exact choice and the last block's refine are those of
+// fit_pass, so the two give the same tables bit for bit.
+constexpr int kRStages = 2;                  // ring rows per warp
+constexpr uint64_t kRoundWaitNs = 2000000000ull;
+
+__device__ unsigned int g_fit_timeout = 0;
+
+struct __align__(16) RoundRing {
+  unsigned char w[kRStages][kWarpCols * 2];
+  unsigned long long bar[kRStages];
+  int fifo[8];
+  int fifoc[8];
+};
+constexpr size_t kRoundSmem = kFitWarps * (sizeof(RoundRing) + kWarpBinBytes);
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void bar_init(unsigned long long* b) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(b)) : "memory");
+}
+__device__ __forceinline__ bool bar_test(unsigned long long* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait (about 2 s of the global timer); false and the device flag set
+// when it runs out.
+__device__ __forceinline__ bool bar_wait(unsigned long long* b, uint32_t parity) {
+  if (bar_test(b, parity)) return true;
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  while (!bar_test(b, parity)) {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (t - t0 > kRoundWaitNs) {
+      atomicExch(&g_fit_timeout, 1u);
+      return false;
+    }
+  }
+  return true;
+}
+
+// One row segment (bytes: a multiple of 16, both ends 16-byte aligned) into a
+// ring slot, issued by the lane for which `on` holds (guard predicates, no
+// branch): the barrier's arrival with the byte count, then the copy.
+__device__ __forceinline__ void issue_row(bool on, unsigned long long* b, void* dst,
+                                          const void* src, uint32_t bytes) {
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " setp.ne.u32 p, %0, 0;\n"
+      " @p fence.proxy.async.shared::cta;\n"
+      " @p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %4;\n"
+      " @p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3], %4, [%1];\n"
+      "}\n" ::"r"((uint32_t)on),
+      "r"(smem_addr(b)), "r"(smem_addr(dst)), "l"(src), "r"(bytes)
+      : "memory");
+}
+
+// Merged cells of one lane-row's 16 weights (u as 8 column pairs): the fp32
+// errors D0 / D1 of both books over columns 0-7 and 8-15 (the summation
+// structure fit_pass uses, so the same rounding bound holds), and the cells'
+// bin offsets.
+__device__ __forceinline__ void assign_row(const Tables& tb, const float2 (&u2)[8],
+                                           const float2 (&Ip)[8], float la, float (&D0)[2],
+                                           float (&D1)[2], uint32_t (&moffs)[16]) {
+  const unsigned char* mthr_b = reinterpret_cast<const unsigned char*>(tb.mthr);
+  const unsigned char* mv0_b = reinterpret_cast<const unsigned char*>(tb.mv0);
+  const unsigned char* mv1_b = reinterpret_cast<const unsigned char*>(tb.mv1);
+  const unsigned char* moff_b = reinterpret_cast<const unsigned char*>(tb.moff);
+  const float cc = kBucketMagic + (float)(kNB / 2);
+  const float2 la2 = make_float2(la, la), cc2 = make_float2(cc, cc), neg1 = make_float2(-1.f, -1.f);
+  float2 dd0[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 dd1[2] = {dd0[0], dd0[1]};
+#pragma unroll
+  for (int p = 0; p < 8; p++) {
+    const float2 bf = __ffma2_rn(u2[p], la2, cc2);
+    const uint32_t cx = tb.mlut4[__float_as_uint(bf.x) & (kNB - 1)];
+    const uint32_t cy = tb.mlut4[__float_as_uint(bf.y) & (kNB - 1)];
+    const uint32_t mx = cx + (u2[p].x >= *reinterpret_cast<const float*>(mthr_b + cx) ? 4u : 0u);
+    const uint32_t my = cy + (u2[p].y >= *reinterpret_cast<const float*>(mthr_b + cy) ? 4u : 0u);
+    const float2 v0 = make_float2(*reinterpret_cast<const float*>(mv0_b + mx),
+                                  *reinterpret_cast<const float*>(mv0_b + my));
+    const float2 v1 = make_float2(*reinterpret_cast<const float*>(mv1_b + mx),
+                                  *reinterpret_cast<const float*>(mv1_b + my));
+    moffs[2 * p] = *reinterpret_cast<const uint32_t*>(moff_b + mx);
+    moffs[2 * p + 1] = *reinterpret_cast<const uint32_t*>(moff_b + my);
+    const float2 e0 = __ffma2_rn(v0, neg1, u2[p]);
+    const float2 e1 = __ffma2_rn(v1, neg1, u2[p]);
+    dd0[p >> 2] = __ffma2_rn(Ip[p], __fmul2_rn(e0, e0), dd0[p >> 2]);
+    dd1[p >> 2] = __ffma2_rn(Ip[p], __fmul2_rn(e1, e1), dd1[p >> 2]);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; h++) {
+    D0[h] = __fadd_rn(dd0[h].x, dd0[h].y);
+    D1[h] = __fadd_rn(dd1[h].x, dd1[h].y);
+  }
+}
+
+// The same by binary search over the merged thresholds (crowded buckets).
+__device__ __forceinline__ void assign_row_search(const Tables& tb, const float2 (&u2)[8],
+                                                  const float2 (&Ip)[8], float (&D0)[2],
+                                                  float (&D1)[2], uint32_t (&moffs)[16]) {
+  float2 dd0[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 dd1[2] = {dd0[0], dd0[1]};
+  const float2 neg1 = make_float2(-1.f, -1.f);
+#pragma unroll
+  for (int p = 0; p < 8; p++) {
+    const uint32_t mx = merged_search(tb, u2[p].x), my = merged_search(tb, u2[p].y);
+    const float2 v0 = make_float2(tb.mv0[mx], tb.mv0[my]);
+    const float2 v1 = make_float2(tb.mv1[mx], tb.mv1[my]);
+    moffs[2 * p] = tb.moff[mx];
+    moffs[2 * p + 1] = tb.moff[my];
+    const float2 e0 = __ffma2_rn(v0, neg1, u2[p]);
+    const float2 e1 = __ffma2_rn(v1, neg1, u2[p]);
+    dd0[p >> 2] = __ffma2_rn(Ip[p], __fmul2_rn(e0, e0), dd0[p >> 2]);
+    dd1[p >> 2] = __ffma2_rn(Ip[p], __fmul2_rn(e1, e1), dd1[p >> 2]);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; h++) {
+    D0[h] = __fadd_rn(dd0[h].x, dd0[h].y);
+    D1[h] = __fadd_rn(dd1[h].x, dd1[h].y);
+  }
+}
+
+// The objective of a group decided in fp32 (its d is an fp32 sum already):
+// fp32_RN(s^2 d) in fixed point, added only when the group is counted here.
+__device__ __forceinline__ void fast_objective(GroupStats& gs, bool on, float s2, float d,
+                                               double twoLe) {
+  const double e = on ? (double)__fmul_rn(s2, d) : 0.0;
+  gs.err += (unsigned long long)__double2ll_rn(e * twoLe);
+  gs.errf += (unsigned long long)__double2ll_rn(e * (twoLe * kFineScale));
+}
+
+// SC: the selection group size when it is 8 or 16, or 0 for S >= 32 (S_rt).
+// finalize 0: the row-sharded fit (the sums are reduced over the shards and
+// a separate kernel refines).
+template <int FMT, int SC>
+__global__ void __launch_bounds__(kFitThreads, kFitBlocksPerSM)
+fit_round(const uint16_t* __restrict__ W, int N, int K, const float* __restrict__ I,
+          const float2* __restrict__ rsc, int g, int S_rt, uint32_t flags, FitCtl* ctl, int cpc,
+          int n_items, int max_items, float tau, RoundOut ro, const float* __restrict__ gsc,
+          int finalize) {
+  const int S = SC ? SC : S_rt;
+  __shared__ Tables tb;
+  __shared__ int s_last;
+  extern __shared__ __align__(128) unsigned char smem[];
+  RoundRing* rings = reinterpret_cast<RoundRing*>(smem);
+  unsigned char* bins = smem + kFitWarps * sizeof(RoundRing);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned full = 0xffffffffu;
+  RoundRing& rg = rings[warp];
+
+  // ---- up to the dependency wait nothing is read that the previous round
+  // writes (W, I and the scale pairs are the layer's)
+  {
+    double2* b = reinterpret_cast<double2*>(bins);
+    for (int i = threadIdx.x; i < kFitWarps * kWarpBinBytes / 16; i += blockDim.x)
+      b[i] = make_double2(kNumBias, kDenBias);
+    // stale ring bytes are finite weights: an inactive lane's garbage times
+    // its zero reciprocal must not make a NaN
+    uint4* r = reinterpret_cast<uint4*>(rg.w);
+    for (int i = lane; i < kRStages * kWarpCols * 2 / 16; i += 32) r[i] = make_uint4(0u, 0u, 0u, 0u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before the copies overwrite it
+  }
+  if (lane < kRStages) bar_init(&rg.bar[lane]);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __syncwarp();
+
+  const int G = K / g;
+  const int lg = __ffs(g) - 1;
+  const int lanes_s = S >> 4;
+  const int leader_lane = S >= 16 ? (lane & ~(lanes_s - 1)) : lane;
+  const bool single = (flags & AAAC_SINGLE_CODEBOOK) != 0;
+  const float gsv = FMT == kNvfp4G ? __ldg(gsc) : 1.0f;
+  unsigned char* mybins = bins + warp * kWarpBinBytes + lane * 16;
+
+  // ---- work items (as in fit_pass): a fixed first item, then claims
+  int* fifo = rg.fifo;
+  int* fifoc = rg.fifoc;
+  const int ncb = n_items / cpc;
+  const bool per_strip = ncb <= kMaxStrips;
+  const int gw = (int)blockIdx.x * kFitWarps + warp;
+  int cur_strip = gw % ncb, tried = 0;
+  int first = -1, first_c = 0;
+  if (per_strip) {
+    if (gw / ncb < cpc) {
+      first = cur_strip;
+      first_c = gw / ncb;
+    }
+  } else if (gw < n_items) {
+    first = gw / cpc;
+    first_c = gw - first * cpc;
+  }
+  unsigned pend = 0u;
+  bool pend_ok = false, no_more = first < 0;
+  int claimed = first >= 0 ? 1 : 0, tail = 1;
+  if (lane == 0) {
+    fifo[0] = first;
+    fifoc[0] = first_c;
+  }
+  __syncwarp();
+  auto claim = [&]() {
+    pend_ok = !no_more && claimed < max_items;
+    if (pend_ok) {
+      if (lane == 0)
+        pend = per_strip ? atomicAdd(&ctl->strip_next[cur_strip], 1u) : atomicAdd(&ctl->next_item, 1u);
+      claimed++;
+    }
+  };
+  auto land_push = [&]() {
+    int it = -1, itc = 0;
+    while (pend_ok) {
+      const int v = __shfl_sync(full, (int)pend, 0);
+      if (!per_strip) {
+        if (v < n_items) {
+          it = v / cpc;
+          itc = v - it * cpc;
+        }
+        break;
+      }
+      if (v < cpc) {
+        it = cur_strip;
+        itc = v;
+        break;
+      }
+      claimed--;
+      if (++tried >= ncb) break;
+      cur_strip = cur_strip + 1 == ncb ? 0 : cur_strip + 1;
+      claim();
+    }
+    if (it < 0) no_more = true;
+    if (lane == 0) {
+      fifo[tail & 7] = it;
+      fifoc[tail & 7] = itc;
+    }
+    tail++;
+    __syncwarp();
+    claim();
+  };
+
+  // prefetch cursor: the row's W segment into a slot by a bulk copy, and its
+  // scale pair into the L1 cache (the row loads it when it runs: a register
+  // holding a load in flight would stall the loop at its first move)
+  int pq = 0, pr = 0, pe = 0, pseg = 0, pgi = 0;
+  uint32_t pbytes = 0;
+  bool pact = false;
+  const int Gs = pair_stride(G);
+  auto enter = [&](int it, int itc) {
+    if (it < 0) return;
+    pseg = it * kWarpCols;
+    pr = itc * kItemRows;
+    pe = min(N, pr + kItemRows);
+    pbytes = 2u * (uint32_t)min(kWarpCols, K - pseg);
+    const int pcol0 = pseg + lane * kLaneCols;
+    pact = pcol0 < K;
+    pgi = pact ? (pcol0 >> lg) : 0;
+  };
+  auto issue = [&](int ps) {
+    issue_row(lane == 0, &rg.bar[ps], rg.w[ps], W + (int64_t)pr * K + pseg, pbytes);
+    const float2* sp = rsc + (pact ? (int64_t)pr * Gs + pgi : 0);
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(sp));
+  };
+  auto prefetch = [&](int ps) {
+    if (fifo[pq & 7] >= 0) {
+      issue(ps);
+      if (++pr >= pe) {
+        pq++;
+        if (pq == tail) land_push();
+        enter(fifo[pq & 7], fifoc[pq & 7]);
+      }
+    }
+  };
+  enter(first, first_c);
+  int npre = 0;
+#pragma unroll
+  for (int k = 0; k < kRStages; k++) {
+    if (first >= 0 && npre == k && pr + 1 < pe) {
+      issue(k);
+      pr++;
+      npre++;
+    }
+  }
+
+  int cq = 0, cr = 0, ce = 0, ccb = 0;
+  auto centre = [&](int it, int itc) {
+    if (it < 0) return;
+    ccb = it;
+    cr = itc * kItemRows;
+    ce = min(N, cr + kItemRows);
+  };
+  centre(first, first_c);
+  int cur_cb = -1, col0 = 0;
+  bool active = false;
+  float2 Ip[8];
+  double Id[16];
+  auto load_importance = [&](int cb) {
+    cur_cb = cb;
+    col0 = cb * kWarpCols + lane * kLaneCols;
+    active = col0 < K;
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+      const float4 a = active ? __ldg(reinterpret_cast<const float4*>(I + col0) + q)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      Ip[2 * q] = make_float2(a.x, a.y);
+      Ip[2 * q + 1] = make_float2(a.z, a.w);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; i++) Id[i] = (double)((i & 1) ? Ip[i >> 1].y : Ip[i >> 1].x);
+  };
+  if (first >= 0) load_importance(ccb);
+
+  // ---- the previous round's results
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  {
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(&ctl->tb);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(&tb);
+    for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 4); i += blockDim.x) dst[i] = src[i];
+  }
+  const double twoL = ctl->twoL;
+  const double twoLe = ctl->twoLe;
+  __syncthreads();
+  const float la = tb.la;
+  claim();
+#pragma unroll
+  for (int k = 0; k < kRStages; k++)
+    if (k >= npre) prefetch(k);
+
+  GroupStats gs{0u, 0u, 0u, 0ull, 0ull};
+  int slot = 0;
+  uint32_t phase = 0;  // bit k: parity of slot k's next phase
+  bool timed_out = false;
+  while (!timed_out) {  // warp-uniform
+    if (fifo[cq & 7] < 0) break;
+    const int r = cr;
+    if (ccb != cur_cb) load_importance(ccb);
+    if (++cr >= ce) {
+      cq++;
+      centre(fifo[cq & 7], fifoc[cq & 7]);
+    }
+    timed_out = __any_sync(full, !bar_wait(&rg.bar[slot], (phase >> slot) & 1u));
+    phase ^= 1u << slot;
+    const uint4 va = *reinterpret_cast<const uint4*>(rg.w[slot] + 32 * lane);       // columns 0-7
+    const uint4 vb = *reinterpret_cast<const uint4*>(rg.w[slot] + 32 * lane + 16);  // 8-15
+    const float2 sr = __ldg(rsc + (active ? (int64_t)r * Gs + (col0 >> lg) : 0));
+    __syncwarp();  // every lane has read the slot before it is refilled
+    if (!timed_out) prefetch(slot);
+    slot = (slot + 1 == kRStages) ? 0 : slot + 1;
+    if (timed_out) break;
+
+    const float s = active ? sr.x : 0.0f, rcp = active ? sr.y : 0.0f;
+    const bool live = active && rcp > 0.0f;  // dead groups carry rcp = 0: u = 0
+    const uint32_t wv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+    const float2 rr = make_float2(rcp, rcp);
+    float2 u2[8];
+#pragma unroll
+    for (int p = 0; p < 8; p++) u2[p] = __fmul2_rn(make_float2(bf16_lo(wv[p]), bf16_hi(wv[p])), rr);
+
+    float D0[2], D1[2];
+    uint32_t moffs[16];
+    assign_row(tb, u2, Ip, la, D0, D1, moffs);
+    const bool crowded = active && isnan(__fadd_rn(D0[0], D0[1]));
+    if (__any_sync(full, crowded)) {
+      // a crowded bucket (rare): the lane's weights by binary search
+      if (crowded) assign_row_search(tb, u2, Ip, D0, D1, moffs);
+    }
+
+    // the choice (section 2, core mechanism 2): fp32 when the gap clears the
+    // rounding bound, else the sequential fp64 rule
+    int ch[2] = {0, 0};
+    bool ex[2] = {false, false};
+    float g0[2] = {D0[0], D0[1]}, g1[2] = {D1[0], D1[1]};
+    if (S == 8) {
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int c = fast_choice(D0[h], D1[h], tau, &ex[h]);
+        ch[h] = (live && !single) ? c : 0;
+        ex[h] = live && ex[h];
+      }
+    } else {
+      float d0 = __fadd_rn(D0[0], D0[1]), d1 = __fadd_rn(D1[0], D1[1]);
+      for (int o = 1; o < lanes_s; o <<= 1) {
+        d0 = __fadd_rn(d0, __shfl_xor_sync(full, d0, o));
+        d1 = __fadd_rn(d1, __shfl_xor_sync(full, d1, o));
+      }
+      g0[0] = g0[1] = d0;
+      g1[0] = g1[1] = d1;
+      const int c = fast_choice(d0, d1, tau, &ex[0]);
+      ch[0] = ch[1] = (live && !single) ? c : 0;
+      ex[0] = ex[1] = live && ex[0];
+    }
+    const float s2 = __fmul_rn(s, s);  // exact: at most 16 significant bits
+    if (__any_sync(full, ex[0] || ex[1])) {
+      const uint16_t* wrow = W + (int64_t)r * K + col0;
+      double E0[2] = {0.0, 0.0}, E1[2] = {0.0, 0.0};
+      if (S == 8) {
+#pragma unroll
+        for (int h = 0; h < 2; h++)
+          if (ex[h]) {
+            exact_group_errors(wrow + 8 * h, I + col0 + 8 * h, 8, rcp, tb, &E0[h], &E1[h]);
+            ch[h] = (!single && E1[h] < E0[h]) ? 1 : 0;
+          }
+      } else {
+        if (ex[0] && lane == leader_lane) {
+          exact_group_errors(wrow, I + col0, S, rcp, tb, &E0[0], &E1[0]);
+          ch[0] = (!single && E1[0] < E0[0]) ? 1 : 0;
+        }
+        ch[0] = __shfl_sync(full, ch[0], leader_lane);
+        ch[1] = ch[0];
+      }
+      // the exactly decided groups' counters and objective s^2 E (fp64)
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const bool mine = ex[h] && (S == 8 || (h == 0 && lane == leader_lane));
+        if (mine) {
+          gs.exact++;
+          if (fabs(E1[h] - E0[h]) < 1e-6 * fmax(E0[h], E1[h])) gs.near++;
+          add_objective(gs, (double)s2 * (ch[h] ? E1[h] : E0[h]), twoLe);
+        }
+      }
+    }
+    // the groups decided in fp32: their objective and T1 counts (branch-free)
+    if (S == 8) {
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        fast_objective(gs, live && !ex[h], s2, ch[h] ? g1[h] : g0[h], twoLe);
+        gs.t1 += live ? ch[h] : 0;
+      }
+    } else {
+      const bool lead = live && lane == leader_lane;
+      fast_objective(gs, lead && !ex[0], s2, ch[0] ? g1[0] : g0[0], twoLe);
+      gs.t1 += lead ? ch[0] : 0;
+    }
+
+    // refine sums (section 2, core mechanism 4): R_k(A 2^L u) and R_k(A 2^L)
+    // into the lane's bin of (chosen book, entry); a dead or inactive lane
+    // adds exact zeros (A = 0)
+    const uint32_t sel0 = ch[0] ? 0x4432u : 0x4410u;
+    const uint32_t sel1 = ch[1] ? 0x4432u : 0x4410u;
+    const double s2L = live ? (double)s2 * twoL : 0.0;
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+      const uint32_t off = __byte_perm(moffs[i], 0u, i < 8 ? sel0 : sel1);
+      double2* bp = reinterpret_cast<double2*>(mybins + off);
+      const double ud = (double)((i & 1) ? u2[i >> 1].y : u2[i >> 1].x);
+      const double A = __dmul_rn(Id[i], s2L);  // exact: 24 + 16 bits
+      double2 b = *bp;
+      if (i & 1) {  // odd column: ceil
+        b.x = __fma_ru(A, ud, b.x);
+        b.y = __dadd_ru(b.y, A);
+      } else {  // even column: floor
+        b.x = __fma_rd(A, ud, b.x);
+        b.y = __dadd_rd(b.y, A);
+      }
+      *bp = b;
+    }
+  }
+  // the next round may start its blocks
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // every phase of the ring has been waited on: the barriers are released
+  // before the last block reuses their memory
+  __syncwarp();
+  if (lane < kRStages)
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_addr(&rg.bar[lane])) : "memory");
+
+  for (int o = 16; o > 0; o >>= 1) {
+    gs.near += __shfl_xor_sync(full, gs.near, o);
+    gs.exact += __shfl_xor_sync(full, gs.exact, o);
+    gs.t1 += __shfl_xor_sync(full, gs.t1, o);
+  }
+  if (lane == 0) {
+    if (gs.near) atomicAdd(&ctl->near_ties, (unsigned long long)gs.near);
+    if (gs.exact) atomicAdd(&ctl->exact_groups, (unsigned long long)gs.exact);
+    if (gs.t1) atomicAdd(&ctl->groups_t1, (unsigned long long)gs.t1);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    gs.err += __shfl_xor_sync(full, gs.err, o);
+    gs.errf += __shfl_xor_sync(full, gs.errf, o);
+  }
+  if (lane == 0 && gs.err) atomicAdd(&ctl->err_acc, gs.err);
+  if (lane == 0 && gs.errf) atomicAdd(&ctl->err_fine, gs.errf);
+  __syncthreads();  // every lane's bins are complete
+  if (threadIdx.x < 64) {
+    // lane bins -> exact integer partials (bias removed exactly), one
+    // (book, entry, num | den) per thread, summed over the block's lanes
+    const int bc = threadIdx.x >> 1, which = threadIdx.x & 1;
+    const double bias = which ? kDenBias : kNumBias;
+    long long sum = 0;
+    for (int w = 0; w < kFitWarps; w++) {
+      const unsigned char* p = bins + w * kWarpBinBytes + bc * kCellBytes + which * 8;
+      for (int j = 0; j < 32; j++) {
+        const int l = (j + bc) & 31;  // staggered: fewer bank conflicts
+        sum += __double2ll_rn(__dsub_rn(*reinterpret_cast<const double*>(p + l * 16), bias));
+      }
+    }
+    if (sum) atomicAdd(reinterpret_cast<unsigned long long*>(&ctl->bins[0][0][0]) + threadIdx.x,
+                       (unsigned long long)sum);
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&ctl->ticket, 1u) == gridDim.x - 1) ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int wt = (int)gridDim.x * kFitWarps;
+  static_assert(sizeof(FinalizeScratch) <= kFitWarps * sizeof(RoundRing), "finalize scratch in the rings");
+  if (!finalize) {
+    if (threadIdx.x == 0) ctl->ticket = 0;
+    seed_claims(ctl, wt, cpc, n_items);
+  } else {
+    round_finalize(ctl, tb, flags, ro, wt, cpc, n_items, __dmul_rn((double)gsv, (double)gsv),
+                   *reinterpret_cast<FinalizeScratch*>(rings));  // the rings are idle now
   }
 }
 
@@ -1264,9 +1841,9 @@ shard_round_end(FitCtl* ctl, uint32_t flags, RoundOut ro, int wt, int cpc, int n
 
 __global__ void shard_pack_end(FitCtl* ctl, double* err_final) {
   if (threadIdx.x != 0) return;
-  const long long acc = (long long)ctl->err_acc;
-  if (err_final) *err_final = (double)acc / ctl->twoLe;
+  if (err_final) *err_final = objective_value(ctl->err_acc, ctl->err_fine, ctl->twoLe);
   ctl->err_acc = 0ull;
+  ctl->err_fine = 0ull;
 }
 
 static float choice_tau(int S) {
@@ -1290,6 +1867,55 @@ static cudaError_t fit_kernel(int S, FitPassFn* out) {
                               (int)smem_bytes(PACK));
 }
 
+using FitRoundFn = void (*)(const uint16_t*, int, int, const float*, const float2*, int, int,
+                            uint32_t, FitCtl*, int, int, int, float, RoundOut, const float*, int);
+template <int FMT>
+static cudaError_t round_kernel(int S, FitRoundFn* out) {
+  const FitRoundFn k = S == 8 ? fit_round<FMT, 8> : S == 16 ? fit_round<FMT, 16> : fit_round<FMT, 0>;
+  *out = k;
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRoundSmem);
+}
+
+// The fit on fit_round: rsc (N * K/g pairs of the caller's workspace) holds
+// the scale pairs fit_prep writes.
+template <int FMT>
+static cudaError_t launch_fit_round_t(const uint16_t* W, int64_t N, int64_t K, const float* I,
+                                      const void* scales, int g, int S, int iters, uint32_t flags,
+                                      float* T, double* err_hist, aaac_stats* stats, void* ws,
+                                      float2* rsc, const float* gsc, cudaStream_t st) {
+  FitRoundFn kern;
+  const cudaError_t attr = round_kernel<FMT>(S, &kern);
+  if (attr != cudaSuccess) return attr;
+  const FitPlan pp = fit_plan(N, K, N * K, (flags & AAAC_CONCURRENT) != 0);
+  const PassPlan pprep = plan_pass(N, K);
+  FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
+  cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
+  fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
+                                                   pprep.ncb, pprep.rows_per_chunk, gsc, rsc);
+  fit_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), stats, pp.blocks * kFitWarps,
+                                       pp.cpc, pp.items);
+  const float tau = choice_tau(S);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)pp.blocks);
+  lc.blockDim = dim3(kFitThreads);
+  lc.dynamicSmemBytes = kRoundSmem;
+  lc.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  for (int it = 0; it < iters; it++) {
+    const cudaError_t e = cudaLaunchKernelEx(&lc, kern, W, (int)N, (int)K, I,
+                                             (const float2*)rsc, g, S, flags, ctl, pp.cpc,
+                                             pp.items, pp.max_items, tau,
+                                             RoundOut{err_hist, T, stats, it}, gsc, 1);
+    if (e != cudaSuccess) return e;
+  }
+  count_launches(2 + iters);
+  return cudaSuccess;
+}
+
 template <int FMT>
 static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const float* I,
                                 const void* scales, int g, int S, int iters, uint32_t flags,
@@ -1304,7 +1930,7 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
-                                                   pprep.ncb, pprep.rows_per_chunk, gsc);
+                                                   pprep.ncb, pprep.rows_per_chunk, gsc, nullptr);
   fit_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), stats, pp.blocks * kFitWarps,
                                        pp.cpc, pp.items);
   const float tau = choice_tau(S);
@@ -1334,8 +1960,19 @@ static cudaError_t launch_fit_t(const uint16_t* W, int64_t N, int64_t K, const f
 
 cudaError_t launch_fit(const uint16_t* W, int64_t N, int64_t K, const float* I,
                        const void* scales, int fmt, int g, int S, int iters, uint32_t flags,
-                       float* T, double* err_hist, aaac_stats* stats, void* ws, const float* gsc,
-                       cudaStream_t st) {
+                       float* T, double* err_hist, aaac_stats* stats, void* ws, float2* rsc,
+                       const float* gsc, cudaStream_t st) {
+  if (rsc) {
+    const cudaError_t e =
+        (fmt == kInt4) ? launch_fit_round_t<kInt4>(W, N, K, I, scales, g, S, iters, flags, T,
+                                                   err_hist, stats, ws, rsc, gsc, st)
+        : (fmt == kNvfp4) ? launch_fit_round_t<kNvfp4>(W, N, K, I, scales, g, S, iters, flags, T,
+                                                       err_hist, stats, ws, rsc, gsc, st)
+                          : launch_fit_round_t<kNvfp4G>(W, N, K, I, scales, g, S, iters, flags,
+                                                        T, err_hist, stats, ws, rsc, gsc, st);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   cudaError_t e =
       (fmt == kInt4) ? launch_fit_t<kInt4>(W, N, K, I, scales, g, S, iters, flags, T, err_hist,
                                            stats, ws, gsc, st)
@@ -1359,15 +1996,16 @@ static cudaError_t launch_fit_sharded_t(const uint16_t* W, int64_t N, int64_t K,
                                         int iters, uint32_t flags, float* T, double* err_hist,
                                         aaac_stats* stats, void* ws, const float* gsc,
                                         Reducer& red, cudaStream_t st) {
-  FitPassFn kern;
-  const cudaError_t attr = fit_kernel<FMT, false>(S, &kern);
+  FitRoundFn kern;
+  const cudaError_t attr = round_kernel<FMT>(S, &kern);
   if (attr != cudaSuccess) return attr;
+  float2* rsc = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(ws) + fit_ctl_bytes());
   const FitPlan pp = fit_plan(N, K, M_total, (flags & AAAC_CONCURRENT) != 0);
   const PassPlan pprep = plan_pass(N, K);
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
-                                                   pprep.ncb, pprep.rows_per_chunk, gsc);
+                                                   pprep.ncb, pprep.rows_per_chunk, gsc, rsc);
   shard_maxima<<<1, 32, 0, st>>>(ctl, 0);
   int launches = 3;
   if (!red.run(ctl->shard_max, 3, AAAC_REDUCE_MAX_I64, st)) return cudaGetLastError();
@@ -1378,10 +2016,9 @@ static cudaError_t launch_fit_sharded_t(const uint16_t* W, int64_t N, int64_t K,
   launches += 2;
   const float tau = choice_tau(S);
   for (int it = 0; it < iters; it++) {
-    kern<<<pp.blocks, kFitThreads, smem_bytes(false), st>>>(
-        W, (int)N, (int)K, I, scales, g, S, flags, ctl, pp.cpc, pp.items, pp.max_items, tau,
-        PackOut{nullptr, nullptr, nullptr, nullptr}, RoundOut{nullptr, nullptr, nullptr, it}, gsc,
-        0);
+    kern<<<pp.blocks, kFitThreads, kRoundSmem, st>>>(
+        W, (int)N, (int)K, I, (const float2*)rsc, g, S, flags, ctl, pp.cpc, pp.items,
+        pp.max_items, tau, RoundOut{nullptr, nullptr, nullptr, it}, gsc, 0);
     if (!red.run(&ctl->bins[0][0][0], kShardSums, AAAC_REDUCE_SUM_I64, st)) break;
     shard_round_end<<<1, kFitThreads, 0, st>>>(ctl, flags, RoundOut{err_hist, T, stats, it},
                                                pp.blocks * kFitWarps, pp.cpc, pp.items, gsc, FMT);
@@ -1485,6 +2122,7 @@ pack_setup(FitCtl* ctl, const float* T_user, int64_t M, int n, uint16_t* T_bf16,
     const double gs = gsc ? (double)*gsc : 1.0;  // the pack's error is in weight space
     ctl->twoLe = objective_scale(ctl, M, gs * gs);
     ctl->err_acc = 0ull;
+    ctl->err_fine = 0ull;
     tb.la = bucket_scale(ctl);
   }
   if (threadIdx.x < 32) sT[threadIdx.x >> 4][threadIdx.x & 15] = T_user[threadIdx.x];
@@ -1527,10 +2165,10 @@ static cudaError_t launch_pack_t(const uint16_t* W, int64_t N, int64_t K, const 
   const FitPlan pp = fit_plan(N, K, N * K, (flags & AAAC_CONCURRENT) != 0);
   const PassPlan pprep = plan_pass(N, K);
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
-  uint8_t* cbytes = reinterpret_cast<uint8_t*>(ws) + fit_ws_bytes(N, K);
+  uint8_t* cbytes = reinterpret_cast<uint8_t*>(ws) + fit_ctl_bytes();
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
-                                                   pprep.ncb, pprep.rows_per_chunk, gsc);
+                                                   pprep.ncb, pprep.rows_per_chunk, gsc, nullptr);
   pack_setup<<<1, kFitThreads, 0, st>>>(ctl, T, N * K, ncodes(FMT), T_bf16,
                                         pp.blocks * kFitWarps, pp.cpc, pp.items,
                                         FMT == kNvfp4G ? gsc : nullptr);
@@ -1566,10 +2204,10 @@ static cudaError_t launch_pack_sharded_t(const uint16_t* W, int64_t N, int64_t K
   const FitPlan pp = fit_plan(N, K, M_total, (flags & AAAC_CONCURRENT) != 0);
   const PassPlan pprep = plan_pass(N, K);
   FitCtl* ctl = reinterpret_cast<FitCtl*>(ws);
-  uint8_t* cbytes = reinterpret_cast<uint8_t*>(ws) + fit_ws_bytes(N, K);
+  uint8_t* cbytes = reinterpret_cast<uint8_t*>(ws) + fit_ctl_bytes();
   cudaMemsetAsync(ctl, 0, sizeof(FitCtl), st);
   fit_prep<FMT><<<pprep.blocks, kThreads, 0, st>>>(W, (int)N, (int)K, I, scales, g, ctl,
-                                                   pprep.ncb, pprep.rows_per_chunk, gsc);
+                                                   pprep.ncb, pprep.rows_per_chunk, gsc, nullptr);
   shard_maxima<<<1, 32, 0, st>>>(ctl, 0);
   int launches = 2;
   if (red.run(ctl->shard_max, 3, AAAC_REDUCE_MAX_I64, st)) {
@@ -1588,7 +2226,7 @@ static cudaError_t launch_pack_sharded_t(const uint16_t* W, int64_t N, int64_t K
       pack_bits<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(cbytes, N, KS, choice_bits);
       launches++;
     }
-    if (red.run(&ctl->err_acc, 1, AAAC_REDUCE_SUM_I64, st)) {
+    if (red.run(&ctl->err_acc, 2, AAAC_REDUCE_SUM_I64, st)) {  // err_acc, err_fine
       shard_pack_end<<<1, 32, 0, st>>>(ctl, err_final);
       launches++;
     }

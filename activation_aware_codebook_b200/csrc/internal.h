@@ -34,7 +34,8 @@ PassPlan plan_pass(int64_t N, int64_t K, int target_blocks = 148 * 4, int seg_co
 size_t fit_ctl_bytes();
 size_t init_ctl_bytes();
 size_t pack_extra_bytes(int64_t N, int64_t K, int S);
-size_t fit_ws_bytes(int64_t N, int64_t K);
+// the fit's workspace: control block + the (s, 1/s_eff) pair of every scale group
+size_t fit_ws_bytes(int64_t N, int64_t K, int g);
 // the fit/pack launch plan: blocks, strips, items per strip, rows per item,
 // items per warp
 void fit_launch_plan(int64_t N, int64_t K, int64_t M_total, uint32_t flags, int32_t out[5]);
@@ -53,10 +54,12 @@ cudaError_t launch_importance(const uint16_t* X, int64_t T, int64_t K, int64_t l
 // ignored for the other formats.
 cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* scales,
                         float* T, void* ws, float* gs_out, cudaStream_t st);
+// rsc: N * K/g float2 of workspace for the scale pairs of fit_round (NULL:
+// the rounds run fit_pass, with only the control block in ws)
 cudaError_t launch_fit(const uint16_t* W, int64_t N, int64_t K, const float* I,
                        const void* scales, int fmt, int g, int S, int iters, uint32_t flags,
-                       float* T, double* err_hist, aaac_stats* stats, void* ws, const float* gsc,
-                       cudaStream_t st);
+                       float* T, double* err_hist, aaac_stats* stats, void* ws, float2* rsc,
+                       const float* gsc, cudaStream_t st);
 cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const float* I,
                         const void* scales, int fmt, int g, int S, uint32_t flags, const float* T,
                         uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,

@@ -353,6 +353,56 @@ def fit_alone_ms(blk, lin, reps=5):
     return statistics.median(times[1:])
 
 
+def timed_ms(fn, reps=5):
+    """Median CUDA-event time of fn() on the current stream, after one warm-up."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    for _ in range(reps + 1):
+        torch.cuda.synchronize()
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times[1:])
+
+
+def other_kernels(blk, wl, probe, peak):
+    """The importance pass over the probe's activations and the probe's pack,
+    each timed alone: algorithmic GB/s against the HBM peak.  Importance: 2 B
+    per X element.  Pack (prep pass, setup, final assign and pack, choice
+    bits): W read twice, the codes (0.5 B/weight), the scales read and the
+    tagged scales and choice bits written."""
+    bb = blk.bb
+    X = blk.Xs[probe.x_key]
+    I = torch_zeros_like(blk.I[probe.x_key])
+    imp_ms = timed_ms(lambda: bb.importance(X, I=I, ws=blk.kws[probe.x_key]))
+    imp_bytes = X.shape[0] * X.shape[1] * 2
+    W = blk.Ws[probe.name]
+    cfg = dataclasses.replace(blk.cfgs[probe.name], flags=0)  # alone: full grid
+    out = blk.out[probe.name]
+    pack_ms = timed_ms(lambda: bb.pack(W, blk.I[probe.x_key], blk.scales[probe.name],
+                                       blk.T[probe.name], cfg, ws=blk.ws, out=out))
+    sb = 2 if wl.fmt == bb.INT4 else 1
+    n, k = probe.N, probe.K
+    pack_bytes = (2 * n * k * 2 + n * k // 2 + 2 * n * (k // wl.g) * sb
+                  + (n * ((k // wl.S + 7) // 8) if wl.S != wl.g else 0))
+    return {
+        "importance": {"tokens": X.shape[0], "K": X.shape[1], "ms": imp_ms,
+                       "GB_per_s": imp_bytes / (imp_ms * 1e-3) / 1e9,
+                       "frac": imp_bytes / (imp_ms * 1e-3) / 1e9 / peak},
+        "pack": {"layer": f"{probe.name} {n}x{k}", "ms": pack_ms,
+                 "GB_per_s": pack_bytes / (pack_ms * 1e-3) / 1e9,
+                 "frac": pack_bytes / (pack_ms * 1e-3) / 1e9 / peak},
+    }
+
+
+def torch_zeros_like(t):
+    import torch
+    return torch.zeros_like(t)
+
+
 def per_linear_fit(blk, wl, peak):
     """Every linear's fit timed alone (prep and setup subtracted): per round,
     weights/s and algorithmic GB/s against the HBM peak.  W of every linear
@@ -363,7 +413,9 @@ def per_linear_fit(blk, wl, peak):
     for l in wl.linears:
         it_ms = (fit_alone_ms(blk, l) - fit_setup_ms(blk, l)) / wl.iters
         b = l.N * l.K * 2 + l.N * (l.K // wl.g) * scale_bytes + l.K * 4
+        st = bb.decode_stats(blk.st[l.name])  # the fit just timed alone
         rows[l.name] = {"shape": f"{l.N}x{l.K}", "round_us": it_ms * 1e3,
+                        "near_ties": st["near_ties"], "exact_groups": st["exact_groups"],
                         "weights_per_s": l.N * l.K / (it_ms * 1e-3),
                         "GB_per_s": b / (it_ms * 1e-3) / 1e9,
                         "frac": b / (it_ms * 1e-3) / 1e9 / peak,
@@ -448,6 +500,7 @@ def run_ours(args, rank, local_rank, world):
                      "source": "warp instructions from the committed ncu capture"}
 
     per_linear = None if args.no_per_linear else per_linear_fit(blk, wl, peak)
+    kernels = other_kernels(blk, wl, probe, peak)
 
     # end to end through the C ABI with host buffers (pinned), copies timed
     e2e = None
@@ -473,7 +526,7 @@ def run_ours(args, rank, local_rank, world):
                                                       "the linears of a block on concurrent streams",
                        "l2": "inputs larger than L2 (activations %.1f GiB per step)" % (
                            sum(x.numel() * 2 for x in Xs.values()) / 2 ** 30)},
-            "roofline": {"kernel": "fit_pass (one fit round; refine fused in its last block)",
+            "roofline": {"kernel": "fit_round (one fit round; refine fused in its last block)",
                          "layer": f"{probe.name} {probe.N}x{probe.K}",
                          "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
@@ -481,6 +534,7 @@ def run_ours(args, rank, local_rank, world):
                          "round_ms": iter_ms, "timing": "the probe's fit alone, CUDA events",
                          "round_ms_in_step": iter_in_step_ms, "issue": issue},
             **({"per_linear_fit": per_linear} if per_linear is not None else {}),
+            "other_kernels": kernels,
             "gpu_launches": int(launches),
             "clocks": clocks,
         }

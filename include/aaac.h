@@ -295,7 +295,7 @@ aaac_status aaac_awq_fit(const void* W, int64_t N, int64_t K, const float* I, in
  * the result does not depend on the reduction's order: every shard ends
  * with the tables of the unsharded call on the whole layer, bit for bit,
  * and packs its own rows exactly as the unsharded pack would.  Per fit round
- * the exchange is 68 int64 values (544 bytes).
+ * the exchange is 69 int64 values (552 bytes).
  *   op AAAC_REDUCE_SUM_I64 / MAX_I64: int64 elements; SUM_I32 / MAX_I32: int32.
  *   The callback returns 0 on success; any other value stops the call, which
  *   returns AAAC_ERR_COLLECTIVE (work already enqueued stays enqueued).

@@ -45,9 +45,12 @@ def test_workspace_size_monotone(lib):
     small = binding.workspace_size(cfg, 256, 512, 128)
     big = binding.workspace_size(cfg, 14336, 4096, 262144)
     assert 256 <= small < big
-    # the pack's choice bytes are part of it for S < g
-    assert binding.workspace_size(cfg, 4096, 4096) > binding.workspace_size(
-        binding.Config(binding.INT4, 128, 128, 20), 4096, 4096)
+    # the fit keeps an fp32 (s, 1/s) pair per scale group, the pack one choice
+    # byte per selection group (S < g): the workspace holds either
+    assert binding.workspace_size(cfg, 4096, 4096) >= 4096 * (4096 // 128) * 8
+    assert binding.workspace_size(cfg, 4096, 4096) >= 4096 * (4096 // 16)
+    nv = binding.Config(binding.NVFP4, 16, 16, 20)
+    assert binding.workspace_size(nv, 4096, 4096) >= 4096 * (4096 // 16) * 8
     assert lib.aaac_workspace_size(None, 0, 0, 0) == 256
 
 
