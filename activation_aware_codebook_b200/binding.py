@@ -27,7 +27,11 @@ STATUS = {0: "AAAC_OK", 1: "AAAC_ERR_INVALID_ARG", 2: "AAAC_ERR_SHAPE", 3: "AAAC
           4: "AAAC_ERR_UNSUPPORTED", 5: "AAAC_ERR_CUDA", 6: "AAAC_ERR_WORKSPACE",
           7: "AAAC_ERR_TIMEOUT", 8: "AAAC_ERR_COLLECTIVE"}
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaaac.so")
+# AAAC_CHECKED=1 selects the debugging build with device-side index checks
+# (built by `python -m activation_aware_codebook_b200.csrc.build --checks`).
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libaaac_checked.so" if os.environ.get("AAAC_CHECKED") == "1"
+                        else "libaaac.so")
 
 EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaac_fit_layer",
            "aaac_pack", "aaac_last_error", "aaac_version", "aaac_kernel_launches",
@@ -35,7 +39,8 @@ EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaa
            "aaac_device_timeouts", "aaac_awq_prescale", "aaac_awq_workspace_size",
            "aaac_awq_fit", "aaac_init_codebooks_sharded", "aaac_fit_layer_sharded",
            "aaac_pack_sharded", "aaac_linear_workspace_size", "aaac_linear_ws",
-           "aaac_fit_launch_plan")
+           "aaac_fit_launch_plan", "aaac_inject_fault", "aaac_device_checks",
+           "aaac_checked_build")
 
 
 # reduction callback of the row-sharded calls: (user, buf, count, op, stream) -> 0 | error
@@ -127,6 +132,12 @@ def load(path: str = LIB_PATH):
     L.aaac_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     L.aaac_kernel_launches.restype = ctypes.c_uint64
     L.aaac_kernel_launches.argtypes = []
+    L.aaac_inject_fault.restype = ctypes.c_int
+    L.aaac_inject_fault.argtypes = [ctypes.c_char_p]
+    L.aaac_device_checks.restype = ctypes.c_int
+    L.aaac_device_checks.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    L.aaac_checked_build.restype = ctypes.c_int
+    L.aaac_checked_build.argtypes = []
     L.aaac_fit_launch_plan.restype = ctypes.c_int
     L.aaac_fit_launch_plan.argtypes = [P, i64, i64, i64, ctypes.POINTER(ctypes.c_int32)]
     L.aaac_awq_prescale.restype = ctypes.c_int
@@ -149,6 +160,19 @@ def load(path: str = LIB_PATH):
     L.aaac_pack_sharded.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, P, P, P, R, P, P, sz, P]
     _lib = L
     return L
+
+
+def device_checks() -> int:
+    """The first failed device-side check of a checked build (0: none)."""
+    v = ctypes.c_uint32(0)
+    _check(load().aaac_device_checks(ctypes.byref(v)))
+    return int(v.value)
+
+
+def inject_fault(kind: Optional[str]) -> None:
+    """Test hook: the next call that would launch work fails on the host
+    ("alloc", "launch" or "sync"; None disarms); see aaac_inject_fault."""
+    _check(load().aaac_inject_fault(None if kind is None else kind.encode()))
 
 
 def kernel_launches() -> int:

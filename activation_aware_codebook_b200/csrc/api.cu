@@ -4,10 +4,14 @@
 // invalid call leaves all outputs untouched.
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 #include <string>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -84,6 +88,48 @@ aaac_status check_ws(void* ws, size_t have, size_t need) {
   if (!aligned16(ws)) return fail(AAAC_ERR_ALIGN, "workspace is not 16-byte aligned");
   if (have < need) return fail(AAAC_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", have, need);
   return AAAC_OK;
+}
+
+// NVTX range around a call (named in profiler timelines; no cost without a tool).
+struct CallScope {
+  explicit CallScope(const char* name) { nvtxRangePushA(name); }
+  ~CallScope() { nvtxRangePop(); }
+  CallScope(const CallScope&) = delete;
+  CallScope& operator=(const CallScope&) = delete;
+};
+
+// Host-side fault injection, for tests of callers' error paths: one fault is
+// armed by AAAC_FAULT=alloc|launch|sync in the environment when the library
+// first runs a call, or by aaac_inject_fault().  The next call that would
+// launch work then returns the matching status after its argument checks,
+// before anything reaches the GPU, and leaves every output untouched.
+enum { kFaultNone = 0, kFaultAlloc = 1, kFaultLaunch = 2, kFaultSync = 3 };
+std::atomic<int> g_fault{kFaultNone};
+std::once_flag g_fault_env;
+
+int fault_kind(const char* k) {
+  if (!k || !*k) return kFaultNone;
+  if (!strcmp(k, "alloc")) return kFaultAlloc;
+  if (!strcmp(k, "launch")) return kFaultLaunch;
+  if (!strcmp(k, "sync")) return kFaultSync;
+  return -1;
+}
+
+aaac_status take_fault() {
+  std::call_once(g_fault_env, [] {
+    const int k = fault_kind(getenv("AAAC_FAULT"));
+    if (k > 0) g_fault.store(k);
+  });
+  switch (g_fault.exchange(kFaultNone)) {
+    case kFaultAlloc:
+      return fail(AAAC_ERR_WORKSPACE, "injected fault: workspace allocation failed");
+    case kFaultLaunch:
+      return fail(AAAC_ERR_CUDA, "injected fault: kernel launch failed");
+    case kFaultSync:
+      return fail(AAAC_ERR_CUDA, "injected fault: stream synchronisation failed");
+    default:
+      return AAAC_OK;
+  }
 }
 
 aaac_status from_cuda(cudaError_t e, const char* where) {
@@ -172,6 +218,7 @@ size_t aaac_workspace_size(const aaac_config* cfg, int64_t N, int64_t K, int64_t
 
 aaac_status aaac_importance(const void* X, int64_t T, int64_t K, int64_t ldx, uint32_t flags,
                             float* I, void* ws, size_t ws_bytes, void* stream) {
+  CallScope cs_("aaac_importance");
   CHECK(check_ptr(X, "X"));
   CHECK(check_ptr(I, "I"));
   if (T <= 0 || K <= 0) return fail(AAAC_ERR_SHAPE, "T and K must be positive");
@@ -181,6 +228,7 @@ aaac_status aaac_importance(const void* X, int64_t T, int64_t K, int64_t ldx, ui
     return fail(AAAC_ERR_SHAPE, "K or T out of range");
   if (flags & ~3u) return fail(AAAC_ERR_INVALID_ARG, "unknown importance flags 0x%x", flags);
   CHECK(check_ws(ws, ws_bytes, aaac::plan_importance(T, K).total));
+  CHECK(take_fault());
   return from_cuda(aaac::launch_importance(reinterpret_cast<const uint16_t*>(X), T, K, ldx, flags,
                                            I, ws, (cudaStream_t)stream),
                    "aaac_importance");
@@ -189,12 +237,14 @@ aaac_status aaac_importance(const void* X, int64_t T, int64_t K, int64_t ldx, ui
 aaac_status aaac_init_codebooks(const void* W, int64_t N, int64_t K, const aaac_config* cfg,
                                 void* scales, float* T, void* ws, size_t ws_bytes,
                                 void* stream) {
+  CallScope cs_("aaac_init_codebooks");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   CHECK(check_ptr(W, "W"));
   CHECK(check_ptr(scales, "scales"));
   CHECK(check_ptr(T, "T"));
   CHECK(check_ws(ws, ws_bytes, aaac::init_ctl_bytes()));
+  CHECK(take_fault());
   return from_cuda(aaac::launch_init(reinterpret_cast<const uint16_t*>(W), N, K, cfg->fmt, cfg->g,
                                      scales, T, ws, cfg->global_scale, (cudaStream_t)stream),
                    "aaac_init_codebooks");
@@ -204,6 +254,7 @@ aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
                            const void* scales, const aaac_config* cfg, float* T,
                            double* err_hist, aaac_stats* stats, void* ws, size_t ws_bytes,
                            void* stream) {
+  CallScope cs_("aaac_fit_layer");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   CHECK(check_ptr(W, "W"));
@@ -214,6 +265,7 @@ aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
   CHECK(check_ptr(stats, "stats", false));
   CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K, cfg->g)));
   float2* rsc = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(ws) + aaac::fit_ctl_bytes());
+  CHECK(take_fault());
   return from_cuda(aaac::launch_fit(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
                                     cfg->fmt, cfg->g, cfg->S, cfg->iters, cfg->flags, T, err_hist,
                                     stats, ws, rsc, cfg->global_scale, (cudaStream_t)stream),
@@ -223,6 +275,7 @@ aaac_status aaac_fit_layer(const void* W, int64_t N, int64_t K, const float* I,
 aaac_status aaac_fit_layer_fixed_scratch(const void* W, int64_t N, int64_t K, const float* I,
                                          const void* scales, const aaac_config* cfg, float* T,
                                          double* err_hist, aaac_stats* stats, void* stream) {
+  CallScope cs_("aaac_fit_layer_fixed_scratch");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   CHECK(check_ptr(W, "W"));
@@ -240,6 +293,7 @@ aaac_status aaac_fit_layer_fixed_scratch(const void* W, int64_t N, int64_t K, co
                 "scratch holds %zu; call aaac_fit_layer with a workspace instead",
                 (long long)N, (long long)K, need, aaac::fixed_scratch_bytes());
   void* ws = nullptr;
+  CHECK(take_fault());
   cudaError_t e = aaac::fixed_scratch_ptr(&ws);
   if (e != cudaSuccess) return from_cuda(e, "aaac_fit_layer_fixed_scratch: scratch address");
   return from_cuda(aaac::launch_fit(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
@@ -252,6 +306,7 @@ aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const
                       const aaac_config* cfg, const float* T, uint16_t* T_bf16, uint8_t* codes,
                       void* scales_tagged, uint8_t* choice_bits, double* err_final, void* ws,
                       size_t ws_bytes, void* stream) {
+  CallScope cs_("aaac_pack");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   CHECK(check_ptr(W, "W"));
@@ -264,6 +319,7 @@ aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const
   CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
   CHECK(check_ptr(err_final, "err_final", false));
   CHECK(check_ws(ws, ws_bytes, aaac::fit_ctl_bytes() + aaac::pack_extra_bytes(N, K, cfg->S)));
+  CHECK(take_fault());
   return from_cuda(aaac::launch_pack(reinterpret_cast<const uint16_t*>(W), N, K, I, scales,
                                      cfg->fmt, cfg->g, cfg->S, cfg->flags, T, T_bf16, codes,
                                      scales_tagged, choice_bits, err_final, ws, cfg->global_scale,
@@ -274,6 +330,7 @@ aaac_status aaac_pack(const void* W, int64_t N, int64_t K, const float* I, const
 aaac_status aaac_dequant(const uint8_t* codes, const void* scales_tagged,
                          const uint8_t* choice_bits, const uint16_t* T_bf16, int64_t N, int64_t K,
                          const aaac_config* cfg, uint16_t* W_hat, void* stream) {
+  CallScope cs_("aaac_dequant");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   CHECK(check_ptr(codes, "codes"));
@@ -281,6 +338,7 @@ aaac_status aaac_dequant(const uint8_t* codes, const void* scales_tagged,
   CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
   CHECK(check_ptr(T_bf16, "T_bf16"));
   CHECK(check_ptr(W_hat, "W_hat"));
+  CHECK(take_fault());
   return from_cuda(aaac::launch_dequant(codes, scales_tagged, choice_bits, T_bf16, N, K, cfg->fmt,
                                         cfg->g, cfg->S, W_hat, cfg->global_scale,
                                         (cudaStream_t)stream),
@@ -291,6 +349,7 @@ aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* co
                         const void* scales_tagged, const uint8_t* choice_bits,
                         const uint16_t* T_bf16, int64_t N, int64_t K, const aaac_config* cfg,
                         float* Y, void* stream) {
+  CallScope cs_("aaac_linear");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   if (M < 1 || M > ((int64_t)1 << 20))
@@ -306,6 +365,7 @@ aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* co
   CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
   CHECK(check_ptr(T_bf16, "T_bf16"));
   CHECK(check_ptr(Y, "Y"));
+  CHECK(take_fault());
   return from_cuda(aaac::launch_linear(reinterpret_cast<const uint16_t*>(X), M, ldx, codes,
                                        scales_tagged, choice_bits, T_bf16, N, K, cfg->fmt,
                                        cfg->g, cfg->S, Y, cfg->global_scale, (cudaStream_t)stream),
@@ -315,6 +375,7 @@ aaac_status aaac_linear(const void* X, int64_t M, int64_t ldx, const uint8_t* co
 aaac_status aaac_awq_prescale(const void* W, int64_t N, int64_t K, const float* I,
                               int64_t tokens, int alpha16, float* c, float* I_scaled,
                               void* W_scaled, void* stream) {
+  CallScope cs_("aaac_awq_prescale");
   if (N <= 0 || K <= 0) return fail(AAAC_ERR_SHAPE, "N and K must be positive");
   if (K % 8) return fail(AAAC_ERR_ALIGN, "K=%lld is not a multiple of 8", (long long)K);
   if (N > INT32_MAX || K > INT32_MAX || N * K >= ((int64_t)1 << 31))
@@ -328,6 +389,7 @@ aaac_status aaac_awq_prescale(const void* W, int64_t N, int64_t K, const float* 
   CHECK(check_ptr(c, "c"));
   CHECK(check_ptr(I_scaled, "I_scaled"));
   CHECK(check_ptr(W_scaled, "W_scaled"));
+  CHECK(take_fault());
   return from_cuda(aaac::launch_awq_prescale(reinterpret_cast<const uint16_t*>(W), N, K, I,
                                              tokens, alpha16, c, I_scaled,
                                              reinterpret_cast<uint16_t*>(W_scaled),
@@ -345,6 +407,7 @@ aaac_status aaac_awq_fit(const void* W, int64_t N, int64_t K, const float* I, in
                          uint16_t* T_bf16, uint8_t* codes, void* scales_tagged,
                          uint8_t* choice_bits, double* err_final, double* err_alpha,
                          int32_t* best, void* ws, size_t ws_bytes, void* stream) {
+  CallScope cs_("aaac_awq_fit");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   if (tokens <= 0) return fail(AAAC_ERR_SHAPE, "tokens must be positive (%lld)", (long long)tokens);
@@ -389,6 +452,7 @@ aaac_status aaac_awq_fit(const void* W, int64_t N, int64_t K, const float* I, in
   void* dst[6] = {codes, scales_tagged, T_bf16, c, choice_bits, cfg->global_scale};
   const size_t bytes[6] = {(size_t)(N * K / 2), (size_t)(N * G) * es, 2 * 16 * 2, (size_t)K * 4,
                            bits ? (size_t)N * ((K / cfg->S + 7) / 8) : 0, gs ? sizeof(float) : 0};
+  CHECK(take_fault());
   for (int i = 0; i < n_alpha; i++) {
     cudaError_t e = aaac::launch_awq_prescale(reinterpret_cast<const uint16_t*>(W), N, K, I,
                                               tokens, alpha16[i], cc, Is, Ws, st);
@@ -422,6 +486,7 @@ aaac_status aaac_init_codebooks_sharded(const void* W, int64_t N, int64_t K, int
                                         const aaac_config* cfg, void* scales, float* T,
                                         aaac_reduce_fn reduce, void* user, void* ws,
                                         size_t ws_bytes, void* stream) {
+  CallScope cs_("aaac_init_codebooks_sharded");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   CHECK(check_shards(N, K, N_total, cfg, reduce));
@@ -429,6 +494,7 @@ aaac_status aaac_init_codebooks_sharded(const void* W, int64_t N, int64_t K, int
   CHECK(check_ptr(scales, "scales"));
   CHECK(check_ptr(T, "T"));
   CHECK(check_ws(ws, ws_bytes, aaac::init_ctl_bytes()));
+  CHECK(take_fault());
   aaac::Reducer red{reduce, user, false};
   const cudaError_t e = aaac::launch_init_sharded(reinterpret_cast<const uint16_t*>(W), N, K,
                                                   N_total * K, cfg->fmt, cfg->g, scales, T, ws,
@@ -442,6 +508,7 @@ aaac_status aaac_fit_layer_sharded(const void* W, int64_t N, int64_t K, int64_t 
                                    float* T, double* err_hist, aaac_stats* stats,
                                    aaac_reduce_fn reduce, void* user, void* ws, size_t ws_bytes,
                                    void* stream) {
+  CallScope cs_("aaac_fit_layer_sharded");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   CHECK(check_shards(N, K, N_total, cfg, reduce));
@@ -452,6 +519,7 @@ aaac_status aaac_fit_layer_sharded(const void* W, int64_t N, int64_t K, int64_t 
   CHECK(check_ptr(err_hist, "err_hist", false));
   CHECK(check_ptr(stats, "stats", false));
   CHECK(check_ws(ws, ws_bytes, aaac::fit_ws_bytes(N, K, cfg->g)));
+  CHECK(take_fault());
   aaac::Reducer red{reduce, user, false};
   const cudaError_t e = aaac::launch_fit_sharded(
       reinterpret_cast<const uint16_t*>(W), N, K, N_total * K, I, scales, cfg->fmt, cfg->g,
@@ -467,6 +535,7 @@ aaac_status aaac_pack_sharded(const void* W, int64_t N, int64_t K, int64_t N_tot
                               void* scales_tagged, uint8_t* choice_bits, double* err_final,
                               aaac_reduce_fn reduce, void* user, void* ws, size_t ws_bytes,
                               void* stream) {
+  CallScope cs_("aaac_pack_sharded");
   CHECK(check_cfg(cfg));
   CHECK(check_layer(N, K, cfg));
   CHECK(check_shards(N, K, N_total, cfg, reduce));
@@ -480,6 +549,7 @@ aaac_status aaac_pack_sharded(const void* W, int64_t N, int64_t K, int64_t N_tot
   CHECK(check_ptr(choice_bits, "choice_bits", cfg->S != cfg->g));
   CHECK(check_ptr(err_final, "err_final", false));
   CHECK(check_ws(ws, ws_bytes, aaac::fit_ctl_bytes() + aaac::pack_extra_bytes(N, K, cfg->S)));
+  CHECK(take_fault());
   aaac::Reducer red{reduce, user, false};
   const cudaError_t e = aaac::launch_pack_sharded(
       reinterpret_cast<const uint16_t*>(W), N, K, N_total * K, I, scales, cfg->fmt, cfg->g,
@@ -502,6 +572,7 @@ aaac_status aaac_linear_ws(const void* X, int64_t M, int64_t ldx, const uint8_t*
                            const void* scales_tagged, const uint8_t* choice_bits,
                            const uint16_t* T_bf16, int64_t N, int64_t K, const aaac_config* cfg,
                            float* Y, void* ws, size_t ws_bytes, void* stream) {
+  CallScope cs_("aaac_linear_ws");
   const size_t need = aaac_linear_workspace_size(cfg, M, N, K);
   if (need == 0 || !ws || ws_bytes < need || !aligned16(ws))
     return aaac_linear(X, M, ldx, codes, scales_tagged, choice_bits, T_bf16, N, K, cfg, Y, stream);
@@ -521,6 +592,7 @@ aaac_status aaac_linear_ws(const void* X, int64_t M, int64_t ldx, const uint8_t*
   CHECK(check_ptr(T_bf16, "T_bf16"));
   CHECK(check_ptr(Y, "Y"));
   uint16_t* Wh = static_cast<uint16_t*>(ws);
+  CHECK(take_fault());
   cudaError_t e = aaac::launch_dequant(codes, scales_tagged, choice_bits, T_bf16, N, K, cfg->fmt,
                                        cfg->g, cfg->S, Wh, cfg->global_scale,
                                        (cudaStream_t)stream);
@@ -529,6 +601,33 @@ aaac_status aaac_linear_ws(const void* X, int64_t M, int64_t ldx, const uint8_t*
                                       (cudaStream_t)stream);
   if (e == cudaSuccess) aaac::count_launches(1);
   return from_cuda(e, "aaac_linear_ws");
+}
+
+aaac_status aaac_device_checks(uint32_t* flag) {
+  if (!flag) return fail(AAAC_ERR_INVALID_ARG, "flag is NULL");
+  unsigned int vf = 0, vi = 0;
+  cudaError_t e = aaac::fit_check_flag(&vf);
+  if (e == cudaSuccess) e = aaac::init_check_flag(&vi);
+  if (e != cudaSuccess) return from_cuda(e, "aaac_device_checks");
+  *flag = vf ? vf : vi;
+  return ok();
+}
+
+int aaac_checked_build(void) {
+#ifdef AAAC_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+aaac_status aaac_inject_fault(const char* kind) {
+  const int k = fault_kind(kind);
+  if (k < 0)
+    return fail(AAAC_ERR_INVALID_ARG, "unknown fault kind '%s' (alloc, launch, sync or empty)",
+                kind);
+  g_fault.store(k);
+  return ok();
 }
 
 aaac_status aaac_device_timeouts(uint32_t* flag) {

@@ -15,6 +15,29 @@
 
 namespace aaac {
 
+// Checked builds (compiled with -DAAAC_CHECKS, `build.py --checks`): kernels
+// test the indices they compute and record the first failed check -- its
+// code in the low byte, the offending value above it -- in g_check_fail,
+// which aaac_device_checks reads.  No trap: the kernel goes on (a debugging
+// aid for cases known to stay in bounds).  In normal builds the checks
+// compile to nothing and the flag stays 0.
+#ifdef AAAC_CHECKS
+// one flag per translation unit (the library is built without relocatable
+// device code); each unit that checks exposes it through a reader
+static __device__ unsigned int g_check_fail = 0;
+static inline cudaError_t read_check_flag(unsigned int* out) {
+  return cudaMemcpyFromSymbol(out, g_check_fail, sizeof(unsigned int));
+}
+#define AAAC_CHECK(cond, code, value)                                                   \
+  do {                                                                                  \
+    if (!(cond)) atomicCAS(&::aaac::g_check_fail, 0u, ((unsigned)(value) << 8) | (code)); \
+  } while (0)
+#else
+#define AAAC_CHECK(cond, code, value) \
+  do {                                \
+  } while (0)
+#endif
+
 constexpr int kInt4 = 0;
 constexpr int kNvfp4 = 1;
 constexpr int kNvfp4G = 2;            // NVFP4 with a per-tensor fp32 scale

@@ -9,14 +9,18 @@
 //   core mechanism 4  alternating assign (nearest entry, Voronoi cells) and
 //                     refine (activation-weighted centroid of each cell).
 //
-// One fit round is ONE launch of fit_pass<false>: a streaming pass over W whose
-// last block to finish (atomic ticket, no waiting) does the refine, sorts the
-// books, rebuilds the tables and records the error.  Per block: 3 warps; a warp
-// covers 512 columns of a row, 16 per lane (32 bytes), and walks the rows of
-// its work items with a 2-deep cp.async ring.  The grid is one wave (4 blocks,
-// 12 warps, per SM, bounded by the refine bins' shared memory: 16 KB a warp;
-// the last block's table rebuild borrows the idle ring for its scratch, so
-// the pass holds almost no static shared memory).
+// One fit round is ONE launch of fit_round: a streaming pass over W whose last
+// block to finish (atomic ticket, no waiting) does the refine, sorts the books,
+// rebuilds the tables and records the error.  Per block: 3 warps; a warp covers
+// 512 columns of a row, 16 per lane (32 bytes), and walks the rows of its work
+// items with a 2-slot ring filled by cp.async.bulk (one lane issues a row's
+// 1 KB copy on an mbarrier).  The grid is one wave (4 blocks, 12 warps, per SM,
+// bounded by the refine bins' shared memory: 16 KB a warp; the last block's
+// table rebuild borrows the idle rings for its scratch).  fit_pass<PACK> is the
+// pack's pass (final assign, codes, choice bits, weight-space error) on the
+// same work distribution with a cp.async ring; fit_pass<fit> is kept as the
+// round of the fixed-scratch entry point, which has no room for the per-fit
+// scale pairs fit_round reads.
 //
 // Nearest entry in both books at once (exact):
 //   the midpoint thresholds of both books, merged and deduplicated (at most
@@ -1284,6 +1288,14 @@ constexpr int kRStages = 2;                  // ring rows per warp
 constexpr uint64_t kRoundWaitNs = 2000000000ull;
 
 __device__ unsigned int g_fit_timeout = 0;
+cudaError_t fit_check_flag(unsigned int* out) {
+#ifdef AAAC_CHECKS
+  return read_check_flag(out);
+#else
+  *out = 0u;
+  return cudaSuccess;
+#endif
+}
 
 struct __align__(16) RoundRing {
   unsigned char w[kRStages][kWarpCols * 2];
@@ -1362,6 +1374,7 @@ __device__ __forceinline__ void assign_row(const Tables& tb, const float2 (&u2)[
     const float2 bf = __ffma2_rn(u2[p], la2, cc2);
     const uint32_t cx = tb.mlut4[__float_as_uint(bf.x) & (kNB - 1)];
     const uint32_t cy = tb.mlut4[__float_as_uint(bf.y) & (kNB - 1)];
+    AAAC_CHECK(cx < 4u * kMerged - 4u && cy < 4u * kMerged - 4u, 5, cx | (cy << 8));
     const uint32_t mx = cx + (u2[p].x >= *reinterpret_cast<const float*>(mthr_b + cx) ? 4u : 0u);
     const uint32_t my = cy + (u2[p].y >= *reinterpret_cast<const float*>(mthr_b + cy) ? 4u : 0u);
     const float2 v0 = make_float2(*reinterpret_cast<const float*>(mv0_b + mx),
@@ -1618,6 +1631,9 @@ fit_round(const uint16_t* __restrict__ W, int N, int K, const float* __restrict_
   while (!timed_out) {  // warp-uniform
     if (fifo[cq & 7] < 0) break;
     const int r = cr;
+    AAAC_CHECK(r >= 0 && r < N, 2, r);
+    AAAC_CHECK(ccb >= 0 && ccb < ncb, 3, ccb);
+    AAAC_CHECK(tail - cq <= 8, 4, tail - cq);
     if (ccb != cur_cb) load_importance(ccb);
     if (++cr >= ce) {
       cq++;
@@ -1726,6 +1742,7 @@ fit_round(const uint16_t* __restrict__ W, int N, int K, const float* __restrict_
 #pragma unroll
     for (int i = 0; i < 16; i++) {
       const uint32_t off = __byte_perm(moffs[i], 0u, i < 8 ? sel0 : sel1);
+      AAAC_CHECK(off < (uint32_t)(32 * kCellBytes) && (off & (kCellBytes - 1)) == 0, 1, off);
       double2* bp = reinterpret_cast<double2*>(mybins + off);
       const double ud = (double)((i & 1) ? u2[i >> 1].y : u2[i >> 1].x);
       const double A = __dmul_rn(Id[i], s2L);  // exact: 24 + 16 bits

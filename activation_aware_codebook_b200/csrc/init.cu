@@ -232,6 +232,7 @@ __device__ __forceinline__ void radix_rows(const RadixArgs& a, uint32_t (*sh)[25
             hit = lo < nslots && sp[lo] == pre;
             slot = (uint32_t)lo;
           }
+          AAAC_CHECK(!hit || slot < (uint32_t)nslots, 6, slot);
           shared_add_at(sh_base, slot * 256u + ((key >> shift) & 255u), 1u, hit);
         }
       }
@@ -438,6 +439,15 @@ static void radix_pass_launch(int pass, int blocks, const RadixArgs& a, InitCtl*
                               cudaStream_t st) {
   if (pass == 0) radix_pass<FMT, true><<<blocks, kThreads, 0, st>>>(a, c);
   else radix_pass<FMT, false><<<blocks, kThreads, 0, st>>>(a, c);
+}
+
+cudaError_t init_check_flag(unsigned int* out) {
+#ifdef AAAC_CHECKS
+  return read_check_flag(out);
+#else
+  *out = 0u;
+  return cudaSuccess;
+#endif
 }
 
 cudaError_t launch_init(const uint16_t* W, int64_t N, int64_t K, int fmt, int g, void* scales,

@@ -111,6 +111,10 @@ cudaError_t launch_gemm_dequantised(const uint16_t* X, int64_t M, int64_t ldx,
                                     const uint16_t* Wh, int64_t N, int64_t K, float* Y,
                                     cudaStream_t st);
 cudaError_t gemm_timeout_flag(unsigned int* out);
+// the first failed device-side check of a checked build in the fit and the
+// init kernels (0: none, or not a checked build)
+cudaError_t fit_check_flag(unsigned int* out);
+cudaError_t init_check_flag(unsigned int* out);
 
 cudaError_t launch_awq_prescale(const uint16_t* W, int64_t N, int64_t K, const float* I,
                                 int64_t tokens, int j, float* c, float* Is, uint16_t* Wout,

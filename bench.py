@@ -110,9 +110,9 @@ def source_hash(*names):
 
 
 def committed_traffic(kernel_src_hash):
-    """DRAM bytes per fit pass from the committed ncu summary, when it was taken
-    on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "fit_pass_traffic.json")
+    """DRAM bytes per fit round from the committed ncu summary, when it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "fit_round_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)

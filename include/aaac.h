@@ -342,6 +342,26 @@ aaac_status aaac_linear_ws(const void* X, int64_t M, int64_t ldx, const uint8_t*
  * Synchronises with the device (reads a device variable). */
 aaac_status aaac_device_timeouts(uint32_t* flag);
 
+/* Debug builds: 1 when the library was compiled with AAAC_CHECKS
+ * (build.py --checks), else 0.  In such a build the fit and init kernels test
+ * the indices they compute (rows, strips, work-item FIFO depth, table cells,
+ * refine-bin offsets, radix slots) and record the first failure; *flag gets
+ * that record (the check's code in the low byte, the offending value above
+ * it), 0 when every check has held -- and always 0 in a normal build.
+ * aaac_device_checks synchronises with the device (reads a device variable). */
+int aaac_checked_build(void);
+aaac_status aaac_device_checks(uint32_t* flag);
+
+/* Test hook: arms one host-side fault (kind "alloc", "launch" or "sync"; NULL
+ * or "" disarms).  The next call that would launch work -- on any thread --
+ * returns AAAC_ERR_WORKSPACE ("alloc") or AAAC_ERR_CUDA ("launch", "sync")
+ * after its argument checks, launches nothing, touches no output, and
+ * disarms the fault.  The environment variable AAAC_FAULT with the same
+ * kinds arms one fault when the library first runs a call.  For testing a
+ * caller's error paths; nothing reaches the GPU.
+ * Errors: AAAC_ERR_INVALID_ARG for an unknown kind. */
+aaac_status aaac_inject_fault(const char* kind);
+
 /* Message describing the last failed call on the calling thread ("" after a
  * successful call).  Valid until the next call on the thread. */
 const char* aaac_last_error(void);
