@@ -826,6 +826,9 @@ def run_linear(args):
     hbm, hbm_kind = measured_peak()
     tflops_peak, tf_kind = measured_tensor_peak()
     code_bytes = N * K // 2 + N * (K // 128) * 2 + N * (K // 16 // 8)
+    # context: cuBLAS bf16 (torch.matmul) on the dequantised weights, same
+    # flush and timing, 4x the weight bytes
+    W_hat = bb.dequant(packed, cfg, N, K).view(torch.bfloat16)
     points = []
     launches0 = bb.kernel_launches()
     sampler = ClockSampler(0)
@@ -848,6 +851,17 @@ def run_linear(args):
             torch.cuda.synchronize()
             times.append(e0.elapsed_time(e1))
         ms = statistics.median(times)
+        ctimes = []
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            torch.matmul(x, W_hat.t())
+            e1.record(st)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ctimes.append(e0.elapsed_time(e1))
+        cublas_us = statistics.median(ctimes) * 1e3
         byts = code_bytes + M * K * 2 + M * N * 4
         flops = 2.0 * M * N * K
         if M <= 64:
@@ -857,9 +871,12 @@ def run_linear(args):
             roof = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": tflops_peak,
                     "peak_kind": tf_kind, "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
+        path = ("tcgen05, clusters splitting K" if M <= 64 and K % 32 == 0
+                else "gemv" if M <= 4 else "tcgen05 fused expansion" if not need
+                else "dequant + TMA-fed tcgen05")
         points.append({"tokens": M, "us": ms * 1e3, "tokens_per_s": M / (ms * 1e-3),
-                       "path": ("gemv" if M <= 4 else "tcgen05 fused expansion" if not need
-                                else "dequant + TMA-fed tcgen05"), "roofline": roof})
+                       "path": path, "roofline": roof,
+                       "cublas_bf16_dequantised_us": cublas_us})
     clocks = sampler.stop()
     launches = bb.kernel_launches() - launches0
     head = points[0]
