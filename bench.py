@@ -871,8 +871,7 @@ def run_linear(args):
             roof = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": tflops_peak,
                     "peak_kind": tf_kind, "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
-        path = ("tcgen05, clusters splitting K" if M <= 64 and K % 32 == 0
-                else "gemv" if M <= 4 else "tcgen05 fused expansion" if not need
+        path = ("gemv" if M <= 4 else "tcgen05 fused expansion" if not need
                 else "dequant + TMA-fed tcgen05")
         points.append({"tokens": M, "us": ms * 1e3, "tokens_per_s": M / (ms * 1e-3),
                        "path": path, "roofline": roof,

@@ -122,10 +122,9 @@ GEMM_CASES = [(oracle.INT4, 128, 16, 200, 640), (oracle.INT4, 128, 128, 130, 384
 @pytest.mark.parametrize("fmt,g,S,N,K", GEMM_CASES)
 @pytest.mark.parametrize("M", [5, 9, 32, 64, 100, 257, 600])
 def test_linear_tensor_core_path(fmt, g, S, N, K, M):
-    """Token counts above 4 take a tcgen05 kernel (up to 64 tokens with
-    K % 32 == 0 the cluster kernel, else the fused one): partial weight-row
-    tiles (N not a multiple of 128), partial token tiles, and a last K block
-    that is only partly inside K (K = 208, 96)."""
+    """Token counts above 4 take the tcgen05 kernel: partial weight-row tiles
+    (N not a multiple of 128), partial token tiles, and a last K block that
+    is only partly inside K (K = 208, 96)."""
     host, dev = packed_layer(N, K, fmt, g, S, seed=M + N)
     X = synth.make_activations(M, K, seed=200 + M, heavy=True).cuda()
     Y = bb.linear(X, dev, dev["cfg"], N, K)
@@ -136,11 +135,11 @@ def test_linear_tensor_core_path(fmt, g, S, N, K, M):
 
 @pytest.mark.parametrize("fmt,g,S", CASES)
 @pytest.mark.parametrize("N,K,Ms", [(300, 4096, (1, 24, 64)), (130, 1024, (16, 40))])
-def test_linear_small_token_cluster_path(fmt, g, S, N, K, Ms):
-    """Up to 64 tokens with K % 32 == 0 take the cluster kernel: several K
-    blocks per CTA (the 4-stage ring wraps), 16-, 32- and 64-token tiles,
-    partial weight-row tiles, and the cluster's partials summed in rank order,
-    so that two runs agree bit for bit."""
+def test_linear_small_token_counts(fmt, g, S, N, K, Ms):
+    """1 to 64 tokens on a layer with many K blocks (K = 4096: 64 blocks, so
+    every stage ring wraps many times) and partial weight-row tiles: the GEMV
+    (1 token) and the fused tcgen05 kernel (its K split in two onto a zeroed
+    Y); two runs agree bit for bit."""
     host, dev = packed_layer(N, K, fmt, g, S, seed=N + K + S + 5, iters=2)
     ref_w = ref_dequant(host, N, K, fmt, g, S)
     for M in Ms:
