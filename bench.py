@@ -636,7 +636,7 @@ def run_sharded(args, rank, local_rank, world):
             "config": {"workload": wl.name, "tokens": tokens,
                        "weights_per_block": sum(l.N * l.K for l in wl.linears),
                        "iters": wl.iters,
-                       "parallelism": f"row-sharded x{world} (one int64 all-reduce of 68 values "
+                       "parallelism": f"row-sharded x{world} (one int64 all-reduce of 69 values "
                                       "per fit round; importance replicated)",
                        "l2": "inputs larger than L2 (activations %.1f GiB per step)" % (
                            sum(x.numel() * 2 for x in Xs.values()) / 2 ** 30)},
