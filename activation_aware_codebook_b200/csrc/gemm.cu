@@ -12,7 +12,7 @@
 // with tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in TMEM).  Per 64-wide
 // K block (one 128-byte swizzle row per operand row):
 //   warp 0      one lane issues the TMA load of the X tile (SWIZZLE_128B) into
-//               stage s, no multicast;
+//               stage s (a plain copy into this CTA only);
 //   warps 2..9  256 producer threads, two per weight row (32 columns each):
 //               16 bytes of codes, the scales and the
 //               choice byte, loaded up to 2 x kPre stages ahead into two
@@ -447,7 +447,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
 //   one CTA per SM walks the 128 x 256 output tiles t = blockIdx.x, +grid, ...
 //   (weight-row tile major, so the CTAs in flight share their W rows in L2);
 //   warp 0      one lane issues the TMA loads of the W_hat tile (128 rows x 64)
-//               and the X tile (256 x 64) of every stage, no multicast;
+//               and the X tile (256 x 64) of every stage, each into this CTA only;
 //   warp 1      allocates all 512 TMEM columns: two 256-column accumulators,
 //               tiles alternating between them; one lane issues the MMAs and
 //               commits each tile's accumulator to acc_full[b];
