@@ -255,16 +255,16 @@ template <int FMT>
 void launch_gemv(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                  const void* tagged, const uint8_t* cbits, const uint16_t* Tb, int64_t N,
                  int64_t K, int lg, int ls, float* Y, const float* gsc, cudaStream_t st) {
-  // rows a warp and unrolled K steps as measured on gate_proj (us for 1 / 2 /
-  // 4 tokens): unrolling by 2 (1 token) or 4 (2 tokens) takes 29.5 -> 27.7
-  // and 35.8 -> 32.2; 3-4 tokens run best with four rows a warp, not unrolled
-  // (45 us, against 53 with one row and 51-64 unrolled)
+  // rows a warp and unrolled K steps as measured on gate_proj (us): 1 token
+  // unrolled by 2, 29.5 -> 28.0; 2 tokens unrolled by 4, 35.8 -> 31.5; 3-4
+  // tokens with two rows a warp unrolled by 2, 43.9 (one row: 53; four rows:
+  // 46; one row unrolled by 2 or 4: 50)
   if (M == 1)
     launch_gemv_t<FMT, 1, 2, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
   else if (M == 2)
     launch_gemv_t<FMT, 2, 2, 4>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
   else
-    launch_gemv_t<FMT, 4, 4, 1>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
+    launch_gemv_t<FMT, 4, 2, 2>(X, M, ldx, codes, tagged, cbits, Tb, N, K, lg, ls, Y, gsc, st);
 }
 
 }  // namespace
