@@ -582,6 +582,305 @@ gemm_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------
+// Small token counts (5 to 32 tokens): the work is the stream of 4-bit codes,
+// so the kernel is laid out to keep HBM busy and to spend few instructions
+// per weight.  A cluster of C = 2 CTAs (along grid y) shares one 128-row tile
+// of W; CTA r of the cluster takes a contiguous half of the 64-wide K blocks.
+//   warp 0      one lane issues, per stage, the TMA copies of the code tile
+//               (128 rows x 32 bytes, no swizzle) and of the X tile (BT x 64,
+//               SWIZZLE_128B), each into this CTA only, on ld_full[s];
+//   warp 1      allocates TMEM and issues the MMAs (M = 128, N = BT) of a
+//               stage once the producers have filled it (a_full[s]), then
+//               commits the stage to empty[s] and, after the last, accum;
+//   warps 2..9  producers: two threads per weight row, 32 columns each;
+//               codes from the stage's code tile, the row's scales and choice
+//               bits from shared memory (staged once at the start), expanded
+//               into the stage's swizzled bf16 A tile (expand8 as in the
+//               fused kernel), then fence.proxy.async and one arrive per warp.
+// The row's partial (128 x BT fp32) goes from TMEM to the CTA's shared memory;
+// after a cluster barrier each CTA sums 1/C of the tile's outputs over the
+// cluster's partials in rank order (distributed shared memory, fixed order:
+// the result does not depend on timing) and stores Y.  A second cluster
+// barrier keeps every partial alive until all CTAs have read it.  Waits on
+// mbarriers are bounded as in gemm_kernel; a CTA that gives up writes NaN
+// partials but still reaches both cluster barriers.
+// ---------------------------------------------------------------------------
+constexpr int kStagesS = 4;
+constexpr int kSmallSmemMax = 227 * 1024;
+constexpr int kCodeTileBytes = kBN * kBK / 2;  // 4 KB: 128 rows x 32 bytes
+
+struct SmallArgs {
+  const void* tagged;
+  const uint8_t* cbits;
+  const uint16_t* Tb;
+  float* Y;
+  int M, N, K, lg, ls;
+  int nkb_all;        // 64-wide K blocks of the layer
+  int sc_stride;      // shared bytes per row for its scales
+  int cb_stride;      // shared bytes per row for its choice bits
+  const float* gsc;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NC]);
+template <>
+__device__ __forceinline__ void tmem_ld_cols<8>(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <int BT>
+__host__ __device__ constexpr uint32_t small_tmem_cols() {
+  return BT < 32 ? 32u : (uint32_t)BT;
+}
+
+template <int FMT, int BT>
+__global__ void __launch_bounds__(kGemmThreads, 2)
+gemm_small_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap,
+                  SmallArgs a) {
+  extern __shared__ __align__(1024) unsigned char gsm[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(gsm) + 1023) & ~(uintptr_t)1023);
+  unsigned char* sA = base;                                  // kStagesS x 16 KB
+  unsigned char* sB = sA + kStagesS * kATileBytes;           // kStagesS x BT*128
+  unsigned char* sC = sB + kStagesS * BT * 128;              // kStagesS x 4 KB
+  unsigned char* sSc = sC + kStagesS * kCodeTileBytes;       // 128 x sc_stride
+  unsigned char* sCb = sSc + kBN * a.sc_stride;              // 128 x cb_stride
+  uint64_t* ld_full = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(sCb + kBN * a.cb_stride) + 7) & ~(uintptr_t)7);
+  uint64_t* a_full = ld_full + kStagesS;
+  uint64_t* empty = a_full + kStagesS;
+  uint64_t* accum = empty + kStagesS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  float* P = reinterpret_cast<float*>(sA);  // the partial tile [BT][128], after the MMAs
+  __shared__ unsigned short sT[32];
+  __shared__ int s_fail;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t crank = cluster_rank(), csize = cluster_size();
+  const int n0 = blockIdx.x * kBN;
+  const int kb_lo = (int)(crank * (uint32_t)a.nkb_all / csize);
+  const int kb_hi = (int)((crank + 1) * (uint32_t)a.nkb_all / csize);
+  const int nkb = kb_hi - kb_lo;  // >= 1: the host takes csize <= nkb_all
+  const int col_lo = kb_lo * kBK;
+  const int col_hi = min(a.K, kb_hi * kBK);
+  const int gi_lo = col_lo >> a.lg;
+  const int bb_lo = (col_lo >> a.ls) >> 3;
+  const bool sign_choice = a.lg == a.ls;
+
+  if (threadIdx.x < 32) sT[threadIdx.x] = a.Tb[threadIdx.x];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStagesS; s++) {
+      mbar_init(&ld_full[s], 1);          // the TMA lane's expect_tx
+      mbar_init(&a_full[s], kProdWarps);  // one arrive per producer warp
+      mbar_init(&empty[s], 1);            // MMA commit
+    }
+    mbar_init(accum, 1);
+    s_fail = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(small_tmem_cols<BT>()));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (warp >= 2) {
+    // stage the tile rows' scales and choice bits of this CTA's K range
+    const int p = threadIdx.x - 64, row = p >> 1, h = p & 1;
+    const int n = n0 + row;
+    const int ng = ((col_hi - 1) >> a.lg) - gi_lo + 1;
+    const int G = a.K >> a.lg;
+    if (FMT == kInt4) {
+      const unsigned short* src = reinterpret_cast<const unsigned short*>(a.tagged) + (int64_t)n * G + gi_lo;
+      unsigned short* dst = reinterpret_cast<unsigned short*>(sSc + row * a.sc_stride);
+      for (int i = h; i < ng; i += 2) dst[i] = n < a.N ? __ldg(src + i) : (unsigned short)0;
+    } else {
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(a.tagged) + (int64_t)n * G + gi_lo;
+      unsigned char* dst = sSc + row * a.sc_stride;
+      for (int i = h; i < ng; i += 2) dst[i] = n < a.N ? __ldg(src + i) : (unsigned char)0;
+    }
+    if (!sign_choice) {
+      const int nb = ((a.K >> a.ls) + 7) >> 3;
+      const int nbb = (((col_hi - 1) >> a.ls) >> 3) - bb_lo + 1;
+      const uint8_t* src = a.cbits + (int64_t)n * nb + bb_lo;
+      unsigned char* dst = sCb + row * a.cb_stride;
+      for (int i = h; i < nbb; i += 2) dst[i] = n < a.N ? __ldg(src + i) : (unsigned char)0;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {  // code and X tiles by TMA
+      int issued = 0;
+      for (int kb = 0; kb < nkb; kb++) {
+        const int s = kb % kStagesS;
+        if (kb >= kStagesS && !mbar_wait(&empty[s], ((kb / kStagesS) - 1) & 1)) { s_fail = 1; break; }
+        mbar_arrive_expect_tx(&ld_full[s], BT * 128 + kCodeTileBytes);
+        tma_load_2d(sB + s * BT * 128, &xmap, &ld_full[s], (kb_lo + kb) * kBK, 0);
+        tma_load_2d(sC + s * kCodeTileBytes, &cmap, &ld_full[s], (kb_lo + kb) * (kBK / 2), n0);
+        issued = kb + 1;
+      }
+      // the last copies have landed before the CTA can exit (bounded)
+      for (int kb = issued > kStagesS ? issued - kStagesS : 0; kb < issued; kb++)
+        if (!mbar_wait(&ld_full[kb % kStagesS], (kb / kStagesS) & 1)) { s_fail = 1; break; }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issue
+      const uint32_t idesc = mma_idesc(kBN, BT);
+      for (int kb = 0; kb < nkb; kb++) {
+        const int s = kb % kStagesS;
+        const uint32_t ph = (kb / kStagesS) & 1;
+        if (!mbar_wait(&ld_full[s], ph) || !mbar_wait(&a_full[s], ph)) { s_fail = 1; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * kATileBytes), b0 = smem_u32(sB + s * BT * 128);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; k++)
+          mma_bf16(tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
+                   (kb > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accum);
+    }
+  } else {
+    // producers: thread p fills half h = p & 1 (32 columns) of weight row p >> 1
+    const int p = threadIdx.x - 64;
+    const int h = p & 1, rowi = p >> 1;
+    const bool rok = n0 + rowi < a.N;
+    const float gsv = FMT == kNvfp4G ? __ldg(a.gsc) : 1.0f;
+    const uint32_t rsw = (uint32_t)(rowi & 7);
+    const uint32_t roff = (uint32_t)(rowi >> 3) * 1024u + rsw * 128u;
+    const unsigned char* scrow = sSc + rowi * a.sc_stride;
+    const unsigned char* cbrow = sCb + rowi * a.cb_stride;
+    for (int kb = 0; kb < nkb; kb++) {
+      const int s = kb % kStagesS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[s], (kb / kStagesS) & 1))) {
+        s_fail = 1;
+        break;
+      }
+      const uint4 cw = *reinterpret_cast<const uint4*>(sC + s * kCodeTileBytes + rowi * 32 + h * 16);
+      const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+      unsigned char* dst = sA + s * kATileBytes + roff;
+      const int k0 = (kb_lo + kb) * kBK + h * 32;
+      // the choice bits of the thread's 32 columns (at most 4 groups of 8)
+      // from one staged byte: S >= 8 and k0 a multiple of 32 keep them in it
+      uint32_t cbyte = 0u;
+      if (!sign_choice && rok && k0 < a.K) {
+        const int bit0 = k0 >> a.ls;
+        cbyte = (uint32_t)cbrow[(bit0 >> 3) - bb_lo] >> (bit0 & 7);
+      }
+      // the scale of the thread's first column: with g >= 32 it covers all 32
+      uint32_t sraw0 = 0u;
+      if (rok && k0 < a.K) {
+        const int gl0 = (k0 >> a.lg) - gi_lo;
+        sraw0 = FMT == kInt4 ? (uint32_t)reinterpret_cast<const unsigned short*>(scrow)[gl0]
+                             : (uint32_t)scrow[gl0];
+      }
+      const bool one_scale = a.lg >= 5;
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const int k = k0 + 8 * j;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (rok && k < a.K) {
+          uint32_t tag, sraw = sraw0;
+          if (!one_scale && j > 0) {
+            const int gl = (k >> a.lg) - gi_lo;
+            sraw = FMT == kInt4 ? (uint32_t)reinterpret_cast<const unsigned short*>(scrow)[gl]
+                                : (uint32_t)scrow[gl];
+          }
+          const uint32_t cbit = (cbyte >> ((8 * j) >> a.ls)) & 1u;
+          if (FMT == kNvfp4G) {
+            tag = sraw >> 7;
+            v = expand8g(words[j], __fmul_rn(gsv, e4m3_mag(sraw & 0x7fu)), sign_choice ? tag : cbit, sT);
+          } else {
+            const uint32_t sbf = scale_bits<FMT>(sraw, &tag);
+            v = expand8(words[j], sbf, sign_choice ? tag : cbit, sT);
+          }
+        }
+        const uint32_t c = (uint32_t)(h * 4 + j);
+        *reinterpret_cast<uint4*>(dst + ((c ^ rsw) << 4)) = v;
+      }
+      fence_proxy_async();  // generic-proxy stores -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[s]);
+    }
+    // the partial tile: TMEM lane quadrant of this warp = 32 weight rows
+    const bool got = __all_sync(0xffffffffu, mbar_wait(accum, 0));
+    tc_fence_after();
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const bool fail = !got || s_fail;
+    constexpr int NC = BT / 2;
+    uint32_t r[NC];
+    if (!fail) tmem_ld_cols<NC>(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * NC), r);
+    // all MMAs are complete (accum), so the A stages are free for the partials
+#pragma unroll
+    for (int j = 0; j < NC; j++)
+      P[(half * NC + j) * kBN + q * 32 + lane] = fail ? __int_as_float(0x7fc00000) : __uint_as_float(r[j]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(small_tmem_cols<BT>()));
+  }
+  cluster_sync_all();  // every CTA's partial is in its shared memory
+  {
+    const int E = BT * kBN;
+    const int e0 = (int)(crank * (uint32_t)E / csize), e1 = (int)((crank + 1) * (uint32_t)E / csize);
+    for (int e = e0 + threadIdx.x; e < e1; e += kGemmThreads) {
+      const int t = e / kBN, row = e % kBN;
+      if (t < a.M && n0 + row < a.N) {
+        float v = 0.0f;
+        for (uint32_t c = 0; c < csize; c++) v = __fadd_rn(v, ld_cluster_f32(P + e, c));
+        a.Y[(int64_t)t * a.N + n0 + row] = v;
+      }
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while another may still read its partial
+}
+
+// ---------------------------------------------------------------------------
 // host: tensor map for X through the driver entry point (no link to libcuda)
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -681,6 +980,89 @@ cudaError_t launch_gemm_tma(const uint16_t* X, int64_t M, int64_t ldx, const uin
   return cudaGetLastError();
 }
 
+template <int BT>
+size_t small_smem(int sc_stride, int cb_stride) {
+  return 1024 + (size_t)kStagesS * (kATileBytes + BT * 128 + kCodeTileBytes) +
+         (size_t)kBN * (sc_stride + cb_stride) + 8 + (3 * kStagesS + 1) * 8 + 16;
+}
+
+// Cluster size: two CTAs split a tile's K blocks (one when the layer has a
+// single K block).  Measured on gate_proj (us at 1 / 16 / 32 / 64 tokens):
+// C = 1: 54 / 56 / 57 / 59; 2: 42 / 43 / 45 / 68; 4: 46 / 47 / 49 / 80;
+// 8: 53 / 55 / 57 / 106 -- more, shorter CTAs spend more of their time
+// filling and draining their stage rings.
+int small_cluster(int nkb) { return nkb < 2 ? nkb : 2; }
+
+// Per-row staging of the largest CTA's scales and choice bytes (+2 for a
+// range that straddles group and byte boundaries), rounded to 4 bytes.
+void small_strides(int nkb_all, int fmt, int lg, int ls, int* sc_stride, int* cb_stride) {
+  const int C = small_cluster(nkb_all);
+  const int nkb_max = (nkb_all + C - 1) / C;
+  const int esz = fmt == kInt4 ? 2 : 1;
+  const int ng_max = (nkb_max * kBK) / (1 << lg) + 2;
+  *sc_stride = (ng_max * esz + 3) & ~3;
+  const int nbb_max = (nkb_max * kBK / (1 << ls)) / 8 + 2;
+  *cb_stride = lg == ls ? 0 : ((nbb_max + 3) & ~3);
+}
+
+template <int FMT, int BT>
+cudaError_t launch_gemm_small_t(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                                SmallArgs sa, cudaStream_t st) {
+  EncodeTiledFn enc;
+  cudaError_t e = encode_fn(&enc);
+  if (e != cudaSuccess) return e;
+  CUtensorMap xmap, cmap;
+  const cuuint32_t estr[2] = {1, 1};
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)sa.K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BT};
+    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // codes as bytes: K / 2 per row (a multiple of 16: K % 32 == 0 is checked
+    // by the caller); rows past N and bytes past K / 2 read as zero
+    const cuuint64_t dims[2] = {(cuuint64_t)(sa.K / 2), (cuuint64_t)sa.N};
+    const cuuint64_t strides[1] = {(cuuint64_t)(sa.K / 2)};
+    const cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), (cuuint32_t)kBN};
+    if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const int tiles = (int)((sa.N + kBN - 1) / kBN);
+  const int C = small_cluster(sa.nkb_all);
+  small_strides(sa.nkb_all, FMT, sa.lg, sa.ls, &sa.sc_stride, &sa.cb_stride);
+  const size_t smem = small_smem<BT>(sa.sc_stride, sa.cb_stride);
+  if (smem > (size_t)kSmallSmemMax) return cudaErrorInvalidValue;  // gemm_small_fits checks it
+  e = cudaFuncSetAttribute(gemm_small_kernel<FMT, BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)tiles, (unsigned)C, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = (unsigned)C;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_small_kernel<FMT, BT>, xmap, cmap, sa);
+}
+
+template <int FMT>
+cudaError_t launch_gemm_small_f(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                                const SmallArgs& sa, cudaStream_t st) {
+  if (M <= 16) return launch_gemm_small_t<FMT, 16>(X, M, ldx, codes, sa, st);
+  return launch_gemm_small_t<FMT, 32>(X, M, ldx, codes, sa, st);
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
@@ -704,6 +1086,26 @@ cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
   return bt == 64 ? launch_gemm_t<kNvfp4G, 64>(X, M, ldx, ga, st)
        : bt == 128 ? launch_gemm_t<kNvfp4G, 128>(X, M, ldx, ga, st)
                    : launch_gemm_t<kNvfp4G, 256>(X, M, ldx, ga, st);
+}
+
+bool gemm_small_fits(int64_t M, int64_t K, int fmt, int lg, int ls) {
+  if (M < kSmallMinM || M > kSmallMaxM || K % 32 != 0) return false;
+  // the staged scales and choice bytes grow with K: past the shared-memory
+  // limit the fused kernel takes the layer
+  int sc = 0, cb = 0;
+  small_strides((int)((K + kBK - 1) / kBK), fmt, lg, ls, &sc, &cb);
+  return small_smem<32>(sc, cb) <= (size_t)kSmallSmemMax;
+}
+
+cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                              const void* tagged, const uint8_t* cbits, const uint16_t* Tb,
+                              int64_t N, int64_t K, int fmt, int lg, int ls, float* Y,
+                              const float* gsc, cudaStream_t st) {
+  SmallArgs sa{tagged, cbits, Tb, Y, (int)M, (int)N, (int)K, lg, ls,
+               (int)((K + kBK - 1) / kBK), 0, 0, gsc};
+  if (fmt == kInt4) return launch_gemm_small_f<kInt4>(X, M, ldx, codes, sa, st);
+  if (fmt == kNvfp4) return launch_gemm_small_f<kNvfp4>(X, M, ldx, codes, sa, st);
+  return launch_gemm_small_f<kNvfp4G>(X, M, ldx, codes, sa, st);
 }
 
 cudaError_t launch_gemm_dequantised(const uint16_t* X, int64_t M, int64_t ldx,

@@ -107,6 +107,16 @@ cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
                         int64_t K, int fmt, int lg, int ls, float* Y, const float* gsc,
                         cudaStream_t st);
 // Y = X W_hat^T from an already dequantised bf16 W_hat [N][K] (both operands by TMA)
+// W4A16 linear for 5 to 32 tokens (K % 32 == 0): one 128-row tile per
+// cluster of two CTAs splitting K, codes and X by TMA, the two partials summed
+// in rank order over distributed shared memory
+constexpr int64_t kSmallMinM = 5;
+constexpr int64_t kSmallMaxM = 32;
+bool gemm_small_fits(int64_t M, int64_t K, int fmt, int lg, int ls);
+cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
+                              const void* tagged, const uint8_t* cbits, const uint16_t* Tb,
+                              int64_t N, int64_t K, int fmt, int lg, int ls, float* Y,
+                              const float* gsc, cudaStream_t st);
 cudaError_t launch_gemm_dequantised(const uint16_t* X, int64_t M, int64_t ldx,
                                     const uint16_t* Wh, int64_t N, int64_t K, float* Y,
                                     cudaStream_t st);

@@ -871,8 +871,9 @@ def run_linear(args):
             roof = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": tflops_peak,
                     "peak_kind": tf_kind, "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
-        path = ("gemv" if M <= 4 else "tcgen05 fused expansion" if not need
-                else "dequant + TMA-fed tcgen05")
+        path = ("gemv" if M <= 4
+                else "tcgen05, two CTAs a tile split K (cluster)" if M <= 32 and K % 32 == 0
+                else "tcgen05 fused expansion" if not need else "dequant + TMA-fed tcgen05")
         points.append({"tokens": M, "us": ms * 1e3, "tokens_per_s": M / (ms * 1e-3),
                        "path": path, "roofline": roof,
                        "cublas_bf16_dequantised_us": cublas_us})
