@@ -39,7 +39,8 @@ EXPORTS = ("aaac_workspace_size", "aaac_importance", "aaac_init_codebooks", "aaa
            "aaac_device_timeouts", "aaac_awq_prescale", "aaac_awq_workspace_size",
            "aaac_awq_fit", "aaac_init_codebooks_sharded", "aaac_fit_layer_sharded",
            "aaac_pack_sharded", "aaac_linear_workspace_size", "aaac_linear_ws",
-           "aaac_fit_launch_plan", "aaac_inject_fault", "aaac_device_checks",
+           "aaac_fit_launch_plan", "aaac_linear_launch_plan", "aaac_inject_fault",
+           "aaac_device_checks",
            "aaac_checked_build")
 
 
@@ -140,6 +141,8 @@ def load(path: str = LIB_PATH):
     L.aaac_checked_build.argtypes = []
     L.aaac_fit_launch_plan.restype = ctypes.c_int
     L.aaac_fit_launch_plan.argtypes = [P, i64, i64, i64, ctypes.POINTER(ctypes.c_int32)]
+    L.aaac_linear_launch_plan.restype = ctypes.c_int
+    L.aaac_linear_launch_plan.argtypes = [P, i64, i64, i64, ctypes.POINTER(ctypes.c_int32)]
     L.aaac_awq_prescale.restype = ctypes.c_int
     L.aaac_awq_prescale.argtypes = [P, i64, i64, P, i64, ctypes.c_int, P, P, P, P]
     L.aaac_awq_workspace_size.restype = sz
@@ -207,6 +210,20 @@ def _need_cuda():
 def workspace_size(cfg: Optional[Config], N: int = 0, K: int = 0, T: int = 0) -> int:
     c = cfg.c() if cfg is not None else None
     return int(load().aaac_workspace_size(ctypes.byref(c) if c is not None else None, N, K, T))
+
+
+LINEAR_PATHS = {0: "gemv", 1: "cluster", 2: "fused"}
+
+
+def linear_launch_plan(cfg: Config, M: int, N: int, K: int) -> dict:
+    """Host-only: the kernel aaac_linear runs and the cluster kernel's plan."""
+    out = (ctypes.c_int32 * 8)()
+    _check(load().aaac_linear_launch_plan(ctypes.byref(cfg.c()), M, N, K, out))
+    keys = ("path", "cluster", "kblocks", "scale_stride", "choice_stride", "smem16", "smem32",
+            "smem_limit")
+    d = dict(zip(keys, list(out)))
+    d["path"] = LINEAR_PATHS[d["path"]]
+    return d
 
 
 def fit_launch_plan(cfg: Config, N: int, K: int, N_total: Optional[int] = None) -> dict:

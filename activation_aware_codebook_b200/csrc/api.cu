@@ -207,6 +207,21 @@ aaac_status aaac_fit_launch_plan(const aaac_config* cfg, int64_t N, int64_t K, i
   return ok();
 }
 
+aaac_status aaac_linear_launch_plan(const aaac_config* cfg, int64_t M, int64_t N, int64_t K,
+                                    int32_t* out) {
+  if (!out) return fail(AAAC_ERR_INVALID_ARG, "out is NULL");
+  CHECK(check_cfg(cfg));
+  CHECK(check_layer(N, K, cfg));
+  if (M < 1 || M > ((int64_t)1 << 20))
+    return fail(AAAC_ERR_SHAPE, "M=%lld must be in [1, 2^20]", (long long)M);
+  int lg = 0, ls = 0;
+  while ((1 << lg) < cfg->g) lg++;
+  while ((1 << ls) < cfg->S) ls++;
+  out[0] = aaac::linear_path(M, K, cfg->fmt, cfg->g, cfg->S);
+  aaac::small_linear_plan(K, cfg->fmt, lg, ls, out + 1);
+  return ok();
+}
+
 size_t aaac_workspace_size(const aaac_config* cfg, int64_t N, int64_t K, int64_t T) {
   size_t need = weight_side_bytes(cfg, N, K);
   if (T > 0 && K > 0) {

@@ -1097,6 +1097,19 @@ bool gemm_small_fits(int64_t M, int64_t K, int fmt, int lg, int ls) {
   return small_smem<32>(sc, cb) <= (size_t)kSmallSmemMax;
 }
 
+void small_linear_plan(int64_t K, int fmt, int lg, int ls, int32_t* out) {
+  const int nkb = (int)((K + kBK - 1) / kBK);
+  int sc = 0, cb = 0;
+  small_strides(nkb, fmt, lg, ls, &sc, &cb);
+  out[0] = small_cluster(nkb);
+  out[1] = nkb;
+  out[2] = sc;
+  out[3] = cb;
+  out[4] = (int32_t)small_smem<16>(sc, cb);
+  out[5] = (int32_t)small_smem<32>(sc, cb);
+  out[6] = kSmallSmemMax;
+}
+
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                               const void* tagged, const uint8_t* cbits, const uint16_t* Tb,
                               int64_t N, int64_t K, int fmt, int lg, int ls, float* Y,

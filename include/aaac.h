@@ -385,6 +385,24 @@ const char* aaac_version(void);
 aaac_status aaac_fit_launch_plan(const aaac_config* cfg, int64_t N, int64_t K, int64_t N_total,
                                  int32_t* out);
 
+/* The kernel aaac_linear runs for M tokens of a layer of N x K weights, and
+ * the plan of the cluster kernel it uses for 5 to 32 tokens.  A host-only
+ * query: no GPU work, no device memory.  out (host int32[8]):
+ *   out[0]  0 GEMV (up to 4 tokens), 1 cluster kernel (5 to 32 tokens, K a
+ *           multiple of 32, its shared memory within the limit), 2 the
+ *           fused tcgen05 kernel (aaac_linear_ws may dequantise instead)
+ *   out[1]  CTAs of a cluster; each takes a contiguous share of the K blocks
+ *   out[2]  64-column K blocks of the layer
+ *   out[3]  bytes per weight row staged for its scales, out[4] for its
+ *           choice bits (0 when S == g)
+ *   out[5]  shared memory of the 16-token kernel, out[6] of the 32-token one
+ *   out[7]  the shared-memory limit the plan must keep
+ * out[1..7] describe the cluster kernel whatever out[0] is.  Errors:
+ * AAAC_ERR_INVALID_ARG (NULL cfg or out), AAAC_ERR_UNSUPPORTED / SHAPE as
+ * aaac_linear's. */
+aaac_status aaac_linear_launch_plan(const aaac_config* cfg, int64_t M, int64_t N, int64_t K,
+                                    int32_t* out);
+
 /* Number of CUDA kernels this library has launched in the process so far
  * (all threads, all devices).  A measurement aid: the difference across a
  * region counts the library's kernel launches in it. */
