@@ -505,7 +505,7 @@ def run_ours(args, rank, local_rank, world):
     # end to end through the C ABI with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(blk, args.e2e_steps, dev)
+        e2e = run_e2e(blk, args.e2e_steps, dev, world)
 
     out = None
     if rank == 0:
@@ -655,10 +655,13 @@ def run_sharded(args, rank, local_rank, world):
     return out
 
 
-def run_e2e(blk, steps, dev):
+def run_e2e(blk, steps, dev, world=1):
     """Same step through the public API with host-resident inputs: pinned H2D
     of every activation and weight, the four calls, D2H of every output, with
-    the copies overlapping the compute (three streams)."""
+    the copies overlapping the compute (three streams).  With several ranks
+    each copies and fits its own block; a barrier starts the timed steps
+    together, the time is the slowest rank's, and the value counts every
+    rank's weights."""
     import torch
     hostX = {k: torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for k, x in blk.Xs.items()}
     hostW = {k: torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for k, w in blk.Ws.items()}
@@ -718,6 +721,10 @@ def run_e2e(blk, steps, dev):
 
     one()
     torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(comp)
     h2d_s.wait_event(e0)
@@ -727,9 +734,10 @@ def run_e2e(blk, steps, dev):
     comp.wait_stream(h2d_s)
     e1.record(comp)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    return {"value": blk.weight_iters / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
-            "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+    return {"value": world * blk.weight_iters / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": int(world * h2d),
+            "d2h_bytes_per_step": int(world * d2h)}
 
 
 # ---------------------------------------------------------------------------
