@@ -1,6 +1,9 @@
-// gemm.cu -- the W4A16 linear for larger token counts on the 5th-generation
-// tensor cores: Y[m][n] = sum_k X[m][k] * W_hat[n][k] with W_hat expanded from
-// the packed format tile by tile in shared memory.
+// gemm.cu -- the W4A16 linear above 4 tokens on the 5th-generation tensor
+// cores: Y[m][n] = sum_k X[m][k] * W_hat[n][k] with W_hat expanded from the
+// packed format tile by tile in shared memory.  Three kernels: gemm_kernel
+// (the fused expansion, below), gemm_small_kernel (5 to 32 tokens: a cluster
+// of two CTAs splits K, codes by TMA), and gemm_tma_kernel (dequantised
+// weights, a persistent TMA-fed GEMM for 192 tokens and more).
 //
 // "Technical summary: AAAC", section 1 (weight-only W4A16 inference: the
 // dequantised values from the tables decide the weights used) and section 2,
