@@ -217,8 +217,8 @@ aaac_status aaac_linear_launch_plan(const aaac_config* cfg, int64_t M, int64_t N
   int lg = 0, ls = 0;
   while ((1 << lg) < cfg->g) lg++;
   while ((1 << ls) < cfg->S) ls++;
-  out[0] = aaac::linear_path(M, K, cfg->fmt, cfg->g, cfg->S);
-  aaac::small_linear_plan(K, cfg->fmt, lg, ls, out + 1);
+  out[0] = aaac::linear_path(M, N, K, cfg->fmt, cfg->g, cfg->S);
+  aaac::small_linear_plan(N, K, cfg->fmt, lg, ls, out + 1);
   return ok();
 }
 

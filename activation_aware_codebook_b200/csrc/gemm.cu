@@ -2,7 +2,7 @@
 // cores: Y[m][n] = sum_k X[m][k] * W_hat[n][k] with W_hat expanded from the
 // packed format tile by tile in shared memory.  Three kernels: gemm_kernel
 // (the fused expansion, below), gemm_small_kernel (5 to 32 tokens: a cluster
-// of two CTAs splits K, codes by TMA), and gemm_tma_kernel (dequantised
+// of 2 to 8 CTAs splits K, codes by TMA), and gemm_tma_kernel (dequantised
 // weights, a persistent TMA-fed GEMM for 192 tokens and more).
 //
 // "Technical summary: AAAC", section 1 (weight-only W4A16 inference: the
@@ -587,8 +587,9 @@ gemm_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
 // ---------------------------------------------------------------------------
 // Small token counts (5 to 32 tokens): the work is the stream of 4-bit codes,
 // so the kernel is laid out to keep HBM busy and to spend few instructions
-// per weight.  A cluster of C = 2 CTAs (along grid y) shares one 128-row tile
-// of W; CTA r of the cluster takes a contiguous half of the 64-wide K blocks.
+// per weight.  A cluster of C CTAs (2 to 8, along grid y) shares one 128-row
+// tile of W; CTA r of the cluster takes a contiguous 1/C of the 64-wide K
+// blocks.
 //   warp 0      one lane issues, per stage, the TMA copies of the code tile
 //               (128 rows x 32 bytes, no swizzle) and of the X tile (BT x 64,
 //               SWIZZLE_128B), each into this CTA only, on ld_full[s];
@@ -989,17 +990,24 @@ size_t small_smem(int sc_stride, int cb_stride) {
          (size_t)kBN * (sc_stride + cb_stride) + 8 + (3 * kStagesS + 1) * 8 + 16;
 }
 
-// Cluster size: two CTAs split a tile's K blocks (one when the layer has a
-// single K block).  Measured on gate_proj (us at 1 / 16 / 32 / 64 tokens):
-// C = 1: 54 / 56 / 57 / 59; 2: 42 / 43 / 45 / 68; 4: 46 / 47 / 49 / 80;
-// 8: 53 / 55 / 57 / 106 -- more, shorter CTAs spend more of their time
-// filling and draining their stage rings.
-int small_cluster(int nkb) { return nkb < 2 ? nkb : 2; }
+// Cluster size: about 240 CTAs over the layer's 128-row tiles, at least 2 and
+// at most 8 (and no more than the K blocks).  Measured at 16 tokens (us):
+// gate_proj 14336x4096 (112 tiles): C = 1 56, 2 43, 4 47, 8 55; q_proj
+// 4096x4096 (32 tiles): C = 2 32.8, 4 22.6, 8 21.3; down_proj 4096x14336:
+// 86.9, 51.1, 39.6; k_proj 1024x4096 (8 tiles): 32.6, 21.3, 17.1.  Fewer CTAs
+// leave SMs idle; more, shorter ones spend more of their time filling and
+// draining their stage rings.
+int small_cluster(int tiles, int nkb) {
+  int c = (240 + tiles / 2) / tiles;
+  c = c < 2 ? 2 : (c > 8 ? 8 : c);
+  return c < nkb ? c : nkb;
+}
 
 // Per-row staging of the largest CTA's scales and choice bytes (+2 for a
 // range that straddles group and byte boundaries), rounded to 4 bytes.
-void small_strides(int nkb_all, int fmt, int lg, int ls, int* sc_stride, int* cb_stride) {
-  const int C = small_cluster(nkb_all);
+void small_strides(int tiles, int nkb_all, int fmt, int lg, int ls, int* sc_stride,
+                   int* cb_stride) {
+  const int C = small_cluster(tiles, nkb_all);
   const int nkb_max = (nkb_all + C - 1) / C;
   const int esz = fmt == kInt4 ? 2 : 1;
   const int ng_max = (nkb_max * kBK) / (1 << lg) + 2;
@@ -1037,8 +1045,8 @@ cudaError_t launch_gemm_small_t(const uint16_t* X, int64_t M, int64_t ldx, const
       return cudaErrorInvalidValue;
   }
   const int tiles = (int)((sa.N + kBN - 1) / kBN);
-  const int C = small_cluster(sa.nkb_all);
-  small_strides(sa.nkb_all, FMT, sa.lg, sa.ls, &sa.sc_stride, &sa.cb_stride);
+  const int C = small_cluster(tiles, sa.nkb_all);
+  small_strides(tiles, sa.nkb_all, FMT, sa.lg, sa.ls, &sa.sc_stride, &sa.cb_stride);
   const size_t smem = small_smem<BT>(sa.sc_stride, sa.cb_stride);
   if (smem > (size_t)kSmallSmemMax) return cudaErrorInvalidValue;  // gemm_small_fits checks it
   e = cudaFuncSetAttribute(gemm_small_kernel<FMT, BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1091,20 +1099,21 @@ cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
                    : launch_gemm_t<kNvfp4G, 256>(X, M, ldx, ga, st);
 }
 
-bool gemm_small_fits(int64_t M, int64_t K, int fmt, int lg, int ls) {
+bool gemm_small_fits(int64_t M, int64_t N, int64_t K, int fmt, int lg, int ls) {
   if (M < kSmallMinM || M > kSmallMaxM || K % 32 != 0) return false;
   // the staged scales and choice bytes grow with K: past the shared-memory
   // limit the fused kernel takes the layer
   int sc = 0, cb = 0;
-  small_strides((int)((K + kBK - 1) / kBK), fmt, lg, ls, &sc, &cb);
+  small_strides((int)((N + kBN - 1) / kBN), (int)((K + kBK - 1) / kBK), fmt, lg, ls, &sc, &cb);
   return small_smem<32>(sc, cb) <= (size_t)kSmallSmemMax;
 }
 
-void small_linear_plan(int64_t K, int fmt, int lg, int ls, int32_t* out) {
+void small_linear_plan(int64_t N, int64_t K, int fmt, int lg, int ls, int32_t* out) {
   const int nkb = (int)((K + kBK - 1) / kBK);
+  const int tiles = (int)((N + kBN - 1) / kBN);
   int sc = 0, cb = 0;
-  small_strides(nkb, fmt, lg, ls, &sc, &cb);
-  out[0] = small_cluster(nkb);
+  small_strides(tiles, nkb, fmt, lg, ls, &sc, &cb);
+  out[0] = small_cluster(tiles, nkb);
   out[1] = nkb;
   out[2] = sc;
   out[3] = cb;

@@ -108,17 +108,17 @@ cudaError_t launch_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
                         cudaStream_t st);
 // Y = X W_hat^T from an already dequantised bf16 W_hat [N][K] (both operands by TMA)
 // W4A16 linear for 5 to 32 tokens (K % 32 == 0): one 128-row tile per
-// cluster of two CTAs splitting K, codes and X by TMA, the two partials summed
+// cluster of 2 to 8 CTAs splitting K, codes and X by TMA, the two partials summed
 // in rank order over distributed shared memory
 constexpr int64_t kSmallMinM = 5;
 constexpr int64_t kSmallMaxM = 32;
-bool gemm_small_fits(int64_t M, int64_t K, int fmt, int lg, int ls);
-// the cluster kernel's plan for a layer of K columns: out[0] cluster size,
+bool gemm_small_fits(int64_t M, int64_t N, int64_t K, int fmt, int lg, int ls);
+// the cluster kernel's plan for a layer of N x K: out[0] cluster size,
 // [1] 64-column K blocks, [2] / [3] staged bytes per row for scales / choice
 // bits, [4] / [5] shared memory of the 16- / 32-token kernel, [6] its limit
-void small_linear_plan(int64_t K, int fmt, int lg, int ls, int32_t* out);
+void small_linear_plan(int64_t N, int64_t K, int fmt, int lg, int ls, int32_t* out);
 // which kernel aaac_linear runs for M tokens: 0 GEMV, 1 cluster, 2 fused
-int linear_path(int64_t M, int64_t K, int fmt, int g, int S);
+int linear_path(int64_t M, int64_t N, int64_t K, int fmt, int g, int S);
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* codes,
                               const void* tagged, const uint8_t* cbits, const uint16_t* Tb,
                               int64_t N, int64_t K, int fmt, int lg, int ls, float* Y,

@@ -297,8 +297,8 @@ cudaError_t launch_dequant(const uint8_t* codes, const void* tagged, const uint8
   return cudaGetLastError();
 }
 
-int linear_path(int64_t M, int64_t K, int fmt, int g, int S) {
-  if (gemm_small_fits(M, K, fmt, log2_of(g), log2_of(S))) return 1;
+int linear_path(int64_t M, int64_t N, int64_t K, int fmt, int g, int S) {
+  if (gemm_small_fits(M, N, K, fmt, log2_of(g), log2_of(S))) return 1;
   return M > kGemvMaxM ? 2 : 0;
 }
 
@@ -307,8 +307,8 @@ cudaError_t launch_linear(const uint16_t* X, int64_t M, int64_t ldx, const uint8
                           int64_t K, int fmt, int g, int S, float* Y, const float* gsc,
                           cudaStream_t st) {
   const int lg = log2_of(g), ls = log2_of(S);
-  const int path = linear_path(M, K, fmt, g, S);
-  if (path == 1) {  // 5-32 tokens: two CTAs a tile split K
+  const int path = linear_path(M, N, K, fmt, g, S);
+  if (path == 1) {  // 5-32 tokens: a cluster of CTAs splits a tile's K
     const cudaError_t e =
         launch_gemm_small(X, M, ldx, codes, tagged, cbits, Tb, N, K, fmt, lg, ls, Y, gsc, st);
     if (e == cudaSuccess) count_launches(1);

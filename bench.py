@@ -880,7 +880,7 @@ def run_linear(args):
                     "peak_kind": tf_kind, "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
         path = ("gemv" if M <= 4
-                else "tcgen05, two CTAs a tile split K (cluster)" if M <= 32 and K % 32 == 0
+                else "tcgen05, a cluster of CTAs splits a tile's K" if M <= 32 and K % 32 == 0
                 else "tcgen05 fused expansion" if not need else "dequant + TMA-fed tcgen05")
         points.append({"tokens": M, "us": ms * 1e3, "tokens_per_s": M / (ms * 1e-3),
                        "path": path, "roofline": roof,

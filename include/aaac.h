@@ -226,8 +226,8 @@ aaac_status aaac_dequant(const uint8_t* codes, const void* scales_tagged,
  *   Y   device fp32 [M][N]
  * The dequantised weights never reach memory: each kernel expands its codes
  * on the fly (a GEMV on CUDA cores up to 4 tokens; tcgen05 kernels above:
- * 5 to 32 tokens on clusters of two CTAs splitting K when K is a multiple of
- * 32, else a fused kernel; aaac_linear_launch_plan reports which).
+ * 5 to 32 tokens on clusters of 2 to 8 CTAs splitting K when K is a
+ * multiple of 32, else a fused kernel; aaac_linear_launch_plan reports which).
  * Accumulation is fp32 in the library's order, the same on every run; every
  * result is within K * 2^-24 * sum_k |X[m][k] W_hat[n][k]| of the exact sum.
  * M in [1, 2^20].  No workspace. */

@@ -1,9 +1,10 @@
 """The W4A16 linear's choice of kernel and the cluster kernel's plan (host
 code, no GPU), from aaac_linear_launch_plan.
 
-aaac_linear takes the GEMV up to 4 tokens, the cluster kernel (two CTAs split
-a 128-row tile's 64-column K blocks; the rows' scales and choice bits of a
-CTA's K range are staged in shared memory) from 5 to 32 tokens when K is a
+aaac_linear takes the GEMV up to 4 tokens, the cluster kernel (2 to 8 CTAs
+split a 128-row tile's 64-column K blocks, about 240 CTAs in all; the rows'
+scales and choice bits of a CTA's K range are staged in shared memory) from 5
+to 32 tokens when K is a
 multiple of 32 and that staging fits, and the fused tcgen05 kernel otherwise.
 The emulation below takes each CTA's share of the K blocks as the kernel does
 (CTA r of C: blocks [r*nkb/C, (r+1)*nkb/C)) and checks that the shares cover
@@ -60,7 +61,8 @@ def test_linear_path_and_cluster_plan(fmt, g, S, N, K):
         p = bb.linear_launch_plan(cfg, M, N, K)
         p["fmt"] = fmt
         assert p["kblocks"] == (K + 63) // 64
-        assert p["cluster"] == min(2, p["kblocks"])
+        tiles = (N + 127) // 128  # about 240 CTAs, 2 to 8 a cluster, at most the K blocks
+        assert p["cluster"] == min(max(2, min(8, (240 + tiles // 2) // tiles)), p["kblocks"])
         fits = p["smem32"] <= p["smem_limit"]
         assert p["smem16"] <= p["smem32"]
         if M <= 4:
@@ -73,9 +75,11 @@ def test_linear_path_and_cluster_plan(fmt, g, S, N, K):
 
 
 def test_wide_nvfp4_layer_falls_back_to_the_fused_kernel():
-    """NVFP4 g=16 with K = 27648 and S = 8: a CTA's half of K stages 866 scale
-    bytes and 110 choice bytes per row, past shared memory at 32 tokens."""
-    p = bb.linear_launch_plan(bb.Config(bb.NVFP4, 16, 8, 0), 16, 5120, 27648)
+    """NVFP4 g=16 with K = 27648 and S = 8 on a layer of 216 row tiles (two
+    CTAs a cluster): a CTA's half of K stages 866 scale bytes and 110 choice
+    bytes per row, past shared memory at 32 tokens."""
+    p = bb.linear_launch_plan(bb.Config(bb.NVFP4, 16, 8, 0), 16, 27648, 27648)
+    assert p["cluster"] == 2
     assert p["smem32"] > p["smem_limit"]
     assert p["path"] == "fused"
 
